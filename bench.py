@@ -1,0 +1,343 @@
+"""Benchmark of the B200 FP8 x FP4 MoE expert layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--workload ID]
+
+A step is one moe_forward (routing + gather, GEMM1 + SwiGLU + requant, GEMM2,
+combine) over one batch of seeded synthetic inputs already resident in HBM.
+The default workload is the decode case (T=8, E=384, top-6, H=7168, I=3072);
+``--workload`` picks another row of the workload table.  With N > 1 (torchrun,
+one process per GPU) every rank runs an independent replica of the layer (the
+single-GPU layer has no exchange step) and the value is the whole job's
+throughput.  Prints one JSON line on rank 0.
+
+``--impl reference`` times the CPU oracle on the host cores instead (a bounded
+sample of the same workload per step), as the comparison arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer µs & TFLOP/s (E=384,k=6,H=7168,I=3072); % of HBM/TC roofline"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    p.add_argument("--workload", type=int, default=1)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the oracle's timed sample")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def expert_bytes(w):
+    """FP4 + UE8M0 bytes of one expert's L1 and L2 (0.5 + 1/32 byte per weight)."""
+    l1 = 2 * w.I * w.H * 17 // 32
+    l2 = w.H * w.I * 17 // 32
+    return l1, l2
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = f"/tmp/moe_bench_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def build_layer(w, device):
+    """Seeded bf16 draws quantised and packed by the CUDA library, resident in HBM."""
+    import moe_expert_layer_08_b200 as moe
+    x = W.gen_x(w, device)
+    idx, tw = W.gen_routing(w, device)
+    xq, xs = moe.quantize_fp8(x)
+    n1, n2 = moe.transformed_weight_bytes(w.E, w.H, w.I)
+    l1_t = torch.empty(n1, dtype=torch.uint8, device=device)
+    l2_t = torch.empty(n2, dtype=torch.uint8, device=device)
+    p1, p2 = n1 // w.E, n2 // w.E
+    for e in range(w.E):
+        a, b = moe.quantize_fp4(W.gen_l1(w, e, device))
+        c, d = moe.quantize_fp4(W.gen_l2(w, e, device))
+        moe.transform_weights(a[None], b[None], c[None], d[None],
+                              out=(l1_t[e * p1:(e + 1) * p1], l2_t[e * p2:(e + 1) * p2]))
+    torch.cuda.synchronize()
+    return dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw, l1_t=l1_t, l2_t=l2_t)
+
+
+def oracle_sample(w, ntok, device):
+    """Host inputs of the oracle for the first ``ntok`` tokens (oracle-quantised)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    x = W.gen_x(w, device)
+    idx, tw = W.gen_routing(w, device)
+    idx, tw = idx.cpu().numpy(), tw.cpu().numpy()
+    tokens = np.arange(min(ntok, w.T), dtype=np.int32)
+    xq, xs = oracle.quantize_e4m3(x.float().cpu().numpy())
+    need = sorted(set(int(e) for e in idx[tokens].ravel()))
+
+    def quant(item):
+        e, a, b = item
+        return e, oracle.quantize_e2m1(a) + oracle.quantize_e2m1(b)
+
+    with ThreadPoolExecutor(max(1, min(len(need), os.cpu_count() or 1))) as pool:
+        futs = [pool.submit(quant, (e, W.gen_l1(w, e, device).float().cpu().numpy(),
+                                    W.gen_l2(w, e, device).float().cpu().numpy())) for e in need]
+        experts = dict(f.result() for f in futs)
+    return dict(xq=xq, xs=xs, idx=idx, tw=tw, experts=experts, tokens=tokens)
+
+
+def time_oracle(w, s, steps):
+    import oracle
+    threads = min(len(s["tokens"]), oracle.num_threads(0))
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.forward(s["xq"], s["xs"], s["idx"], s["tw"], s["experts"], w.E, w.H, w.I,
+                       tokens=s["tokens"], threads=threads)
+        times.append(time.perf_counter() - t0)
+    flops = 2 * len(s["tokens"]) * w.k * 3 * w.H * w.I
+    return flops, times, threads
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    s = oracle_sample(w, args.cpu_tokens, device)
+    flops, times, threads = time_oracle(w, s, args.warmup + args.steps)
+    t = float(np.mean(times[args.warmup:])) if args.steps > 0 else float(np.mean(times))
+    value = flops / t / 1e12
+    sample = f"first {len(s['tokens'])} of {w.T} tokens (all {w.k} experts each) per step"
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")}},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_b200(args, w, rank, world, local_rank):
+    import moe_expert_layer_08_b200 as moe
+    from moe_expert_layer_08_b200 import build as mbuild
+    if rank == 0:
+        mbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    g = build_layer(w, device)
+    layer = moe.MoELayer(g["l1_t"], g["l2_t"], w.E, w.k, w.H, w.I, T_max=w.T, device=device)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.NUM_STAGE_EVENTS)]
+          for _ in range(args.steps)]
+
+    def step(events=None):
+        layer(g["xq"], g["xs"], g["idx"], g["tw"], out=out, events=events, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = moe.check_device_error(layer.workspace)
+    if st != 0:
+        raise RuntimeError(f"device error after warm-up: {moe.STATUS.get(st, st)}")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clocks:
+        barrier()
+        start.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        stop.record(stream)
+        barrier()
+    total_ms = start.elapsed_time(stop)
+    stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(moe.NUM_STAGE_EVENTS - 1)] for e in ev])
+    ms = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs -> device -> layer -> host output
+    h_xq = g["xq"].cpu().pin_memory()
+    h_xs = g["xs"].cpu().pin_memory()
+    h_idx = g["idx"].cpu().pin_memory()
+    h_tw = g["tw"].cpu().pin_memory()
+    h_out = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+    d_xq, d_xs = torch.empty_like(g["xq"]), torch.empty_like(g["xs"])
+    d_idx, d_tw = torch.empty_like(g["idx"]), torch.empty_like(g["tw"])
+    h2d = sum(t.numel() * t.element_size() for t in (h_xq, h_xs, h_idx, h_tw))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        d_xq.copy_(h_xq, non_blocking=True)
+        d_xs.copy_(h_xs, non_blocking=True)
+        d_idx.copy_(h_idx, non_blocking=True)
+        d_tw.copy_(h_tw, non_blocking=True)
+        layer(d_xq, d_xs, d_idx, d_tw, out=out, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    stop.record(stream)
+    barrier()
+    e2e_ms = start.elapsed_time(stop) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    st = moe.check_device_error(layer.workspace)
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {moe.STATUS.get(st, st)}")
+
+    if rank != 0:
+        return
+    # roofline of the dominant kernel (GEMM1 or GEMM2), timed by the stage events
+    touched = len(W.touched_experts(g["idx"].cpu(), w.E))
+    b1, b2 = expert_bytes(w)
+    g1_ms, g2_ms = float(stage_ms[:, 1].mean()), float(stage_ms[:, 2].mean())
+    pk = peaks()
+    if g1_ms >= g2_ms:
+        kname, kms, kbytes = "moe_gemm_kernel<gemm1>", g1_ms, touched * b1
+    else:
+        kname, kms, kbytes = "moe_gemm_kernel<gemm2>", g2_ms, touched * b2
+    achieved = kbytes / (kms * 1e-3) / 1e9
+    layer_bytes = touched * (b1 + b2) + w.T * w.H * 33 // 32 + w.T * w.k * 12 + w.T * w.H * 2
+    flops = w.flops
+    value = world * flops / (ms * 1e-3) / 1e12
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8xfp4 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")},
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (touched expert weights per step >> 126 MB)"
+                   if touched * (b1 + b2) > 256e6 else "inputs fit in L2 (not flushed)"},
+        "us_per_layer": ms * 1e3,
+        "effective_GBps": layer_bytes / (ms * 1e-3) / 1e9,
+        "hbm_frac_layer": layer_bytes / (ms * 1e-3) / 1e9 / pk["hbm"],
+        "touched_experts": touched,
+        "stage_us": {"route_gather": float(stage_ms[:, 0].mean() * 1e3), "gemm1": g1_ms * 1e3,
+                     "gemm2": g2_ms * 1e3, "combine": float(stage_ms[:, 3].mean() * 1e3)},
+        "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm"], "peak_source": pk["source"], "traffic": None},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        s = oracle_sample(w, args.cpu_tokens, device)
+        cflops, times, threads = time_oracle(w, s, 1)
+        line["cpu_baseline"] = {"value": cflops / times[0] / 1e12, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "seconds": times[0],
+                                "sample": f"first {len(s['tokens'])} of {w.T} tokens, all {w.k} experts each"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if args.impl == "b200" else "gloo",
+                                             timeout=datetime.timedelta(seconds=120))
+    w = W.WORKLOADS[args.workload]
+    try:
+        if args.impl == "reference":
+            run_reference(args, w, rank, world)
+        else:
+            run_b200(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

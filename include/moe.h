@@ -1,0 +1,186 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) FP8 x FP4 MoE expert layer.
+ *
+ * One MoE expert layer on one GPU: top-k routing to a per-expert token
+ * permutation, grouped GEMM1 of FP8 E4M3 activations against FP4 E2M1 expert
+ * weights (both with one UE8M0 scale per 32 elements along K), SwiGLU fused
+ * with an FP8 E4M3 + UE8M0 requantisation, grouped GEMM2, and a top-k-weighted
+ * combine back to bf16 tokens.  It restates, for a single GPU, the five-phase
+ * "Mega MoE" pipeline of the pages "Mega moe fusion with symmetric memory"
+ * (Procedure, step 5: dispatch, GEMM1, SwiGLU, GEMM2, combine) and MATE's
+ * "Mega MoE" API page (API: get_symm_buffer_for_mega_moe,
+ * transform_weights_for_mega_moe, fp8_fp8_mega_moe); the cross-rank dispatch
+ * and combine become a local gather and a local weighted scatter.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers (cudaMalloc / torch CUDA tensors)
+ *    unless stated otherwise; arrays are dense, row-major, contiguous.
+ *  - The caller owns every buffer; no entry point allocates device memory.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the host is never synchronised, except by
+ *    moe_check_device_error and moe_read_routing, which say so.
+ *  - Arguments are validated on the host before any CUDA call.  A rejected
+ *    call returns a non-zero moe_status_t and touches no memory.
+ *  - FP4 E2M1 is packed two per byte, element 2c in the low nibble of byte c.
+ *  - UE8M0 scale bytes b mean 2^(b-127) and are stored in K order: byte g of
+ *    a row scales elements 32g .. 32g+31 of that row.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,        /* null / misaligned pointer, negative size */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* H or I not a multiple of 128, I > 8192, E > 1024, ... */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+    MOE_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed */
+    MOE_ERR_BAD_ROUTING = 5,        /* device-detected expert id outside [0, E) */
+    MOE_ERR_DEVICE_TIMEOUT = 6      /* a bounded device-side wait gave up */
+} moe_status_t;
+
+/* Number of events moe_forward records when given an event array. */
+#define MOE_NUM_STAGE_EVENTS 5
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *moe_status_string(int status);
+
+/* Library ABI version (increments on any signature change). */
+int moe_abi_version(void);
+
+/*
+ * moe_quantize_fp8 -- per-row, per-32 FP8 E4M3 quantisation with UE8M0 scales
+ * (the activation cast `per_token_cast_to_fp8(x, use_ue8m0=True, gran_k=32)`
+ * of the DeepGEMM PR #416 review thread, test body).
+ *   x      : bf16 [rows, cols], cols % 32 == 0, 16-byte aligned
+ *   q      : u8   [rows, cols]      E4M3 codes (out)
+ *   sf     : u8   [rows, cols/32]   UE8M0 bytes (out)
+ * Per group of 32: e = smallest integer with amax <= 448 * 2^e (amax = 0 gives
+ * e = 0), scale byte e+127 clamped to [0, 254]; code = round-to-nearest-even
+ * of v * 2^-e, sign bit = sign bit of v.  Same rule as the layer's SwiGLU
+ * requantisation.
+ */
+moe_status_t moe_quantize_fp8(const void *x, int64_t rows, int64_t cols,
+                              void *q, void *sf, moe_stream_t stream);
+
+/*
+ * moe_quantize_fp4 -- per-row, per-32 FP4 E2M1 quantisation with UE8M0 scales
+ * (the weight cast `_cast_weights_to_fp4` of the same test body), same rule
+ * with format maximum 6.
+ *   w      : bf16 [rows, cols], cols % 32 == 0, 16-byte aligned
+ *   q      : u8   [rows, cols/2]    packed E2M1 (out)
+ *   sf     : u8   [rows, cols/32]   UE8M0 bytes (out)
+ */
+moe_status_t moe_quantize_fp4(const void *w, int64_t rows, int64_t cols,
+                              void *q, void *sf, moe_stream_t stream);
+
+/*
+ * moe_transformed_weight_bytes -- sizes of the two tile-major weight buffers
+ * that moe_transform_weights writes for E experts (host-only, no CUDA call).
+ */
+moe_status_t moe_transformed_weight_bytes(int E, int H, int I,
+                                          size_t *l1_bytes, size_t *l2_bytes);
+
+/*
+ * moe_transform_weights -- model-load-time layout transform
+ * (`transform_weights_for_mega_moe(l1, l2, tile_pack=True)`: MATE "Mega MoE"
+ * API; DeepGEMM PR #394 "cluster-paired FP4 weight packets", Summary and
+ * Motivation).  Packs each expert's logical FP4 weights and their UE8M0
+ * scales into packets of one 128-row x 128-K tile followed by the 512 scale
+ * bytes that tile consumes, so body and scales share one allocation and one
+ * access stream.  Packet order: expert -> output tile -> K tile -> (gate, up)
+ * for L1; expert -> output tile -> K tile for L2.
+ *   l1    : u8 [E, 2I, H/2]   rows 0..I-1 gate, I..2I-1 up     (in)
+ *   l1_sf : u8 [E, 2I, H/32]                                   (in)
+ *   l2    : u8 [E, H, I/2]                                     (in)
+ *   l2_sf : u8 [E, H, I/32]                                    (in)
+ *   l1_t, l2_t : outputs of moe_transformed_weight_bytes size, 256-byte aligned
+ * H % 128 == 0, I % 128 == 0, I <= 8192.  To transform one expert at a time,
+ * call with E = 1 and pointers offset to that expert: the packets of expert e
+ * start at e * (l1_bytes / E) and e * (l2_bytes / E).
+ */
+moe_status_t moe_transform_weights(const void *l1, const void *l1_sf,
+                                   const void *l2, const void *l2_sf,
+                                   int E, int H, int I,
+                                   void *l1_t, void *l2_t, moe_stream_t stream);
+
+/*
+ * moe_workspace_bytes -- device workspace moe_forward needs for up to T_max
+ * tokens (host-only).  Holds the routing metadata (counts, offsets,
+ * permutation and inverse, tile list), the gathered FP8 activations, the FP8
+ * SwiGLU output with its scales and the bf16 GEMM2 rows: the runtime workspace
+ * of MATE's "Mega MoE" page (Typical Flow), sized for the worst case.
+ */
+moe_status_t moe_workspace_bytes(int T_max, int E, int k, int H, int I, size_t *bytes);
+
+/*
+ * moe_forward -- one MoE expert layer (`fp8_fp4_mega_moe(y, l1, l2, buffer)`;
+ * the five phases of "Mega moe fusion with symmetric memory", Procedure step 5,
+ * on one GPU).
+ *   x_fp8    : u8  [T, H]      E4M3 activations, 16-byte aligned
+ *   x_sf     : u8  [T, H/32]   UE8M0 activation scales, 4-byte aligned
+ *   topk_idx : i64 [T, k]      expert ids; an id outside [0, E) is dropped
+ *                              (contributes nothing) and reported by
+ *                              moe_check_device_error as MOE_ERR_BAD_ROUTING;
+ *                              a repeated id counts as separate routed rows
+ *   topk_w   : f32 [T, k]      combine weights
+ *   l1_t, l2_t : buffers written by moe_transform_weights
+ *   out_bf16 : bf16 [T, H]     out[t] = bf16_rne(sum_j topk_w[t,j] * Y(t,j)),
+ *                              fully overwritten, 16-byte aligned
+ *   workspace: >= moe_workspace_bytes(T, E, k, H, I) bytes, 256-byte aligned;
+ *              its contents after the call are the routing metadata of this
+ *              call (moe_read_routing) and scratch
+ *   expert_stats : nullable i32 [E]; when given, expert_stats[e] += rows routed
+ *              to e (the `cumulative_local_expert_recv_stats` of the API page)
+ *   stage_events : nullable array of MOE_NUM_STAGE_EVENTS cudaEvent_t; when
+ *              given, recorded on `stream` before routing, before GEMM1,
+ *              before GEMM2, before the combine and after the combine
+ * Computes per routed row r = (t, j, e): C1 = x[t] . L1[e]^T (fp32),
+ * h = silu(C1[:, :I]) * C1[:, I:], h -> FP8 E4M3 + UE8M0 per 32 (the
+ * moe_quantize_fp8 rule), Y = h . L2[e]^T (fp32, stored bf16), then the
+ * weighted combine in ascending j.  T = 0 is a no-op.  The call is
+ * asynchronous and performs no host synchronisation.
+ */
+moe_status_t moe_forward(const void *x_fp8, const void *x_sf,
+                         const int64_t *topk_idx, const float *topk_w,
+                         const void *l1_t, const void *l2_t, void *out_bf16,
+                         int T, int E, int k, int H, int I,
+                         void *workspace, size_t ws_bytes,
+                         int32_t *expert_stats, void *const *stage_events,
+                         moe_stream_t stream);
+
+/*
+ * moe_read_routing -- copies the routing metadata of the last moe_forward that
+ * used `workspace` with these (T, E, k, H, I) into HOST arrays (test and
+ * inspection hook; synchronises `stream`).  Any output may be NULL.
+ *   count  : i32 [E]     rows routed to each expert
+ *   offset : i32 [E+1]   exclusive scan of count
+ *   perm   : i32 [T*k]   perm[r] = t*k+j of routed row r, rows of one expert
+ *                        in ascending t*k+j; entries >= offset[E] unused
+ *   inv    : i32 [T*k]   inv[t*k+j] = r, or -1 for a dropped slot
+ */
+moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H, int I,
+                              int32_t *count, int32_t *offset, int32_t *perm,
+                              int32_t *inv, moe_stream_t stream);
+
+/*
+ * moe_check_device_error -- synchronises `stream`, then reads the device error
+ * word of the last moe_forward on `workspace`: MOE_OK, MOE_ERR_BAD_ROUTING
+ * (an expert id was out of range) or MOE_ERR_DEVICE_TIMEOUT (a bounded wait
+ * inside a kernel gave up; that call's output is undefined).
+ */
+moe_status_t moe_check_device_error(const void *workspace, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,231 @@
+"""B200 (sm_100a) FP8 x FP4 MoE expert layer -- Python binding of include/moe.h.
+
+Every entry point of the C ABI has a function of the same name here (without
+the ``moe_`` prefix).  This module only marshals torch tensors into pointers
+and sizes and allocates outputs with torch; every step of the layer runs in the
+CUDA library ``libmoe_b200.so`` next to this file.  There is no fallback: if
+the library is missing, loading fails with an error naming the build command.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "MoEError", "load", "status_string", "abi_version", "quantize_fp8", "quantize_fp4",
+    "transformed_weight_bytes", "transform_weights", "workspace_bytes", "forward",
+    "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+NUM_STAGE_EVENTS = 5
+STATUS = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+    3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_ROUTING",
+    6: "MOE_ERR_DEVICE_TIMEOUT",
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+def _declare(lib):
+    c = ctypes
+    P, I32, I64, SZ = c.c_void_p, c.c_int, c.c_int64, c.c_size_t
+    sig = {
+        "moe_status_string": (c.c_char_p, [I32]),
+        "moe_abi_version": (I32, []),
+        "moe_quantize_fp8": (I32, [P, I64, I64, P, P, P]),
+        "moe_quantize_fp4": (I32, [P, I64, I64, P, P, P]),
+        "moe_transformed_weight_bytes": (I32, [I32, I32, I32, c.POINTER(SZ), c.POINTER(SZ)]),
+        "moe_transform_weights": (I32, [P, P, P, P, I32, I32, I32, P, P, P]),
+        "moe_workspace_bytes": (I32, [I32, I32, I32, I32, I32, c.POINTER(SZ)]),
+        "moe_forward": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P]),
+        "moe_read_routing": (I32, [P, I32, I32, I32, I32, I32, P, P, P, P, P]),
+        "moe_check_device_error": (I32, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+def load():
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"{LIB_PATH} is missing; build it with `python -m moe_expert_layer_08_b200.build`")
+            _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MoEError(status, what)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+def status_string(status: int) -> str:
+    return load().moe_status_string(status).decode()
+
+
+def abi_version() -> int:
+    return load().moe_abi_version()
+
+
+def quantize_fp8(x: torch.Tensor, stream=None):
+    """bf16 [rows, cols] -> (E4M3 codes u8 [rows, cols], UE8M0 u8 [rows, cols/32])."""
+    _need(x, torch.bfloat16, "x", 2)
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
+    _check(load().moe_quantize_fp8(_ptr(x), rows, cols, _ptr(q), _ptr(sf), _stream(stream)), "moe_quantize_fp8")
+    return q, sf
+
+
+def quantize_fp4(w: torch.Tensor, stream=None):
+    """bf16 [rows, cols] -> (packed E2M1 u8 [rows, cols/2], UE8M0 u8 [rows, cols/32])."""
+    _need(w, torch.bfloat16, "w", 2)
+    rows, cols = w.shape
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=w.device)
+    sf = torch.empty((rows, cols // 32), dtype=torch.uint8, device=w.device)
+    _check(load().moe_quantize_fp4(_ptr(w), rows, cols, _ptr(q), _ptr(sf), _stream(stream)), "moe_quantize_fp4")
+    return q, sf
+
+
+def transformed_weight_bytes(E: int, H: int, I: int):
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().moe_transformed_weight_bytes(E, H, I, ctypes.byref(a), ctypes.byref(b)),
+           "moe_transformed_weight_bytes")
+    return a.value, b.value
+
+
+def transform_weights(l1, l1_sf, l2, l2_sf, out=None, stream=None):
+    """[E, 2I, H/2], [E, 2I, H/32], [E, H, I/2], [E, H, I/32] (u8) -> (l1_t, l2_t)
+    tile-packet buffers (u8, 1-D).  ``out`` may give the two destination views."""
+    for t, n in ((l1, "l1"), (l1_sf, "l1_sf"), (l2, "l2"), (l2_sf, "l2_sf")):
+        _need(t, torch.uint8, n, 3)
+    E, twoI, Hh = l1.shape
+    H, I = Hh * 2, twoI // 2
+    if l1_sf.shape != (E, 2 * I, H // 32) or l2.shape != (E, H, I // 2) or l2_sf.shape != (E, H, I // 32):
+        raise ValueError("inconsistent weight shapes")
+    n1, n2 = transformed_weight_bytes(E, H, I)
+    if out is None:
+        l1_t = torch.empty(n1, dtype=torch.uint8, device=l1.device)
+        l2_t = torch.empty(n2, dtype=torch.uint8, device=l1.device)
+    else:
+        l1_t, l2_t = out
+        if l1_t.numel() < n1 or l2_t.numel() < n2:
+            raise ValueError("output buffers too small")
+    _check(load().moe_transform_weights(_ptr(l1), _ptr(l1_sf), _ptr(l2), _ptr(l2_sf), E, H, I,
+                                        _ptr(l1_t), _ptr(l2_t), _stream(stream)), "moe_transform_weights")
+    return l1_t, l2_t
+
+
+def workspace_bytes(T: int, E: int, k: int, H: int, I: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().moe_workspace_bytes(T, E, k, H, I, ctypes.byref(n)), "moe_workspace_bytes")
+    return n.value
+
+
+def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
+            out=None, workspace=None, expert_stats=None, events=None, stream=None):
+    """One layer; returns out (bf16 [T, H]).  ``events``: optional list of
+    NUM_STAGE_EVENTS torch.cuda.Event recorded at the stage boundaries."""
+    _need(x_fp8, torch.uint8, "x_fp8", 2)
+    _need(x_sf, torch.uint8, "x_sf", 2)
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(l1_t, torch.uint8, "l1_t")
+    _need(l2_t, torch.uint8, "l2_t")
+    T, k = topk_idx.shape
+    if x_fp8.shape != (T, H) or x_sf.shape != (T, H // 32) or topk_w.shape != (T, k):
+        raise ValueError("inconsistent activation / routing shapes")
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x_fp8.device)
+    else:
+        _need(out, torch.bfloat16, "out", 2)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(T, E, k, H, I), dtype=torch.uint8, device=x_fp8.device)
+    else:
+        _need(workspace, torch.uint8, "workspace")
+    if expert_stats is not None:
+        _need(expert_stats, torch.int32, "expert_stats", 1)
+    ev = None
+    if events is not None:
+        if len(events) != NUM_STAGE_EVENTS:
+            raise ValueError(f"events must hold {NUM_STAGE_EVENTS} torch.cuda.Event")
+        ev = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[e.cuda_event for e in events])
+    st = load().moe_forward(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t), _ptr(l2_t),
+                            _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),
+                            _ptr(expert_stats), ev, _stream(stream))
+    _check(st, "moe_forward")
+    return out
+
+
+def read_routing(workspace, T: int, E: int, k: int, H: int, I: int, stream=None):
+    """Routing metadata of the last forward on ``workspace`` (host int32 tensors)."""
+    count = torch.empty(E, dtype=torch.int32)
+    offset = torch.empty(E + 1, dtype=torch.int32)
+    perm = torch.empty(max(T * k, 1), dtype=torch.int32)
+    inv = torch.empty(max(T * k, 1), dtype=torch.int32)
+    _check(load().moe_read_routing(_ptr(workspace), T, E, k, H, I, _ptr(count), _ptr(offset), _ptr(perm),
+                                   _ptr(inv), _stream(stream)), "moe_read_routing")
+    n = int(offset[E])
+    return dict(count=count, offset=offset, perm=perm[:n].clone(), inv=inv[: T * k].clone())
+
+
+def check_device_error(workspace, stream=None) -> int:
+    """Synchronises the stream and returns the status of the last forward on
+    ``workspace`` (0, MOE_ERR_BAD_ROUTING or MOE_ERR_DEVICE_TIMEOUT)."""
+    return load().moe_check_device_error(_ptr(workspace), _stream(stream))
+
+
+class MoELayer:
+    """Holds one layer's transformed weights and a workspace for up to T_max tokens."""
+
+    def __init__(self, l1_t, l2_t, E: int, k: int, H: int, I: int, T_max: int, device=None):
+        self.l1_t, self.l2_t = l1_t, l2_t
+        self.E, self.k, self.H, self.I, self.T_max = E, k, H, I, T_max
+        device = device or l1_t.device
+        self.workspace = torch.empty(workspace_bytes(T_max, E, k, H, I), dtype=torch.uint8, device=device)
+
+    def __call__(self, x_fp8, x_sf, topk_idx, topk_w, out=None, expert_stats=None, events=None, stream=None):
+        if topk_idx.shape[0] > self.T_max:
+            raise ValueError(f"T={topk_idx.shape[0]} exceeds T_max={self.T_max}")
+        return forward(x_fp8, x_sf, topk_idx, topk_w, self.l1_t, self.l2_t, self.E, self.H, self.I,
+                       out=out, workspace=self.workspace, expert_stats=expert_stats, events=events,
+                       stream=stream)

@@ -1,0 +1,301 @@
+// api.cu -- the C ABI declared in include/moe.h: host validation (fails closed
+// before any CUDA call, as the DeepGEMM PR #394 "Scope and fallback" section
+// asks of unsupported shapes), workspace layout, TMA descriptor encoding and
+// the launch sequence of one layer.
+#include <mutex>
+
+#include "moe.h"
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+WsLayout ws_layout(int T, int E, int k, int H, int I) {
+    WsLayout L;
+    L.R = int64_t(T) * k;
+    L.nb = int((L.R + kRouteBlock - 1) / kRouteBlock);
+    if (L.nb < 1) L.nb = 1;
+    L.max_chunks = (L.R + kChunkRows - 1) / kChunkRows + (L.R < E ? L.R : E);
+    const size_t R = size_t(L.R > 0 ? L.R : 1);
+    const size_t MC = size_t(L.max_chunks > 0 ? L.max_chunks : 1);
+    size_t o = kHdrBytes;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o += align_up(bytes, 256);
+        return at;
+    };
+    L.off_count = take(sizeof(int) * size_t(E));
+    L.off_offset = take(sizeof(int) * size_t(E + 1));
+    L.off_chunk_base = take(sizeof(int) * size_t(E + 1));
+    L.off_chunks = take(sizeof(int4) * MC);
+    L.off_hist = take(sizeof(int) * size_t(L.nb) * size_t(E));
+    L.off_bad = take(sizeof(int) * size_t(L.nb));
+    L.off_lrank = take(sizeof(int) * R);
+    L.off_perm = take(sizeof(int) * R);
+    L.off_inv = take(sizeof(int) * R);
+    L.off_xg = take(R * size_t(H));
+    L.off_xg_sf = take(MC * size_t(H / kTileK) * kSfBlockBytes);
+    L.off_hq = take(R * size_t(I));
+    L.off_hq_sf = take(MC * size_t(I / kTileK) * kSfBlockBytes);
+    L.off_y = take(R * size_t(H) * 2);
+    L.total = o;
+    return L;
+}
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// Tile packets as a 3D tensor of 4-bit elements: (128 K, 128 rows, packet),
+// one 128 x 128 box per load, expanded to one byte per element in shared
+// memory with the 128-byte swizzle.
+bool encode_packets(CUtensorMap *m, const void *base, int64_t num_packets) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(kTileK), cuuint64_t(kTileRows), cuuint64_t(num_packets)};
+    const cuuint64_t strides[2] = {cuuint64_t(kTileK / 2), cuuint64_t(kPacketBytes)};
+    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(kTileRows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major FP8 activations [rows, cols] as bytes, 128 x 16 boxes.
+bool encode_rows(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(cols)};
+    const cuuint32_t box[2] = {cuuint32_t(kTileK), cuuint32_t(kBoxRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t check_shape(int E, int H, int I) {
+    if (E <= 0 || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+    if (H % kTileK != 0 || I % kTileK != 0 || I > kMaxI || E > kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (int64_t(H) * 2 * I > (int64_t(1) << 40)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+// Make the device that owns `p` current (the library carries its own runtime
+// state, so the caller's current device is not visible to it).
+moe_status_t use_device_of(const void *p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return MOE_ERR_INVALID_ARG;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cur != attr.device && cudaSetDevice(attr.device) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int num_sms() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_status_string(int status) {
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_BAD_ROUTING: return "MOE_ERR_BAD_ROUTING";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+        default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+int moe_abi_version(void) { return 1; }
+
+moe_status_t moe_quantize_fp8(const void *x, int64_t rows, int64_t cols, void *q, void *sf, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!x || !q || !sf || !aligned(x, 16) || !aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = use_device_of(q);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_quantize(x, rows, cols, q, sf, true, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_quantize_fp4(const void *w, int64_t rows, int64_t cols, void *q, void *sf, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!w || !q || !sf || !aligned(w, 16) || !aligned(q, 16)) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = use_device_of(q);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_quantize(w, rows, cols, q, sf, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_transformed_weight_bytes(int E, int H, int I, size_t *l1_bytes, size_t *l2_bytes) {
+    const moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    const size_t per_tile_k = size_t(H / kTileK) * size_t(I / kTileRows);  // packets per expert per half
+    if (l1_bytes) *l1_bytes = size_t(E) * per_tile_k * 2 * kPacketBytes;
+    if (l2_bytes) *l2_bytes = size_t(E) * per_tile_k * kPacketBytes;
+    return MOE_OK;
+}
+
+moe_status_t moe_transform_weights(const void *l1, const void *l1_sf, const void *l2, const void *l2_sf, int E,
+                                   int H, int I, void *l1_t, void *l2_t, moe_stream_t stream) {
+    const moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    if (!l1 || !l1_sf || !l2 || !l2_sf || !l1_t || !l2_t) return MOE_ERR_INVALID_ARG;
+    if (!aligned(l1, 16) || !aligned(l2, 16) || !aligned(l1_sf, 4) || !aligned(l2_sf, 4) || !aligned(l1_t, 256) ||
+        !aligned(l2_t, 256))
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t d = use_device_of(l1_t);
+    if (d != MOE_OK) return d;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_transform(l1, l1_sf, E, 2 * I, H, I / kTileRows, 2, I, l1_t, st);
+    if (e == cudaSuccess) e = launch_transform(l2, l2_sf, E, H, I, H / kTileRows, 1, 0, l2_t, st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_workspace_bytes(int T_max, int E, int k, int H, int I, size_t *bytes) {
+    const moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    if (T_max < 0 || k <= 0 || k > E || !bytes) return MOE_ERR_INVALID_ARG;
+    if (int64_t(T_max) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+    *bytes = ws_layout(T_max, E, k, H, I).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_forward(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
+                         const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                         void *workspace, size_t ws_bytes, int32_t *expert_stats, void *const *stage_events,
+                         moe_stream_t stream) {
+    moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    if (T < 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+    if (int64_t(T) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!x_fp8 || !x_sf || !topk_idx || !topk_w || !l1_t || !l2_t || !out_bf16 || !workspace)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_fp8, 16) || !aligned(x_sf, 4) || !aligned(topk_idx, 8) || !aligned(topk_w, 4) ||
+        !aligned(l1_t, 256) || !aligned(l2_t, 256) || !aligned(out_bf16, 16) || !aligned(workspace, 256) ||
+        (expert_stats && !aligned(expert_stats, 4)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, E, k, H, I);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    size_t l1_bytes = 0, l2_bytes = 0;
+    moe_transformed_weight_bytes(E, H, I, &l1_bytes, &l2_bytes);
+
+    CUtensorMap tm_w1, tm_w2, tm_xg, tm_hq;
+    if (!encode_packets(&tm_w1, l1_t, int64_t(l1_bytes / kPacketBytes)) ||
+        !encode_packets(&tm_w2, l2_t, int64_t(l2_bytes / kPacketBytes)) ||
+        !encode_rows(&tm_xg, ws + L.off_xg, L.R, H) || !encode_rows(&tm_hq, ws + L.off_hq, L.R, I))
+        return MOE_ERR_CUDA;
+
+    auto record = [&](int i) -> cudaError_t {
+        if (!stage_events || !stage_events[i]) return cudaSuccess;
+        return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st);
+    };
+    const int sms = num_sms();
+    const int64_t items1 = L.max_chunks * (I / kTileRows);
+    const int64_t items2 = L.max_chunks * (H / kTileRows);
+    const int grid1 = int(items1 < sms ? items1 : sms);
+    const int grid2 = int(items2 < sms ? items2 : sms);
+
+    cudaError_t e = record(0);
+    if (e == cudaSuccess)
+        e = launch_route(topk_idx, static_cast<const uint8_t *>(x_fp8), static_cast<const uint8_t *>(x_sf), T, k, E,
+                         H, ws, L, expert_stats, st);
+    if (e == cudaSuccess) e = record(1);
+    if (e == cudaSuccess)
+        e = launch_gemm(true, tm_w1, tm_xg, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
+    if (e == cudaSuccess) e = record(2);
+    if (e == cudaSuccess)
+        e = launch_gemm(false, tm_w2, tm_hq, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
+    if (e == cudaSuccess) e = record(3);
+    if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
+    if (e == cudaSuccess) e = record(4);
+    return cuda_status(e);
+}
+
+moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H, int I, int32_t *count,
+                              int32_t *offset, int32_t *perm, int32_t *inv, moe_stream_t stream) {
+    moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    if (!workspace || T < 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    const WsLayout L = ws_layout(T, E, k, H, I);
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (count) e = cudaMemcpyAsync(count, ws + L.off_count, sizeof(int32_t) * E, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && offset)
+        e = cudaMemcpyAsync(offset, ws + L.off_offset, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && perm && L.R > 0)
+        e = cudaMemcpyAsync(perm, ws + L.off_perm, sizeof(int32_t) * L.R, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && inv && L.R > 0)
+        e = cudaMemcpyAsync(inv, ws + L.off_inv, sizeof(int32_t) * L.R, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_check_device_error(const void *workspace, moe_stream_t stream) {
+    if (!workspace) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    int word = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (word & kDevErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+    if (word & kDevErrBadRouting) return MOE_ERR_BAD_ROUTING;
+    return MOE_OK;
+}
+
+}  // extern "C"

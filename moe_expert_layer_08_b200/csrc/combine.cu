@@ -1,0 +1,55 @@
+// combine.cu -- the top-k-weighted combine back to token order (phase 5 of
+// "Mega moe fusion with symmetric memory", Procedure step 5, on one GPU: a
+// local gather through the inverse permutation instead of cross-rank stores).
+// out[t] = bf16_rne(sum_{j ascending} topk_w[t, j] * Y[inv[t*k + j]]), fp32
+// sum, no atomics, so the result is deterministic.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+constexpr int kCombineThreads = 128;
+constexpr int kCombineCols = kCombineThreads * 8;  // 8 bf16 (16 bytes) per thread
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfloat16 *__restrict__ y,
+                                                                  const int *__restrict__ inv,
+                                                                  const float *__restrict__ topk_w, int k, int H,
+                                                                  int col_blocks, __nv_bfloat16 *__restrict__ out) {
+    const int64_t t = blockIdx.x / col_blocks;
+    const int col = (blockIdx.x % col_blocks) * kCombineCols + threadIdx.x * 8;
+    if (col >= H) return;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const int r = __ldg(inv + t * k + j);
+        if (r < 0) continue;  // dropped slot
+        const float wv = __ldg(topk_w + t * k + j);
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col));
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += wv * __uint_as_float(u[i] << 16);
+            acc[2 * i + 1] += wv * __uint_as_float(u[i] & 0xFFFF0000u);
+        }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        o[i] = *reinterpret_cast<const uint32_t *>(&b);
+    }
+    *reinterpret_cast<uint4 *>(out + t * H + col) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
+                           void *out, cudaStream_t stream) {
+    const int col_blocks = (H + kCombineCols - 1) / kCombineCols;
+    const int64_t grid = int64_t(T) * col_blocks;
+    combine_kernel<<<unsigned(grid), kCombineThreads, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(ws + L.off_y), reinterpret_cast<const int *>(ws + L.off_inv),
+        topk_w, k, H, col_blocks, static_cast<__nv_bfloat16 *>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,115 @@
+// quant.cu -- the per-32 UE8M0 quantisers (activation cast to FP8 E4M3 and
+// weight cast to FP4 E2M1, the casts of the DeepGEMM PR #416 review thread's
+// test body) and the model-load weight transform into tile packets (DeepGEMM
+// PR #394, "cluster-paired FP4 weight packets": body and scale words of one
+// tile stored together, in the order the GEMM reads them).
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+// One thread per group of 32 consecutive elements of a row: 64 bytes of bf16
+// in, 32 bytes (FP8) or 16 bytes (FP4) of codes and one scale byte out.
+template <bool kFp8>
+__global__ void __launch_bounds__(256) quantize_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
+                                                       int64_t cols, uint8_t *__restrict__ q,
+                                                       uint8_t *__restrict__ sf) {
+    const int64_t gpr = cols / 32;
+    const int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (g >= rows * gpr) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + g * 32);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 w = __ldg(src + i);
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[i * 8 + j * 2] = __uint_as_float(u[j] << 16);
+            v[i * 8 + j * 2 + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+        }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e = scale_exponent<kFp8>(amax);
+    const float m = exp2_neg(e);
+    sf[g] = uint8_t(e + 127);
+    if (kFp8) {
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            w[i] = to_e4m3(v[4 * i] * m) | (to_e4m3(v[4 * i + 1] * m) << 8) | (to_e4m3(v[4 * i + 2] * m) << 16) |
+                   (to_e4m3(v[4 * i + 3] * m) << 24);
+        uint4 *dst = reinterpret_cast<uint4 *>(q + g * 32);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc |= to_e2m1(v[8 * i + j] * m) << (4 * j);
+            w[i] = acc;
+        }
+        *reinterpret_cast<uint4 *>(q + g * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, void *q, void *sf, bool fp8,
+                            cudaStream_t stream) {
+    const int64_t groups = rows * (cols / 32);
+    if (groups == 0) return cudaSuccess;
+    const int64_t blocks = (groups + 255) / 256;
+    if (fp8)
+        quantize_kernel<true><<<unsigned(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(x), rows, cols, static_cast<uint8_t *>(q), static_cast<uint8_t *>(sf));
+    else
+        quantize_kernel<false><<<unsigned(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(x), rows, cols, static_cast<uint8_t *>(q), static_cast<uint8_t *>(sf));
+    return cudaGetLastError();
+}
+
+// One 128-thread block per packet (grid-stride): thread r copies the 64 bytes
+// of row r of the tile and writes that row's 4 scale bytes into the packet's
+// 512-byte scale block.  Packet p = ((e * tiles + tile) * KB + kb) * halves + half
+// holds source rows half * half_rows + tile * 128 + [0, 128) of expert e,
+// K columns kb * 128 + [0, 128).
+__global__ void __launch_bounds__(128) transform_kernel(const uint8_t *__restrict__ w, const uint8_t *__restrict__ w_sf,
+                                                        int rows_per_expert, int K, int tiles, int halves,
+                                                        int half_rows, int64_t num_packets, uint8_t *__restrict__ out) {
+    const int KB = K / kTileK;
+    const int r = threadIdx.x;
+    for (int64_t p = blockIdx.x; p < num_packets; p += gridDim.x) {
+        int64_t q = p;
+        const int half = int(q % halves);
+        q /= halves;
+        const int kb = int(q % KB);
+        q /= KB;
+        const int tile = int(q % tiles);
+        const int64_t e = q / tiles;
+        const int64_t src_row = e * rows_per_expert + int64_t(half) * half_rows + int64_t(tile) * kTileRows + r;
+        const uint4 *src = reinterpret_cast<const uint4 *>(w + src_row * (K / 2) + kb * (kTileK / 2));
+        uint8_t *pkt = out + p * kPacketBytes;
+        uint4 *dst = reinterpret_cast<uint4 *>(pkt + r * (kTileK / 2));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
+        const uint32_t s = __ldg(reinterpret_cast<const uint32_t *>(w_sf + src_row * (K / 32) + kb * 4));
+        *reinterpret_cast<uint32_t *>(pkt + kPacketBody + sf_block_offset(r, 0)) = s;
+    }
+}
+
+cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int tiles,
+                             int halves, int half_rows, void *out, cudaStream_t stream) {
+    const int64_t num_packets = int64_t(E) * tiles * (K / kTileK) * halves;
+    if (num_packets == 0) return cudaSuccess;
+    const int64_t grid = num_packets < 65536 ? num_packets : 65536;
+    transform_kernel<<<unsigned(grid), 128, 0, stream>>>(static_cast<const uint8_t *>(w),
+                                                         static_cast<const uint8_t *>(w_sf), rows_per_expert, K,
+                                                         tiles, halves, half_rows, num_packets,
+                                                         static_cast<uint8_t *>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

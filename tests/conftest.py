@@ -16,3 +16,12 @@ def pytest_configure(config):
 def olib():
     import oracle
     return oracle.load()
+
+
+@pytest.fixture(scope="session")
+def moelib():
+    """The CUDA library, built in place if missing (nvcc cross-compiles here)."""
+    from moe_expert_layer_08_b200 import build
+    build.build()
+    import moe_expert_layer_08_b200 as m
+    return m.load()

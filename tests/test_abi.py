@@ -1,0 +1,98 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/moe.h declares, and validates arguments on the host (before any CUDA
+call, so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for need in ("moe_forward", "moe_transform_weights", "moe_workspace_bytes", "moe_read_routing",
+                 "moe_check_device_error", "moe_quantize_fp8", "moe_quantize_fp4"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(moelib):
+    for name in declared_functions():
+        assert hasattr(moelib, name), name
+
+
+def test_status_strings(moelib):
+    assert moelib.moe_status_string(0) == b"MOE_OK"
+    assert moelib.moe_status_string(3) == b"MOE_ERR_WORKSPACE_TOO_SMALL"
+    assert moelib.moe_status_string(99) == b"MOE_ERR_UNKNOWN"
+    assert moelib.moe_abi_version() >= 1
+
+
+def test_sizes_are_host_only_and_consistent(moelib):
+    import moe_expert_layer_08_b200 as m
+    l1, l2 = m.transformed_weight_bytes(384, 7168, 3072)
+    per_expert = (2 * 3072 * 7168 + 7168 * 3072) // 2 + (2 * 3072 * 7168 + 7168 * 3072) // 32
+    assert l1 + l2 == 384 * per_expert == 384 * 35094528
+    a = m.workspace_bytes(8, 384, 6, 7168, 3072)
+    b = m.workspace_bytes(8192, 384, 6, 7168, 3072)
+    assert 0 < a < b
+    assert m.workspace_bytes(0, 8, 2, 256, 256) > 0
+
+
+@pytest.mark.parametrize("E,H,I,status", [(8, 200, 256, 2), (8, 256, 200, 2), (8, 256, 8320, 2),
+                                          (2000, 256, 256, 2), (0, 256, 256, 1)])
+def test_bad_shapes_fail_closed(moelib, E, H, I, status):
+    import moe_expert_layer_08_b200 as m
+    with pytest.raises(m.MoEError) as ei:
+        m.transformed_weight_bytes(E, H, I)
+    assert ei.value.status == status
+    n = ctypes.c_size_t()
+    assert moelib.moe_workspace_bytes(4, E, 2, H, I, ctypes.byref(n)) == status
+
+
+def test_forward_validation_before_any_cuda_call(moelib):
+    f = moelib.moe_forward
+    p = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+    # unsupported shape
+    assert f(p, p, p, p, p, p, p, 4, 8, 2, 200, 256, p, 1 << 30, None, None, None) == 2
+    # k > E, negative T
+    assert f(p, p, p, p, p, p, p, 4, 8, 9, 256, 256, p, 1 << 30, None, None, None) == 1
+    assert f(p, p, p, p, p, p, p, -1, 8, 2, 256, 256, p, 1 << 30, None, None, None) == 1
+    # T = 0 is a no-op
+    assert f(None, None, None, None, None, None, None, 0, 8, 2, 256, 256, None, 0, None, None, None) == 0
+    # null / misaligned pointers
+    assert f(None, p, p, p, p, p, p, 4, 8, 2, 256, 256, p, 1 << 30, None, None, None) == 1
+    q = ctypes.c_void_p(0x10001)
+    assert f(q, p, p, p, p, p, p, 4, 8, 2, 256, 256, p, 1 << 30, None, None, None) == 1
+    # workspace too small
+    assert f(p, p, p, p, p, p, p, 4, 8, 2, 256, 256, p, 16, None, None, None) == 3
+
+
+def test_quantize_and_transform_validation(moelib):
+    p = ctypes.c_void_p(0x10000)
+    assert moelib.moe_quantize_fp8(p, 4, 33, p, p, None) == 2
+    assert moelib.moe_quantize_fp4(p, -1, 32, p, p, None) == 1
+    assert moelib.moe_quantize_fp8(None, 0, 32, None, None, None) == 0
+    assert moelib.moe_transform_weights(p, p, p, p, 4, 256, 200, p, p, None) == 2
+    assert moelib.moe_transform_weights(None, p, p, p, 4, 256, 256, p, p, None) == 1
+    odd = ctypes.c_void_p(0x10080)  # 128- but not 256-byte aligned destination
+    assert moelib.moe_transform_weights(p, p, p, p, 4, 256, 256, odd, p, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import moe_expert_layer_08_b200 as m
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(m, "_lib", None)
+    with pytest.raises(ImportError):
+        m.load()

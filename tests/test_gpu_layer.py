@@ -1,0 +1,131 @@
+"""GPU parity of the whole layer (moe_forward through the C ABI) against the
+oracle, element by element per token row: rel L2 <= 1e-2 and max abs <=
+5e-2 * max|row| (the tolerance the layer is specified with).  Small cases are
+checked on every token; the full-size workloads on sampled tokens, each of
+which the oracle evaluates exactly (a token's output depends only on its own
+row and its experts)."""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from cases import compare_rows, experts_of, gpu_layer, oracle_side
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe(moelib):
+    import moe_expert_layer_08_b200 as m
+    return m
+
+
+def run_and_compare(moe, w, routing=None, tokens=None, gen_device="cuda", check_repeat=True):
+    g = gpu_layer(w, routing=routing, gen_device=gen_device)
+    ws = torch.empty(moe.workspace_bytes(w.T, w.E, w.k, w.H, w.I), dtype=torch.uint8, device="cuda")
+    out = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, workspace=ws)
+    status = moe.check_device_error(ws)
+    idx = g["idx"].cpu().numpy()
+    if check_repeat:
+        out2 = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, workspace=ws)
+        assert torch.equal(out.view(torch.int16), out2.view(torch.int16)), "not deterministic"
+    tok = np.arange(w.T) if tokens is None else np.asarray(tokens)
+    xq, xs, ex = oracle_side(w, g["x"], g["idx"], experts_of(idx, tok, w.E), gen_device=gen_device)
+    ref = oracle.forward(xq, xs, idx, g["tw"].cpu().numpy(), ex, w.E, w.H, w.I,
+                         tokens=None if tokens is None else tok.astype(np.int32))
+    worst = compare_rows(out[torch.as_tensor(tok, device="cuda")], ref["out_bf16"], w.name)
+    del g, ws, out
+    gc.collect()
+    torch.cuda.empty_cache()
+    return status, worst
+
+
+SMALL = [
+    W.WORKLOADS[0],
+    W.custom("ragged", T=37, E=5, k=3, H=384, I=256, seed=21),              # chunk rows not /16
+    W.custom("multichunk", T=300, E=2, k=2, H=256, I=128, seed=22),         # experts with > 128 rows
+    W.custom("k_eq_E", T=20, E=4, k=4, H=256, I=384, seed=23),
+    W.custom("one_token", T=1, E=16, k=4, H=512, I=256, seed=24),
+    W.custom("wide", T=33, E=3, k=2, H=1024, I=1024, seed=25),
+    W.custom("zipf_small", T=512, E=32, k=4, H=256, I=256, seed=26, routing="zipf"),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_layer_small_all_tokens(moe, w):
+    status, _ = run_and_compare(moe, w)
+    assert status == 0
+
+
+def test_layer_single_expert_all_tokens_many_chunks(moe):
+    w = W.custom("hot", T=700, E=3, k=1, H=256, I=256, seed=27)
+    idx = torch.full((w.T, 1), 1, dtype=torch.int64)
+    tw = torch.ones((w.T, 1), dtype=torch.float32)
+    status, _ = run_and_compare(moe, w, routing=(idx, tw))
+    assert status == 0
+
+
+def test_layer_structured_routing(moe):
+    w = W.custom("structured", T=96, E=12, k=4, H=256, I=256, seed=28)
+    status, _ = run_and_compare(moe, w, routing=W.structured_routing(w.T, w.k, w.E))
+    assert status == 0
+
+
+def test_layer_duplicate_and_dropped_slots(moe):
+    w = W.custom("dup_drop", T=24, E=6, k=3, H=256, I=256, seed=29)
+    idx, tw = W.gen_routing(w)
+    idx[0, 1] = idx[0, 0]        # same expert twice
+    idx[5, 2] = 99               # dropped
+    idx[7] = -1                  # a token with every slot dropped
+    status, _ = run_and_compare(moe, w, routing=(idx, tw))
+    assert status == 5  # MOE_ERR_BAD_ROUTING is reported, the rest is computed
+
+
+def test_layer_decode_full(moe):
+    w = W.WORKLOADS[1]            # T=8, E=384, k=6, H=7168, I=3072: every token
+    status, _ = run_and_compare(moe, w)
+    assert status == 0
+
+
+@pytest.mark.parametrize("cfg,ntok", [(2, 12), (3, 8), (4, 8)])
+def test_layer_full_size_sampled(moe, cfg, ntok):
+    w = W.WORKLOADS[cfg]
+    idx, tw = W.gen_routing(w, "cuda")
+    ic = idx.cpu().numpy()
+    rng = np.random.default_rng(cfg)
+    tokens = set(rng.choice(w.T, ntok - 2, replace=False).tolist()) | {0, w.T - 1}
+    if cfg == 4:
+        # include tokens of the hottest expert, whose rows span many chunks
+        hot = np.bincount(ic.ravel(), minlength=w.E).argmax()
+        users = np.nonzero((ic == hot).any(axis=1))[0]
+        tokens |= {int(users[0]), int(users[len(users) // 2]), int(users[-1])}
+    status, _ = run_and_compare(moe, w, routing=(idx, tw), tokens=sorted(tokens), check_repeat=False)
+    assert status == 0
+
+
+def test_expert_stats_accumulate(moe):
+    w = W.custom("stats", T=40, E=8, k=2, H=128, I=128, seed=30)
+    g = gpu_layer(w)
+    stats = torch.zeros(w.E, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, expert_stats=stats)
+    ref = np.bincount(g["idx"].cpu().numpy().ravel(), minlength=w.E) * 3
+    assert np.array_equal(stats.cpu().numpy(), ref)
+
+
+def test_stage_events_and_stream(moe):
+    w = W.WORKLOADS[0]
+    g = gpu_layer(w)
+    s = torch.cuda.Stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(moe.NUM_STAGE_EVENTS)]
+    with torch.cuda.stream(s):
+        out = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I,
+                          events=ev, stream=s)
+    s.synchronize()
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(moe.NUM_STAGE_EVENTS - 1)]
+    assert all(t >= 0 for t in times)
+    ref = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I)
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
