@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--workload", type=int, default=1)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the oracle's timed sample")
+    p.add_argument("--experts", type=int, default=0,
+                   help="override E (a smaller resident weight set for profiler captures)")
     return p.parse_args()
 
 
@@ -329,6 +331,9 @@ def main():
         torch.distributed.init_process_group("nccl" if args.impl == "b200" else "gloo",
                                              timeout=datetime.timedelta(seconds=120))
     w = W.WORKLOADS[args.workload]
+    if args.experts:
+        w = W.custom(f"{w.name}_E{args.experts}", T=w.T, E=args.experts, k=w.k, H=w.H, I=w.I, seed=w.seed,
+                     routing=w.routing, zipf_s=w.zipf_s)
     try:
         if args.impl == "reference":
             run_reference(args, w, rank, world)

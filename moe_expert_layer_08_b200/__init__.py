@@ -188,6 +188,9 @@ def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
     if events is not None:
         if len(events) != NUM_STAGE_EVENTS:
             raise ValueError(f"events must hold {NUM_STAGE_EVENTS} torch.cuda.Event")
+        for e in events:
+            if e.cuda_event == 0:  # torch creates events lazily, on first record
+                e.record(stream if stream is not None else torch.cuda.current_stream())
         ev = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[e.cuda_event for e in events])
     st = load().moe_forward(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t), _ptr(l2_t),
                             _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),

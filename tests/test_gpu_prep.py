@@ -27,7 +27,7 @@ def special_rows(cols, gen):
     rows.append(torch.randn(cols, generator=gen) * 3e4)
     r = torch.randn(cols, generator=gen)
     r[5] = 448.0                             # exactly on a scale boundary
-    r[40] = 6.0
+    r[min(40, cols - 1)] = 6.0
     rows.append(r)
     rows.append(torch.full((cols,), -0.0))
     return torch.stack(rows)
@@ -111,7 +111,7 @@ def route_through_forward(moe, T, k, E, idx, H=128, I=128):
 
 ROUTING_CASES = [
     ("uniform", 64, 2, 8), ("uniform", 8, 6, 384), ("uniform", 1000, 6, 384), ("uniform", 8192, 6, 384),
-    ("zipf", 4096, 8, 256), ("structured", 96, 4, 12), ("one_expert", 300, 1, 5), ("dups", 77, 4, 3),
+    ("zipf", 4096, 8, 256), ("structured", 96, 4, 12), ("one_expert", 300, 1, 5), ("dups", 77, 3, 3),
 ]
 
 
