@@ -179,6 +179,49 @@ moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H,
  */
 moe_status_t moe_check_device_error(const void *workspace, moe_stream_t stream);
 
+/*
+ * moe_forward_static -- moe_forward without a caller-provided workspace, for
+ * callers that cannot allocate device memory.  The pages have no counterpart
+ * of this entry point; it exists for this library's users.
+ *
+ * Who cannot allocate: code that runs while a CUDA graph is being captured
+ * (cudaMalloc is not a stream operation and is not allowed there), serving
+ * runtimes that reserve all device memory for their own pools at start-up and
+ * forbid allocation on the request path, and plug-ins called from inside
+ * another framework's operator that cannot reach that framework's allocator
+ * and must not call cudaMalloc, which can synchronise the device.
+ *
+ * Arguments and results are those of moe_forward, minus the workspace: the
+ * caller still passes (and owns) every input and the output.  The layer's
+ * scratch is one file-scope device array of MOE_STATIC_WORKSPACE_BYTES inside
+ * this library, which every GPU that loads the library holds until the
+ * process exits.  This entry point allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *  - The first call on a device looks up the array's device address on that
+ *    device (cudaGetSymbolAddress); make that first call before any stream
+ *    capture on that device.
+ *  - A (T, E, k, H, I) whose moe_workspace_bytes exceeds
+ *    MOE_STATIC_WORKSPACE_BYTES is rejected with MOE_ERR_WORKSPACE_TOO_SMALL
+ *    before any device work (decode-sized batches fit: T = 128 tokens at
+ *    E = 384, top-6, H = 7168, I = 3072 needs 33.3 MiB).
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents; nothing in it needs to start at zero.  Calls that overlap on
+ *    the GPU (different streams, or threads without ordering between their
+ *    streams) race on it and give undefined results: issue them in order on
+ *    one stream.
+ *  - Out-of-range expert ids are dropped as in moe_forward, but the device
+ *    error word lives in the shared array, so moe_check_device_error cannot
+ *    report it for this entry point.
+ */
+#define MOE_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
+
+moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf,
+                                const int64_t *topk_idx, const float *topk_w,
+                                const void *l1_t, const void *l2_t, void *out_bf16,
+                                int T, int E, int k, int H, int I,
+                                int32_t *expert_stats, void *const *stage_events,
+                                moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,10 +18,12 @@ __all__ = [
     "MoEError", "load", "status_string", "abi_version", "quantize_fp8", "quantize_fp4",
     "transformed_weight_bytes", "transform_weights", "workspace_bytes", "forward",
     "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
+    "forward_static", "STATIC_WORKSPACE_BYTES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
 NUM_STAGE_EVENTS = 5
+STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024  # MOE_STATIC_WORKSPACE_BYTES
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_BAD_ROUTING",
@@ -52,6 +54,7 @@ def _declare(lib):
         "moe_forward": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P]),
         "moe_read_routing": (I32, [P, I32, I32, I32, I32, I32, P, P, P, P, P]),
         "moe_check_device_error": (I32, [P, P]),
+        "moe_forward_static": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -196,6 +199,35 @@ def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
                             _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),
                             _ptr(expert_stats), ev, _stream(stream))
     _check(st, "moe_forward")
+    return out
+
+
+def forward_static(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
+                   out=None, expert_stats=None, stream=None):
+    """The layer for callers that cannot allocate device memory: the scratch is
+    the library's fixed STATIC_WORKSPACE_BYTES device array (see
+    moe_forward_static in include/moe.h; calls on one device must not overlap
+    on the GPU).  ``out`` must be given by such callers; when it is None this
+    helper allocates it with torch for convenience."""
+    _need(x_fp8, torch.uint8, "x_fp8", 2)
+    _need(x_sf, torch.uint8, "x_sf", 2)
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(l1_t, torch.uint8, "l1_t")
+    _need(l2_t, torch.uint8, "l2_t")
+    T, k = topk_idx.shape
+    if x_fp8.shape != (T, H) or x_sf.shape != (T, H // 32) or topk_w.shape != (T, k):
+        raise ValueError("inconsistent activation / routing shapes")
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x_fp8.device)
+    else:
+        _need(out, torch.bfloat16, "out", 2)
+    if expert_stats is not None:
+        _need(expert_stats, torch.int32, "expert_stats", 1)
+    st = load().moe_forward_static(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t),
+                                   _ptr(l2_t), _ptr(out), T, E, k, H, I, _ptr(expert_stats), None,
+                                   _stream(stream))
+    _check(st, "moe_forward_static")
     return out
 
 

@@ -88,6 +88,25 @@ bool encode_rows(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int num_sms() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 moe_status_t check_shape(int E, int H, int I) {
@@ -112,24 +131,48 @@ moe_status_t use_device_of(const void *p) {
     return MOE_OK;
 }
 
-int num_sms() {
-    static std::mutex mu;
-    static int cache[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    std::lock_guard<std::mutex> g(mu);
-    if (dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cache[dev] = n > 0 ? n : 148;
-    }
-    return cache[dev];
+// The launch sequence of one layer on a validated workspace (shared by the
+// entry points that run the layer).  The workspace's device must be current.
+moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
+                       const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                       uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream) {
+    const WsLayout L = ws_layout(T, E, k, H, I);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    size_t l1_bytes = 0, l2_bytes = 0;
+    moe_transformed_weight_bytes(E, H, I, &l1_bytes, &l2_bytes);
+
+    CUtensorMap tm_w1, tm_w2, tm_xg, tm_hq;
+    if (!encode_packets(&tm_w1, l1_t, int64_t(l1_bytes / kPacketBytes)) ||
+        !encode_packets(&tm_w2, l2_t, int64_t(l2_bytes / kPacketBytes)) ||
+        !encode_rows(&tm_xg, ws + L.off_xg, L.R, H) || !encode_rows(&tm_hq, ws + L.off_hq, L.R, I))
+        return MOE_ERR_CUDA;
+
+    auto record = [&](int i) -> cudaError_t {
+        if (!stage_events || !stage_events[i]) return cudaSuccess;
+        return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st);
+    };
+    const int sms = num_sms();
+    const int64_t items1 = L.max_chunks * (I / kTileRows);
+    const int64_t items2 = L.max_chunks * (H / kTileRows);
+    const int grid1 = int(items1 < sms ? items1 : sms);
+    const int grid2 = int(items2 < sms ? items2 : sms);
+
+    cudaError_t e = record(0);
+    if (e == cudaSuccess)
+        e = launch_route(topk_idx, static_cast<const uint8_t *>(x_fp8), static_cast<const uint8_t *>(x_sf), T, k, E,
+                         H, ws, L, expert_stats, st);
+    if (e == cudaSuccess) e = record(1);
+    if (e == cudaSuccess)
+        e = launch_gemm(true, tm_w1, tm_xg, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
+    if (e == cudaSuccess) e = record(2);
+    if (e == cudaSuccess)
+        e = launch_gemm(false, tm_w2, tm_hq, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
+    if (e == cudaSuccess) e = record(3);
+    if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
+    if (e == cudaSuccess) e = record(4);
+    return cuda_status(e);
 }
 
-moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
-
-}  // namespace
 }  // namespace moe
 
 using namespace moe;
@@ -224,42 +267,8 @@ moe_status_t moe_forward(const void *x_fp8, const void *x_sf, const int64_t *top
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     s = use_device_of(workspace);
     if (s != MOE_OK) return s;
-
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    size_t l1_bytes = 0, l2_bytes = 0;
-    moe_transformed_weight_bytes(E, H, I, &l1_bytes, &l2_bytes);
-
-    CUtensorMap tm_w1, tm_w2, tm_xg, tm_hq;
-    if (!encode_packets(&tm_w1, l1_t, int64_t(l1_bytes / kPacketBytes)) ||
-        !encode_packets(&tm_w2, l2_t, int64_t(l2_bytes / kPacketBytes)) ||
-        !encode_rows(&tm_xg, ws + L.off_xg, L.R, H) || !encode_rows(&tm_hq, ws + L.off_hq, L.R, I))
-        return MOE_ERR_CUDA;
-
-    auto record = [&](int i) -> cudaError_t {
-        if (!stage_events || !stage_events[i]) return cudaSuccess;
-        return cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st);
-    };
-    const int sms = num_sms();
-    const int64_t items1 = L.max_chunks * (I / kTileRows);
-    const int64_t items2 = L.max_chunks * (H / kTileRows);
-    const int grid1 = int(items1 < sms ? items1 : sms);
-    const int grid2 = int(items2 < sms ? items2 : sms);
-
-    cudaError_t e = record(0);
-    if (e == cudaSuccess)
-        e = launch_route(topk_idx, static_cast<const uint8_t *>(x_fp8), static_cast<const uint8_t *>(x_sf), T, k, E,
-                         H, ws, L, expert_stats, st);
-    if (e == cudaSuccess) e = record(1);
-    if (e == cudaSuccess)
-        e = launch_gemm(true, tm_w1, tm_xg, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
-    if (e == cudaSuccess) e = record(2);
-    if (e == cudaSuccess)
-        e = launch_gemm(false, tm_w2, tm_hq, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
-    if (e == cudaSuccess) e = record(3);
-    if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
-    if (e == cudaSuccess) e = record(4);
-    return cuda_status(e);
+    return run_layer(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, out_bf16, T, E, k, H, I,
+                     static_cast<uint8_t *>(workspace), expert_stats, stage_events, stream);
 }
 
 moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H, int I, int32_t *count,

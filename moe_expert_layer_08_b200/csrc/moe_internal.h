@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "moe.h"
+
 namespace moe {
 
 constexpr int kRouteBlock = 256;  // routed slots per routing block
@@ -38,5 +40,16 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
                         cudaStream_t stream);
 cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
                            void *out, cudaStream_t stream);
+
+// Argument checks shared by the entry points.
+bool aligned(const void *p, uintptr_t a);
+moe_status_t check_shape(int E, int H, int I);
+moe_status_t use_device_of(const void *p);
+
+// The launch sequence of one layer on a validated, large-enough workspace of
+// the current device.
+moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
+                       const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                       uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream);
 
 }  // namespace moe

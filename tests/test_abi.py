@@ -96,3 +96,12 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(m, "_lib", None)
     with pytest.raises(ImportError):
         m.load()
+
+
+def test_static_entry_point_rejects_oversize_before_any_cuda_call(moelib):
+    p = ctypes.c_void_p(0x10000)
+    # T = 4096 at E = 384, top-6, H = 7168, I = 3072 does not fit the fixed array
+    assert moelib.moe_forward_static(p, p, p, p, p, p, p, 4096, 384, 6, 7168, 3072, None, None, None) == 3
+    assert moelib.moe_forward_static(p, p, p, p, p, p, p, 4, 8, 2, 200, 256, None, None, None) == 2
+    assert moelib.moe_forward_static(None, None, None, None, None, None, None, 0, 8, 2, 256, 256,
+                                     None, None, None) == 0
