@@ -203,7 +203,7 @@ moe_status_t moe_check_device_error(const void *workspace, moe_stream_t stream);
  *  - A (T, E, k, H, I) whose moe_workspace_bytes exceeds
  *    MOE_STATIC_WORKSPACE_BYTES is rejected with MOE_ERR_WORKSPACE_TOO_SMALL
  *    before any device work (decode-sized batches fit: T = 128 tokens at
- *    E = 384, top-6, H = 7168, I = 3072 needs 33.3 MiB).
+ *    E = 384, top-6, H = 7168, I = 3072 needs 34 MiB).
  *  - All calls on a device share the one array, which keeps the last call's
  *    contents; nothing in it needs to start at zero.  Calls that overlap on
  *    the GPU (different streams, or threads without ordering between their

@@ -15,7 +15,11 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.R = int64_t(T) * k;
     L.nb = int((L.R + kRouteBlock - 1) / kRouteBlock);
     if (L.nb < 1) L.nb = 1;
-    L.max_chunks = (L.R + kChunkRows - 1) / kChunkRows + (L.R < E ? L.R : E);
+    // Small per-expert loads (decode) use 32-row chunks and the kN = 32 GEMMs;
+    // the chunk bound is taken for 32-row chunks either way, so the workspace
+    // size grows monotonically with T.
+    L.chunk_rows = L.R <= int64_t(8) * E ? kChunkRowsSmall : kChunkRows;
+    L.max_chunks = (L.R + kChunkRowsSmall - 1) / kChunkRowsSmall + (L.R < E ? L.R : E);
     const size_t R = size_t(L.R > 0 ? L.R : 1);
     const size_t MC = size_t(L.max_chunks > 0 ? L.max_chunks : 1);
     size_t o = kHdrBytes;
@@ -33,9 +37,13 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.off_lrank = take(sizeof(int) * R);
     L.off_perm = take(sizeof(int) * R);
     L.off_inv = take(sizeof(int) * R);
-    L.off_xg = take(R * size_t(H));
+    L.off_rowinfo = take(sizeof(int4) * R);
+    L.Rp = L.R > kActBoxRows ? L.R : kActBoxRows;
+    L.kbh = H / kTileK > 2 ? H / kTileK : 2;
+    L.kbi = I / kTileK > 2 ? I / kTileK : 2;
+    L.off_xg = take(size_t(L.Rp) * size_t(L.kbh) * kTileK);
     L.off_xg_sf = take(MC * size_t(H / kTileK) * kSfBlockBytes);
-    L.off_hq = take(R * size_t(I));
+    L.off_hq = take(size_t(L.Rp) * size_t(L.kbi) * kTileK);
     L.off_hq_sf = take(MC * size_t(I / kTileK) * kSfBlockBytes);
     L.off_y = take(R * size_t(H) * 2);
     L.total = o;
@@ -60,30 +68,46 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Tile packets as a 3D tensor of 4-bit elements: (128 K, 128 rows, packet),
-// one 128 x 128 box per load, expanded to one byte per element in shared
-// memory with the 128-byte swizzle.
-bool encode_packets(CUtensorMap *m, const void *base, int64_t num_packets) {
+// Tile packets as a 3D tensor of 4-bit elements: (128 K, 128 rows, packet);
+// one box moves `depth` consecutive 128 x 128 packet bodies, expanded to one
+// byte per element in shared memory with the 128-byte swizzle.
+bool encode_packets(CUtensorMap *m, const void *base, int64_t num_packets, int depth) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     const cuuint64_t dims[3] = {cuuint64_t(kTileK), cuuint64_t(kTileRows), cuuint64_t(num_packets)};
     const cuuint64_t strides[2] = {cuuint64_t(kTileK / 2), cuuint64_t(kPacketBytes)};
-    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(kTileRows), 1};
+    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(kTileRows), cuuint32_t(depth)};
     const cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major FP8 activations [rows, cols] as bytes, 128 x 16 boxes.
-bool encode_rows(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+// The same packets as 32-bit words [packet][2176]; a box of 128 words at word
+// 2048 is one packet's 512-byte scale block, `depth` packets per load.
+bool encode_packet_sf(CUtensorMap *m, const void *base, int64_t num_packets, int depth) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-    const cuuint64_t strides[1] = {cuuint64_t(cols)};
-    const cuuint32_t box[2] = {cuuint32_t(kTileK), cuuint32_t(kBoxRows)};
+    const cuuint64_t dims[2] = {cuuint64_t(kPacketBytes / 4), cuuint64_t(num_packets)};
+    const cuuint64_t strides[1] = {cuuint64_t(kPacketBytes)};
+    const cuuint32_t box[2] = {cuuint32_t(kPacketSf / 4), cuuint32_t(depth)};
     const cuuint32_t estr[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// FP8 activations stored K-block-major, [kblocks][rows][128] bytes, as a 3D
+// tensor (128 bytes, rows, K blocks); one box moves kActBoxRows rows of
+// `depth` consecutive K blocks.
+bool encode_act(CUtensorMap *m, const void *base, int64_t rows, int64_t kblocks, int depth) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(kTileK), cuuint64_t(rows), cuuint64_t(kblocks)};
+    const cuuint64_t strides[2] = {cuuint64_t(kTileK), cuuint64_t(rows) * kTileK};
+    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(kActBoxRows), cuuint32_t(depth)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -141,10 +165,13 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
     size_t l1_bytes = 0, l2_bytes = 0;
     moe_transformed_weight_bytes(E, H, I, &l1_bytes, &l2_bytes);
 
-    CUtensorMap tm_w1, tm_w2, tm_xg, tm_hq;
-    if (!encode_packets(&tm_w1, l1_t, int64_t(l1_bytes / kPacketBytes)) ||
-        !encode_packets(&tm_w2, l2_t, int64_t(l2_bytes / kPacketBytes)) ||
-        !encode_rows(&tm_xg, ws + L.off_xg, L.R, H) || !encode_rows(&tm_hq, ws + L.off_hq, L.R, I))
+    const int64_t np1 = int64_t(l1_bytes / kPacketBytes), np2 = int64_t(l2_bytes / kPacketBytes);
+    const int d1 = gemm_packets_per_stage(true, L.chunk_rows), d2 = gemm_packets_per_stage(false, L.chunk_rows);
+    CUtensorMap tm_w1, tm_w2, tm_s1, tm_s2, tm_xg, tm_hq;
+    if (!encode_packets(&tm_w1, l1_t, np1, d1) || !encode_packets(&tm_w2, l2_t, np2, d2) ||
+        !encode_packet_sf(&tm_s1, l1_t, np1, d1) || !encode_packet_sf(&tm_s2, l2_t, np2, d2) ||
+        !encode_act(&tm_xg, ws + L.off_xg, L.Rp, L.kbh, gemm_kblocks_per_stage(L.chunk_rows)) ||
+        !encode_act(&tm_hq, ws + L.off_hq, L.Rp, L.kbi, gemm_kblocks_per_stage(L.chunk_rows)))
         return MOE_ERR_CUDA;
 
     auto record = [&](int i) -> cudaError_t {
@@ -163,10 +190,10 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
                          H, ws, L, expert_stats, st);
     if (e == cudaSuccess) e = record(1);
     if (e == cudaSuccess)
-        e = launch_gemm(true, tm_w1, tm_xg, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
+        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
     if (e == cudaSuccess) e = record(2);
     if (e == cudaSuccess)
-        e = launch_gemm(false, tm_w2, tm_hq, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
+        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
     if (e == cudaSuccess) e = record(3);
     if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
     if (e == cudaSuccess) e = record(4);

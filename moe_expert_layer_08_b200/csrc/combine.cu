@@ -15,6 +15,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfl
                                                                   const int *__restrict__ inv,
                                                                   const float *__restrict__ topk_w, int k, int H,
                                                                   int col_blocks, __nv_bfloat16 *__restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t t = blockIdx.x / col_blocks;
     const int col = (blockIdx.x % col_blocks) * kCombineCols + threadIdx.x * 8;
     if (col >= H) return;
@@ -22,10 +24,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfl
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
     for (int j = 0; j < k; ++j) {
-        const int r = __ldg(inv + t * k + j);
+        const int r = __ldcg(inv + t * k + j);
         if (r < 0) continue;  // dropped slot
         const float wv = __ldg(topk_w + t * k + j);
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col));
+        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col));
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -46,10 +48,10 @@ cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *to
                            void *out, cudaStream_t stream) {
     const int col_blocks = (H + kCombineCols - 1) / kCombineCols;
     const int64_t grid = int64_t(T) * col_blocks;
-    combine_kernel<<<unsigned(grid), kCombineThreads, 0, stream>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(ws + L.off_y), reinterpret_cast<const int *>(ws + L.off_inv),
-        topk_w, k, H, col_blocks, static_cast<__nv_bfloat16 *>(out));
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
+                      reinterpret_cast<const __nv_bfloat16 *>(ws + L.off_y),
+                      reinterpret_cast<const int *>(ws + L.off_inv), topk_w, k, H, col_blocks,
+                      static_cast<__nv_bfloat16 *>(out));
 }
 
 }  // namespace moe

@@ -32,23 +32,45 @@
 
 namespace moe {
 
-template <bool kGemm1>
+// kN = the largest token chunk an item can hold (the MMA's N).  Small-batch
+// launches (kN = 32) take 256-K stages and two MMA-issuing warps: each
+// tcgen05.mma / tcgen05.cp costs a fixed issue slot whatever its N, so at
+// decode sizes the issue rate of a single thread, not HBM, would set the pace.
+template <bool kGemm1, int kN>
 struct GemmCfg {
-    static constexpr int kNumA = kGemm1 ? 2 : 1;        // accumulators (gate, up) or (down)
-    static constexpr int kStages = kGemm1 ? 4 : 6;
+    static constexpr bool kSmall = kN == kChunkRowsSmall;
+    static constexpr int kNumA = kGemm1 ? 2 : 1;        // weight tiles per K block: (gate, up) or (down)
+    static constexpr int kKB = kSmall ? 2 : 1;          // 128-K blocks per pipeline stage
+    static constexpr int kIssuers = kSmall ? 2 : 1;     // MMA-issuing warps
+    static constexpr int kStages = kSmall ? (kGemm1 ? 3 : 5) : (kGemm1 ? 4 : 6);
     static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 one-byte elements
-    static constexpr int kBTile = kChunkRows * kTileK;  // 16 KB: up to 128 token rows
-    static constexpr int kStageTiles = kNumA * kATile + kBTile;
-    static constexpr int kStageSf = (kNumA + 1) * kSfBlockBytes;
+    static constexpr int kBTile = kN * kTileK;          // token rows x 128 bytes, per K block
+    static constexpr int kStageTiles = kNumA * kKB * kATile + kKB * kBTile;
+    static constexpr int kStageSf = (kNumA * kKB + kKB) * kSfBlockBytes;
     static constexpr int kSmemTiles = kStages * kStageTiles;
     static constexpr int kSmemSf = kStages * kStageSf;
     static constexpr int kSmemMisc = 256;
     static constexpr int kSmemBytes = 1024 + kSmemTiles + kSmemSf + kSmemMisc;
-    static constexpr int kAccCols = kNumA * kChunkRows;
-    static constexpr int kSfCols = kStages * (kNumA + 1) * 4;
-    static constexpr int kTmemCols = (kAccCols + kSfCols) <= 256 ? 256 : 512;
-    static_assert(kAccCols + kSfCols <= kTmemCols, "TMEM budget");
+    // Accumulators per buffer: GEMM1 (gate, up); GEMM2 one per issuer (a
+    // K split, summed by the epilogue).
+    static constexpr int kNumAcc = kGemm1 ? 2 : kIssuers;
+    static constexpr int kAccCols = kNumAcc * kN;
+    // Per issuer and stage: the scale blocks of the weight tiles it consumes
+    // and of the activation K blocks it consumes, 4 TMEM columns each.
+    static constexpr int kIssuerKB = (!kGemm1 && kIssuers == 2) ? 1 : kKB;
+    static constexpr int kIssuerAcc = (kGemm1 && kIssuers == 1) ? 2 : 1;
+    static constexpr int kSfColsIssuer = kIssuerKB * (kIssuerAcc + 1) * 4;
+    static constexpr int kSfCols = kStages * kIssuers * kSfColsIssuer;
+    static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
+    static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
+    static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                   : kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kThreads = 224 + 32 * (kIssuers - 1);  // + activation producer, + second issuer
+    static_assert(kTmemUsed <= 512, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kBTile % 1024 == 0, "swizzle atoms");
+    static_assert(kKB == 1 || kN == kActBoxRows, "one activation box per stage when a stage spans K blocks");
+    static_assert(kGemm1 || kIssuers == 1 || kKB == kIssuers, "GEMM2 K split needs one K block per issuer");
 };
 
 struct GemmArgs {
@@ -62,6 +84,7 @@ struct GemmArgs {
     int K;                     // reduction length (H for GEMM1, I for GEMM2)
     int n_tiles;               // output tiles per expert (I/128 or H/128)
     int out_ld;                // row length of the output (I or H)
+    int rows;                  // row extent of the K-block-major FP8 operands
 };
 
 // After the call lane l holds max over the warp's lanes of a[l] (the input
@@ -81,36 +104,40 @@ __device__ __forceinline__ float warp_transpose_max(float (&a)[32], int lane) {
     return a[0];
 }
 
-template <bool kGemm1>
-__global__ void __launch_bounds__(192, 1)
-    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_act,
-                    const GemmArgs args) {
-    using C = GemmCfg<kGemm1>;
-    constexpr int kNumA = C::kNumA, kStages = C::kStages;
+template <bool kGemm1, int kN>
+__global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_wsf,
+                    const __grid_constant__ CUtensorMap tmap_act, const GemmArgs args) {
+    using C = GemmCfg<kGemm1, kN>;
+    constexpr int kNumA = C::kNumA, kKB = C::kKB, kStages = C::kStages, kBufs = C::kAccBufs;
+    constexpr int kIssuers = C::kIssuers;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tiles = smem;
     uint8_t *sfs = tiles + C::kSmemTiles;
     uint64_t *full = reinterpret_cast<uint64_t *>(sfs + C::kSmemSf);
     uint64_t *empty = full + kStages;
-    uint64_t *tmem_full = empty + kStages;
-    uint64_t *tmem_empty = tmem_full + 1;
-    uint64_t *mma_done = tmem_empty + 1;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *tmem_full = empty + kStages;   // [2]
+    uint64_t *tmem_empty = tmem_full + 2;    // [2]
+    uint64_t *mma_done = tmem_empty + 2;     // [kIssuers]
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&full[s], 2);  // weight producer + activation producer
+            mbar_init(&empty[s], kIssuers);
         }
-        mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 4);
-        mbar_init(mma_done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], kIssuers);
+            mbar_init(&tmem_empty[b], 4);
+        }
+        for (int i = 0; i < 2; ++i) mbar_init(&mma_done[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_wsf);
         prefetch_tmap(&tmap_act);
     }
     if (warp == 1) {
@@ -122,46 +149,69 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // GEMM2's weights do not depend on GEMM1, so its producer streams the
+    // first stages' weight tiles before waiting for GEMM1 to finish; every
+    // other access to memory written by earlier kernels comes after pdl_wait.
+    const bool early_weights = !kGemm1;
+    const bool is_w_producer = warp == 0 && lane == 0;
+    if (!(early_weights && is_w_producer)) pdl_wait();
+    if (threadIdx.x == 32) pdl_trigger();
+
     const int n_tiles = args.n_tiles;
-    const int num_items = args.hdr[kHdrNumChunks] * n_tiles;
+    const int num_items = __ldcg(args.hdr + kHdrNumChunks) * n_tiles;
     const int KB = args.K / kTileK;
+    const int n_steps = (KB + kKB - 1) / kKB;  // pipeline stages per item
     int *err = args.hdr;
 
-    if (warp == 0) {
+    // which MMA issuer this warp is (-1: none)
+    const int issuer = warp == 1 ? 0 : (kIssuers == 2 && warp == 7) ? 1 : -1;
+
+    if (warp == 0 || warp == 6) {
         if (lane == 0) {
-            // ------------------------------------------------------------ producer
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_a = policy_evict_last();
+            // ------------------------------------------------------------ producers
+            // warp 0: weight packets and their scale blocks (one box each per
+            // stage); warp 6: the chunk's activation K blocks (one 3D box of
+            // kKB K blocks x 32 rows per 32 rows) and their scale blocks.
+            const bool weights = warp == 0;
+            const uint64_t pol = weights ? policy_evict_first() : policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0, fill_parity = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
                 const int c = item / n_tiles, tile = item % n_tiles;
-                const int4 ch = args.chunks[c];
-                const int nbox = (ch.z + kBoxRows - 1) / kBoxRows;
-                const uint32_t bytes = kNumA * (kPacketBody + kPacketSf) + nbox * kBoxRows * kTileK + kSfBlockBytes;
+                const int4 ch = __ldcg(args.chunks + c);
+                const int nbox = (ch.z + kActBoxRows - 1) / kActBoxRows;
                 const int64_t pkt0 = (int64_t(ch.x) * n_tiles + tile) * KB * kNumA;
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, 1)) {
+                for (int step = 0; step < n_steps; ++step) {
+                    const int kb0 = step * kKB;
+                    const int nkb = min(kKB, KB - kb0);
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, weights ? 1 : 5)) {
                         ok = false;
                         break;
                     }
                     uint8_t *st = tiles + stage * C::kStageTiles;
                     uint8_t *sf = sfs + stage * C::kStageSf;
-                    mbar_arrive_expect_tx(&full[stage], bytes);
-#pragma unroll
-                    for (int a = 0; a < kNumA; ++a) {
-                        const int64_t pkt = pkt0 + int64_t(kb) * kNumA + a;
-                        tma_load_3d(st + a * C::kATile, &tmap_w, &full[stage], 0, 0, int(pkt), pol_w);
-                        bulk_load(sf + a * kSfBlockBytes, args.w_packets + pkt * kPacketBytes + kPacketBody,
-                                  kSfBlockBytes, &full[stage], pol_w);
+                    if (weights) {
+                        // the weight boxes always move kNumA * kKB packets (a
+                        // last odd K block loads one packet it then ignores)
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(kNumA * kKB * (kPacketBody + kPacketSf)));
+                        const int pkt = int(pkt0 + int64_t(kb0) * kNumA);
+                        tma_load_3d(st, &tmap_w, &full[stage], 0, 0, pkt, pol);
+                        tma_load_2d(sf, &tmap_wsf, &full[stage], kPacketBody / 4, pkt, pol);
+                    } else {
+                        // the activation box always moves kKB K blocks (a K
+                        // block past the end reads zeros)
+                        mbar_arrive_expect_tx(&full[stage],
+                                              uint32_t(nbox * kKB * kActBoxRows * kTileK + nkb * kSfBlockBytes));
+                        uint8_t *bt = st + kNumA * kKB * C::kATile;
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_3d(bt + j * kActBoxRows * kTileK, &tmap_act, &full[stage], 0,
+                                        ch.y + j * kActBoxRows, kb0, pol);
+                        bulk_load(sf + kNumA * kKB * kSfBlockBytes,
+                                  args.act_sf + (int64_t(c) * KB + kb0) * kSfBlockBytes, nkb * kSfBlockBytes,
+                                  &full[stage], pol);
                     }
-                    for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(st + kNumA * C::kATile + j * kBoxRows * kTileK, &tmap_act, &full[stage],
-                                    kb * kTileK, ch.y + j * kBoxRows, pol_a);
-                    bulk_load(sf + kNumA * kSfBlockBytes, args.act_sf + (int64_t(c) * KB + kb) * kSfBlockBytes,
-                              kSfBlockBytes, &full[stage], pol_a);
                     filled |= 1u << stage;
                     fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) {
@@ -180,41 +230,62 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (issuer >= 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
+            // GEMM1: issuer 0 owns the gate accumulator, issuer 1 the up one
+            // (a single issuer owns both).  GEMM2: issuer i owns accumulator i
+            // and the stage's K block i.
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            uint32_t phase = 0;
+            int li = 0;  // items handled by this CTA so far
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
-                const int4 ch = args.chunks[item / n_tiles];
-                const uint32_t n = uint32_t((ch.z + kBoxRows - 1) / kBoxRows * kBoxRows);
-                if (!mbar_wait(tmem_empty, acc_phase ^ 1u, abort_flag, err, 2)) break;
+            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++li) {
+                const int4 ch = __ldcg(args.chunks + item / n_tiles);
+                const uint32_t n = uint32_t((ch.z + 15) / 16 * 16);
+                const int buf = li % kBufs;
+                const uint32_t use = uint32_t(li / kBufs) & 1u;  // how often this buffer was used, mod 2
+                if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 2)) break;
                 tc_fence_after();
-                for (int kb = 0; kb < KB; ++kb) {
+                const uint32_t acc = tmem + uint32_t(buf * C::kAccCols);
+                for (int step = 0; step < n_steps; ++step) {
+                    const int kb0 = step * kKB;
+                    const int nkb = min(kKB, KB - kb0);
                     if (!mbar_wait(&full[stage], phase, abort_flag, err, 3)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint8_t *st = tiles + stage * C::kStageTiles;
-                    const uint8_t *sf = sfs + stage * C::kStageSf;
-                    const uint32_t sf_col = tmem + C::kAccCols + stage * (kNumA + 1) * 4;
+                    const uint8_t *sfa = sfs + stage * C::kStageSf;
+                    const uint8_t *sfb = sfa + kNumA * kKB * kSfBlockBytes;
+                    const uint8_t *bt = st + kNumA * kKB * C::kATile;
+                    uint32_t col = tmem + uint32_t(kBufs * C::kAccCols + (stage * kIssuers + issuer) * C::kSfColsIssuer);
+                    const int b_lo = (!kGemm1 && kIssuers == 2) ? issuer : 0;
+                    const int b_hi = (!kGemm1 && kIssuers == 2) ? issuer + 1 : nkb;
+                    for (int b = b_lo; b < b_hi && b < nkb; ++b) {
+                        // scale blocks of this K block into TMEM: weight tile(s), then activations
+                        const int a_lo = kGemm1 ? (kIssuers == 2 ? issuer : 0) : 0;
+                        const int a_n = C::kIssuerAcc;
+                        for (int a = 0; a < a_n; ++a)
+                            tc_cp_sf(col + a * 4, smem_desc_sf(smem_u32(sfa + (b * kNumA + a_lo + a) * kSfBlockBytes)));
+                        const uint32_t sfb_col = col + a_n * 4;
+                        tc_cp_sf(sfb_col, smem_desc_sf(smem_u32(sfb + b * kSfBlockBytes)));
+                        const uint64_t bdesc = smem_desc_sw128(smem_u32(bt + b * C::kBTile));
 #pragma unroll
-                    for (int a = 0; a <= kNumA; ++a)
-                        tc_cp_sf(sf_col + a * 4, smem_desc_sf(smem_u32(sf + a * kSfBlockBytes)));
-                    const uint64_t bdesc = smem_desc_sw128(smem_u32(st + kNumA * C::kATile));
-#pragma unroll
-                    for (int ks = 0; ks < kTileK / 32; ++ks) {
-                        const uint32_t idesc = idesc_mxf8f6f4(n, uint32_t(ks));
-#pragma unroll
-                        for (int a = 0; a < kNumA; ++a) {
-                            const uint64_t adesc = smem_desc_sw128(smem_u32(st + a * C::kATile));
-                            // +32 bytes of K per step inside the 128-byte swizzled row
-                            tc_mma_mxf8f6f4(tmem + a * kChunkRows, adesc + uint64_t(2 * ks),
-                                            bdesc + uint64_t(2 * ks), idesc, sf_col + a * 4, sf_col + kNumA * 4,
-                                            (kb | ks) != 0 ? 1u : 0u);
+                        for (int ks = 0; ks < kTileK / 32; ++ks) {
+                            const uint32_t idesc = idesc_mxf8f6f4(n, uint32_t(ks));
+                            for (int a = 0; a < a_n; ++a) {
+                                const int acc_i = kGemm1 ? a_lo + a : issuer;
+                                const uint64_t adesc = smem_desc_sw128(smem_u32(st + (b * kNumA + a_lo + a) * C::kATile));
+                                const bool first = (kb0 + b == (kGemm1 ? 0 : b_lo)) && ks == 0;
+                                // +32 bytes of K per step inside the 128-byte swizzled row
+                                tc_mma_mxf8f6f4(acc + uint32_t(acc_i * kN), adesc + uint64_t(2 * ks),
+                                                bdesc + uint64_t(2 * ks), idesc, col + a * 4, sfb_col,
+                                                first ? 0u : 1u);
+                            }
                         }
+                        col += uint32_t((a_n + 1) * 4);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -223,34 +294,39 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
                 if (!ok) break;
-                tc_commit(tmem_full);
-                acc_phase ^= 1u;
+                tc_commit(&tmem_full[buf]);
             }
             // All issued MMAs must be finished before TMEM is released.
-            tc_commit(mma_done);
+            tc_commit(&mma_done[issuer]);
             const unsigned long long t0 = global_timer_ns();
-            while (!mbar_try_wait(mma_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+            while (!mbar_try_wait(&mma_done[issuer], 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        uint32_t acc_phase = 0;
-        for (int item = blockIdx.x; item < num_items; item += gridDim.x) {
+        // GEMM2 with a K split: the second accumulator holds a partial sum
+        // only when there is a second K block
+        const bool add_second = !kGemm1 && kIssuers == 2 && KB > 1;
+        int li = 0;
+        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
             const int c = item / n_tiles, tile = item % n_tiles;
-            const int4 ch = args.chunks[c];
-            if (!mbar_wait(tmem_full, acc_phase, abort_flag, err, 4)) break;
+            const int4 ch = __ldcg(args.chunks + c);
+            const int buf = li % kBufs;
+            const uint32_t use = uint32_t(li / kBufs) & 1u;
+            if (!mbar_wait(&tmem_full[buf], use, abort_flag, err, 4)) break;
             tc_fence_after();
+            const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
             const int ncb = (ch.z + 31) / 32;
             const int row_out = tile * kTileRows + q * 32 + lane;  // this thread's output column
             for (int cb = 0; cb < ncb; ++cb) {
                 uint32_t g[32];
-                tmem_ld_32x32(tmem + lane_base + uint32_t(cb * 32), g);
+                tmem_ld_32x32(acc + uint32_t(cb * 32), g);
                 if constexpr (kGemm1) {
                     uint32_t u[32];
-                    tmem_ld_32x32(tmem + lane_base + uint32_t(kChunkRows + cb * 32), u);
+                    tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
                     tmem_ld_wait();
                     float h[32], a[32];
 #pragma unroll
@@ -272,22 +348,33 @@ __global__ void __launch_bounds__(192, 1)
                     for (int j = 0; j < 32; ++j) {
                         const float mj = __shfl_sync(0xFFFFFFFFu, mult, j);
                         const uint32_t code = to_e4m3(h[j] * mj);
+                        // K-block-major [I/128][rows][128]: GEMM2 reads two K blocks per box
                         if (cb * 32 + j < ch.z)
-                            args.out_q[int64_t(ch.y + cb * 32 + j) * args.out_ld + row_out] = uint8_t(code);
+                            args.out_q[(int64_t(tile) * args.rows + ch.y + cb * 32 + j) * kTileK + q * 32 + lane] =
+                                uint8_t(code);
                     }
                 } else {
-                    tmem_ld_wait();
+                    float y[32];
+                    if (add_second) {
+                        uint32_t g2[32];
+                        tmem_ld_32x32(acc + uint32_t(kN + cb * 32), g2);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(g[j]) + __uint_as_float(g2[j]);
+                    } else {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(g[j]);
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (cb * 32 + j < ch.z)
-                            args.out_y[int64_t(ch.y + cb * 32 + j) * args.out_ld + row_out] =
-                                __float2bfloat16_rn(__uint_as_float(g[j]));
+                            args.out_y[int64_t(ch.y + cb * 32 + j) * args.out_ld + row_out] = __float2bfloat16_rn(y[j]);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tmem_empty);
-            acc_phase ^= 1u;
+            if (lane == 0) mbar_arrive(&tmem_empty[buf]);
         }
     }
 
@@ -297,30 +384,42 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <bool kGemm1>
-static cudaError_t launch_gemm_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, const GemmArgs &args,
-                                 int grid, cudaStream_t stream) {
-    using C = GemmCfg<kGemm1>;
+template <bool kGemm1, int kN>
+static cudaError_t launch_gemm_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf, const CUtensorMap &tmap_act,
+                                 const GemmArgs &args, int grid, cudaStream_t stream) {
+    using C = GemmCfg<kGemm1, kN>;
     static int configured_for = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_for != dev) {
-        const cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kGemm1>,
+        const cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kGemm1, kN>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (e != cudaSuccess) return e;
         configured_for = dev;
     }
-    moe_gemm_kernel<kGemm1><<<grid, 192, C::kSmemBytes, stream>>>(tmap_w, tmap_act, args);
-    return cudaGetLastError();
+    return launch_pdl(moe_gemm_kernel<kGemm1, kN>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
+                      tmap_w, tmap_wsf, tmap_act, args);
 }
 
-cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act,
-                        const uint8_t *w_packets, uint8_t *ws, const WsLayout &L, int H, int I, int grid,
-                        cudaStream_t stream) {
+int gemm_kblocks_per_stage(int chunk_rows) {
+    return chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall>::kKB : GemmCfg<true, kChunkRows>::kKB;
+}
+
+int gemm_packets_per_stage(bool gemm1, int chunk_rows) {
+    return gemm1 ? (chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall>::kNumA * GemmCfg<true, kChunkRowsSmall>::kKB
+                                                  : GemmCfg<true, kChunkRows>::kNumA * GemmCfg<true, kChunkRows>::kKB)
+                 : (chunk_rows == kChunkRowsSmall ? GemmCfg<false, kChunkRowsSmall>::kNumA * GemmCfg<false, kChunkRowsSmall>::kKB
+                                                  : GemmCfg<false, kChunkRows>::kNumA * GemmCfg<false, kChunkRows>::kKB);
+}
+
+cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
+                        const CUtensorMap &tmap_act, const uint8_t *w_packets, uint8_t *ws, const WsLayout &L, int H,
+                        int I, int grid, cudaStream_t stream) {
     GemmArgs a{};
     a.w_packets = w_packets;
     a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
     a.hdr = reinterpret_cast<int *>(ws);
+    const bool small = L.chunk_rows == kChunkRowsSmall;
     if (gemm1) {
         a.act_sf = ws + L.off_xg_sf;
         a.out_q = ws + L.off_hq;
@@ -328,14 +427,18 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
         a.K = H;
         a.n_tiles = I / kTileRows;
         a.out_ld = I;
-        return launch_gemm_t<true>(tmap_w, tmap_act, a, grid, stream);
+        a.rows = int(L.Rp);
+        return small ? launch_gemm_t<true, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, a, grid, stream)
+                     : launch_gemm_t<true, kChunkRows>(tmap_w, tmap_wsf, tmap_act, a, grid, stream);
     }
     a.act_sf = ws + L.off_hq_sf;
     a.out_y = reinterpret_cast<__nv_bfloat16 *>(ws + L.off_y);
     a.K = I;
     a.n_tiles = H / kTileRows;
     a.out_ld = H;
-    return launch_gemm_t<false>(tmap_w, tmap_act, a, grid, stream);
+    a.rows = int(L.Rp);
+    return small ? launch_gemm_t<false, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, a, grid, stream)
+                 : launch_gemm_t<false, kChunkRows>(tmap_w, tmap_wsf, tmap_act, a, grid, stream);
 }
 
 }  // namespace moe

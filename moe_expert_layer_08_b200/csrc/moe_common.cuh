@@ -15,7 +15,8 @@ namespace moe {
 // ---------------------------------------------------------------- layout constants
 constexpr int kTileRows = 128;        // weight rows per MMA (M) and per packet
 constexpr int kTileK = 128;           // K elements per pipeline stage and per packet
-constexpr int kChunkRows = 128;       // max routed rows (tokens) per work item (MMA N)
+constexpr int kChunkRows = 128;       // max routed rows (tokens) per work item (MMA N), large batches
+constexpr int kChunkRowsSmall = 32;   // the same for small batches (decode)
 constexpr int kBoxRows = 16;          // activation rows per TMA box
 constexpr int kPacketBody = kTileRows * kTileK / 2;   // 8192 B of packed FP4
 constexpr int kPacketSf = kTileRows * 4;              // 512 B of UE8M0 (4 groups x 128 rows)
@@ -145,6 +146,14 @@ static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, vo
         }
     }
 }
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Block until the preceding kernel on the stream has completed and its memory
+// is visible (no-op when the kernel was not launched as a dependent).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next kernel on the stream to be scheduled once every CTA of this
+// grid has issued this (or exited).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------- TMA (no multicast)
 __device__ __forceinline__ uint64_t policy_evict_first() {

@@ -11,7 +11,27 @@
 
 namespace moe {
 
-constexpr int kRouteBlock = 256;  // routed slots per routing block
+constexpr int kRouteBlock = 256;       // routed slots per routing block (large batches)
+constexpr int kRouteSmallMax = 1024;   // batches of at most this many slots route in one block
+
+// Launch `kernel` as a programmatic dependent of the preceding work on `stream`
+// (its CTAs may start before that work ends; the kernel orders itself with
+// griddepcontrol.wait before touching dependent memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -20,8 +40,11 @@ struct WsLayout {
     int64_t R = 0;          // routed slots T*k
     int64_t max_chunks = 0; // upper bound of (expert, <=128-row) work chunks
     int nb = 0;             // routing blocks
+    int chunk_rows = 0;     // routed rows per chunk (32 or 128)
+    int64_t Rp = 0;         // rows of the K-block-major FP8 operands (R, at least one TMA box)
+    int kbh = 0, kbi = 0;   // K blocks of those operands (H/128, I/128, at least 2)
     size_t off_count = 0, off_offset = 0, off_chunk_base = 0, off_chunks = 0;
-    size_t off_hist = 0, off_bad = 0, off_lrank = 0, off_perm = 0, off_inv = 0;
+    size_t off_hist = 0, off_bad = 0, off_lrank = 0, off_perm = 0, off_inv = 0, off_rowinfo = 0;
     size_t off_xg = 0, off_xg_sf = 0, off_hq = 0, off_hq_sf = 0, off_y = 0;
     size_t total = 0;
 };
@@ -35,9 +58,14 @@ cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_pe
                              int halves, int half_rows, void *out, cudaStream_t stream);
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
                          int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream);
-cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act,
-                        const uint8_t *w_packets, uint8_t *ws, const WsLayout &L, int H, int I, int grid,
-                        cudaStream_t stream);
+cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
+                        const CUtensorMap &tmap_act, const uint8_t *w_packets, uint8_t *ws, const WsLayout &L, int H,
+                        int I, int grid, cudaStream_t stream);
+// Weight packets one pipeline stage of that GEMM variant moves (TMA box depth).
+int gemm_packets_per_stage(bool gemm1, int chunk_rows);
+// 128-K blocks one pipeline stage moves (the activation box depth).
+int gemm_kblocks_per_stage(int chunk_rows);
+constexpr int kActBoxRows = 32;  // activation rows per TMA box
 cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
                            void *out, cudaStream_t stream);
 

@@ -2,25 +2,142 @@
 // permutation and its inverse, chunk list) and the local gather that replaces
 // the cross-rank dispatch of the "Mega MoE" pipeline ("Mega moe fusion with
 // symmetric memory", Procedure step 5, phase 1; the "gather-by-expert" step of
-// What / Why).  Three launches, no host synchronisation:
-//   1. route_count: per 256-slot block, per-expert counts and each slot's rank
-//      among the block's earlier slots of the same expert;
-//   2. route_scan (one block): counts, offsets, per-block base positions,
-//      the list of <=128-row chunks per expert, expert statistics, error word;
-//   3. route_place_gather: perm / inv, then the FP8 rows of x copied into
-//      permuted order and their UE8M0 scales into per-chunk 512-byte blocks in
-//      the layout tcgen05.cp copies into TMEM.
+// What / Why).  No host synchronisation anywhere.
+//
+// Small batches (T*k <= 1024 slots): one block does everything
+// (route_small_kernel).  Large batches: route_count (per 256-slot block,
+// per-expert counts and each slot's rank among the block's earlier slots of
+// its expert), route_scan (one block: counts, offsets, per-block bases, chunk
+// list, statistics, error word), route_place (perm, inv, per-row gather
+// descriptor).  Then gather_kernel copies the FP8 rows of x into permuted
+// order (stored K-block-major, [H/128][R][128]) and the UE8M0 scales into per-chunk 512-byte blocks laid out as the
+// image tcgen05.cp copies into TMEM.
+//
+// Within an expert, routed rows keep ascending slot order t*k+j (a stable
+// counting sort), so the metadata is unique and compared bit-exactly.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
 namespace moe {
 
+// Exclusive scan of one int per thread over a block of blockDim.x (<= 1024,
+// multiple of 32) threads; every thread must call it.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;  // inclusive totals of warps 0..lane
+    }
+    __syncthreads();
+    const int before = warp > 0 ? s_warp[warp - 1] : 0;
+    const int r = before + x - v;
+    __syncthreads();
+    return r;
+}
+
+// Per expert e (one thread each): count c, offset, chunk base, chunk list
+// entries, statistics.  Shared by both routing paths.
+__device__ __forceinline__ void write_expert_meta(int e, int E, int c, int off, int cbase, int chunk_rows,
+                                                 int *count, int *offset, int *chunk_base, int4 *chunks, int *hdr,
+                                                 int32_t *expert_stats) {
+    const int nch = (c + chunk_rows - 1) / chunk_rows;
+    count[e] = c;
+    offset[e] = off;
+    chunk_base[e] = cbase;
+    for (int q = 0; q < nch; ++q)
+        chunks[cbase + q] = make_int4(e, off + q * chunk_rows, min(chunk_rows, c - q * chunk_rows), 0);
+    if (expert_stats) expert_stats[e] += c;
+    if (e == E - 1) {
+        offset[E] = off + c;
+        chunk_base[E] = cbase + nch;
+        hdr[kHdrNumChunks] = cbase + nch;
+    }
+}
+
+// ------------------------------------------------------------------ small batches
+// One 1024-thread block, one slot per thread (R <= 1024).  Shared memory:
+// cnt[32 warps][E] per-warp per-expert counts, turned into per-warp bases.
+__global__ void __launch_bounds__(1024) route_small_kernel(const int64_t *__restrict__ topk_idx, int R, int k, int E,
+                                                           int chunk_rows, int *__restrict__ count,
+                                                           int *__restrict__ offset, int *__restrict__ chunk_base,
+                                                           int4 *__restrict__ chunks, int *__restrict__ perm,
+                                                           int *__restrict__ inv, int4 *__restrict__ rowinfo,
+                                                           int *__restrict__ hdr, int32_t *__restrict__ expert_stats) {
+    extern __shared__ int cnt[];
+    __shared__ int s_warp[32];
+    __shared__ int s_off[kMaxExperts], s_cbase[kMaxExperts];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_wait();
+    pdl_trigger();
+    for (int i = tid; i < 32 * E; i += 1024) cnt[i] = 0;
+    __syncthreads();
+    bool valid = false;
+    int e = 0;
+    if (tid < R) {
+        const int64_t v = __ldcg(topk_idx + tid);
+        valid = v >= 0 && v < E;
+        e = valid ? int(v) : 0;
+    }
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, valid ? unsigned(e) : 0xFFFFFFFFu);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (valid && rank_w == 0) cnt[warp * E + e] = __popc(peers);
+    const int nbad = __syncthreads_count(tid < R && !valid);
+    // per expert: per-warp exclusive bases and the total
+    int c = 0;
+    if (tid < E)
+        for (int w = 0; w < 32; ++w) {
+            const int x = cnt[w * E + tid];
+            cnt[w * E + tid] = c;
+            c += x;
+        }
+    const int off = block_exclusive_scan(tid < E ? c : 0, s_warp);
+    const int cbase = block_exclusive_scan(tid < E ? (c + chunk_rows - 1) / chunk_rows : 0, s_warp);
+    if (tid < E) {
+        s_off[tid] = off;
+        s_cbase[tid] = cbase;
+        write_expert_meta(tid, E, c, off, cbase, chunk_rows, count, offset, chunk_base, chunks, hdr, expert_stats);
+    }
+    __syncthreads();
+    if (tid < R) {
+        if (valid) {
+            const int local = cnt[warp * E + e] + rank_w;
+            const int pos = s_off[e] + local;
+            perm[pos] = tid;
+            inv[tid] = pos;
+            rowinfo[pos] = make_int4(tid / k, s_cbase[e] + local / chunk_rows, local % chunk_rows, 0);
+        } else {
+            inv[tid] = -1;
+        }
+    }
+    if (tid == 0) {
+        hdr[kHdrDropped] = nbad;
+        hdr[kHdrError] = nbad ? kDevErrBadRouting : 0;
+        hdr[kHdrTimeoutWhere] = 0;
+    }
+}
+
+// ------------------------------------------------------------------ large batches
 __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const int64_t *__restrict__ topk_idx, int R,
                                                                   int E, int *__restrict__ hist,
                                                                   int *__restrict__ lrank, int *__restrict__ bad) {
     extern __shared__ int cnt[];  // [kRouteBlock / 32][E]
     constexpr int kWarps = kRouteBlock / 32;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_wait();
+    pdl_trigger();
     for (int i = tid; i < kWarps * E; i += kRouteBlock) cnt[i] = 0;
     __syncthreads();
 
@@ -28,13 +145,12 @@ __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const int64_t 
     bool valid = false;
     int e = 0;
     if (s < R) {
-        const int64_t v = topk_idx[s];
+        const int64_t v = __ldcg(topk_idx + s);
         valid = v >= 0 && v < E;
         e = valid ? int(v) : 0;
     }
     // rank among this warp's earlier lanes routed to the same expert
-    const unsigned key = valid ? unsigned(e) : 0xFFFFFFFFu;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, valid ? unsigned(e) : 0xFFFFFFFFu);
     const int rank_w = __popc(peers & ((1u << lane) - 1u));
     if (valid && rank_w == 0) cnt[warp * E + e] = __popc(peers);
     __syncthreads();
@@ -52,71 +168,35 @@ __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const int64_t 
     if (tid == 0) bad[blockIdx.x] = nbad;
 }
 
-// Exclusive scan of one int per thread over a 1024-thread block.
-__device__ __forceinline__ int block_exclusive_scan(int v, int *s_warp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = s_warp[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
-            if (lane >= o) w += y;
-        }
-        s_warp[lane] = w;  // inclusive totals of warps 0..lane
-    }
-    __syncthreads();
-    const int before = warp > 0 ? s_warp[warp - 1] : 0;
-    const int r = before + x - v;
-    __syncthreads();
-    return r;
-}
-
 __global__ void __launch_bounds__(1024) route_scan_kernel(int *__restrict__ hist, const int *__restrict__ bad,
-                                                          int nb, int E, int *__restrict__ count,
+                                                          int nb, int E, int chunk_rows, int *__restrict__ count,
                                                           int *__restrict__ offset, int *__restrict__ chunk_base,
                                                           int4 *__restrict__ chunks, int *__restrict__ hdr,
                                                           int32_t *__restrict__ expert_stats) {
     __shared__ int s_warp[32];
     __shared__ int s_bad;
     const int e = threadIdx.x;
+    pdl_wait();
+    pdl_trigger();
     int c = 0;
     if (e < E)
-        for (int b = 0; b < nb; ++b) c += hist[size_t(b) * E + e];
-    const int nch = (c + kChunkRows - 1) / kChunkRows;
+        for (int b = 0; b < nb; ++b) c += __ldcg(hist + size_t(b) * E + e);
     const int off = block_exclusive_scan(c, s_warp);
-    const int cbase = block_exclusive_scan(nch, s_warp);
+    const int cbase = block_exclusive_scan((c + chunk_rows - 1) / chunk_rows, s_warp);
     if (e < E) {
-        count[e] = c;
-        offset[e] = off;
-        chunk_base[e] = cbase;
         int run = off;  // per-block base position of this expert's slots
         for (int b = 0; b < nb; ++b) {
             const size_t ix = size_t(b) * E + e;
-            const int h = hist[ix];
+            const int h = __ldcg(hist + ix);
             hist[ix] = run;
             run += h;
         }
-        for (int q = 0; q < nch; ++q)
-            chunks[cbase + q] = make_int4(e, off + q * kChunkRows, min(kChunkRows, c - q * kChunkRows), 0);
-        if (expert_stats) expert_stats[e] += c;
-        if (e == E - 1) {
-            offset[E] = off + c;
-            chunk_base[E] = cbase + nch;
-            hdr[kHdrNumChunks] = cbase + nch;
-        }
+        write_expert_meta(e, E, c, off, cbase, chunk_rows, count, offset, chunk_base, chunks, hdr, expert_stats);
     }
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
     int d = 0;
-    for (int b = threadIdx.x; b < nb; b += blockDim.x) d += bad[b];
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) d += __ldcg(bad + b);
     if (d) atomicAdd(&s_bad, d);
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -126,49 +206,53 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int *__restrict__ hist
     }
 }
 
-__global__ void __launch_bounds__(kRouteBlock) route_place_gather_kernel(
-    const int64_t *__restrict__ topk_idx, int R, int k, int E, int H, const int *__restrict__ base,
+__global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
+    const int64_t *__restrict__ topk_idx, int R, int k, int E, int chunk_rows, const int *__restrict__ base,
     const int *__restrict__ lrank, const int *__restrict__ offset, const int *__restrict__ chunk_base,
-    int *__restrict__ perm, int *__restrict__ inv, const uint8_t *__restrict__ x, const uint8_t *__restrict__ x_sf,
-    uint8_t *__restrict__ xg, uint8_t *__restrict__ xg_sf) {
-    __shared__ int s_t[kRouteBlock], s_pos[kRouteBlock], s_chunk[kRouteBlock], s_rl[kRouteBlock];
-    const int tid = threadIdx.x;
-    const int64_t s = int64_t(blockIdx.x) * kRouteBlock + tid;
-    int pos = -1, t = 0, chunk = 0, rl = 0;
-    if (s < R) {
-        const int64_t v = topk_idx[s];
-        if (v >= 0 && v < E) {
-            const int e = int(v);
-            pos = base[size_t(blockIdx.x) * E + e] + lrank[s];
-            perm[pos] = int(s);
-            inv[s] = pos;
-            t = int(s / k);
-            const int local = pos - offset[e];
-            chunk = chunk_base[e] + local / kChunkRows;
-            rl = local % kChunkRows;
-        } else {
-            inv[s] = -1;
-        }
+    int *__restrict__ perm, int *__restrict__ inv, int4 *__restrict__ rowinfo) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t s = int64_t(blockIdx.x) * kRouteBlock + threadIdx.x;
+    if (s >= R) return;
+    const int64_t v = __ldcg(topk_idx + s);
+    if (v < 0 || v >= E) {
+        inv[s] = -1;
+        return;
     }
-    s_t[tid] = t;
-    s_pos[tid] = pos;
-    s_chunk[tid] = chunk;
-    s_rl[tid] = rl;
-    __syncthreads();
+    const int e = int(v);
+    const int pos = __ldcg(base + size_t(blockIdx.x) * E + e) + __ldcg(lrank + s);
+    perm[pos] = int(s);
+    inv[s] = pos;
+    const int local = pos - __ldcg(offset + e);
+    rowinfo[pos] = make_int4(int(s / k), __ldcg(chunk_base + e) + local / chunk_rows, local % chunk_rows, 0);
+}
 
-    const int warp = tid >> 5, lane = tid & 31;
-    const int nvec = H / 16;
-    const int KB = H / kTileK;
-    for (int j = warp; j < kRouteBlock; j += kRouteBlock / 32) {
-        const int p = s_pos[j];
-        if (p < 0) continue;
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + size_t(s_t[j]) * H);
-        uint4 *dst = reinterpret_cast<uint4 *>(xg + size_t(p) * H);
-        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
-        const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + size_t(s_t[j]) * (H / 32));
-        for (int kb = lane; kb < KB; kb += 32) {
-            uint8_t *blk = xg_sf + (size_t(s_chunk[j]) * KB + kb) * kSfBlockBytes;
-            *reinterpret_cast<uint32_t *>(blk + sf_block_offset(s_rl[j], 0)) = __ldg(sfs + kb);
+// ------------------------------------------------------------------ gather
+// One 128-thread block per (routed row, 2048-byte segment of the row); the
+// first segment's block also moves the row's scale words.
+constexpr int kGatherSeg = 2048;
+
+__global__ void __launch_bounds__(128) gather_kernel(const int4 *__restrict__ rowinfo, const int *__restrict__ offset,
+                                                     int E, int H, int64_t R, int segs, const uint8_t *__restrict__ x,
+                                                     const uint8_t *__restrict__ x_sf, uint8_t *__restrict__ xg,
+                                                     uint8_t *__restrict__ xg_sf) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t pos = blockIdx.x / segs;
+    const int seg = blockIdx.x % segs;
+    if (pos >= __ldcg(offset + E)) return;  // dropped slots leave no row
+    const int4 ri = __ldcg(rowinfo + pos);
+    const int col = seg * kGatherSeg + threadIdx.x * 16;
+    // K-block-major destination [H/128][Rp][128]
+    if (col < H)
+        *reinterpret_cast<uint4 *>(xg + ((col / kTileK) * R + pos) * kTileK + col % kTileK) =
+            __ldcg(reinterpret_cast<const uint4 *>(x + int64_t(ri.x) * H + col));
+    if (seg == 0) {
+        const int KB = H / kTileK;
+        const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * (H / 32));
+        for (int kb = threadIdx.x; kb < KB; kb += 128) {
+            uint8_t *blk = xg_sf + (int64_t(ri.y) * KB + kb) * kSfBlockBytes;
+            *reinterpret_cast<uint32_t *>(blk + sf_block_offset(ri.z, 0)) = __ldcg(sfs + kb);
         }
     }
 }
@@ -186,14 +270,38 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
     int4 *chunks = reinterpret_cast<int4 *>(ws + L.off_chunks);
     int *perm = reinterpret_cast<int *>(ws + L.off_perm);
     int *inv = reinterpret_cast<int *>(ws + L.off_inv);
-    const size_t cnt_smem = size_t(kRouteBlock / 32) * E * sizeof(int);
-    route_count_kernel<<<L.nb, kRouteBlock, cnt_smem, stream>>>(topk_idx, R, E, hist, lrank, bad);
-    route_scan_kernel<<<1, 1024, 0, stream>>>(hist, bad, L.nb, E, count, offset, chunk_base, chunks, hdr,
-                                              expert_stats);
-    route_place_gather_kernel<<<L.nb, kRouteBlock, 0, stream>>>(topk_idx, R, k, E, H, hist, lrank, offset,
-                                                                chunk_base, perm, inv, x, x_sf, ws + L.off_xg,
-                                                                ws + L.off_xg_sf);
-    return cudaGetLastError();
+    int4 *rowinfo = reinterpret_cast<int4 *>(ws + L.off_rowinfo);
+    const int cr = L.chunk_rows;
+    cudaError_t e;
+    if (R <= kRouteSmallMax) {
+        const size_t smem = size_t(32) * E * sizeof(int);
+        static int configured_for = -1;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (configured_for != dev) {
+            e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     32 * kMaxExperts * int(sizeof(int)));
+            if (e != cudaSuccess) return e;
+            configured_for = dev;
+        }
+        e = launch_pdl(route_small_kernel, dim3(1), dim3(1024), smem, stream, topk_idx, R, k, E, cr, count, offset,
+                       chunk_base, chunks, perm, inv, rowinfo, hdr, expert_stats);
+    } else {
+        const size_t cnt_smem = size_t(kRouteBlock / 32) * E * sizeof(int);
+        e = launch_pdl(route_count_kernel, dim3(L.nb), dim3(kRouteBlock), cnt_smem, stream, topk_idx, R, E, hist,
+                       lrank, bad);
+        if (e == cudaSuccess)
+            e = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, hist, bad, L.nb, E, cr, count, offset,
+                           chunk_base, chunks, hdr, expert_stats);
+        if (e == cudaSuccess)
+            e = launch_pdl(route_place_kernel, dim3(L.nb), dim3(kRouteBlock), 0, stream, topk_idx, R, k, E, cr, hist,
+                           lrank, offset, chunk_base, perm, inv, rowinfo);
+    }
+    if (e != cudaSuccess) return e;
+    const int segs = (H + kGatherSeg - 1) / kGatherSeg;
+    return launch_pdl(gather_kernel, dim3(unsigned(int64_t(R) * segs)), dim3(128), 0, stream,
+                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, L.Rp, segs, x, x_sf,
+                      ws + L.off_xg, ws + L.off_xg_sf);
 }
 
 }  // namespace moe
