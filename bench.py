@@ -118,6 +118,18 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.sm)}
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks (the job is as slow as its slowest
+    replica); identity without a process group."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def build_layer(w, device):
     """Seeded bf16 draws quantised and packed by the CUDA library, resident in HBM."""
     import moe_expert_layer_08_b200 as moe
@@ -232,11 +244,7 @@ def run_b200(args, w, rank, world, local_rank):
         barrier()
     total_ms = start.elapsed_time(stop)
     stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(moe.NUM_STAGE_EVENTS - 1)] for e in ev])
-    ms = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(total_ms / args.steps, device)
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host output
     h_xq = g["xq"].cpu().pin_memory()
@@ -265,11 +273,7 @@ def run_b200(args, w, rank, world, local_rank):
         e2e_step()
     stop.record(stream)
     barrier()
-    e2e_ms = start.elapsed_time(stop) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(start.elapsed_time(stop) / args.steps, device)
     st = moe.check_device_error(layer.workspace)
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {moe.STATUS.get(st, st)}")
