@@ -118,6 +118,26 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.sm)}
 
 
+def kernel_source_hash() -> str:
+    import hashlib
+    files = ["gemm.cu", "moe_common.cuh", "moe_internal.h"]
+    src = b"".join(open(os.path.join(ROOT, "moe_expert_layer_08_b200", "csrc", f), "rb").read() for f in files)
+    return hashlib.sha256(src).hexdigest()
+
+
+def measured_traffic(w, touched, gemm1: bool):
+    """DRAM bytes per launch of the dominant GEMM from the committed ncu
+    capture (scaled by touched experts, which the traffic is proportional
+    to), or None when the kernel changed since or another variant runs."""
+    path = os.path.join(ROOT, "profiles", "gemm_decode_traffic.json")
+    if not os.path.exists(path) or w.T * w.k > 8 * w.E:
+        return None
+    d = json.load(open(path))
+    if d.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    return touched * d["gemm1_bytes_per_touched_expert" if gemm1 else "gemm2_bytes_per_touched_expert"]
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """The largest `value` over all ranks (the job is as slow as its slowest
     replica); identity without a process group."""
@@ -290,6 +310,7 @@ def run_b200(args, w, rank, world, local_rank):
     else:
         kname, kms, kbytes = "moe_gemm_kernel<gemm2>", g2_ms, touched * b2
     achieved = kbytes / (kms * 1e-3) / 1e9
+    traffic = measured_traffic(w, touched, g1_ms >= g2_ms)
     layer_bytes = touched * (b1 + b2) + w.T * w.H * 33 // 32 + w.T * w.k * 12 + w.T * w.H * 2
     flops = w.flops
     value = world * flops / (ms * 1e-3) / 1e12
@@ -309,7 +330,8 @@ def run_b200(args, w, rank, world, local_rank):
         "stage_us": {"route_gather": float(stage_ms[:, 0].mean() * 1e3), "gemm1": g1_ms * 1e3,
                      "gemm2": g2_ms * 1e3, "combine": float(stage_ms[:, 3].mean() * 1e3)},
         "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm"], "peak_source": pk["source"], "traffic": None},
+                     "frac": achieved / pk["hbm"], "peak_source": pk["source"], "algorithmic_bytes": kbytes,
+                     "traffic": traffic},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": 6 * args.steps,
