@@ -42,9 +42,14 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.kbh = H / kTileK > 2 ? H / kTileK : 2;
     L.kbi = I / kTileK > 2 ? I / kTileK : 2;
     L.off_xg = take(size_t(L.Rp) * size_t(L.kbh) * kTileK);
-    L.off_xg_sf = take(MC * size_t(H / kTileK) * kSfBlockBytes);
+    // scale blocks per (chunk, K block): the larger of the two chunkings' needs
+    const size_t sf_small = MC * size_t(act_sf_bytes(kChunkRowsSmall));
+    const size_t mc_large = size_t((L.R + kChunkRows - 1) / kChunkRows + (L.R < E ? L.R : E));
+    const size_t sf_large = (mc_large > 0 ? mc_large : 1) * size_t(act_sf_bytes(kChunkRows));
+    const size_t sf_per_kb = sf_small > sf_large ? sf_small : sf_large;
+    L.off_xg_sf = take(sf_per_kb * size_t(H / kTileK));
     L.off_hq = take(size_t(L.Rp) * size_t(L.kbi) * kTileK);
-    L.off_hq_sf = take(MC * size_t(I / kTileK) * kSfBlockBytes);
+    L.off_hq_sf = take(sf_per_kb * size_t(I / kTileK));
     L.off_y = take(R * size_t(H) * 2);
     L.total = o;
     return L;

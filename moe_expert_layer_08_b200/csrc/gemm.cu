@@ -41,12 +41,14 @@ struct GemmCfg {
     static constexpr bool kSmall = kN == kChunkRowsSmall;
     static constexpr int kNumA = kGemm1 ? 2 : 1;        // weight tiles per K block: (gate, up) or (down)
     static constexpr int kKB = kSmall ? 2 : 1;          // 128-K blocks per pipeline stage
-    static constexpr int kIssuers = kSmall ? 2 : 1;     // MMA-issuing warps
+    static constexpr int kIssuers = (kSmall || kGemm1) ? 2 : 1;  // MMA-issuing warps
     static constexpr int kStages = kSmall ? (kGemm1 ? 3 : 5) : (kGemm1 ? 4 : 6);
     static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 one-byte elements
     static constexpr int kBTile = kN * kTileK;          // token rows x 128 bytes, per K block
     static constexpr int kStageTiles = kNumA * kKB * kATile + kKB * kBTile;
-    static constexpr int kStageSf = (kNumA * kKB + kKB) * kSfBlockBytes;
+    static constexpr int kActSf = act_sf_bytes(kN);     // activation scale bytes per K block
+    static constexpr int kSfbImages = kActSf / kSfBlockBytes;
+    static constexpr int kStageSf = kNumA * kKB * kSfBlockBytes + kKB * kActSf;
     static constexpr int kSmemTiles = kStages * kStageTiles;
     static constexpr int kSmemSf = kStages * kStageSf;
     static constexpr int kSmemMisc = 256;
@@ -59,7 +61,7 @@ struct GemmCfg {
     // and of the activation K blocks it consumes, 4 TMEM columns each.
     static constexpr int kIssuerKB = (!kGemm1 && kIssuers == 2) ? 1 : kKB;
     static constexpr int kIssuerAcc = (kGemm1 && kIssuers == 1) ? 2 : 1;
-    static constexpr int kSfColsIssuer = kIssuerKB * (kIssuerAcc + 1) * 4;
+    static constexpr int kSfColsIssuer = kIssuerKB * (kIssuerAcc + kSfbImages) * 4;
     static constexpr int kSfCols = kStages * kIssuers * kSfColsIssuer;
     static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
@@ -203,13 +205,13 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         // the activation box always moves kKB K blocks (a K
                         // block past the end reads zeros)
                         mbar_arrive_expect_tx(&full[stage],
-                                              uint32_t(nbox * kKB * kActBoxRows * kTileK + nkb * kSfBlockBytes));
+                                              uint32_t(nbox * kKB * kActBoxRows * kTileK + nkb * C::kActSf));
                         uint8_t *bt = st + kNumA * kKB * C::kATile;
                         for (int j = 0; j < nbox; ++j)
                             tma_load_3d(bt + j * kActBoxRows * kTileK, &tmap_act, &full[stage], 0,
                                         ch.y + j * kActBoxRows, kb0, pol);
                         bulk_load(sf + kNumA * kKB * kSfBlockBytes,
-                                  args.act_sf + (int64_t(c) * KB + kb0) * kSfBlockBytes, nkb * kSfBlockBytes,
+                                  args.act_sf + (int64_t(c) * KB + kb0) * C::kActSf, nkb * C::kActSf,
                                   &full[stage], pol);
                     }
                     filled |= 1u << stage;
@@ -270,7 +272,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         for (int a = 0; a < a_n; ++a)
                             tc_cp_sf(col + a * 4, smem_desc_sf(smem_u32(sfa + (b * kNumA + a_lo + a) * kSfBlockBytes)));
                         const uint32_t sfb_col = col + a_n * 4;
-                        tc_cp_sf(sfb_col, smem_desc_sf(smem_u32(sfb + b * kSfBlockBytes)));
+#pragma unroll
+                        for (int im = 0; im < C::kSfbImages; ++im)
+                            tc_cp_sf(sfb_col + im * 4, smem_desc_sf(smem_u32(sfb + b * C::kActSf + im * kSfBlockBytes)));
                         const uint64_t bdesc = smem_desc_sw128(smem_u32(bt + b * C::kBTile));
 #pragma unroll
                         for (int ks = 0; ks < kTileK / 32; ++ks) {
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                                                 first ? 0u : 1u);
                             }
                         }
-                        col += uint32_t((a_n + 1) * 4);
+                        col += uint32_t((a_n + C::kSfbImages) * 4);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -333,7 +337,10 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     for (int j = 0; j < 32; ++j) {
                         const float gv = __uint_as_float(g[j]);
                         const float uv = __uint_as_float(u[j]);
-                        h[j] = gv / (1.0f + expf(-gv)) * uv;
+                        // silu(g) * u with the fast exponential and division (within
+                        // the layer's tolerance; the division returns 0 where 1 + e^-g
+                        // overflows, the limit of silu)
+                        h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
                         a[j] = fabsf(h[j]);
                     }
                     // lane l: amax of token cb*32+l over this warp's 32 rows of h
@@ -342,7 +349,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     const float mult = exp2_neg(e);
                     const int tok = cb * 32 + lane;
                     if (tok < ch.z)
-                        args.out_sf[(int64_t(c) * n_tiles + tile) * kSfBlockBytes + sf_block_offset(tok, q)] =
+                        args.out_sf[(int64_t(c) * n_tiles + tile) * C::kActSf + act_sf_offset(tok, q)] =
                             uint8_t(e + 127);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {

@@ -15,13 +15,19 @@ namespace moe {
 // ---------------------------------------------------------------- layout constants
 constexpr int kTileRows = 128;        // weight rows per MMA (M) and per packet
 constexpr int kTileK = 128;           // K elements per pipeline stage and per packet
-constexpr int kChunkRows = 128;       // max routed rows (tokens) per work item (MMA N), large batches
+constexpr int kChunkRows = 160;       // max routed rows (tokens) per work item (MMA N), large batches
 constexpr int kChunkRowsSmall = 32;   // the same for small batches (decode)
 constexpr int kBoxRows = 16;          // activation rows per TMA box
 constexpr int kPacketBody = kTileRows * kTileK / 2;   // 8192 B of packed FP4
 constexpr int kPacketSf = kTileRows * 4;              // 512 B of UE8M0 (4 groups x 128 rows)
 constexpr int kPacketBytes = kPacketBody + kPacketSf; // 8704 B
-constexpr int kSfBlockBytes = kChunkRows * 4;         // 512 B activation scale block
+constexpr int kSfBlockBytes = 128 * 4;                // 512 B scale image of 128 rows x 4 groups
+
+// Bytes of the activation scale blocks of one (chunk, 128-K block): one
+// 128-row image per 128 rows of the chunk.
+__host__ __device__ constexpr int act_sf_bytes(int chunk_rows) { return (chunk_rows + 127) / 128 * kSfBlockBytes; }
+// Offset of (row r < 256, group g) inside those blocks.
+__host__ __device__ __forceinline__ int act_sf_offset(int r, int g);
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxI = 8192;
 
@@ -44,6 +50,9 @@ constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 // where lane r%32 holds rows r%32, r%32+32, r%32+64, r%32+96 in its 4 words.
 __host__ __device__ __forceinline__ int sf_block_offset(int r, int g) {
     return (r & 31) * 16 + (r >> 5) * 4 + g;
+}
+__host__ __device__ __forceinline__ int act_sf_offset(int r, int g) {
+    return (r >> 7) * kSfBlockBytes + sf_block_offset(r & 127, g);
 }
 
 // ---------------------------------------------------------------- UE8M0 scale rule

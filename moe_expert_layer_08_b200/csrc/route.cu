@@ -10,7 +10,7 @@
 // its expert), route_scan (one block: counts, offsets, per-block bases, chunk
 // list, statistics, error word), route_place (perm, inv, per-row gather
 // descriptor).  Then gather_kernel copies the FP8 rows of x into permuted
-// order (stored K-block-major, [H/128][R][128]) and the UE8M0 scales into per-chunk 512-byte blocks laid out as the
+// order (stored K-block-major, [H/128][R][128]) and the UE8M0 scales into per-chunk blocks of 512-byte images laid out as the
 // image tcgen05.cp copies into TMEM.
 //
 // Within an expert, routed rows keep ascending slot order t*k+j (a stable
@@ -233,7 +233,8 @@ __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
 constexpr int kGatherSeg = 2048;
 
 __global__ void __launch_bounds__(128) gather_kernel(const int4 *__restrict__ rowinfo, const int *__restrict__ offset,
-                                                     int E, int H, int64_t R, int segs, const uint8_t *__restrict__ x,
+                                                     int E, int H, int64_t R, int segs, int sf_bytes,
+                                                     const uint8_t *__restrict__ x,
                                                      const uint8_t *__restrict__ x_sf, uint8_t *__restrict__ xg,
                                                      uint8_t *__restrict__ xg_sf) {
     pdl_wait();
@@ -251,8 +252,8 @@ __global__ void __launch_bounds__(128) gather_kernel(const int4 *__restrict__ ro
         const int KB = H / kTileK;
         const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * (H / 32));
         for (int kb = threadIdx.x; kb < KB; kb += 128) {
-            uint8_t *blk = xg_sf + (int64_t(ri.y) * KB + kb) * kSfBlockBytes;
-            *reinterpret_cast<uint32_t *>(blk + sf_block_offset(ri.z, 0)) = __ldcg(sfs + kb);
+            uint8_t *blk = xg_sf + (int64_t(ri.y) * KB + kb) * sf_bytes;
+            *reinterpret_cast<uint32_t *>(blk + act_sf_offset(ri.z, 0)) = __ldcg(sfs + kb);
         }
     }
 }
@@ -300,7 +301,7 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
     if (e != cudaSuccess) return e;
     const int segs = (H + kGatherSeg - 1) / kGatherSeg;
     return launch_pdl(gather_kernel, dim3(unsigned(int64_t(R) * segs)), dim3(128), 0, stream,
-                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, L.Rp, segs, x, x_sf,
+                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, L.Rp, segs, act_sf_bytes(L.chunk_rows), x, x_sf,
                       ws + L.off_xg, ws + L.off_xg_sf);
 }
 
