@@ -32,17 +32,19 @@
 
 namespace moe {
 
-// kN = the largest token chunk an item can hold (the MMA's N).  Small-batch
-// launches (kN = 32) take 256-K stages and two MMA-issuing warps: each
-// tcgen05.mma / tcgen05.cp costs a fixed issue slot whatever its N, so at
-// decode sizes the issue rate of a single thread, not HBM, would set the pace.
+// kN = the largest token chunk an item can hold (the MMA's N).  Every item
+// owns two 128-row weight tiles that share the chunk's activations: GEMM1 the
+// gate and up tiles of one intermediate block, GEMM2 two adjacent output
+// tiles.  Each tile has its own accumulator and its own MMA-issuing warp, since
+// every tcgen05.mma / tcgen05.cp costs a fixed issue slot whatever its N.
+// Small-batch launches (kN = 32) take 256-K stages.
 template <bool kGemm1, int kN>
 struct GemmCfg {
     static constexpr bool kSmall = kN == kChunkRowsSmall;
-    static constexpr int kNumA = kGemm1 ? 2 : 1;        // weight tiles per K block: (gate, up) or (down)
+    static constexpr int kNumA = 2;                     // weight tiles (accumulators, issuers) per item
     static constexpr int kKB = kSmall ? 2 : 1;          // 128-K blocks per pipeline stage
-    static constexpr int kIssuers = (kSmall || kGemm1) ? 2 : 1;  // MMA-issuing warps
-    static constexpr int kStages = kSmall ? (kGemm1 ? 3 : 5) : (kGemm1 ? 4 : 6);
+    static constexpr int kIssuers = 2;
+    static constexpr int kStages = kSmall ? 3 : 4;
     static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 one-byte elements
     static constexpr int kBTile = kN * kTileK;          // token rows x 128 bytes, per K block
     static constexpr int kStageTiles = kNumA * kKB * kATile + kKB * kBTile;
@@ -53,27 +55,30 @@ struct GemmCfg {
     static constexpr int kSmemSf = kStages * kStageSf;
     static constexpr int kSmemMisc = 256;
     static constexpr int kSmemBytes = 1024 + kSmemTiles + kSmemSf + kSmemMisc;
-    // Accumulators per buffer: GEMM1 (gate, up); GEMM2 one per issuer (a
-    // K split, summed by the epilogue).
-    static constexpr int kNumAcc = kGemm1 ? 2 : kIssuers;
-    static constexpr int kAccCols = kNumAcc * kN;
-    // Per issuer and stage: the scale blocks of the weight tiles it consumes
-    // and of the activation K blocks it consumes, 4 TMEM columns each.
-    static constexpr int kIssuerKB = (!kGemm1 && kIssuers == 2) ? 1 : kKB;
-    static constexpr int kIssuerAcc = (kGemm1 && kIssuers == 1) ? 2 : 1;
-    static constexpr int kSfColsIssuer = kIssuerKB * (kIssuerAcc + kSfbImages) * 4;
+    static constexpr int kAccCols = kNumA * kN;          // one accumulator buffer
+    // per issuer and stage: its weight tile's and the activations' scale images
+    static constexpr int kSfColsIssuer = kKB * (1 + kSfbImages) * 4;
     static constexpr int kSfCols = kStages * kIssuers * kSfColsIssuer;
     static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
-    static constexpr int kThreads = 224 + 32 * (kIssuers - 1);  // + activation producer, + second issuer
+    static constexpr int kThreads = 256;  // producers (2), issuers (2), epilogue (4)
+    // weight packets one TMA box moves: GEMM1's gate and up packets of
+    // consecutive K tiles are adjacent, GEMM2's two tiles are not
+    static constexpr int kBoxPackets = kGemm1 ? kNumA * kKB : kKB;
     static_assert(kTmemUsed <= 512, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kBTile % 1024 == 0, "swizzle atoms");
     static_assert(kKB == 1 || kN == kActBoxRows, "one activation box per stage when a stage spans K blocks");
-    static_assert(kGemm1 || kIssuers == 1 || kKB == kIssuers, "GEMM2 K split needs one K block per issuer");
 };
+
+// Shared-memory slot of weight tile a (0, 1) of K block b within a stage:
+// the order in which the TMA boxes land.
+template <bool kGemm1, int kKB>
+__device__ __forceinline__ int a_slot(int a, int b) {
+    return kGemm1 ? b * 2 + a : a * kKB + b;
+}
 
 struct GemmArgs {
     const uint8_t *w_packets;  // transformed weights (for the scale blocks)
@@ -84,7 +89,8 @@ struct GemmArgs {
     uint8_t *out_sf;           // GEMM1: h scale blocks [chunk][I/128][512]
     __nv_bfloat16 *out_y;      // GEMM2: Y [R, H]
     int K;                     // reduction length (H for GEMM1, I for GEMM2)
-    int n_tiles;               // output tiles per expert (I/128 or H/128)
+    int n_tiles;               // 128-row weight tiles per expert and half (GEMM1: I/128, GEMM2: H/128)
+    int n_items;               // items per chunk (GEMM1: I/128, GEMM2: tile pairs)
     int out_ld;                // row length of the output (I or H)
     int rows;                  // row extent of the K-block-major FP8 operands
 };
@@ -159,14 +165,14 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
     if (!(early_weights && is_w_producer)) pdl_wait();
     if (threadIdx.x == 32) pdl_trigger();
 
-    const int n_tiles = args.n_tiles;
-    const int num_items = __ldcg(args.hdr + kHdrNumChunks) * n_tiles;
+    const int n_tiles = args.n_tiles, n_items = args.n_items;
+    const int num_items = __ldcg(args.hdr + kHdrNumChunks) * n_items;
     const int KB = args.K / kTileK;
     const int n_steps = (KB + kKB - 1) / kKB;  // pipeline stages per item
     int *err = args.hdr;
 
     // which MMA issuer this warp is (-1: none)
-    const int issuer = warp == 1 ? 0 : (kIssuers == 2 && warp == 7) ? 1 : -1;
+    const int issuer = warp == 1 ? 0 : warp == 7 ? 1 : -1;
 
     if (warp == 0 || warp == 6) {
         if (lane == 0) {
@@ -181,10 +187,13 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
             uint32_t filled = 0, fill_parity = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
-                const int c = item / n_tiles, tile = item % n_tiles;
+                const int c = item / n_items, it = item % n_items;
                 const int4 ch = __ldcg(args.chunks + c);
                 const int nbox = (ch.z + kActBoxRows - 1) / kActBoxRows;
-                const int64_t pkt0 = (int64_t(ch.x) * n_tiles + tile) * KB * kNumA;
+                // GEMM1: gate/up packets of tile `it`, interleaved per K tile;
+                // GEMM2: tiles 2*it and 2*it+1 (the second may not exist)
+                const int t0 = kGemm1 ? it : 2 * it;
+                const int n_valid = kGemm1 ? 2 : (t0 + 1 < n_tiles ? 2 : 1);
                 for (int step = 0; step < n_steps; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
@@ -195,12 +204,21 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     uint8_t *st = tiles + stage * C::kStageTiles;
                     uint8_t *sf = sfs + stage * C::kStageSf;
                     if (weights) {
-                        // the weight boxes always move kNumA * kKB packets (a
-                        // last odd K block loads one packet it then ignores)
-                        mbar_arrive_expect_tx(&full[stage], uint32_t(kNumA * kKB * (kPacketBody + kPacketSf)));
-                        const int pkt = int(pkt0 + int64_t(kb0) * kNumA);
-                        tma_load_3d(st, &tmap_w, &full[stage], 0, 0, pkt, pol);
-                        tma_load_2d(sf, &tmap_wsf, &full[stage], kPacketBody / 4, pkt, pol);
+                        // a box always moves kBoxPackets packets (a last odd K
+                        // block loads a packet it then ignores)
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(n_valid * kKB * (kPacketBody + kPacketSf)));
+                        if (kGemm1) {
+                            const int pkt = int((int64_t(ch.x) * n_tiles + t0) * KB * 2 + int64_t(kb0) * 2);
+                            tma_load_3d(st, &tmap_w, &full[stage], 0, 0, pkt, pol);
+                            tma_load_2d(sf, &tmap_wsf, &full[stage], kPacketBody / 4, pkt, pol);
+                        } else {
+                            for (int a = 0; a < n_valid; ++a) {
+                                const int pkt = int((int64_t(ch.x) * n_tiles + t0 + a) * KB + kb0);
+                                tma_load_3d(st + a * kKB * C::kATile, &tmap_w, &full[stage], 0, 0, pkt, pol);
+                                tma_load_2d(sf + a * kKB * kSfBlockBytes, &tmap_wsf, &full[stage], kPacketBody / 4, pkt,
+                                            pol);
+                            }
+                        }
                     } else {
                         // the activation box always moves kKB K blocks (a K
                         // block past the end reads zeros)
@@ -235,21 +253,22 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
     } else if (issuer >= 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
-            // GEMM1: issuer 0 owns the gate accumulator, issuer 1 the up one
-            // (a single issuer owns both).  GEMM2: issuer i owns accumulator i
-            // and the stage's K block i.
+            // Issuer a owns weight tile a of every item and its accumulator.
+            const int a = issuer;
             int stage = 0;
             uint32_t phase = 0;
             int li = 0;  // items handled by this CTA so far
             bool ok = true;
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++li) {
-                const int4 ch = __ldcg(args.chunks + item / n_tiles);
+                const int4 ch = __ldcg(args.chunks + item / n_items);
+                const int it = item % n_items;
+                const bool valid = kGemm1 || 2 * it + a < n_tiles;  // GEMM2's last pair may hold one tile
                 const uint32_t n = uint32_t((ch.z + 15) / 16 * 16);
                 const int buf = li % kBufs;
                 const uint32_t use = uint32_t(li / kBufs) & 1u;  // how often this buffer was used, mod 2
                 if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 2)) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + uint32_t(buf * C::kAccCols);
+                const uint32_t acc = tmem + uint32_t(buf * C::kAccCols + a * kN);
                 for (int step = 0; step < n_steps; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
@@ -258,38 +277,33 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint8_t *st = tiles + stage * C::kStageTiles;
-                    const uint8_t *sfa = sfs + stage * C::kStageSf;
-                    const uint8_t *sfb = sfa + kNumA * kKB * kSfBlockBytes;
-                    const uint8_t *bt = st + kNumA * kKB * C::kATile;
-                    uint32_t col = tmem + uint32_t(kBufs * C::kAccCols + (stage * kIssuers + issuer) * C::kSfColsIssuer);
-                    const int b_lo = (!kGemm1 && kIssuers == 2) ? issuer : 0;
-                    const int b_hi = (!kGemm1 && kIssuers == 2) ? issuer + 1 : nkb;
-                    for (int b = b_lo; b < b_hi && b < nkb; ++b) {
-                        // scale blocks of this K block into TMEM: weight tile(s), then activations
-                        const int a_lo = kGemm1 ? (kIssuers == 2 ? issuer : 0) : 0;
-                        const int a_n = C::kIssuerAcc;
-                        for (int a = 0; a < a_n; ++a)
-                            tc_cp_sf(col + a * 4, smem_desc_sf(smem_u32(sfa + (b * kNumA + a_lo + a) * kSfBlockBytes)));
-                        const uint32_t sfb_col = col + a_n * 4;
+                    if (valid) {
+                        const uint8_t *st = tiles + stage * C::kStageTiles;
+                        const uint8_t *sfa = sfs + stage * C::kStageSf;
+                        const uint8_t *sfb = sfa + kNumA * kKB * kSfBlockBytes;
+                        const uint8_t *bt = st + kNumA * kKB * C::kATile;
+                        uint32_t col =
+                            tmem + uint32_t(kBufs * C::kAccCols + (stage * kIssuers + a) * C::kSfColsIssuer);
+                        for (int b = 0; b < nkb; ++b) {
+                            const int slot = a_slot<kGemm1, kKB>(a, b);
+                            // scale images of this K block into TMEM: weight tile, then activations
+                            tc_cp_sf(col, smem_desc_sf(smem_u32(sfa + slot * kSfBlockBytes)));
+                            const uint32_t sfb_col = col + 4;
 #pragma unroll
-                        for (int im = 0; im < C::kSfbImages; ++im)
-                            tc_cp_sf(sfb_col + im * 4, smem_desc_sf(smem_u32(sfb + b * C::kActSf + im * kSfBlockBytes)));
-                        const uint64_t bdesc = smem_desc_sw128(smem_u32(bt + b * C::kBTile));
+                            for (int im = 0; im < C::kSfbImages; ++im)
+                                tc_cp_sf(sfb_col + im * 4,
+                                         smem_desc_sf(smem_u32(sfb + b * C::kActSf + im * kSfBlockBytes)));
+                            const uint64_t adesc = smem_desc_sw128(smem_u32(st + slot * C::kATile));
+                            const uint64_t bdesc = smem_desc_sw128(smem_u32(bt + b * C::kBTile));
 #pragma unroll
-                        for (int ks = 0; ks < kTileK / 32; ++ks) {
-                            const uint32_t idesc = idesc_mxf8f6f4(n, uint32_t(ks));
-                            for (int a = 0; a < a_n; ++a) {
-                                const int acc_i = kGemm1 ? a_lo + a : issuer;
-                                const uint64_t adesc = smem_desc_sw128(smem_u32(st + (b * kNumA + a_lo + a) * C::kATile));
-                                const bool first = (kb0 + b == (kGemm1 ? 0 : b_lo)) && ks == 0;
+                            for (int ks = 0; ks < kTileK / 32; ++ks) {
                                 // +32 bytes of K per step inside the 128-byte swizzled row
-                                tc_mma_mxf8f6f4(acc + uint32_t(acc_i * kN), adesc + uint64_t(2 * ks),
-                                                bdesc + uint64_t(2 * ks), idesc, col + a * 4, sfb_col,
-                                                first ? 0u : 1u);
+                                tc_mma_mxf8f6f4(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks),
+                                                idesc_mxf8f6f4(n, uint32_t(ks)), col, sfb_col,
+                                                (kb0 + b == 0 && ks == 0) ? 0u : 1u);
                             }
+                            col += uint32_t((1 + C::kSfbImages) * 4);
                         }
-                        col += uint32_t((a_n + C::kSfbImages) * 4);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -301,9 +315,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                 tc_commit(&tmem_full[buf]);
             }
             // All issued MMAs must be finished before TMEM is released.
-            tc_commit(&mma_done[issuer]);
+            tc_commit(&mma_done[a]);
             const unsigned long long t0 = global_timer_ns();
-            while (!mbar_try_wait(&mma_done[issuer], 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+            while (!mbar_try_wait(&mma_done[a], 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
             }
         }
         __syncwarp();
@@ -311,12 +325,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        // GEMM2 with a K split: the second accumulator holds a partial sum
-        // only when there is a second K block
-        const bool add_second = !kGemm1 && kIssuers == 2 && KB > 1;
         int li = 0;
         for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
-            const int c = item / n_tiles, tile = item % n_tiles;
+            const int c = item / n_items, it = item % n_items;
             const int4 ch = __ldcg(args.chunks + c);
             const int buf = li % kBufs;
             const uint32_t use = uint32_t(li / kBufs) & 1u;
@@ -324,15 +335,13 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
             tc_fence_after();
             const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
             const int ncb = (ch.z + 31) / 32;
-            const int row_out = tile * kTileRows + q * 32 + lane;  // this thread's output column
             for (int cb = 0; cb < ncb; ++cb) {
-                uint32_t g[32];
-                tmem_ld_32x32(acc + uint32_t(cb * 32), g);
                 if constexpr (kGemm1) {
-                    uint32_t u[32];
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32(acc + uint32_t(cb * 32), g);
                     tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
                     tmem_ld_wait();
-                    float h[32], a[32];
+                    float h[32], amx[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float gv = __uint_as_float(g[j]);
@@ -341,15 +350,15 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         // the layer's tolerance; the division returns 0 where 1 + e^-g
                         // overflows, the limit of silu)
                         h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
-                        a[j] = fabsf(h[j]);
+                        amx[j] = fabsf(h[j]);
                     }
                     // lane l: amax of token cb*32+l over this warp's 32 rows of h
-                    const float amax = warp_transpose_max(a, lane);
+                    const float amax = warp_transpose_max(amx, lane);
                     const int e = scale_exponent<true>(amax);
                     const float mult = exp2_neg(e);
                     const int tok = cb * 32 + lane;
                     if (tok < ch.z)
-                        args.out_sf[(int64_t(c) * n_tiles + tile) * C::kActSf + act_sf_offset(tok, q)] =
+                        args.out_sf[(int64_t(c) * n_tiles + it) * C::kActSf + act_sf_offset(tok, q)] =
                             uint8_t(e + 127);
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -357,26 +366,24 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         const uint32_t code = to_e4m3(h[j] * mj);
                         // K-block-major [I/128][rows][128]: GEMM2 reads two K blocks per box
                         if (cb * 32 + j < ch.z)
-                            args.out_q[(int64_t(tile) * args.rows + ch.y + cb * 32 + j) * kTileK + q * 32 + lane] =
+                            args.out_q[(int64_t(it) * args.rows + ch.y + cb * 32 + j) * kTileK + q * 32 + lane] =
                                 uint8_t(code);
                     }
                 } else {
-                    float y[32];
-                    if (add_second) {
-                        uint32_t g2[32];
-                        tmem_ld_32x32(acc + uint32_t(kN + cb * 32), g2);
-                        tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(g[j]) + __uint_as_float(g2[j]);
-                    } else {
+                    for (int a = 0; a < kNumA; ++a) {
+                        const int tile = 2 * it + a;
+                        if (tile >= n_tiles) break;
+                        uint32_t g[32];
+                        tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), g);
                         tmem_ld_wait();
+                        const int col_out = tile * kTileRows + q * 32 + lane;  // this thread's output column
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(g[j]);
+                        for (int j = 0; j < 32; ++j)
+                            if (cb * 32 + j < ch.z)
+                                args.out_y[int64_t(ch.y + cb * 32 + j) * args.out_ld + col_out] =
+                                    __float2bfloat16_rn(__uint_as_float(g[j]));
                     }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (cb * 32 + j < ch.z)
-                            args.out_y[int64_t(ch.y + cb * 32 + j) * args.out_ld + row_out] = __float2bfloat16_rn(y[j]);
                 }
             }
             tc_fence_before();
@@ -413,10 +420,10 @@ int gemm_kblocks_per_stage(int chunk_rows) {
 }
 
 int gemm_packets_per_stage(bool gemm1, int chunk_rows) {
-    return gemm1 ? (chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall>::kNumA * GemmCfg<true, kChunkRowsSmall>::kKB
-                                                  : GemmCfg<true, kChunkRows>::kNumA * GemmCfg<true, kChunkRows>::kKB)
-                 : (chunk_rows == kChunkRowsSmall ? GemmCfg<false, kChunkRowsSmall>::kNumA * GemmCfg<false, kChunkRowsSmall>::kKB
-                                                  : GemmCfg<false, kChunkRows>::kNumA * GemmCfg<false, kChunkRows>::kKB);
+    return gemm1 ? (chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall>::kBoxPackets
+                                                  : GemmCfg<true, kChunkRows>::kBoxPackets)
+                 : (chunk_rows == kChunkRowsSmall ? GemmCfg<false, kChunkRowsSmall>::kBoxPackets
+                                                  : GemmCfg<false, kChunkRows>::kBoxPackets);
 }
 
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
@@ -433,6 +440,7 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
         a.out_sf = ws + L.off_hq_sf;
         a.K = H;
         a.n_tiles = I / kTileRows;
+        a.n_items = I / kTileRows;
         a.out_ld = I;
         a.rows = int(L.Rp);
         return small ? launch_gemm_t<true, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, a, grid, stream)
@@ -442,6 +450,7 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
     a.out_y = reinterpret_cast<__nv_bfloat16 *>(ws + L.off_y);
     a.K = I;
     a.n_tiles = H / kTileRows;
+    a.n_items = (H / kTileRows + 1) / 2;
     a.out_ld = H;
     a.rows = int(L.Rp);
     return small ? launch_gemm_t<false, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, a, grid, stream)
