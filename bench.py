@@ -44,6 +44,7 @@ def parse():
     p.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the oracle's timed sample")
     p.add_argument("--experts", type=int, default=0,
                    help="override E (a smaller resident weight set for profiler captures)")
+    p.add_argument("--tokens", type=int, default=0, help="override T (with --experts: same rows per expert)")
     return p.parse_args()
 
 
@@ -356,8 +357,9 @@ def main():
         torch.distributed.init_process_group("nccl" if args.impl == "b200" else "gloo",
                                              timeout=datetime.timedelta(seconds=120))
     w = W.WORKLOADS[args.workload]
-    if args.experts:
-        w = W.custom(f"{w.name}_E{args.experts}", T=w.T, E=args.experts, k=w.k, H=w.H, I=w.I, seed=w.seed,
+    if args.experts or args.tokens:
+        E, T = args.experts or w.E, args.tokens or w.T
+        w = W.custom(f"{w.name}_T{T}_E{E}", T=T, E=E, k=w.k, H=w.H, I=w.I, seed=w.seed,
                      routing=w.routing, zipf_s=w.zipf_s)
     try:
         if args.impl == "reference":

@@ -38,7 +38,7 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.off_perm = take(sizeof(int) * R);
     L.off_inv = take(sizeof(int) * R);
     L.off_rowinfo = take(sizeof(int4) * R);
-    L.Rp = L.R > kActBoxRows ? L.R : kActBoxRows;
+    L.Rp = L.R > kChunkRows ? L.R : kChunkRows;  // at least the largest activation box
     L.kbh = H / kTileK > 2 ? H / kTileK : 2;
     L.kbi = I / kTileK > 2 ? I / kTileK : 2;
     L.off_xg = take(size_t(L.Rp) * size_t(L.kbh) * kTileK);
@@ -103,14 +103,14 @@ bool encode_packet_sf(CUtensorMap *m, const void *base, int64_t num_packets, int
 }
 
 // FP8 activations stored K-block-major, [kblocks][rows][128] bytes, as a 3D
-// tensor (128 bytes, rows, K blocks); one box moves kActBoxRows rows of
+// tensor (128 bytes, rows, K blocks); one box moves `box_rows` rows of
 // `depth` consecutive K blocks.
-bool encode_act(CUtensorMap *m, const void *base, int64_t rows, int64_t kblocks, int depth) {
+bool encode_act(CUtensorMap *m, const void *base, int64_t rows, int64_t kblocks, int depth, int box_rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     const cuuint64_t dims[3] = {cuuint64_t(kTileK), cuuint64_t(rows), cuuint64_t(kblocks)};
     const cuuint64_t strides[2] = {cuuint64_t(kTileK), cuuint64_t(rows) * kTileK};
-    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(kActBoxRows), cuuint32_t(depth)};
+    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(box_rows), cuuint32_t(depth)};
     const cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -172,11 +172,14 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
 
     const int64_t np1 = int64_t(l1_bytes / kPacketBytes), np2 = int64_t(l2_bytes / kPacketBytes);
     const int d1 = gemm_packets_per_stage(true, L.chunk_rows), d2 = gemm_packets_per_stage(false, L.chunk_rows);
-    CUtensorMap tm_w1, tm_w2, tm_s1, tm_s2, tm_xg, tm_hq;
+    const int dk = gemm_kblocks_per_stage(L.chunk_rows);
+    CUtensorMap tm_w1, tm_w2, tm_s1, tm_s2, tm_xg, tm_hq, tm_xg_full, tm_hq_full;
     if (!encode_packets(&tm_w1, l1_t, np1, d1) || !encode_packets(&tm_w2, l2_t, np2, d2) ||
         !encode_packet_sf(&tm_s1, l1_t, np1, d1) || !encode_packet_sf(&tm_s2, l2_t, np2, d2) ||
-        !encode_act(&tm_xg, ws + L.off_xg, L.Rp, L.kbh, gemm_kblocks_per_stage(L.chunk_rows)) ||
-        !encode_act(&tm_hq, ws + L.off_hq, L.Rp, L.kbi, gemm_kblocks_per_stage(L.chunk_rows)))
+        !encode_act(&tm_xg, ws + L.off_xg, L.Rp, L.kbh, dk, kActBoxRows) ||
+        !encode_act(&tm_hq, ws + L.off_hq, L.Rp, L.kbi, dk, kActBoxRows) ||
+        !encode_act(&tm_xg_full, ws + L.off_xg, L.Rp, L.kbh, dk, L.chunk_rows) ||
+        !encode_act(&tm_hq_full, ws + L.off_hq, L.Rp, L.kbi, dk, L.chunk_rows))
         return MOE_ERR_CUDA;
 
     auto record = [&](int i) -> cudaError_t {
@@ -195,10 +198,10 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
                          H, ws, L, expert_stats, st);
     if (e == cudaSuccess) e = record(1);
     if (e == cudaSuccess)
-        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
+        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
     if (e == cudaSuccess) e = record(2);
     if (e == cudaSuccess)
-        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
+        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
     if (e == cudaSuccess) e = record(3);
     if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
     if (e == cudaSuccess) e = record(4);

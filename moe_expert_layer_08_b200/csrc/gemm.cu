@@ -115,7 +115,8 @@ __device__ __forceinline__ float warp_transpose_max(float (&a)[32], int lane) {
 template <bool kGemm1, int kN>
 __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_wsf,
-                    const __grid_constant__ CUtensorMap tmap_act, const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_act_full,
+                    const GemmArgs args) {
     using C = GemmCfg<kGemm1, kN>;
     constexpr int kNumA = C::kNumA, kKB = C::kKB, kStages = C::kStages, kBufs = C::kAccBufs;
     constexpr int kIssuers = C::kIssuers;
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
         prefetch_tmap(&tmap_w);
         prefetch_tmap(&tmap_wsf);
         prefetch_tmap(&tmap_act);
+        prefetch_tmap(&tmap_act_full);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, C::kTmemCols);
@@ -221,13 +223,19 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         }
                     } else {
                         // the activation box always moves kKB K blocks (a K
-                        // block past the end reads zeros)
-                        mbar_arrive_expect_tx(&full[stage],
-                                              uint32_t(nbox * kKB * kActBoxRows * kTileK + nkb * C::kActSf));
+                        // block past the end reads zeros); a nearly full large
+                        // chunk takes one kN-row box instead of several 32-row ones
+                        const bool one_box = !C::kSmall && ch.z > kN - 64;
+                        const int rows_moved = one_box ? kN : nbox * kActBoxRows;
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(rows_moved * kKB * kTileK + nkb * C::kActSf));
                         uint8_t *bt = st + kNumA * kKB * C::kATile;
-                        for (int j = 0; j < nbox; ++j)
-                            tma_load_3d(bt + j * kActBoxRows * kTileK, &tmap_act, &full[stage], 0,
-                                        ch.y + j * kActBoxRows, kb0, pol);
+                        if (one_box) {
+                            tma_load_3d(bt, &tmap_act_full, &full[stage], 0, ch.y, kb0, pol);
+                        } else {
+                            for (int j = 0; j < nbox; ++j)
+                                tma_load_3d(bt + j * kActBoxRows * kTileK, &tmap_act, &full[stage], 0,
+                                            ch.y + j * kActBoxRows, kb0, pol);
+                        }
                         bulk_load(sf + kNumA * kKB * kSfBlockBytes,
                                   args.act_sf + (int64_t(c) * KB + kb0) * C::kActSf, nkb * C::kActSf,
                                   &full[stage], pol);
@@ -400,7 +408,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
 
 template <bool kGemm1, int kN>
 static cudaError_t launch_gemm_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf, const CUtensorMap &tmap_act,
-                                 const GemmArgs &args, int grid, cudaStream_t stream) {
+                                 const CUtensorMap &tmap_act_full, const GemmArgs &args, int grid,
+                                 cudaStream_t stream) {
     using C = GemmCfg<kGemm1, kN>;
     static int configured_for = -1;
     int dev = 0;
@@ -412,7 +421,7 @@ static cudaError_t launch_gemm_t(const CUtensorMap &tmap_w, const CUtensorMap &t
         configured_for = dev;
     }
     return launch_pdl(moe_gemm_kernel<kGemm1, kN>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
-                      tmap_w, tmap_wsf, tmap_act, args);
+                      tmap_w, tmap_wsf, tmap_act, tmap_act_full, args);
 }
 
 int gemm_kblocks_per_stage(int chunk_rows) {
@@ -427,8 +436,8 @@ int gemm_packets_per_stage(bool gemm1, int chunk_rows) {
 }
 
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
-                        const CUtensorMap &tmap_act, const uint8_t *w_packets, uint8_t *ws, const WsLayout &L, int H,
-                        int I, int grid, cudaStream_t stream) {
+                        const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const uint8_t *w_packets,
+                        uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream) {
     GemmArgs a{};
     a.w_packets = w_packets;
     a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
@@ -443,8 +452,8 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
         a.n_items = I / kTileRows;
         a.out_ld = I;
         a.rows = int(L.Rp);
-        return small ? launch_gemm_t<true, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, a, grid, stream)
-                     : launch_gemm_t<true, kChunkRows>(tmap_w, tmap_wsf, tmap_act, a, grid, stream);
+        return small ? launch_gemm_t<true, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream)
+                     : launch_gemm_t<true, kChunkRows>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
     }
     a.act_sf = ws + L.off_hq_sf;
     a.out_y = reinterpret_cast<__nv_bfloat16 *>(ws + L.off_y);
@@ -453,8 +462,8 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
     a.n_items = (H / kTileRows + 1) / 2;
     a.out_ld = H;
     a.rows = int(L.Rp);
-    return small ? launch_gemm_t<false, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, a, grid, stream)
-                 : launch_gemm_t<false, kChunkRows>(tmap_w, tmap_wsf, tmap_act, a, grid, stream);
+    return small ? launch_gemm_t<false, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream)
+                 : launch_gemm_t<false, kChunkRows>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
 }
 
 }  // namespace moe

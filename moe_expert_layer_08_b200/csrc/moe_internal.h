@@ -59,8 +59,8 @@ cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_pe
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
                          int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream);
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
-                        const CUtensorMap &tmap_act, const uint8_t *w_packets, uint8_t *ws, const WsLayout &L, int H,
-                        int I, int grid, cudaStream_t stream);
+                        const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const uint8_t *w_packets,
+                        uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream);
 // Weight packets one pipeline stage of that GEMM variant moves (TMA box depth).
 int gemm_packets_per_stage(bool gemm1, int chunk_rows);
 // 128-K blocks one pipeline stage moves (the activation box depth).

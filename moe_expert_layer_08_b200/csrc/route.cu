@@ -7,8 +7,9 @@
 // Small batches (T*k <= 1024 slots): one block does everything
 // (route_small_kernel).  Large batches: route_count (per 256-slot block,
 // per-expert counts and each slot's rank among the block's earlier slots of
-// its expert), route_scan (one block: counts, offsets, per-block bases, chunk
-// list, statistics, error word), route_place (perm, inv, per-row gather
+// its expert), route_colscan (one block per expert: that expert's per-block
+// bases and its count), route_meta (one block: offsets, chunk list,
+// statistics, error word), route_place (perm, inv, per-row gather
 // descriptor).  Then gather_kernel copies the FP8 rows of x into permuted
 // order (stored K-block-major, [H/128][R][128]) and the UE8M0 scales into per-chunk blocks of 512-byte images laid out as the
 // image tcgen05.cp copies into TMEM.
@@ -162,37 +163,51 @@ __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const int64_t 
     for (int x = tid; x < E; x += kRouteBlock) {
         int sum = 0;
         for (int w = 0; w < kWarps; ++w) sum += cnt[w * E + x];
-        hist[size_t(blockIdx.x) * E + x] = sum;
+        hist[size_t(x) * gridDim.x + blockIdx.x] = sum;  // expert-major
     }
     const int nbad = __syncthreads_count(s < R && !valid);
     if (tid == 0) bad[blockIdx.x] = nbad;
 }
 
-__global__ void __launch_bounds__(1024) route_scan_kernel(int *__restrict__ hist, const int *__restrict__ bad,
-                                                          int nb, int E, int chunk_rows, int *__restrict__ count,
-                                                          int *__restrict__ offset, int *__restrict__ chunk_base,
-                                                          int4 *__restrict__ chunks, int *__restrict__ hdr,
-                                                          int32_t *__restrict__ expert_stats) {
+// One block per expert: exclusive prefix over the routing blocks of that
+// expert's counts (in place, expert-major) and the expert's total.
+__global__ void __launch_bounds__(1024) route_colscan_kernel(int *__restrict__ hist, int nb, int *__restrict__ count) {
+    __shared__ int s_warp[32];
+    __shared__ int s_carry;
+    pdl_wait();
+    pdl_trigger();
+    const int e = blockIdx.x;
+    int *row = hist + size_t(e) * nb;
+    if (threadIdx.x == 0) s_carry = 0;
+    __syncthreads();
+    for (int b0 = 0; b0 < nb; b0 += blockDim.x) {
+        const int b = b0 + threadIdx.x;
+        const int v = b < nb ? __ldcg(row + b) : 0;
+        const int ex = block_exclusive_scan(v, s_warp);
+        const int carry = s_carry;
+        if (b < nb) row[b] = carry + ex;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) s_carry = carry + ex + v;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) count[e] = s_carry;
+}
+
+// One block: offsets and chunk bases (scans over experts), chunk list,
+// statistics, dropped count and error word.
+__global__ void __launch_bounds__(1024) route_meta_kernel(const int *__restrict__ bad, int nb, int E, int chunk_rows,
+                                                          int *__restrict__ count, int *__restrict__ offset,
+                                                          int *__restrict__ chunk_base, int4 *__restrict__ chunks,
+                                                          int *__restrict__ hdr, int32_t *__restrict__ expert_stats) {
     __shared__ int s_warp[32];
     __shared__ int s_bad;
     const int e = threadIdx.x;
     pdl_wait();
     pdl_trigger();
-    int c = 0;
-    if (e < E)
-        for (int b = 0; b < nb; ++b) c += __ldcg(hist + size_t(b) * E + e);
+    const int c = e < E ? __ldcg(count + e) : 0;
     const int off = block_exclusive_scan(c, s_warp);
     const int cbase = block_exclusive_scan((c + chunk_rows - 1) / chunk_rows, s_warp);
-    if (e < E) {
-        int run = off;  // per-block base position of this expert's slots
-        for (int b = 0; b < nb; ++b) {
-            const size_t ix = size_t(b) * E + e;
-            const int h = __ldcg(hist + ix);
-            hist[ix] = run;
-            run += h;
-        }
-        write_expert_meta(e, E, c, off, cbase, chunk_rows, count, offset, chunk_base, chunks, hdr, expert_stats);
-    }
+    if (e < E) write_expert_meta(e, E, c, off, cbase, chunk_rows, count, offset, chunk_base, chunks, hdr, expert_stats);
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
     int d = 0;
@@ -220,7 +235,7 @@ __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
         return;
     }
     const int e = int(v);
-    const int pos = __ldcg(base + size_t(blockIdx.x) * E + e) + __ldcg(lrank + s);
+    const int pos = __ldcg(offset + e) + __ldcg(base + size_t(e) * gridDim.x + blockIdx.x) + __ldcg(lrank + s);
     perm[pos] = int(s);
     inv[s] = pos;
     const int local = pos - __ldcg(offset + e);
@@ -291,9 +306,12 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
         const size_t cnt_smem = size_t(kRouteBlock / 32) * E * sizeof(int);
         e = launch_pdl(route_count_kernel, dim3(L.nb), dim3(kRouteBlock), cnt_smem, stream, topk_idx, R, E, hist,
                        lrank, bad);
+        const int cs_threads = L.nb >= 1024 ? 1024 : (L.nb + 31) / 32 * 32;
         if (e == cudaSuccess)
-            e = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, hist, bad, L.nb, E, cr, count, offset,
-                           chunk_base, chunks, hdr, expert_stats);
+            e = launch_pdl(route_colscan_kernel, dim3(E), dim3(cs_threads), 0, stream, hist, L.nb, count);
+        if (e == cudaSuccess)
+            e = launch_pdl(route_meta_kernel, dim3(1), dim3(1024), 0, stream, static_cast<const int *>(bad), L.nb, E,
+                           cr, count, offset, chunk_base, chunks, hdr, expert_stats);
         if (e == cudaSuccess)
             e = launch_pdl(route_place_kernel, dim3(L.nb), dim3(kRouteBlock), 0, stream, topk_idx, R, k, E, cr, hist,
                            lrank, offset, chunk_base, perm, inv, rowinfo);
