@@ -84,7 +84,9 @@ moe_status_t moe_quantize_fp4(const void *w, int64_t rows, int64_t cols,
 
 /*
  * moe_transformed_weight_bytes -- sizes of the two tile-major weight buffers
- * that moe_transform_weights writes for E experts (host-only, no CUDA call).
+ * that moe_transform_weights writes for E experts (host-only, no CUDA call):
+ * 8704 bytes per packet (128 x 128 FP4 body + 512 scale bytes), 2*(I/128)*(H/128)
+ * packets per expert for L1 and 2*ceil(H/256)*(I/128) for L2.
  */
 moe_status_t moe_transformed_weight_bytes(int E, int H, int I,
                                           size_t *l1_bytes, size_t *l2_bytes);
@@ -96,8 +98,11 @@ moe_status_t moe_transformed_weight_bytes(int E, int H, int I,
  * Motivation).  Packs each expert's logical FP4 weights and their UE8M0
  * scales into packets of one 128-row x 128-K tile followed by the 512 scale
  * bytes that tile consumes, so body and scales share one allocation and one
- * access stream.  Packet order: expert -> output tile -> K tile -> (gate, up)
- * for L1; expert -> output tile -> K tile for L2.
+ * access stream.  Packet order: expert -> intermediate tile i -> K tile ->
+ * (gate tile i, up tile i) for L1; expert -> output tile pair p -> K tile ->
+ * (tile 2p, tile 2p+1) for L2, so the two tiles one GEMM work item multiplies
+ * are adjacent for every K tile (an odd H/128 gets one zero-filled padding
+ * tile per expert).
  *   l1    : u8 [E, 2I, H/2]   rows 0..I-1 gate, I..2I-1 up     (in)
  *   l1_sf : u8 [E, 2I, H/32]                                   (in)
  *   l2    : u8 [E, H, I/2]                                     (in)

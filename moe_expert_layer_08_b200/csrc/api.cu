@@ -252,9 +252,12 @@ moe_status_t moe_quantize_fp4(const void *w, int64_t rows, int64_t cols, void *q
 moe_status_t moe_transformed_weight_bytes(int E, int H, int I, size_t *l1_bytes, size_t *l2_bytes) {
     const moe_status_t s = check_shape(E, H, I);
     if (s != MOE_OK) return s;
-    const size_t per_tile_k = size_t(H / kTileK) * size_t(I / kTileRows);  // packets per expert per half
-    if (l1_bytes) *l1_bytes = size_t(E) * per_tile_k * 2 * kPacketBytes;
-    if (l2_bytes) *l2_bytes = size_t(E) * per_tile_k * kPacketBytes;
+    // L1: (I/128 gate/up tile pairs) x (H/128 K tiles) x 2 packets per expert;
+    // L2: (H/128 tiles rounded up to pairs) x (I/128 K tiles) packets per expert
+    const size_t l1_packets = size_t(I / kTileRows) * size_t(H / kTileK) * 2;
+    const size_t l2_packets = size_t((H / kTileRows + 1) / 2) * size_t(I / kTileK) * 2;
+    if (l1_bytes) *l1_bytes = size_t(E) * l1_packets * kPacketBytes;
+    if (l2_bytes) *l2_bytes = size_t(E) * l2_packets * kPacketBytes;
     return MOE_OK;
 }
 
@@ -269,8 +272,8 @@ moe_status_t moe_transform_weights(const void *l1, const void *l1_sf, const void
     const moe_status_t d = use_device_of(l1_t);
     if (d != MOE_OK) return d;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_transform(l1, l1_sf, E, 2 * I, H, I / kTileRows, 2, I, l1_t, st);
-    if (e == cudaSuccess) e = launch_transform(l2, l2_sf, E, H, I, H / kTileRows, 1, 0, l2_t, st);
+    cudaError_t e = launch_transform(l1, l1_sf, E, 2 * I, H, I / kTileRows, false, I, l1_t, st);
+    if (e == cudaSuccess) e = launch_transform(l2, l2_sf, E, H, I, (H / kTileRows + 1) / 2, true, 0, l2_t, st);
     return cuda_status(e);
 }
 

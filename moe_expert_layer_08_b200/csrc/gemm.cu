@@ -64,9 +64,9 @@ struct GemmCfg {
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
     static constexpr int kThreads = 256;  // producers (2), issuers (2), epilogue (4)
-    // weight packets one TMA box moves: GEMM1's gate and up packets of
-    // consecutive K tiles are adjacent, GEMM2's two tiles are not
-    static constexpr int kBoxPackets = kGemm1 ? kNumA * kKB : kKB;
+    // weight packets one TMA box moves: an item's two tiles are adjacent for
+    // every K tile (gate/up for GEMM1, a tile pair for GEMM2)
+    static constexpr int kBoxPackets = kNumA * kKB;
     static_assert(kTmemUsed <= 512, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kBTile % 1024 == 0, "swizzle atoms");
@@ -74,11 +74,8 @@ struct GemmCfg {
 };
 
 // Shared-memory slot of weight tile a (0, 1) of K block b within a stage:
-// the order in which the TMA boxes land.
-template <bool kGemm1, int kKB>
-__device__ __forceinline__ int a_slot(int a, int b) {
-    return kGemm1 ? b * 2 + a : a * kKB + b;
-}
+// the order in which the packets land (K tile major, tile minor).
+__device__ __forceinline__ int a_slot(int a, int b) { return b * 2 + a; }
 
 struct GemmArgs {
     const uint8_t *w_packets;  // transformed weights (for the scale blocks)
@@ -194,8 +191,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                 const int nbox = (ch.z + kActBoxRows - 1) / kActBoxRows;
                 // GEMM1: gate/up packets of tile `it`, interleaved per K tile;
                 // GEMM2: tiles 2*it and 2*it+1 (the second may not exist)
-                const int t0 = kGemm1 ? it : 2 * it;
-                const int n_valid = kGemm1 ? 2 : (t0 + 1 < n_tiles ? 2 : 1);
+                // packet group of the item: gate/up pair `it` (GEMM1) or tile pair `it` (GEMM2)
+                const int groups = kGemm1 ? n_tiles : n_items;
                 for (int step = 0; step < n_steps; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
@@ -207,20 +204,11 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     uint8_t *sf = sfs + stage * C::kStageSf;
                     if (weights) {
                         // a box always moves kBoxPackets packets (a last odd K
-                        // block loads a packet it then ignores)
-                        mbar_arrive_expect_tx(&full[stage], uint32_t(n_valid * kKB * (kPacketBody + kPacketSf)));
-                        if (kGemm1) {
-                            const int pkt = int((int64_t(ch.x) * n_tiles + t0) * KB * 2 + int64_t(kb0) * 2);
-                            tma_load_3d(st, &tmap_w, &full[stage], 0, 0, pkt, pol);
-                            tma_load_2d(sf, &tmap_wsf, &full[stage], kPacketBody / 4, pkt, pol);
-                        } else {
-                            for (int a = 0; a < n_valid; ++a) {
-                                const int pkt = int((int64_t(ch.x) * n_tiles + t0 + a) * KB + kb0);
-                                tma_load_3d(st + a * kKB * C::kATile, &tmap_w, &full[stage], 0, 0, pkt, pol);
-                                tma_load_2d(sf + a * kKB * kSfBlockBytes, &tmap_wsf, &full[stage], kPacketBody / 4, pkt,
-                                            pol);
-                            }
-                        }
+                        // block loads packets it then ignores)
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(kNumA * kKB * (kPacketBody + kPacketSf)));
+                        const int pkt = int((int64_t(ch.x) * groups + it) * KB * 2 + int64_t(kb0) * 2);
+                        tma_load_3d(st, &tmap_w, &full[stage], 0, 0, pkt, pol);
+                        tma_load_2d(sf, &tmap_wsf, &full[stage], kPacketBody / 4, pkt, pol);
                     } else {
                         // the activation box always moves kKB K blocks (a K
                         // block past the end reads zeros); a nearly full large
@@ -293,7 +281,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         uint32_t col =
                             tmem + uint32_t(kBufs * C::kAccCols + (stage * kIssuers + a) * C::kSfColsIssuer);
                         for (int b = 0; b < nkb; ++b) {
-                            const int slot = a_slot<kGemm1, kKB>(a, b);
+                            const int slot = a_slot(a, b);
                             // scale images of this K block into TMEM: weight tile, then activations
                             tc_cp_sf(col, smem_desc_sf(smem_u32(sfa + slot * kSfBlockBytes)));
                             const uint32_t sfb_col = col + 4;

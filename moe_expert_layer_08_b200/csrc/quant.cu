@@ -73,41 +73,52 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, void *q, 
 
 // One 128-thread block per packet (grid-stride): thread r copies the 64 bytes
 // of row r of the tile and writes that row's 4 scale bytes into the packet's
-// 512-byte scale block.  Packet p = ((e * tiles + tile) * KB + kb) * halves + half
-// holds source rows half * half_rows + tile * 128 + [0, 128) of expert e,
-// K columns kb * 128 + [0, 128).
+// 512-byte scale block.  Packet p = ((e * groups + grp) * KB + kb) * 2 + slot
+// holds K columns kb * 128 + [0, 128) of source rows
+//   L1 (halves):  slot * half_rows + grp * 128 + [0, 128)   (slot 0 gate, 1 up)
+//   L2 (pairs):   (2 * grp + slot) * 128 + [0, 128)         (two adjacent tiles)
+// so the two tiles one GEMM item multiplies are adjacent for every K tile.  A
+// pair slot past the last tile (odd tile count) is zero-filled padding.
 __global__ void __launch_bounds__(128) transform_kernel(const uint8_t *__restrict__ w, const uint8_t *__restrict__ w_sf,
-                                                        int rows_per_expert, int K, int tiles, int halves,
+                                                        int rows_per_expert, int K, int groups, bool pairs,
                                                         int half_rows, int64_t num_packets, uint8_t *__restrict__ out) {
     const int KB = K / kTileK;
     const int r = threadIdx.x;
     for (int64_t p = blockIdx.x; p < num_packets; p += gridDim.x) {
         int64_t q = p;
-        const int half = int(q % halves);
-        q /= halves;
+        const int slot = int(q % 2);
+        q /= 2;
         const int kb = int(q % KB);
         q /= KB;
-        const int tile = int(q % tiles);
-        const int64_t e = q / tiles;
-        const int64_t src_row = e * rows_per_expert + int64_t(half) * half_rows + int64_t(tile) * kTileRows + r;
-        const uint4 *src = reinterpret_cast<const uint4 *>(w + src_row * (K / 2) + kb * (kTileK / 2));
+        const int grp = int(q % groups);
+        const int64_t e = q / groups;
+        const int64_t row_in_expert =
+            pairs ? int64_t(2 * grp + slot) * kTileRows + r : int64_t(slot) * half_rows + int64_t(grp) * kTileRows + r;
         uint8_t *pkt = out + p * kPacketBytes;
         uint4 *dst = reinterpret_cast<uint4 *>(pkt + r * (kTileK / 2));
+        uint32_t *dsf = reinterpret_cast<uint32_t *>(pkt + kPacketBody + sf_block_offset(r, 0));
+        if (row_in_expert >= rows_per_expert) {  // padding slot
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+            *dsf = 0;
+            continue;
+        }
+        const int64_t src_row = e * rows_per_expert + row_in_expert;
+        const uint4 *src = reinterpret_cast<const uint4 *>(w + src_row * (K / 2) + kb * (kTileK / 2));
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
-        const uint32_t s = __ldg(reinterpret_cast<const uint32_t *>(w_sf + src_row * (K / 32) + kb * 4));
-        *reinterpret_cast<uint32_t *>(pkt + kPacketBody + sf_block_offset(r, 0)) = s;
+        *dsf = __ldg(reinterpret_cast<const uint32_t *>(w_sf + src_row * (K / 32) + kb * 4));
     }
 }
 
-cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int tiles,
-                             int halves, int half_rows, void *out, cudaStream_t stream) {
-    const int64_t num_packets = int64_t(E) * tiles * (K / kTileK) * halves;
+cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int groups,
+                             bool pairs, int half_rows, void *out, cudaStream_t stream) {
+    const int64_t num_packets = int64_t(E) * groups * (K / kTileK) * 2;
     if (num_packets == 0) return cudaSuccess;
     const int64_t grid = num_packets < 65536 ? num_packets : 65536;
     transform_kernel<<<unsigned(grid), 128, 0, stream>>>(static_cast<const uint8_t *>(w),
                                                          static_cast<const uint8_t *>(w_sf), rows_per_expert, K,
-                                                         tiles, halves, half_rows, num_packets,
+                                                         groups, pairs, half_rows, num_packets,
                                                          static_cast<uint8_t *>(out));
     return cudaGetLastError();
 }

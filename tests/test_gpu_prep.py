@@ -54,32 +54,38 @@ def test_quantize_fp4_matches_oracle(moe, rows, cols):
 
 
 def untransform(l1_t, l2_t, E, H, I):
-    """Host inverse of the packet layout: 128x128 tiles, 64 B rows, 512 scale
-    bytes after each body, lane r%32 word r/32 holding row r's 4 scale bytes."""
+    """Host inverse of the packet layout: packets of a 128x128 tile (64-byte
+    rows) followed by 512 scale bytes (lane r%32, word r//32 holds row r's 4
+    scale bytes).  L1: expert -> I-tile -> K tile -> (gate, up); L2: expert ->
+    H-tile pair -> K tile -> (tile 2p, tile 2p+1), padded to an even count."""
     P = 8704
 
-    def unpack(buf, rows_per_expert, K, tiles, halves, half_rows):
+    def unpack(buf, rows_per_expert, K, groups, row_of):
         KB = K // 128
-        pk = buf.reshape(E, tiles, KB, halves, P)
+        pk = buf.reshape(E, groups, KB, 2, P)
         w = np.zeros((E, rows_per_expert, K // 2), np.uint8)
         s = np.zeros((E, rows_per_expert, K // 32), np.uint8)
-        body = pk[..., :8192].reshape(E, tiles, KB, halves, 128, 64)
-        sfb = pk[..., 8192:].reshape(E, tiles, KB, halves, 32, 4, 4)  # lane, word, byte
-        for h in range(halves):
-            for t in range(tiles):
-                rows = slice(h * half_rows + t * 128, h * half_rows + t * 128 + 128)
-                w[:, rows, :] = body[:, t, :, h].transpose(0, 2, 1, 3).reshape(E, 128, K // 2)
+        body = pk[..., :8192].reshape(E, groups, KB, 2, 128, 64)
+        sfb = pk[..., 8192:].reshape(E, groups, KB, 2, 32, 4, 4)  # lane, word, byte
+        for g in range(groups):
+            for slot in range(2):
+                r0 = row_of(g, slot)
+                if r0 >= rows_per_expert:
+                    assert not body[:, g, :, slot].any() and not sfb[:, g, :, slot].any()  # zero padding
+                    continue
+                rows = slice(r0, r0 + 128)
+                w[:, rows, :] = body[:, g, :, slot].transpose(0, 2, 1, 3).reshape(E, 128, K // 2)
                 for kb in range(KB):
-                    v = sfb[:, t, kb, h]  # [E, lane, word, byte]
+                    v = sfb[:, g, kb, slot]  # [E, lane, word, byte]
                     s[:, rows, kb * 4:kb * 4 + 4] = v.transpose(0, 2, 1, 3).reshape(E, 128, 4)
         return w, s
 
-    w1, s1 = unpack(l1_t, 2 * I, H, I // 128, 2, I)
-    w2, s2 = unpack(l2_t, H, I, H // 128, 1, 0)
+    w1, s1 = unpack(l1_t, 2 * I, H, I // 128, lambda g, slot: slot * I + g * 128)
+    w2, s2 = unpack(l2_t, H, I, (H // 128 + 1) // 2, lambda g, slot: (2 * g + slot) * 128)
     return w1, s1, w2, s2
 
 
-@pytest.mark.parametrize("E,H,I", [(1, 128, 128), (3, 256, 384), (2, 512, 256)])
+@pytest.mark.parametrize("E,H,I", [(1, 128, 128), (3, 256, 384), (2, 512, 256), (2, 384, 128)])
 def test_transform_round_trip(moe, E, H, I):
     g = torch.Generator().manual_seed(E + H + I)
     l1 = torch.randint(0, 256, (E, 2 * I, H // 2), generator=g, dtype=torch.uint8)
