@@ -63,7 +63,8 @@ struct GemmCfg {
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
-    static constexpr int kThreads = 256;  // producers (2), issuers (2), epilogue (4)
+    static constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, alternating 32-token column blocks
+    static constexpr int kThreads = 32 * (4 + kEpiWarps);  // producers (2), issuers (2), epilogue
     // weight packets one TMA box moves: an item's two tiles are adjacent for
     // every K tile (gate/up for GEMM1, a tile pair for GEMM2)
     static constexpr int kBoxPackets = kNumA * kKB;
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tmem_full[b], kIssuers);
-            mbar_init(&tmem_empty[b], 4);
+            mbar_init(&tmem_empty[b], C::kEpiWarps);
         }
         for (int i = 0; i < 2; ++i) mbar_init(&mma_done[i], 1);
         *abort_flag = 0;
@@ -317,9 +318,10 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp >= 2 && warp <= 5) {
+    } else if ((warp >= 2 && warp <= 5) || warp >= 8) {
         // ---------------------------------------------------------------- epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int half = warp >= 8 ? 1 : 0;     // which column blocks of the quarter it handles
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int li = 0;
         for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
@@ -331,7 +333,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
             tc_fence_after();
             const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
             const int ncb = (ch.z + 31) / 32;
-            for (int cb = 0; cb < ncb; ++cb) {
+            for (int cb = half; cb < ncb; cb += 2) {
                 if constexpr (kGemm1) {
                     uint32_t g[32], u[32];
                     tmem_ld_32x32(acc + uint32_t(cb * 32), g);
