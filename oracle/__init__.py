@@ -75,6 +75,12 @@ def _declare(lib):
     lib.oracle_route.argtypes = [P, c.c_int, c.c_int, c.c_int, P, P, P, P]
     lib.oracle_num_threads.restype = c.c_int
     lib.oracle_num_threads.argtypes = [c.c_int]
+    lib.oracle_moe_forward_act.restype = c.c_int
+    lib.oracle_moe_forward_act.argtypes = [P, P, P, P, P, P, P, P,
+                                           c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
+                                           P, c.c_int, c.c_int, c.c_int,
+                                           c.c_int, c.c_double, c.c_double,
+                                           P, P, P, P, P, P]
     lib.oracle_moe_forward.restype = c.c_int
     lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, P, P,
                                        c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
@@ -180,14 +186,17 @@ def route(topk_idx, E: int, lib=None):
 # ---------------------------------------------------------------- layer
 def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: int,
             tokens=None, precision: str = "fp32", threads: int = 0,
-            intermediates: bool = False, lib=None):
+            intermediates: bool = False, activation: str = "swiglu", beta: float = 1.0,
+            linear_beta=None, lib=None):
     """Evaluate the layer for the listed tokens (all when ``tokens`` is None).
 
     ``experts`` maps expert id -> (l1 [2I, H/2] u8, l1_sf [2I, H/32] u8,
     l2 [H, I/2] u8, l2_sf [H, I/32] u8); every expert a listed token uses must
     be present.  Returns dict with ``out_bf16`` (uint16 bits, [ntok, H]) and
-    ``out_f32``; with ``intermediates`` also ``h_pre`` [ntok, k, I] (SwiGLU
-    before requantisation), ``h_q``, ``h_sf`` and ``y`` [ntok, k, H].
+    ``out_f32``; with ``intermediates`` also ``h_pre`` [ntok, k, I] (the
+    activation before requantisation), ``h_q``, ``h_sf`` and ``y`` [ntok, k, H].
+    ``activation``: "swiglu" or "situ" (with ``beta`` and optional
+    ``linear_beta``).
     """
     lib = lib or load()
     x_codes = _c(x_codes, np.uint8)
@@ -217,11 +226,13 @@ def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: i
     h_q = np.empty((ntok, k, I), np.uint8) if intermediates else None
     h_sf = np.empty((ntok, k, I // 32), np.uint8) if intermediates else None
     y = np.empty((ntok, k, H), np.float32) if intermediates else None
-    rc = lib.oracle_moe_forward(
+    act = {"swiglu": 0, "situ": 1}[activation]
+    rc = lib.oracle_moe_forward_act(
         _ptr(x_codes), _ptr(x_sf), _ptr(idx), _ptr(w),
         ctypes.cast(arrs[0], ctypes.c_void_p), ctypes.cast(arrs[1], ctypes.c_void_p),
         ctypes.cast(arrs[2], ctypes.c_void_p), ctypes.cast(arrs[3], ctypes.c_void_p),
         T, E, k, H, I, _ptr(tok), ntok, 1 if precision == "double" else 0, threads,
+        act, float(beta), float(linear_beta or 0.0),
         _ptr(out_bf16), _ptr(out_f32), _ptr(h_pre), _ptr(h_q), _ptr(h_sf), _ptr(y))
     if rc == -1:
         raise KeyError("a listed token routes to an expert whose weights were not given")

@@ -19,6 +19,13 @@
  * DeepGEMM PR #416 review thread (test body: gate = first chunk of L1's
  * output, activation applied to gate; per-token FP8 cast with UE8M0, gran 32).
  *
+ * SiTU (the second activation of MATE's "Mega MoE" page, section Activations;
+ * formula in the DeepGEMM PR #416 test body):
+ *     h = sigmoid(g) * (beta * tanh(g / beta)) * (beta_lin * tanh(u / beta_lin))
+ * with beta > 0 required and beta_lin optional; without beta_lin the up factor
+ * is u itself (the beta_lin -> infinity limit) -- a reading, the pages only
+ * say the coefficient is optional.
+ *
  * Readings where the pages are silent or disagree (all listed in the design
  * notes): SwiGLU is silu(gate)*up (one page writes "gate x silu(up)"; the
  * review thread's test applies the nonlinearity to the gate chunk); the top-k
@@ -268,6 +275,8 @@ typedef struct {
     const int32_t *tokens;            /* which tokens to evaluate (NULL: all) */
     int ntok;
     int use_double;                   /* 0: fp32 accumulation (the method); 1: double */
+    int activation;                   /* 0: SwiGLU, 1: SiTU */
+    double beta, linear_beta;         /* SiTU coefficients; linear_beta <= 0: absent */
     /* outputs, indexed by position p in the token list */
     uint16_t *out_bf16;               /* [ntok, H] */
     float *out_f32;                   /* [ntok, H]       (nullable) */
@@ -335,14 +344,27 @@ static void token_forward(job_t *J, int p, double *xd, double *c1, double *h,
                 c1f[n] = s;
             }
         }
-        /* SwiGLU: h[i] = silu(gate[i]) * up[i], gate = C1[i], up = C1[I+i] */
+        /* activation of gate = C1[i] and up = C1[I+i]:
+         *   SwiGLU: h = silu(gate) * up
+         *   SiTU:   h = sigmoid(gate) * (beta*tanh(gate/beta)) * (beta_lin*tanh(up/beta_lin)) */
         for (int i = 0; i < I; i++) {
             if (J->use_double) {
                 double g = c1[i], u = c1[I + i];
-                h[i] = g / (1.0 + exp(-g)) * u;
+                if (J->activation == 0) {
+                    h[i] = g / (1.0 + exp(-g)) * u;
+                } else {
+                    double up = J->linear_beta > 0 ? J->linear_beta * tanh(u / J->linear_beta) : u;
+                    h[i] = (1.0 / (1.0 + exp(-g))) * (J->beta * tanh(g / J->beta)) * up;
+                }
             } else {
                 float g = c1f[i], u = c1f[I + i];
-                hf[i] = g / (1.0f + expf(-g)) * u;
+                if (J->activation == 0) {
+                    hf[i] = g / (1.0f + expf(-g)) * u;
+                } else {
+                    float bt = (float)J->beta, lb = (float)J->linear_beta;
+                    float up = lb > 0 ? lb * tanhf(u / lb) : u;
+                    hf[i] = (1.0f / (1.0f + expf(-g))) * (bt * tanhf(g / bt)) * up;
+                }
                 h[i] = (double)hf[i];
             }
         }
@@ -435,16 +457,19 @@ int oracle_num_threads(int requested)
  * listed token uses must be present.  Returns 0, or -1 if a needed expert was
  * missing, or -2 on a bad argument.  Each token is evaluated by one thread in
  * a fixed order, so the result does not depend on the thread count. */
-int oracle_moe_forward(const uint8_t *x, const uint8_t *x_sf,
-                       const int64_t *topk_idx, const float *topk_w,
-                       const uint8_t *const *l1, const uint8_t *const *l1_sf,
-                       const uint8_t *const *l2, const uint8_t *const *l2_sf,
-                       int T, int E, int k, int H, int I,
-                       const int32_t *tokens, int ntok, int use_double, int nthreads,
-                       uint16_t *out_bf16, float *out_f32, float *h_pre,
-                       uint8_t *h_q, uint8_t *h_sf, float *y)
+int oracle_moe_forward_act(const uint8_t *x, const uint8_t *x_sf,
+                           const int64_t *topk_idx, const float *topk_w,
+                           const uint8_t *const *l1, const uint8_t *const *l1_sf,
+                           const uint8_t *const *l2, const uint8_t *const *l2_sf,
+                           int T, int E, int k, int H, int I,
+                           const int32_t *tokens, int ntok, int use_double, int nthreads,
+                           int activation, double beta, double linear_beta,
+                           uint16_t *out_bf16, float *out_f32, float *h_pre,
+                           uint8_t *h_q, uint8_t *h_sf, float *y)
 {
     if (H % 32 || I % 32 || H <= 0 || I <= 0 || k <= 0 || E <= 0 || T < 0 || ntok < 0)
+        return -2;
+    if (activation != 0 && !(activation == 1 && beta > 0 && isfinite(beta) && isfinite(linear_beta)))
         return -2;
     if (tokens)
         for (int p = 0; p < ntok; p++)
@@ -456,6 +481,7 @@ int oracle_moe_forward(const uint8_t *x, const uint8_t *x_sf,
     J.l1 = l1; J.l1_sf = l1_sf; J.l2 = l2; J.l2_sf = l2_sf;
     J.T = T; J.E = E; J.k = k; J.H = H; J.I = I;
     J.tokens = tokens; J.ntok = ntok; J.use_double = use_double;
+    J.activation = activation; J.beta = beta; J.linear_beta = linear_beta;
     J.out_bf16 = out_bf16; J.out_f32 = out_f32; J.h_pre = h_pre;
     J.h_q = h_q; J.h_sf = h_sf; J.y = y;
     for (int c = 0; c < 256; c++) {
@@ -474,4 +500,19 @@ int oracle_moe_forward(const uint8_t *x, const uint8_t *x_sf,
         pthread_join(th[i], NULL);
     free(th);
     return J.missing_expert ? -1 : 0;
+}
+
+/* The layer with SwiGLU (see oracle_moe_forward_act). */
+int oracle_moe_forward(const uint8_t *x, const uint8_t *x_sf,
+                       const int64_t *topk_idx, const float *topk_w,
+                       const uint8_t *const *l1, const uint8_t *const *l1_sf,
+                       const uint8_t *const *l2, const uint8_t *const *l2_sf,
+                       int T, int E, int k, int H, int I,
+                       const int32_t *tokens, int ntok, int use_double, int nthreads,
+                       uint16_t *out_bf16, float *out_f32, float *h_pre,
+                       uint8_t *h_q, uint8_t *h_sf, float *y)
+{
+    return oracle_moe_forward_act(x, x_sf, topk_idx, topk_w, l1, l1_sf, l2, l2_sf, T, E, k, H, I,
+                                  tokens, ntok, use_double, nthreads, 0, 1.0, 0.0,
+                                  out_bf16, out_f32, h_pre, h_q, h_sf, y);
 }

@@ -176,3 +176,47 @@ def test_missing_expert_weights_raise():
     partial = {e: ex[e] for e in list(ex)[:1]}
     with pytest.raises(KeyError):
         oracle.forward(xq, xs, idx, tw, partial, w.E, w.H, w.I)
+
+
+# ---------------------------------------------------------------- SiTU
+def situ64(g, u, beta, linear_beta):
+    """SiTU in float64: sigmoid(g) * beta*tanh(g/beta) * beta_lin*tanh(u/beta_lin)
+    (up factor u when beta_lin is absent)."""
+    up = u if linear_beta is None else linear_beta * np.tanh(u / linear_beta)
+    return 1.0 / (1.0 + np.exp(-g)) * (beta * np.tanh(g / beta)) * up
+
+
+@pytest.mark.parametrize("beta,linear_beta", [(1.25, 1.5), (0.5, None), (3.0, 0.25)])
+def test_situ_matches_float64_brute_force(beta, linear_beta):
+    w = W.custom("situ", T=6, E=4, k=2, H=64, I=64, seed=16)
+    xq, xs, idx, tw, ex = make(w)
+    r = oracle.forward(xq, xs, idx, tw, ex, w.E, w.H, w.I, intermediates=True,
+                       activation="situ", beta=beta, linear_beta=linear_beta)
+    xd = dq_e4m3(xq, xs)
+    for t in range(w.T):
+        out = np.zeros(w.H)
+        for j in range(w.k):
+            e = int(idx[t, j])
+            c1 = dq_e2m1(ex[e][0], ex[e][1]) @ xd[t]
+            h = situ64(c1[: w.I], c1[w.I:], beta, linear_beta)
+            assert np.abs(r["h_pre"][t, j] - h).max() <= 1e-5 * max(np.abs(h).max(), 1e-30)
+            y = dq_e2m1(ex[e][2], ex[e][3]) @ dq_e4m3(r["h_q"][t, j], r["h_sf"][t, j])
+            out += float(tw[t, j]) * y
+        assert np.abs(r["out_f32"][t] - out).max() <= 1e-5 * np.abs(out).max()
+
+
+def test_situ_with_large_betas_is_swiglu():
+    w = W.custom("situ_lim", T=5, E=3, k=2, H=64, I=96, seed=17)
+    xq, xs, idx, tw, ex = make(w)
+    a = oracle.forward(xq, xs, idx, tw, ex, w.E, w.H, w.I, intermediates=True, precision="double",
+                       activation="situ", beta=1e9, linear_beta=1e9)
+    b = oracle.forward(xq, xs, idx, tw, ex, w.E, w.H, w.I, intermediates=True, precision="double")
+    assert np.abs(a["h_pre"] - b["h_pre"]).max() <= 1e-6 * np.abs(b["h_pre"]).max()
+
+
+def test_situ_rejects_bad_coefficients():
+    w = W.custom("situ_bad", T=2, E=2, k=1, H=32, I=32, seed=18)
+    xq, xs, idx, tw, ex = make(w)
+    for beta, lb in ((0.0, 1.0), (-1.0, None), (float("inf"), None), (1.0, float("nan"))):
+        with pytest.raises(ValueError):
+            oracle.forward(xq, xs, idx, tw, ex, w.E, w.H, w.I, activation="situ", beta=beta, linear_beta=lb)
