@@ -163,6 +163,37 @@ moe_status_t moe_forward(const void *x_fp8, const void *x_sf,
                          moe_stream_t stream);
 
 /*
+ * Activation between GEMM1 and the FP8 requantisation (MATE "Mega MoE" API,
+ * section Activations: "swiglu" by default, "situ" with a required positive
+ * coefficient and an optional positive linear coefficient).
+ *   MOE_ACT_SWIGLU: h = silu(gate) * up
+ *   MOE_ACT_SITU:   h = sigmoid(gate) * beta*tanh(gate/beta)
+ *                       * linear_beta*tanh(up/linear_beta)   (formula of the
+ *                   DeepGEMM PR #416 test body); linear_beta = 0 means absent,
+ *                   and then the up factor is `up` itself.
+ */
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_SITU = 1 } moe_activation_kind_t;
+typedef struct {
+    int kind;           /* moe_activation_kind_t */
+    float beta;         /* SiTU: > 0 and finite */
+    float linear_beta;  /* SiTU: 0 (absent) or > 0 and finite */
+} moe_activation_t;
+
+/*
+ * moe_forward_act -- moe_forward with a chosen activation.  `activation` is a
+ * HOST pointer (read during the call; NULL = SwiGLU).  Everything else is as
+ * for moe_forward; an invalid kind or coefficient returns MOE_ERR_INVALID_ARG
+ * before any CUDA call.
+ */
+moe_status_t moe_forward_act(const void *x_fp8, const void *x_sf,
+                             const int64_t *topk_idx, const float *topk_w,
+                             const void *l1_t, const void *l2_t, void *out_bf16,
+                             int T, int E, int k, int H, int I,
+                             void *workspace, size_t ws_bytes,
+                             int32_t *expert_stats, void *const *stage_events,
+                             const moe_activation_t *activation, moe_stream_t stream);
+
+/*
  * moe_read_routing -- copies the routing metadata of the last moe_forward that
  * used `workspace` with these (T, E, k, H, I) into HOST arrays (test and
  * inspection hook; synchronises `stream`).  Any output may be NULL.

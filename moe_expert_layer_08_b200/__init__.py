@@ -18,7 +18,7 @@ __all__ = [
     "MoEError", "load", "status_string", "abi_version", "quantize_fp8", "quantize_fp4",
     "transformed_weight_bytes", "transform_weights", "workspace_bytes", "forward",
     "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
-    "forward_static", "STATIC_WORKSPACE_BYTES",
+    "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -32,6 +32,15 @@ STATUS = {
 
 _lib = None
 _lock = threading.Lock()
+
+
+class Activation(ctypes.Structure):
+    """moe_activation_t: kind 0 = SwiGLU, 1 = SiTU (beta, linear_beta; 0 = absent)."""
+    _fields_ = [("kind", ctypes.c_int), ("beta", ctypes.c_float), ("linear_beta", ctypes.c_float)]
+
+
+def activation(kind: str = "swiglu", beta: float = 1.0, linear_beta=None) -> Activation:
+    return Activation({"swiglu": 0, "situ": 1}[kind], float(beta), float(linear_beta or 0.0))
 
 
 class MoEError(RuntimeError):
@@ -55,6 +64,8 @@ def _declare(lib):
         "moe_read_routing": (I32, [P, I32, I32, I32, I32, I32, P, P, P, P, P]),
         "moe_check_device_error": (I32, [P, P]),
         "moe_forward_static": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, P, P]),
+        "moe_forward_act": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P,
+                                  c.POINTER(Activation), P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -165,9 +176,10 @@ def workspace_bytes(T: int, E: int, k: int, H: int, I: int) -> int:
 
 
 def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
-            out=None, workspace=None, expert_stats=None, events=None, stream=None):
+            out=None, workspace=None, expert_stats=None, events=None, stream=None, act=None):
     """One layer; returns out (bf16 [T, H]).  ``events``: optional list of
-    NUM_STAGE_EVENTS torch.cuda.Event recorded at the stage boundaries."""
+    NUM_STAGE_EVENTS torch.cuda.Event recorded at the stage boundaries.
+    ``act``: an Activation (see ``activation()``); None = SwiGLU."""
     _need(x_fp8, torch.uint8, "x_fp8", 2)
     _need(x_sf, torch.uint8, "x_sf", 2)
     _need(topk_idx, torch.int64, "topk_idx", 2)
@@ -195,10 +207,16 @@ def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
             if e.cuda_event == 0:  # torch creates events lazily, on first record
                 e.record(stream if stream is not None else torch.cuda.current_stream())
         ev = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[e.cuda_event for e in events])
-    st = load().moe_forward(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t), _ptr(l2_t),
-                            _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),
-                            _ptr(expert_stats), ev, _stream(stream))
-    _check(st, "moe_forward")
+    if act is None:
+        st = load().moe_forward(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t), _ptr(l2_t),
+                                _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),
+                                _ptr(expert_stats), ev, _stream(stream))
+        _check(st, "moe_forward")
+    else:
+        st = load().moe_forward_act(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t),
+                                    _ptr(l2_t), _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),
+                                    _ptr(expert_stats), ev, ctypes.byref(act), _stream(stream))
+        _check(st, "moe_forward_act")
     return out
 
 
@@ -258,9 +276,10 @@ class MoELayer:
         device = device or l1_t.device
         self.workspace = torch.empty(workspace_bytes(T_max, E, k, H, I), dtype=torch.uint8, device=device)
 
-    def __call__(self, x_fp8, x_sf, topk_idx, topk_w, out=None, expert_stats=None, events=None, stream=None):
+    def __call__(self, x_fp8, x_sf, topk_idx, topk_w, out=None, expert_stats=None, events=None, stream=None,
+                 act=None):
         if topk_idx.shape[0] > self.T_max:
             raise ValueError(f"T={topk_idx.shape[0]} exceeds T_max={self.T_max}")
         return forward(x_fp8, x_sf, topk_idx, topk_w, self.l1_t, self.l2_t, self.E, self.H, self.I,
                        out=out, workspace=self.workspace, expert_stats=expert_stats, events=events,
-                       stream=stream)
+                       stream=stream, act=act)

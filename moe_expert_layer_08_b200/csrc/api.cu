@@ -2,6 +2,7 @@
 // before any CUDA call, as the DeepGEMM PR #394 "Scope and fallback" section
 // asks of unsupported shapes), workspace layout, TMA descriptor encoding and
 // the launch sequence of one layer.
+#include <cmath>
 #include <mutex>
 
 #include "moe.h"
@@ -164,7 +165,8 @@ moe_status_t use_device_of(const void *p) {
 // entry points that run the layer).  The workspace's device must be current.
 moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
                        const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
-                       uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream) {
+                       uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream,
+                       const moe_activation_t &act) {
     const WsLayout L = ws_layout(T, E, k, H, I);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     size_t l1_bytes = 0, l2_bytes = 0;
@@ -198,10 +200,12 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
                          H, ws, L, expert_stats, st);
     if (e == cudaSuccess) e = record(1);
     if (e == cudaSuccess)
-        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st);
+        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st,
+                        act);
     if (e == cudaSuccess) e = record(2);
     if (e == cudaSuccess)
-        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st);
+        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st,
+                        act);
     if (e == cudaSuccess) e = record(3);
     if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
     if (e == cudaSuccess) e = record(4);
@@ -290,6 +294,24 @@ moe_status_t moe_forward(const void *x_fp8, const void *x_sf, const int64_t *top
                          const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
                          void *workspace, size_t ws_bytes, int32_t *expert_stats, void *const *stage_events,
                          moe_stream_t stream) {
+    return moe_forward_act(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, out_bf16, T, E, k, H, I, workspace, ws_bytes,
+                           expert_stats, stage_events, nullptr, stream);
+}
+
+moe_status_t moe_forward_act(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
+                             const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                             void *workspace, size_t ws_bytes, int32_t *expert_stats, void *const *stage_events,
+                             const moe_activation_t *activation, moe_stream_t stream) {
+    moe_activation_t act = {MOE_ACT_SWIGLU, 1.0f, 0.0f};
+    if (activation) {
+        act = *activation;
+        if (act.kind == MOE_ACT_SITU) {
+            if (!(act.beta > 0.0f) || !isfinite(act.beta) || !(act.linear_beta >= 0.0f) || !isfinite(act.linear_beta))
+                return MOE_ERR_INVALID_ARG;
+        } else if (act.kind != MOE_ACT_SWIGLU) {
+            return MOE_ERR_INVALID_ARG;
+        }
+    }
     moe_status_t s = check_shape(E, H, I);
     if (s != MOE_OK) return s;
     if (T < 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
@@ -306,7 +328,7 @@ moe_status_t moe_forward(const void *x_fp8, const void *x_sf, const int64_t *top
     s = use_device_of(workspace);
     if (s != MOE_OK) return s;
     return run_layer(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, out_bf16, T, E, k, H, I,
-                     static_cast<uint8_t *>(workspace), expert_stats, stage_events, stream);
+                     static_cast<uint8_t *>(workspace), expert_stats, stage_events, stream, act);
 }
 
 moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H, int I, int32_t *count,

@@ -91,6 +91,9 @@ struct GemmArgs {
     int n_items;               // items per chunk (GEMM1: I/128, GEMM2: tile pairs)
     int out_ld;                // row length of the output (I or H)
     int rows;                  // row extent of the K-block-major FP8 operands
+    int act_kind;              // GEMM1: MOE_ACT_SWIGLU or MOE_ACT_SITU
+    float beta, inv_beta;      // SiTU coefficients (inv_lbeta = 0: no linear coefficient)
+    float lbeta, inv_lbeta;
 };
 
 // After the call lane l holds max over the warp's lanes of a[l] (the input
@@ -340,16 +343,28 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
                     tmem_ld_wait();
                     float h[32], amx[32];
+                    if (args.act_kind == MOE_ACT_SWIGLU) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float gv = __uint_as_float(g[j]);
-                        const float uv = __uint_as_float(u[j]);
-                        // silu(g) * u with the fast exponential and division (within
-                        // the layer's tolerance; the division returns 0 where 1 + e^-g
-                        // overflows, the limit of silu)
-                        h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
-                        amx[j] = fabsf(h[j]);
+                        for (int j = 0; j < 32; ++j) {
+                            const float gv = __uint_as_float(g[j]);
+                            const float uv = __uint_as_float(u[j]);
+                            // silu(g) * u with the fast exponential and division (within
+                            // the layer's tolerance; the division returns 0 where 1 + e^-g
+                            // overflows, the limit of silu)
+                            h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float gv = __uint_as_float(g[j]);
+                            const float uv = __uint_as_float(u[j]);
+                            // SiTU: sigmoid(g) * beta*tanh(g/beta) * lbeta*tanh(u/lbeta)
+                            const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
+                            h[j] = __fdividef(args.beta * tanhf(gv * args.inv_beta), 1.0f + __expf(-gv)) * up;
+                        }
                     }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
                     // lane l: amax of token cb*32+l over this warp's 32 rows of h
                     const float amax = warp_transpose_max(amx, lane);
                     const int e = scale_exponent<true>(amax);
@@ -427,8 +442,14 @@ int gemm_packets_per_stage(bool gemm1, int chunk_rows) {
 
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
                         const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const uint8_t *w_packets,
-                        uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream) {
+                        uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
+                        const moe_activation_t &act) {
     GemmArgs a{};
+    a.act_kind = act.kind;
+    a.beta = act.beta;
+    a.inv_beta = act.kind == MOE_ACT_SITU ? 1.0f / act.beta : 0.0f;
+    a.lbeta = act.linear_beta;
+    a.inv_lbeta = (act.kind == MOE_ACT_SITU && act.linear_beta > 0.0f) ? 1.0f / act.linear_beta : 0.0f;
     a.w_packets = w_packets;
     a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
     a.hdr = reinterpret_cast<int *>(ws);

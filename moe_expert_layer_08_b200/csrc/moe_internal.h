@@ -60,7 +60,8 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
                          int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream);
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
                         const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const uint8_t *w_packets,
-                        uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream);
+                        uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
+                        const moe_activation_t &act);
 // Weight packets one pipeline stage of that GEMM variant moves (TMA box depth).
 int gemm_packets_per_stage(bool gemm1, int chunk_rows);
 // 128-K blocks one pipeline stage moves (the activation box depth).
@@ -78,6 +79,7 @@ moe_status_t use_device_of(const void *p);
 // the current device.
 moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
                        const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
-                       uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream);
+                       uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream,
+                       const moe_activation_t &act);
 
 }  // namespace moe

@@ -105,3 +105,16 @@ def test_static_entry_point_rejects_oversize_before_any_cuda_call(moelib):
     assert moelib.moe_forward_static(p, p, p, p, p, p, p, 4, 8, 2, 200, 256, None, None, None) == 2
     assert moelib.moe_forward_static(None, None, None, None, None, None, None, 0, 8, 2, 256, 256,
                                      None, None, None) == 0
+
+
+def test_forward_act_validates_activation_before_any_cuda_call(moelib):
+    import moe_expert_layer_08_b200 as m
+    p = ctypes.c_void_p(0x10000)
+    f = moelib.moe_forward_act
+    for kind, beta, lb in ((1, 0.0, 1.0), (1, -2.0, 0.0), (1, float("inf"), 0.0), (1, 1.0, -1.0),
+                           (1, 1.0, float("nan")), (7, 1.0, 0.0)):
+        a = m.Activation(kind, beta, lb)
+        assert f(p, p, p, p, p, p, p, 4, 8, 2, 256, 256, p, 16, None, None, ctypes.byref(a), None) == 1
+    # a valid activation passes to the next check (workspace too small)
+    a = m.activation("situ", 1.25, 1.5)
+    assert f(p, p, p, p, p, p, p, 4, 8, 2, 256, 256, p, 16, None, None, ctypes.byref(a), None) == 3

@@ -23,19 +23,24 @@ def moe(moelib):
     return m
 
 
-def run_and_compare(moe, w, routing=None, tokens=None, gen_device="cuda", check_repeat=True):
+def run_and_compare(moe, w, routing=None, tokens=None, gen_device="cuda", check_repeat=True, situ=None):
+    """situ: None (SwiGLU) or (beta, linear_beta or None)."""
     g = gpu_layer(w, routing=routing, gen_device=gen_device)
     ws = torch.empty(moe.workspace_bytes(w.T, w.E, w.k, w.H, w.I), dtype=torch.uint8, device="cuda")
-    out = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, workspace=ws)
+    act = None if situ is None else moe.activation("situ", situ[0], situ[1])
+    out = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, workspace=ws,
+                      act=act)
     status = moe.check_device_error(ws)
     idx = g["idx"].cpu().numpy()
     if check_repeat:
-        out2 = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, workspace=ws)
+        out2 = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I, workspace=ws,
+                           act=act)
         assert torch.equal(out.view(torch.int16), out2.view(torch.int16)), "not deterministic"
     tok = np.arange(w.T) if tokens is None else np.asarray(tokens)
     xq, xs, ex = oracle_side(w, g["x"], g["idx"], experts_of(idx, tok, w.E), gen_device=gen_device)
+    kw = {} if situ is None else dict(activation="situ", beta=situ[0], linear_beta=situ[1])
     ref = oracle.forward(xq, xs, idx, g["tw"].cpu().numpy(), ex, w.E, w.H, w.I,
-                         tokens=None if tokens is None else tok.astype(np.int32))
+                         tokens=None if tokens is None else tok.astype(np.int32), **kw)
     worst = compare_rows(out[torch.as_tensor(tok, device="cuda")], ref["out_bf16"], w.name)
     del g, ws, out
     gc.collect()
@@ -51,6 +56,9 @@ SMALL = [
     W.custom("one_token", T=1, E=16, k=4, H=512, I=256, seed=24),
     W.custom("wide", T=33, E=3, k=2, H=1024, I=1024, seed=25),
     W.custom("zipf_small", T=512, E=32, k=4, H=256, I=256, seed=26, routing="zipf"),
+    W.custom("max_E_one_block", T=300, E=1024, k=2, H=128, I=128, seed=43),   # 1024 experts, one-block routing
+    W.custom("max_E_multi_block", T=2000, E=1024, k=2, H=128, I=128, seed=45),  # 1024 experts, block-scan routing
+    W.custom("max_I", T=20, E=2, k=2, H=256, I=8192, seed=44),                # largest intermediate size
 ]
 
 
@@ -129,3 +137,26 @@ def test_stage_events_and_stream(moe):
     assert all(t >= 0 for t in times)
     ref = moe.forward(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I)
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
+SITU_CASES = [(W.WORKLOADS[0], (1.25, 1.5)), (W.custom("situ_ragged", T=37, E=5, k=3, H=384, I=256, seed=41), (0.5, None)),
+              (W.custom("situ_multichunk", T=300, E=2, k=2, H=256, I=128, seed=42), (3.0, 0.75))]
+
+
+@pytest.mark.parametrize("w,coef", SITU_CASES, ids=lambda v: getattr(v, "name", str(v)))
+def test_layer_situ_small(moe, w, coef):
+    status, _ = run_and_compare(moe, w, situ=coef)
+    assert status == 0
+
+
+def test_layer_situ_decode_full(moe):
+    status, _ = run_and_compare(moe, W.WORKLOADS[1], situ=(1.25, 1.5))
+    assert status == 0
+
+
+def test_layer_situ_prefill_sampled(moe):
+    w = W.WORKLOADS[3]
+    idx, tw = W.gen_routing(w, "cuda")
+    tokens = sorted(set(np.random.default_rng(5).choice(w.T, 6, replace=False).tolist()) | {0, w.T - 1})
+    status, _ = run_and_compare(moe, w, routing=(idx, tw), tokens=tokens, check_repeat=False, situ=(1.25, None))
+    assert status == 0
