@@ -257,13 +257,24 @@ def run_b200(args, w, rank, world, local_rank):
 
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(device.index) as clocks:
+        # the timed region: K layer calls back to back, nothing else enqueued
+        barrier()
+        start.record(stream)
+        for i in range(args.steps):
+            step()
+        stop.record(stream)
+        barrier()
+        total_ms = start.elapsed_time(stop)
+        # per-kernel durations: the same K calls again with an event between
+        # kernels (an event breaks the programmatic overlap of consecutive
+        # kernels, so this pass is a little slower and is not the headline)
         barrier()
         start.record(stream)
         for i in range(args.steps):
             step(ev[i])
         stop.record(stream)
         barrier()
-    total_ms = start.elapsed_time(stop)
+        staged_ms = start.elapsed_time(stop) / args.steps
     stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(moe.NUM_STAGE_EVENTS - 1)] for e in ev])
     ms = max_over_ranks(total_ms / args.steps, device)
 
@@ -330,12 +341,15 @@ def run_b200(args, w, rank, world, local_rank):
         "touched_experts": touched,
         "stage_us": {"route_gather": float(stage_ms[:, 0].mean() * 1e3), "gemm1": g1_ms * 1e3,
                      "gemm2": g2_ms * 1e3, "combine": float(stage_ms[:, 3].mean() * 1e3)},
+        "stage_timing": {"how": "second pass of the same K steps with a CUDA event on the launch stream "
+                                "between kernels; the roofline's kernel duration comes from it",
+                         "us_per_layer": staged_ms * 1e3},
         "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                      "frac": achieved / pk["hbm"], "peak_source": pk["source"], "algorithmic_bytes": kbytes,
                      "traffic": traffic},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": args.steps * moe.forward_kernel_launches(w.T, w.E, w.k, w.H, w.I),
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:

@@ -127,6 +127,19 @@ moe_status_t moe_transform_weights(const void *l1, const void *l1_sf,
 moe_status_t moe_workspace_bytes(int T_max, int E, int k, int H, int I, size_t *bytes);
 
 /*
+ * moe_forward_kernel_launches -- how many kernels one moe_forward or
+ * moe_forward_act call with these sizes enqueues (host-only; no counterpart on
+ * the pages: it lets a caller that counts launches, such as a benchmark or a
+ * graph builder, know the layer's launch structure).  Routing takes two
+ * kernels when T * k <= 1024 (one block does histogram, scan and placement,
+ * then the gather) and five otherwise (histogram, per-expert scan, metadata,
+ * placement, gather); GEMM1, GEMM2 and the combine add three.  T = 0 enqueues
+ * nothing.  Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE for sizes
+ * moe_forward would reject.
+ */
+moe_status_t moe_forward_kernel_launches(int T, int E, int k, int H, int I, int *launches);
+
+/*
  * moe_forward -- one MoE expert layer (`fp8_fp4_mega_moe(y, l1, l2, buffer)`;
  * the five phases of "Mega moe fusion with symmetric memory", Procedure step 5,
  * on one GPU).

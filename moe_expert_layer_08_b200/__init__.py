@@ -18,7 +18,7 @@ __all__ = [
     "MoEError", "load", "status_string", "abi_version", "quantize_fp8", "quantize_fp4",
     "transformed_weight_bytes", "transform_weights", "workspace_bytes", "forward",
     "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
-    "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation",
+    "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -60,6 +60,7 @@ def _declare(lib):
         "moe_transformed_weight_bytes": (I32, [I32, I32, I32, c.POINTER(SZ), c.POINTER(SZ)]),
         "moe_transform_weights": (I32, [P, P, P, P, I32, I32, I32, P, P, P]),
         "moe_workspace_bytes": (I32, [I32, I32, I32, I32, I32, c.POINTER(SZ)]),
+        "moe_forward_kernel_launches": (I32, [I32, I32, I32, I32, I32, c.POINTER(I32)]),
         "moe_forward": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P]),
         "moe_read_routing": (I32, [P, I32, I32, I32, I32, I32, P, P, P, P, P]),
         "moe_check_device_error": (I32, [P, P]),
@@ -172,6 +173,13 @@ def transform_weights(l1, l1_sf, l2, l2_sf, out=None, stream=None):
 def workspace_bytes(T: int, E: int, k: int, H: int, I: int) -> int:
     n = ctypes.c_size_t()
     _check(load().moe_workspace_bytes(T, E, k, H, I, ctypes.byref(n)), "moe_workspace_bytes")
+    return n.value
+
+
+def forward_kernel_launches(T: int, E: int, k: int, H: int, I: int) -> int:
+    """Kernels one forward call with these sizes enqueues (host-only)."""
+    n = ctypes.c_int()
+    _check(load().moe_forward_kernel_launches(T, E, k, H, I, ctypes.byref(n)), "moe_forward_kernel_launches")
     return n.value
 
 

@@ -290,6 +290,15 @@ moe_status_t moe_workspace_bytes(int T_max, int E, int k, int H, int I, size_t *
     return MOE_OK;
 }
 
+moe_status_t moe_forward_kernel_launches(int T, int E, int k, int H, int I, int *launches) {
+    const moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    if (T < 0 || k <= 0 || k > E || !launches) return MOE_ERR_INVALID_ARG;
+    if (int64_t(T) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+    *launches = T == 0 ? 0 : route_kernel_launches(T * k) + 3;
+    return MOE_OK;
+}
+
 moe_status_t moe_forward(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
                          const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
                          void *workspace, size_t ws_bytes, int32_t *expert_stats, void *const *stage_events,

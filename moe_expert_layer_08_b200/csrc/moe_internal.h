@@ -56,6 +56,10 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, void *q, 
                             cudaStream_t stream);
 cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int groups,
                              bool pairs, int half_rows, void *out, cudaStream_t stream);
+// kernels launch_route enqueues for R = T * k routed rows (one-block routing
+// up to kRouteSmallMax rows, then the gather; else four routing kernels and
+// the gather)
+inline int route_kernel_launches(int64_t R) { return R <= kRouteSmallMax ? 2 : 5; }
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
                          int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream);
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,

@@ -50,6 +50,21 @@ def test_sizes_are_host_only_and_consistent(moelib):
     assert m.workspace_bytes(0, 8, 2, 256, 256) > 0
 
 
+def test_forward_kernel_launches(moelib):
+    """One-block routing up to T*k = 1024 routed rows (2 kernels), block-scan
+    routing above (5), plus GEMM1, GEMM2 and the combine; nothing for T = 0."""
+    import moe_expert_layer_08_b200 as m
+    assert m.forward_kernel_launches(8, 384, 6, 7168, 3072) == 5
+    assert m.forward_kernel_launches(170, 384, 6, 7168, 3072) == 5     # 1020 rows
+    assert m.forward_kernel_launches(171, 384, 6, 7168, 3072) == 8     # 1026 rows
+    assert m.forward_kernel_launches(8192, 384, 6, 7168, 3072) == 8
+    assert m.forward_kernel_launches(0, 8, 2, 256, 256) == 0
+    with pytest.raises(m.MoEError):
+        m.forward_kernel_launches(4, 8, 9, 256, 256)                   # k > E
+    with pytest.raises(m.MoEError):
+        m.forward_kernel_launches(4, 8, 2, 200, 256)                   # H % 128
+
+
 @pytest.mark.parametrize("E,H,I,status", [(8, 200, 256, 2), (8, 256, 200, 2), (8, 256, 8320, 2),
                                           (2000, 256, 256, 2), (0, 256, 256, 1)])
 def test_bad_shapes_fail_closed(moelib, E, H, I, status):
