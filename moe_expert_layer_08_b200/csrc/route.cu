@@ -242,31 +242,50 @@ __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
     rowinfo[pos] = make_int4(int(s / k), __ldcg(chunk_base + e) + local / chunk_rows, local % chunk_rows, 0);
 }
 
-// ------------------------------------------------------------------ gather
-// One 128-thread block per (routed row, 2048-byte segment of the row); the
-// first segment's block also moves the row's scale words.
-constexpr int kGatherSeg = 2048;
+// gather_kernel: one warp per routed row (grid-stride over the rows).  The
+// row's H bytes move in batches of 32 lanes x kGatherVec 16-byte vectors, all
+// loads of a batch issued before its stores; each vector goes to its K block's
+// plane of the K-block-major destination [H/128][Rp][128] (8 lanes fill one
+// 128-byte line).  The lanes then copy the row's scale words into the chunk's
+// scale images.
+constexpr int kGatherThreads = 256;
+constexpr int kGatherVec = 8;
 
-__global__ void __launch_bounds__(128) gather_kernel(const int4 *__restrict__ rowinfo, const int *__restrict__ offset,
-                                                     int E, int H, int64_t R, int segs, int sf_bytes,
-                                                     const uint8_t *__restrict__ x,
-                                                     const uint8_t *__restrict__ x_sf, uint8_t *__restrict__ xg,
-                                                     uint8_t *__restrict__ xg_sf) {
+__global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__restrict__ rowinfo,
+                                                                const int *__restrict__ offset, int E, int H,
+                                                                int64_t Rp, int sf_bytes,
+                                                                const uint8_t *__restrict__ x,
+                                                                const uint8_t *__restrict__ x_sf,
+                                                                uint8_t *__restrict__ xg, uint8_t *__restrict__ xg_sf) {
     pdl_wait();
     pdl_trigger();
-    const int64_t pos = blockIdx.x / segs;
-    const int seg = blockIdx.x % segs;
-    if (pos >= __ldcg(offset + E)) return;  // dropped slots leave no row
-    const int4 ri = __ldcg(rowinfo + pos);
-    const int col = seg * kGatherSeg + threadIdx.x * 16;
-    // K-block-major destination [H/128][Rp][128]
-    if (col < H)
-        *reinterpret_cast<uint4 *>(xg + ((col / kTileK) * R + pos) * kTileK + col % kTileK) =
-            __ldcg(reinterpret_cast<const uint4 *>(x + int64_t(ri.x) * H + col));
-    if (seg == 0) {
-        const int KB = H / kTileK;
+    constexpr int kWarps = kGatherThreads / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = int64_t(gridDim.x) * kWarps;
+    const int64_t nrows = __ldcg(offset + E);  // dropped slots leave no row
+    const int nvec = H / 16;
+    const int KB = H / kTileK;
+    for (int64_t pos = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); pos < nrows; pos += nwarps) {
+        const int4 ri = __ldcg(rowinfo + pos);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + int64_t(ri.x) * H);
+        for (int base = 0; base < nvec; base += 32 * kGatherVec) {
+            uint4 v[kGatherVec];
+#pragma unroll
+            for (int i = 0; i < kGatherVec; ++i) {
+                const int idx = base + i * 32 + lane;
+                if (idx < nvec) v[i] = __ldcg(src + idx);
+            }
+#pragma unroll
+            for (int i = 0; i < kGatherVec; ++i) {
+                const int idx = base + i * 32 + lane;
+                if (idx < nvec) {
+                    const int col = idx * 16;
+                    *reinterpret_cast<uint4 *>(xg + (int64_t(col / kTileK) * Rp + pos) * kTileK + col % kTileK) = v[i];
+                }
+            }
+        }
         const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * (H / 32));
-        for (int kb = threadIdx.x; kb < KB; kb += 128) {
+        for (int kb = lane; kb < KB; kb += 32) {
             uint8_t *blk = xg_sf + (int64_t(ri.y) * KB + kb) * sf_bytes;
             *reinterpret_cast<uint32_t *>(blk + act_sf_offset(ri.z, 0)) = __ldcg(sfs + kb);
         }
@@ -317,10 +336,15 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
                            lrank, offset, chunk_base, perm, inv, rowinfo);
     }
     if (e != cudaSuccess) return e;
-    const int segs = (H + kGatherSeg - 1) / kGatherSeg;
-    return launch_pdl(gather_kernel, dim3(unsigned(int64_t(R) * segs)), dim3(128), 0, stream,
-                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, L.Rp, segs, act_sf_bytes(L.chunk_rows), x, x_sf,
-                      ws + L.off_xg, ws + L.off_xg_sf);
+    // up to 4 blocks per SM; the kernel strides over the rows that routing kept
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (int64_t(R) + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+    const int grid = int(want < int64_t(sms) * 4 ? want : int64_t(sms) * 4);
+    return launch_pdl(gather_kernel, dim3(unsigned(grid)), dim3(kGatherThreads), 0, stream,
+                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, int64_t(L.Rp),
+                      act_sf_bytes(L.chunk_rows), x, x_sf, ws + L.off_xg, ws + L.off_xg_sf);
 }
 
 }  // namespace moe
