@@ -54,7 +54,13 @@ struct GemmCfg {
     static constexpr int kSmemTiles = kStages * kStageTiles;
     static constexpr int kSmemSf = kStages * kStageSf;
     static constexpr int kSmemMisc = 256;
-    static constexpr int kSmemBytes = 1024 + kSmemTiles + kSmemSf + kSmemMisc;
+    // GEMM2 with large chunks: each epilogue warp stages 1 KB of bf16 output in
+    // shared memory and writes whole row pieces with 16-byte stores instead of
+    // 32 two-byte stores per row block (no room with 32-row chunks)
+    static constexpr int kEpiWarpsC = 8;
+    static constexpr bool kStaged = !kSmall && !kGemm1;
+    static constexpr int kEpiStage = kStaged ? kEpiWarpsC * 1024 : 0;
+    static constexpr int kSmemBytes = 1024 + kSmemTiles + kSmemSf + kSmemMisc + kEpiStage;
     static constexpr int kAccCols = kNumA * kN;          // one accumulator buffer
     // per issuer and stage: its weight tile's and the activations' scale images
     static constexpr int kSfColsIssuer = kKB * (1 + kSfbImages) * 4;
@@ -63,7 +69,7 @@ struct GemmCfg {
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
-    static constexpr int kEpiWarps = 8;  // two per TMEM lane quarter, alternating 32-token column blocks
+    static constexpr int kEpiWarps = kEpiWarpsC;  // two per TMEM lane quarter, alternating 32-token column blocks
     static constexpr int kThreads = 32 * (4 + kEpiWarps);  // producers (2), issuers (2), epilogue
     // weight packets one TMA box moves: an item's two tiles are adjacent for
     // every K tile (gate/up for GEMM1, a tile pair for GEMM2)
@@ -132,6 +138,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
     uint64_t *mma_done = tmem_empty + 2;     // [kIssuers]
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    uint8_t *epi_stage = reinterpret_cast<uint8_t *>(full) + C::kSmemMisc;  // [kEpiWarps][1024] (large chunks)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -325,6 +332,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int half = warp >= 8 ? 1 : 0;     // which column blocks of the quarter it handles
+        uint8_t *my_stage = epi_stage + (warp < 8 ? warp - 2 : warp - 4) * 1024;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int li = 0;
         for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
@@ -373,14 +381,15 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     if (tok < ch.z)
                         args.out_sf[(int64_t(c) * n_tiles + it) * C::kActSf + act_sf_offset(tok, q)] =
                             uint8_t(e + 127);
+                    // K-block-major [I/128][rows][128]: this warp's 32 codes of a row are
+                    // bytes q*32 .. q*32+31 of row (ch.y + token) in K block `it`
+                    uint8_t *qbase = args.out_q + (int64_t(it) * args.rows + ch.y) * kTileK + q * 32;
+                    // one store per token: the warp's 32 lanes write 32 contiguous bytes
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float mj = __shfl_sync(0xFFFFFFFFu, mult, j);
                         const uint32_t code = to_e4m3(h[j] * mj);
-                        // K-block-major [I/128][rows][128]: GEMM2 reads two K blocks per box
-                        if (cb * 32 + j < ch.z)
-                            args.out_q[(int64_t(it) * args.rows + ch.y + cb * 32 + j) * kTileK + q * 32 + lane] =
-                                uint8_t(code);
+                        if (cb * 32 + j < ch.z) qbase[int64_t(cb * 32 + j) * kTileK + lane] = uint8_t(code);
                     }
                 } else {
 #pragma unroll
@@ -390,12 +399,33 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         uint32_t g[32];
                         tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), g);
                         tmem_ld_wait();
-                        const int col_out = tile * kTileRows + q * 32 + lane;  // this thread's output column
+                        __nv_bfloat16 *ybase = args.out_y + int64_t(ch.y + cb * 32) * args.out_ld + tile * kTileRows + q * 32;
+                        if constexpr (C::kStaged) {
+                            // two passes of 16 rows: stage [row][32 columns] bf16 (1 KB), then
+                            // 16-byte stores, four lanes per 64-byte row piece
+                            __nv_bfloat16 *sb = reinterpret_cast<__nv_bfloat16 *>(my_stage);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (cb * 32 + j < ch.z)
-                                args.out_y[int64_t(ch.y + cb * 32 + j) * args.out_ld + col_out] =
-                                    __float2bfloat16_rn(__uint_as_float(g[j]));
+                            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    sb[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[hh * 16 + j]));
+                                __syncwarp();
+#pragma unroll
+                                for (int i = 0; i < 2; ++i) {
+                                    const int cidx = i * 32 + lane;  // row hh*16 + cidx / 4, columns (cidx % 4) * 8 ..
+                                    const int r = hh * 16 + (cidx >> 2);
+                                    if (cb * 32 + r < ch.z)
+                                        *reinterpret_cast<uint4 *>(ybase + int64_t(r) * args.out_ld + (cidx & 3) * 8) =
+                                            *reinterpret_cast<const uint4 *>(my_stage + cidx * 16);
+                                }
+                                __syncwarp();
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (cb * 32 + j < ch.z)
+                                    ybase[int64_t(j) * args.out_ld + lane] = __float2bfloat16_rn(__uint_as_float(g[j]));
+                        }
                     }
                 }
             }
