@@ -10,6 +10,7 @@ namespace moe {
 
 constexpr int kCombineThreads = 128;
 constexpr int kCombineCols = kCombineThreads * 8;  // 8 bf16 (16 bytes) per thread
+constexpr int kCombineBatch = 8;                   // top-k up to this many: loads issued together
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfloat16 *__restrict__ y,
                                                                   const int *__restrict__ inv,
@@ -23,16 +24,36 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfl
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        const int r = __ldcg(inv + t * k + j);
-        if (r < 0) continue;  // dropped slot
-        const float wv = __ldg(topk_w + t * k + j);
-        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col));
+    auto add = [&](const uint4 &v, float wv) {
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             acc[2 * i] += wv * __uint_as_float(u[i] << 16);
             acc[2 * i + 1] += wv * __uint_as_float(u[i] & 0xFFFF0000u);
+        }
+    };
+    if (k <= kCombineBatch) {
+        // all of the token's row indices, then all row loads in flight at once;
+        // the sum still runs over j ascending
+        int r[kCombineBatch];
+        float wv[kCombineBatch];
+        uint4 v[kCombineBatch];
+#pragma unroll
+        for (int j = 0; j < kCombineBatch; ++j) {
+            r[j] = j < k ? __ldcg(inv + t * k + j) : -1;
+            wv[j] = j < k ? __ldg(topk_w + t * k + j) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < kCombineBatch; ++j)
+            if (r[j] >= 0) v[j] = __ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r[j]) * H + col));
+#pragma unroll
+        for (int j = 0; j < kCombineBatch; ++j)
+            if (r[j] >= 0) add(v[j], wv[j]);  // r < 0: dropped slot
+    } else {
+        for (int j = 0; j < k; ++j) {
+            const int r = __ldcg(inv + t * k + j);
+            if (r < 0) continue;  // dropped slot
+            add(__ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col)), __ldg(topk_w + t * k + j));
         }
     }
     uint32_t o[4];

@@ -242,18 +242,20 @@ __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
     rowinfo[pos] = make_int4(int(s / k), __ldcg(chunk_base + e) + local / chunk_rows, local % chunk_rows, 0);
 }
 
-// gather_kernel: one warp per routed row (grid-stride over the rows).  The
-// row's H bytes move in batches of 32 lanes x kGatherVec 16-byte vectors, all
-// loads of a batch issued before its stores; each vector goes to its K block's
-// plane of the K-block-major destination [H/128][Rp][128] (8 lanes fill one
-// 128-byte line).  The lanes then copy the row's scale words into the chunk's
-// scale images.
+// gather_kernel: one warp per task, a task being `seg_vec` 16-byte vectors of
+// one routed row (the whole row for large batches; pieces of it when there are
+// few rows, so that enough warps run); warps stride over the tasks.  A task's
+// vectors move in batches of 32 lanes x kGatherVec, all loads of a batch issued
+// before its stores; each vector goes to its K block's plane of the K-block-
+// major destination [H/128][Rp][128] (8 lanes fill one 128-byte line).  The
+// first task of a row also copies the row's scale words into the chunk's scale
+// images.
 constexpr int kGatherThreads = 256;
 constexpr int kGatherVec = 8;
 
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__restrict__ rowinfo,
                                                                 const int *__restrict__ offset, int E, int H,
-                                                                int64_t Rp, int sf_bytes,
+                                                                int64_t Rp, int sf_bytes, int segs, int seg_vec,
                                                                 const uint8_t *__restrict__ x,
                                                                 const uint8_t *__restrict__ x_sf,
                                                                 uint8_t *__restrict__ xg, uint8_t *__restrict__ xg_sf) {
@@ -265,25 +267,29 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__re
     const int64_t nrows = __ldcg(offset + E);  // dropped slots leave no row
     const int nvec = H / 16;
     const int KB = H / kTileK;
-    for (int64_t pos = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); pos < nrows; pos += nwarps) {
+    for (int64_t task = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); task < nrows * segs; task += nwarps) {
+        const int64_t pos = task / segs;
+        const int seg = int(task % segs);
         const int4 ri = __ldcg(rowinfo + pos);
         const uint4 *src = reinterpret_cast<const uint4 *>(x + int64_t(ri.x) * H);
-        for (int base = 0; base < nvec; base += 32 * kGatherVec) {
+        const int vend = (seg + 1) * seg_vec < nvec ? (seg + 1) * seg_vec : nvec;
+        for (int base = seg * seg_vec; base < vend; base += 32 * kGatherVec) {
             uint4 v[kGatherVec];
 #pragma unroll
             for (int i = 0; i < kGatherVec; ++i) {
                 const int idx = base + i * 32 + lane;
-                if (idx < nvec) v[i] = __ldcg(src + idx);
+                if (idx < vend) v[i] = __ldcg(src + idx);
             }
 #pragma unroll
             for (int i = 0; i < kGatherVec; ++i) {
                 const int idx = base + i * 32 + lane;
-                if (idx < nvec) {
+                if (idx < vend) {
                     const int col = idx * 16;
                     *reinterpret_cast<uint4 *>(xg + (int64_t(col / kTileK) * Rp + pos) * kTileK + col % kTileK) = v[i];
                 }
             }
         }
+        if (seg != 0) continue;
         const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * (H / 32));
         for (int kb = lane; kb < KB; kb += 32) {
             uint8_t *blk = xg_sf + (int64_t(ri.y) * KB + kb) * sf_bytes;
@@ -336,15 +342,25 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
                            lrank, offset, chunk_base, perm, inv, rowinfo);
     }
     if (e != cudaSuccess) return e;
-    // up to 4 blocks per SM; the kernel strides over the rows that routing kept
+    // up to 4 blocks per SM, striding over (row, piece) tasks; rows are cut
+    // into pieces of a multiple of 32 vectors until there are about that many
+    // warps' worth of tasks
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t want = (int64_t(R) + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+    const int64_t warps = int64_t(sms) * 4 * (kGatherThreads / 32);
+    const int nvec = H / 16;
+    const int max_segs = (nvec + 31) / 32;
+    int64_t segs = (warps + R - 1) / (R > 0 ? R : 1);
+    if (segs > max_segs) segs = max_segs;
+    if (segs < 1) segs = 1;
+    const int seg_vec = int((max_segs + segs - 1) / segs) * 32;  // vectors per piece, a multiple of 32
+    const int nseg = (nvec + seg_vec - 1) / seg_vec;  // pieces per row with that size
+    const int64_t want = (int64_t(R) * nseg + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
     const int grid = int(want < int64_t(sms) * 4 ? want : int64_t(sms) * 4);
-    return launch_pdl(gather_kernel, dim3(unsigned(grid)), dim3(kGatherThreads), 0, stream,
+    return launch_pdl(gather_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kGatherThreads), 0, stream,
                       static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, int64_t(L.Rp),
-                      act_sf_bytes(L.chunk_rows), x, x_sf, ws + L.off_xg, ws + L.off_xg_sf);
+                      act_sf_bytes(L.chunk_rows), nseg, seg_vec, x, x_sf, ws + L.off_xg, ws + L.off_xg_sf);
 }
 
 }  // namespace moe

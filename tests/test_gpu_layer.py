@@ -59,6 +59,7 @@ SMALL = [
     W.custom("max_E_one_block", T=300, E=1024, k=2, H=128, I=128, seed=43),   # 1024 experts, one-block routing
     W.custom("max_E_multi_block", T=2000, E=1024, k=2, H=128, I=128, seed=45),  # 1024 experts, block-scan routing
     W.custom("max_I", T=20, E=2, k=2, H=256, I=8192, seed=44),                # largest intermediate size
+    W.custom("k10", T=40, E=12, k=10, H=256, I=128, seed=46),                 # top-k above the combine's batch of 8
 ]
 
 
