@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--experts", type=int, default=0,
                    help="override E (a smaller resident weight set for profiler captures)")
     p.add_argument("--tokens", type=int, default=0, help="override T (with --experts: same rows per expert)")
+    p.add_argument("--layout", default="packets", choices=["packets", "rowmajor"],
+                   help="weight layout: tile packets, or row-major bodies with separate scale blocks")
     return p.parse_args()
 
 
@@ -151,23 +153,39 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def build_layer(w, device):
-    """Seeded bf16 draws quantised and packed by the CUDA library, resident in HBM."""
+def build_layer(w, device, layout="packets"):
+    """Seeded bf16 draws quantised and laid out by the CUDA library, resident in
+    HBM: tile packets (l1_t, l2_t) or row-major bodies + scale blocks (rm)."""
     import moe_expert_layer_08_b200 as moe
     x = W.gen_x(w, device)
     idx, tw = W.gen_routing(w, device)
     xq, xs = moe.quantize_fp8(x)
-    n1, n2 = moe.transformed_weight_bytes(w.E, w.H, w.I)
-    l1_t = torch.empty(n1, dtype=torch.uint8, device=device)
-    l2_t = torch.empty(n2, dtype=torch.uint8, device=device)
-    p1, p2 = n1 // w.E, n2 // w.E
+    u8 = dict(dtype=torch.uint8, device=device)
+    if layout == "packets":
+        n1, n2 = moe.transformed_weight_bytes(w.E, w.H, w.I)
+        l1_t, l2_t = torch.empty(n1, **u8), torch.empty(n2, **u8)
+        p1, p2 = n1 // w.E, n2 // w.E
+    else:
+        r1, r2 = torch.empty((w.E, 2 * w.I, w.H // 2), **u8), torch.empty((w.E, w.H, w.I // 2), **u8)
+        m1, m2 = moe.transformed_scale_bytes(w.E, w.H, w.I)
+        s1, s2 = torch.empty(m1, **u8), torch.empty(m2, **u8)
+        q1, q2 = m1 // w.E, m2 // w.E
     for e in range(w.E):
         a, b = moe.quantize_fp4(W.gen_l1(w, e, device))
         c, d = moe.quantize_fp4(W.gen_l2(w, e, device))
-        moe.transform_weights(a[None], b[None], c[None], d[None],
-                              out=(l1_t[e * p1:(e + 1) * p1], l2_t[e * p2:(e + 1) * p2]))
+        if layout == "packets":
+            moe.transform_weights(a[None], b[None], c[None], d[None],
+                                  out=(l1_t[e * p1:(e + 1) * p1], l2_t[e * p2:(e + 1) * p2]))
+        else:
+            r1[e], r2[e] = a, c
+            moe.transform_scales(b[None], d[None], out=(s1[e * q1:(e + 1) * q1], s2[e * q2:(e + 1) * q2]))
     torch.cuda.synchronize()
-    return dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw, l1_t=l1_t, l2_t=l2_t)
+    g = dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw)
+    if layout == "packets":
+        g.update(l1_t=l1_t, l2_t=l2_t, rm=None)
+    else:
+        g.update(l1_t=None, l2_t=None, rm=moe.RowMajorWeights(r1, s1, r2, s2))
+    return g
 
 
 def oracle_sample(w, ntok, device):
@@ -234,8 +252,8 @@ def run_b200(args, w, rank, world, local_rank):
         torch.distributed.barrier()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    g = build_layer(w, device)
-    layer = moe.MoELayer(g["l1_t"], g["l2_t"], w.E, w.k, w.H, w.I, T_max=w.T, device=device)
+    g = build_layer(w, device, args.layout)
+    layer = moe.MoELayer(g["l1_t"], g["l2_t"], w.E, w.k, w.H, w.I, T_max=w.T, device=device, weights=g["rm"])
     out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.NUM_STAGE_EVENTS)]
@@ -345,7 +363,7 @@ def run_b200(args, w, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8xfp4 (fp32 accumulate)", "data": "synthetic",
         "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")},
-                   "parallelism": f"replicas x{world}",
+                   "parallelism": f"replicas x{world}", "weight_layout": args.layout,
                    "l2": "inputs larger than L2 (touched expert weights per step >> 126 MB)"
                    if touched * (b1 + b2) > 256e6 else "inputs fit in L2 (not flushed)"},
         "us_per_layer": ms * 1e3,

@@ -207,6 +207,64 @@ moe_status_t moe_forward_act(const void *x_fp8, const void *x_sf,
                              const moe_activation_t *activation, moe_stream_t stream);
 
 /*
+ * Weight layouts (DeepGEMM PR #394, Summary and API: the packet layout is an
+ * option of the model-load transform; "row-major" weights keep their natural
+ * layout).
+ *   MOE_LAYOUT_PACKETS   l1 / l2 are the buffers of moe_transform_weights
+ *                        (body and scales of each tile in one packet);
+ *                        l1_sf / l2_sf must be NULL.
+ *   MOE_LAYOUT_ROW_MAJOR l1 / l2 are the FP4 weights as moe_quantize_fp4 wrote
+ *                        them (l1 [E, 2I, H/2], rows 0..I-1 gate; l2 [E, H, I/2]),
+ *                        256-byte aligned, read in place; l1_sf / l2_sf are the
+ *                        scale blocks of moe_transform_scales.
+ * Both layouts feed the tensor cores the same bytes, so the layer's output is
+ * bitwise identical between them.
+ */
+typedef enum { MOE_LAYOUT_PACKETS = 0, MOE_LAYOUT_ROW_MAJOR = 1 } moe_layout_t;
+typedef struct {
+    int layout;        /* moe_layout_t */
+    const void *l1, *l1_sf;
+    const void *l2, *l2_sf;
+} moe_weights_t;
+
+/*
+ * moe_transformed_scale_bytes -- sizes of the separate scale arrays of the
+ * row-major layout (host-only): 512 bytes per 128 x 128 weight tile, in the
+ * packet order of moe_transform_weights (L1: E * (I/128) * (H/128) * 2 blocks;
+ * L2: E * ceil(H/256) * 2 * (I/128) blocks, an odd H/128 padded with zero
+ * blocks).
+ */
+moe_status_t moe_transformed_scale_bytes(int E, int H, int I, size_t *l1_sf_bytes, size_t *l2_sf_bytes);
+
+/*
+ * moe_transform_scales -- the scale half of moe_transform_weights: writes each
+ * tile's 512-byte scale block (the image tcgen05.cp copies into TMEM, byte
+ * (r % 32) * 16 + (r / 32) * 4 + g for tile row r, K group g) into l1_sf_t /
+ * l2_sf_t (256-byte aligned, sizes from moe_transformed_scale_bytes) and
+ * leaves the FP4 bodies where they are.  l1_sf [E, 2I, H/32], l2_sf [E, H,
+ * I/32] as moe_quantize_fp4 wrote them.  Same validation as
+ * moe_transform_weights.
+ */
+moe_status_t moe_transform_scales(const void *l1_sf, const void *l2_sf, int E, int H, int I,
+                                  void *l1_sf_t, void *l2_sf_t, moe_stream_t stream);
+
+/*
+ * moe_forward_weights -- moe_forward_act with the weights given by layout
+ * (`weights` is a HOST pointer read during the call).  An unknown layout, a
+ * missing or misaligned weight pointer, or l1_sf / l2_sf given with packets
+ * returns MOE_ERR_INVALID_ARG before any CUDA call.  No counterpart on the
+ * pages beyond the layout option itself: it lets one runtime serve both
+ * layouts for their A/B comparison.
+ */
+moe_status_t moe_forward_weights(const void *x_fp8, const void *x_sf,
+                                 const int64_t *topk_idx, const float *topk_w,
+                                 const moe_weights_t *weights, void *out_bf16,
+                                 int T, int E, int k, int H, int I,
+                                 void *workspace, size_t ws_bytes,
+                                 int32_t *expert_stats, void *const *stage_events,
+                                 const moe_activation_t *activation, moe_stream_t stream);
+
+/*
  * moe_read_routing -- copies the routing metadata of the last moe_forward that
  * used `workspace` with these (T, E, k, H, I) into HOST arrays (test and
  * inspection hook; synchronises `stream`).  Any output may be NULL.

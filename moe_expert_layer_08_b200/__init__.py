@@ -19,6 +19,8 @@ __all__ = [
     "transformed_weight_bytes", "transform_weights", "workspace_bytes", "forward",
     "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
     "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
+    "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
+    "LAYOUT_ROW_MAJOR",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -37,6 +39,31 @@ _lock = threading.Lock()
 class Activation(ctypes.Structure):
     """moe_activation_t: kind 0 = SwiGLU, 1 = SiTU (beta, linear_beta; 0 = absent)."""
     _fields_ = [("kind", ctypes.c_int), ("beta", ctypes.c_float), ("linear_beta", ctypes.c_float)]
+
+
+LAYOUT_PACKETS, LAYOUT_ROW_MAJOR = 0, 1
+
+
+class Weights(ctypes.Structure):
+    """moe_weights_t: a weight layout and its four pointers."""
+    _fields_ = [("layout", ctypes.c_int), ("l1", ctypes.c_void_p), ("l1_sf", ctypes.c_void_p),
+                ("l2", ctypes.c_void_p), ("l2_sf", ctypes.c_void_p)]
+
+
+class RowMajorWeights:
+    """Weights in the row-major layout: the FP4 bodies as quantize_fp4 wrote them
+    (l1 [E, 2I, H/2], l2 [E, H, I/2], u8) and the scale blocks of
+    transform_scales (1-D u8).  Holds the tensors so they outlive the calls."""
+
+    def __init__(self, l1, l1_sf_t, l2, l2_sf_t):
+        for t, n in ((l1, "l1"), (l2, "l2")):
+            _need(t, torch.uint8, n, 3)
+        _need(l1_sf_t, torch.uint8, "l1_sf_t")
+        _need(l2_sf_t, torch.uint8, "l2_sf_t")
+        self.l1, self.l1_sf_t, self.l2, self.l2_sf_t = l1, l1_sf_t, l2, l2_sf_t
+
+    def struct(self) -> Weights:
+        return Weights(LAYOUT_ROW_MAJOR, _ptr(self.l1), _ptr(self.l1_sf_t), _ptr(self.l2), _ptr(self.l2_sf_t))
 
 
 def activation(kind: str = "swiglu", beta: float = 1.0, linear_beta=None) -> Activation:
@@ -67,6 +94,10 @@ def _declare(lib):
         "moe_forward_static": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, P, P]),
         "moe_forward_act": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P,
                                   c.POINTER(Activation), P]),
+        "moe_transformed_scale_bytes": (I32, [I32, I32, I32, c.POINTER(SZ), c.POINTER(SZ)]),
+        "moe_transform_scales": (I32, [P, P, I32, I32, I32, P, P, P]),
+        "moe_forward_weights": (I32, [P, P, P, P, c.POINTER(Weights), P, I32, I32, I32, I32, I32, P, SZ, P, P,
+                                      c.POINTER(Activation), P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -170,6 +201,36 @@ def transform_weights(l1, l1_sf, l2, l2_sf, out=None, stream=None):
     return l1_t, l2_t
 
 
+def transformed_scale_bytes(E: int, H: int, I: int):
+    """Byte sizes of the row-major layout's two scale arrays (host-only)."""
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().moe_transformed_scale_bytes(E, H, I, ctypes.byref(a), ctypes.byref(b)),
+           "moe_transformed_scale_bytes")
+    return a.value, b.value
+
+
+def transform_scales(l1_sf, l2_sf, out=None, stream=None):
+    """[E, 2I, H/32], [E, H, I/32] (u8) -> (l1_sf_t, l2_sf_t) scale-block arrays of
+    the row-major layout (u8, 1-D).  ``out`` may give the two destination views."""
+    _need(l1_sf, torch.uint8, "l1_sf", 3)
+    _need(l2_sf, torch.uint8, "l2_sf", 3)
+    E, twoI, Hg = l1_sf.shape
+    H, I = Hg * 32, twoI // 2
+    if l2_sf.shape != (E, H, I // 32):
+        raise ValueError("inconsistent scale shapes")
+    n1, n2 = transformed_scale_bytes(E, H, I)
+    if out is None:
+        a = torch.empty(n1, dtype=torch.uint8, device=l1_sf.device)
+        b = torch.empty(n2, dtype=torch.uint8, device=l1_sf.device)
+    else:
+        a, b = out
+        if a.numel() < n1 or b.numel() < n2:
+            raise ValueError("output buffers too small")
+    _check(load().moe_transform_scales(_ptr(l1_sf), _ptr(l2_sf), E, H, I, _ptr(a), _ptr(b), _stream(stream)),
+           "moe_transform_scales")
+    return a, b
+
+
 def workspace_bytes(T: int, E: int, k: int, H: int, I: int) -> int:
     n = ctypes.c_size_t()
     _check(load().moe_workspace_bytes(T, E, k, H, I, ctypes.byref(n)), "moe_workspace_bytes")
@@ -184,16 +245,21 @@ def forward_kernel_launches(T: int, E: int, k: int, H: int, I: int) -> int:
 
 
 def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
-            out=None, workspace=None, expert_stats=None, events=None, stream=None, act=None):
+            out=None, workspace=None, expert_stats=None, events=None, stream=None, act=None, weights=None):
     """One layer; returns out (bf16 [T, H]).  ``events``: optional list of
     NUM_STAGE_EVENTS torch.cuda.Event recorded at the stage boundaries.
-    ``act``: an Activation (see ``activation()``); None = SwiGLU."""
+    ``act``: an Activation (see ``activation()``); None = SwiGLU.
+    ``weights``: a RowMajorWeights to run the row-major layout (then l1_t and
+    l2_t are None); by default l1_t / l2_t are the packet buffers."""
     _need(x_fp8, torch.uint8, "x_fp8", 2)
     _need(x_sf, torch.uint8, "x_sf", 2)
     _need(topk_idx, torch.int64, "topk_idx", 2)
     _need(topk_w, torch.float32, "topk_w", 2)
-    _need(l1_t, torch.uint8, "l1_t")
-    _need(l2_t, torch.uint8, "l2_t")
+    if weights is None:
+        _need(l1_t, torch.uint8, "l1_t")
+        _need(l2_t, torch.uint8, "l2_t")
+    elif l1_t is not None or l2_t is not None or not isinstance(weights, RowMajorWeights):
+        raise ValueError("give either packet buffers l1_t / l2_t or weights=RowMajorWeights(...)")
     T, k = topk_idx.shape
     if x_fp8.shape != (T, H) or x_sf.shape != (T, H // 32) or topk_w.shape != (T, k):
         raise ValueError("inconsistent activation / routing shapes")
@@ -215,7 +281,14 @@ def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
             if e.cuda_event == 0:  # torch creates events lazily, on first record
                 e.record(stream if stream is not None else torch.cuda.current_stream())
         ev = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[e.cuda_event for e in events])
-    if act is None:
+    if weights is not None:
+        ws_struct = weights.struct()
+        st = load().moe_forward_weights(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w),
+                                        ctypes.byref(ws_struct), _ptr(out), T, E, k, H, I, _ptr(workspace),
+                                        workspace.numel(), _ptr(expert_stats), ev,
+                                        ctypes.byref(act) if act is not None else None, _stream(stream))
+        _check(st, "moe_forward_weights")
+    elif act is None:
         st = load().moe_forward(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t), _ptr(l2_t),
                                 _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(),
                                 _ptr(expert_stats), ev, _stream(stream))
@@ -278,10 +351,10 @@ def check_device_error(workspace, stream=None) -> int:
 class MoELayer:
     """Holds one layer's transformed weights and a workspace for up to T_max tokens."""
 
-    def __init__(self, l1_t, l2_t, E: int, k: int, H: int, I: int, T_max: int, device=None):
-        self.l1_t, self.l2_t = l1_t, l2_t
+    def __init__(self, l1_t, l2_t, E: int, k: int, H: int, I: int, T_max: int, device=None, weights=None):
+        self.l1_t, self.l2_t, self.weights = l1_t, l2_t, weights
         self.E, self.k, self.H, self.I, self.T_max = E, k, H, I, T_max
-        device = device or l1_t.device
+        device = device or (l1_t.device if weights is None else weights.l1.device)
         self.workspace = torch.empty(workspace_bytes(T_max, E, k, H, I), dtype=torch.uint8, device=device)
 
     def __call__(self, x_fp8, x_sf, topk_idx, topk_w, out=None, expert_stats=None, events=None, stream=None,
@@ -290,4 +363,4 @@ class MoELayer:
             raise ValueError(f"T={topk_idx.shape[0]} exceeds T_max={self.T_max}")
         return forward(x_fp8, x_sf, topk_idx, topk_w, self.l1_t, self.l2_t, self.E, self.H, self.I,
                        out=out, workspace=self.workspace, expert_stats=expert_stats, events=events,
-                       stream=stream, act=act)
+                       stream=stream, act=act, weights=self.weights)

@@ -74,28 +74,35 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Tile packets as a 3D tensor of 4-bit elements: (128 K, 128 rows, packet);
-// one box moves `depth` consecutive 128 x 128 packet bodies, expanded to one
-// byte per element in shared memory with the 128-byte swizzle.
-bool encode_packets(CUtensorMap *m, const void *base, int64_t num_packets, int depth) {
+// FP4 weight bodies as a 4D tensor of 4-bit elements (128 K, rows, tile a,
+// K block b); a box (128, box_rows, box_a, kblocks) lands in shared memory as
+// 128-row slots b * 2 + a, each element expanded to one byte, 128-byte
+// swizzle. The GEMMs read every layout through such a box:
+//   packets:   (128 K, 128 rows, slot [8704 B], K-tile pair [17408 B]), box (128, 128, 2, kKB)
+//   L1 rows:   (128 K, rows E*2I - I [H/2 B], gate/up [I rows], K block [64 B]), box (128, 128, 2, kKB)
+//   L2 rows:   (128 K, rows E*H [I/2 B], 1, K block [64 B]), box (128, 256, 1, kKB): two adjacent
+//              tiles as one 256-row box, so an odd last tile of the last expert reads zeros
+bool encode_weights4(CUtensorMap *m, const void *base, uint64_t rows, uint64_t row_stride, uint64_t a_dim,
+                     uint64_t a_stride, uint64_t b_dim, uint64_t b_stride, int box_rows, int box_a, int kblocks) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    const cuuint64_t dims[3] = {cuuint64_t(kTileK), cuuint64_t(kTileRows), cuuint64_t(num_packets)};
-    const cuuint64_t strides[2] = {cuuint64_t(kTileK / 2), cuuint64_t(kPacketBytes)};
-    const cuuint32_t box[3] = {cuuint32_t(kTileK), cuuint32_t(kTileRows), cuuint32_t(depth)};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(base), dims, strides, box, estr,
+    const cuuint64_t dims[4] = {cuuint64_t(kTileK), rows, a_dim, b_dim};
+    const cuuint64_t strides[3] = {row_stride, a_stride, b_stride};
+    const cuuint32_t box[4] = {cuuint32_t(kTileK), cuuint32_t(box_rows), cuuint32_t(box_a), cuuint32_t(kblocks)};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The same packets as 32-bit words [packet][2176]; a box of 128 words at word
-// 2048 is one packet's 512-byte scale block, `depth` packets per load.
-bool encode_packet_sf(CUtensorMap *m, const void *base, int64_t num_packets, int depth) {
+// Scale blocks as 32-bit words [packet][row_words]: packets (row_words 2176,
+// blocks at word 2048) or the row-major layout's separate arrays (row_words
+// 128); a box of 128 words moves one 512-byte block, `depth` packets per load.
+bool encode_packet_sf(CUtensorMap *m, const void *base, int64_t num_packets, int depth, int row_words) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    const cuuint64_t dims[2] = {cuuint64_t(kPacketBytes / 4), cuuint64_t(num_packets)};
-    const cuuint64_t strides[1] = {cuuint64_t(kPacketBytes)};
+    const cuuint64_t dims[2] = {cuuint64_t(row_words), cuuint64_t(num_packets)};
+    const cuuint64_t strides[1] = {cuuint64_t(row_words) * 4};
     const cuuint32_t box[2] = {cuuint32_t(kPacketSf / 4), cuuint32_t(depth)};
     const cuuint32_t estr[2] = {1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides, box, estr,
@@ -164,7 +171,7 @@ moe_status_t use_device_of(const void *p) {
 // The launch sequence of one layer on a validated workspace (shared by the
 // entry points that run the layer).  The workspace's device must be current.
 moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
-                       const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                       const moe_weights_t &w, void *out_bf16, int T, int E, int k, int H, int I,
                        uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream,
                        const moe_activation_t &act) {
     const WsLayout L = ws_layout(T, E, k, H, I);
@@ -176,8 +183,25 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
     const int d1 = gemm_packets_per_stage(true, L.chunk_rows), d2 = gemm_packets_per_stage(false, L.chunk_rows);
     const int dk = gemm_kblocks_per_stage(L.chunk_rows);
     CUtensorMap tm_w1, tm_w2, tm_s1, tm_s2, tm_xg, tm_hq, tm_xg_full, tm_hq_full;
-    if (!encode_packets(&tm_w1, l1_t, np1, d1) || !encode_packets(&tm_w2, l2_t, np2, d2) ||
-        !encode_packet_sf(&tm_s1, l1_t, np1, d1) || !encode_packet_sf(&tm_s2, l2_t, np2, d2) ||
+    const bool rowmajor = w.layout == MOE_LAYOUT_ROW_MAJOR;
+    bool ok;
+    if (rowmajor) {
+        const uint64_t e = uint64_t(E), h = uint64_t(H), i = uint64_t(I);
+        ok = encode_weights4(&tm_w1, w.l1, e * 2 * i - i, h / 2, 2, i * h / 2, h / kTileK, kTileK / 2, kTileRows, 2,
+                             d1 / 2) &&
+             encode_weights4(&tm_w2, w.l2, e * h, i / 2, 1, e * h * i / 2, i / kTileK, kTileK / 2, 2 * kTileRows, 1,
+                             d2 / 2) &&
+             encode_packet_sf(&tm_s1, w.l1_sf, np1, d1, kPacketSf / 4) &&
+             encode_packet_sf(&tm_s2, w.l2_sf, np2, d2, kPacketSf / 4);
+    } else {
+        ok = encode_weights4(&tm_w1, w.l1, kTileRows, kTileK / 2, 2, kPacketBytes, uint64_t(np1 / 2),
+                             2 * kPacketBytes, kTileRows, 2, d1 / 2) &&
+             encode_weights4(&tm_w2, w.l2, kTileRows, kTileK / 2, 2, kPacketBytes, uint64_t(np2 / 2),
+                             2 * kPacketBytes, kTileRows, 2, d2 / 2) &&
+             encode_packet_sf(&tm_s1, w.l1, np1, d1, kPacketBytes / 4) &&
+             encode_packet_sf(&tm_s2, w.l2, np2, d2, kPacketBytes / 4);
+    }
+    if (!ok ||
         !encode_act(&tm_xg, ws + L.off_xg, L.Rp, L.kbh, dk, kActBoxRows) ||
         !encode_act(&tm_hq, ws + L.off_hq, L.Rp, L.kbi, dk, kActBoxRows) ||
         !encode_act(&tm_xg_full, ws + L.off_xg, L.Rp, L.kbh, dk, L.chunk_rows) ||
@@ -200,12 +224,10 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
                          H, ws, L, expert_stats, st);
     if (e == cudaSuccess) e = record(1);
     if (e == cudaSuccess)
-        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, static_cast<const uint8_t *>(l1_t), ws, L, H, I, grid1, st,
-                        act);
+        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, rowmajor, ws, L, H, I, grid1, st, act);
     if (e == cudaSuccess) e = record(2);
     if (e == cudaSuccess)
-        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, static_cast<const uint8_t *>(l2_t), ws, L, H, I, grid2, st,
-                        act);
+        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, rowmajor, ws, L, H, I, grid2, st, act);
     if (e == cudaSuccess) e = record(3);
     if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
     if (e == cudaSuccess) e = record(4);
@@ -276,8 +298,33 @@ moe_status_t moe_transform_weights(const void *l1, const void *l1_sf, const void
     const moe_status_t d = use_device_of(l1_t);
     if (d != MOE_OK) return d;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_transform(l1, l1_sf, E, 2 * I, H, I / kTileRows, false, I, l1_t, st);
-    if (e == cudaSuccess) e = launch_transform(l2, l2_sf, E, H, I, (H / kTileRows + 1) / 2, true, 0, l2_t, st);
+    cudaError_t e = launch_transform(l1, l1_sf, E, 2 * I, H, I / kTileRows, false, I, l1_t, true, st);
+    if (e == cudaSuccess) e = launch_transform(l2, l2_sf, E, H, I, (H / kTileRows + 1) / 2, true, 0, l2_t, true, st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_transformed_scale_bytes(int E, int H, int I, size_t *l1_sf_bytes, size_t *l2_sf_bytes) {
+    size_t a = 0, b = 0;
+    const moe_status_t s = moe_transformed_weight_bytes(E, H, I, &a, &b);
+    if (s != MOE_OK) return s;
+    if (l1_sf_bytes) *l1_sf_bytes = a / kPacketBytes * kPacketSf;
+    if (l2_sf_bytes) *l2_sf_bytes = b / kPacketBytes * kPacketSf;
+    return MOE_OK;
+}
+
+moe_status_t moe_transform_scales(const void *l1_sf, const void *l2_sf, int E, int H, int I, void *l1_sf_t,
+                                  void *l2_sf_t, moe_stream_t stream) {
+    const moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    if (!l1_sf || !l2_sf || !l1_sf_t || !l2_sf_t) return MOE_ERR_INVALID_ARG;
+    if (!aligned(l1_sf, 4) || !aligned(l2_sf, 4) || !aligned(l1_sf_t, 256) || !aligned(l2_sf_t, 256))
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t d = use_device_of(l1_sf_t);
+    if (d != MOE_OK) return d;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_transform(nullptr, l1_sf, E, 2 * I, H, I / kTileRows, false, I, l1_sf_t, false, st);
+    if (e == cudaSuccess)
+        e = launch_transform(nullptr, l2_sf, E, H, I, (H / kTileRows + 1) / 2, true, 0, l2_sf_t, false, st);
     return cuda_status(e);
 }
 
@@ -311,6 +358,25 @@ moe_status_t moe_forward_act(const void *x_fp8, const void *x_sf, const int64_t 
                              const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
                              void *workspace, size_t ws_bytes, int32_t *expert_stats, void *const *stage_events,
                              const moe_activation_t *activation, moe_stream_t stream) {
+    const moe_weights_t w = {MOE_LAYOUT_PACKETS, l1_t, nullptr, l2_t, nullptr};
+    return moe_forward_weights(x_fp8, x_sf, topk_idx, topk_w, &w, out_bf16, T, E, k, H, I, workspace, ws_bytes,
+                               expert_stats, stage_events, activation, stream);
+}
+
+moe_status_t moe_forward_weights(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
+                                 const moe_weights_t *weights, void *out_bf16, int T, int E, int k, int H, int I,
+                                 void *workspace, size_t ws_bytes, int32_t *expert_stats,
+                                 void *const *stage_events, const moe_activation_t *activation,
+                                 moe_stream_t stream) {
+    if (!weights) return MOE_ERR_INVALID_ARG;
+    const moe_weights_t w = *weights;
+    if (w.layout == MOE_LAYOUT_PACKETS) {
+        if (w.l1_sf || w.l2_sf) return MOE_ERR_INVALID_ARG;
+    } else if (w.layout == MOE_LAYOUT_ROW_MAJOR) {
+        if (!w.l1_sf || !w.l2_sf || !aligned(w.l1_sf, 256) || !aligned(w.l2_sf, 256)) return MOE_ERR_INVALID_ARG;
+    } else {
+        return MOE_ERR_INVALID_ARG;
+    }
     moe_activation_t act = {MOE_ACT_SWIGLU, 1.0f, 0.0f};
     if (activation) {
         act = *activation;
@@ -326,18 +392,18 @@ moe_status_t moe_forward_act(const void *x_fp8, const void *x_sf, const int64_t 
     if (T < 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
     if (int64_t(T) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (T == 0) return MOE_OK;
-    if (!x_fp8 || !x_sf || !topk_idx || !topk_w || !l1_t || !l2_t || !out_bf16 || !workspace)
+    if (!x_fp8 || !x_sf || !topk_idx || !topk_w || !w.l1 || !w.l2 || !out_bf16 || !workspace)
         return MOE_ERR_INVALID_ARG;
     if (!aligned(x_fp8, 16) || !aligned(x_sf, 4) || !aligned(topk_idx, 8) || !aligned(topk_w, 4) ||
-        !aligned(l1_t, 256) || !aligned(l2_t, 256) || !aligned(out_bf16, 16) || !aligned(workspace, 256) ||
+        !aligned(w.l1, 256) || !aligned(w.l2, 256) || !aligned(out_bf16, 16) || !aligned(workspace, 256) ||
         (expert_stats && !aligned(expert_stats, 4)))
         return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(T, E, k, H, I);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     s = use_device_of(workspace);
     if (s != MOE_OK) return s;
-    return run_layer(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, out_bf16, T, E, k, H, I,
-                     static_cast<uint8_t *>(workspace), expert_stats, stage_events, stream, act);
+    return run_layer(x_fp8, x_sf, topk_idx, topk_w, w, out_bf16, T, E, k, H, I, static_cast<uint8_t *>(workspace),
+                     expert_stats, stage_events, stream, act);
 }
 
 moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H, int I, int32_t *count,

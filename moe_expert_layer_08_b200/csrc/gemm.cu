@@ -85,7 +85,12 @@ struct GemmCfg {
 __device__ __forceinline__ int a_slot(int a, int b) { return b * 2 + a; }
 
 struct GemmArgs {
-    const uint8_t *w_packets;  // transformed weights (for the scale blocks)
+    // weight layout: tile packets (body and scale block of each tile together)
+    // or row-major FP4 bodies with the scale blocks in a separate array
+    int w_rowmajor;
+    int w_rows_per_expert;     // row-major: body rows of one expert (2I for L1, H for L2)
+    int w_item_rows;           // row-major: body rows one item steps (128 for L1, 256 for L2)
+    int w_sf_x0;               // word offset of a scale block within a row of the scale map
     const uint8_t *act_sf;     // activation scale blocks [chunk][K/128][512]
     const int4 *chunks;        // (expert, first row, rows, -)
     int *hdr;                  // workspace header (chunk count, error word)
@@ -217,9 +222,14 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         // a box always moves kBoxPackets packets (a last odd K
                         // block loads packets it then ignores)
                         mbar_arrive_expect_tx(&full[stage], uint32_t(kNumA * kKB * (kPacketBody + kPacketSf)));
+                        // 4D box (128 K, 128 rows, tile a, K block b) lands as slots b * 2 + a
                         const int pkt = int((int64_t(ch.x) * groups + it) * KB * 2 + int64_t(kb0) * 2);
-                        tma_load_3d(st, &tmap_w, &full[stage], 0, 0, pkt, pol);
-                        tma_load_2d(sf, &tmap_wsf, &full[stage], kPacketBody / 4, pkt, pol);
+                        if (args.w_rowmajor)
+                            tma_load_4d(st, &tmap_w, &full[stage], 0,
+                                        ch.x * args.w_rows_per_expert + it * args.w_item_rows, 0, kb0, pol);
+                        else
+                            tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol);
+                        tma_load_2d(sf, &tmap_wsf, &full[stage], args.w_sf_x0, pkt, pol);
                     } else {
                         // the activation box always moves kKB K blocks (a K
                         // block past the end reads zeros); a nearly full large
@@ -471,16 +481,19 @@ int gemm_packets_per_stage(bool gemm1, int chunk_rows) {
 }
 
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
-                        const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const uint8_t *w_packets,
+                        const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, bool w_rowmajor,
                         uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
                         const moe_activation_t &act) {
     GemmArgs a{};
+    a.w_rowmajor = w_rowmajor ? 1 : 0;
+    a.w_rows_per_expert = gemm1 ? 2 * I : H;
+    a.w_item_rows = gemm1 ? kTileRows : 2 * kTileRows;
+    a.w_sf_x0 = w_rowmajor ? 0 : kPacketBody / 4;
     a.act_kind = act.kind;
     a.beta = act.beta;
     a.inv_beta = act.kind == MOE_ACT_SITU ? 1.0f / act.beta : 0.0f;
     a.lbeta = act.linear_beta;
     a.inv_lbeta = (act.kind == MOE_ACT_SITU && act.linear_beta > 0.0f) ? 1.0f / act.linear_beta : 0.0f;
-    a.w_packets = w_packets;
     a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
     a.hdr = reinterpret_cast<int *>(ws);
     const bool small = L.chunk_rows == kChunkRowsSmall;

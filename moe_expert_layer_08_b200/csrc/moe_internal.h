@@ -54,8 +54,10 @@ WsLayout ws_layout(int T, int E, int k, int H, int I);
 // Kernel launchers (all asynchronous on `stream`; return cudaGetLastError()).
 cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, void *q, void *sf, bool fp8,
                             cudaStream_t stream);
+// Tile packets (body + scale block, kPacketBytes each) or, with out_body ==
+// nullptr, only the 512-byte scale blocks in the same order (row-major layout).
 cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int groups,
-                             bool pairs, int half_rows, void *out, cudaStream_t stream);
+                             bool pairs, int half_rows, void *out, bool with_body, cudaStream_t stream);
 // kernels launch_route enqueues for R = T * k routed rows (one-block routing
 // up to kRouteSmallMax rows, then the gather; else four routing kernels and
 // the gather)
@@ -63,7 +65,7 @@ inline int route_kernel_launches(int64_t R) { return R <= kRouteSmallMax ? 2 : 5
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
                          int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream);
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
-                        const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const uint8_t *w_packets,
+                        const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, bool w_rowmajor,
                         uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
                         const moe_activation_t &act);
 // Weight packets one pipeline stage of that GEMM variant moves (TMA box depth).
@@ -82,7 +84,7 @@ moe_status_t use_device_of(const void *p);
 // The launch sequence of one layer on a validated, large-enough workspace of
 // the current device.
 moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
-                       const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                       const moe_weights_t &w, void *out_bf16, int T, int E, int k, int H, int I,
                        uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream,
                        const moe_activation_t &act);
 

@@ -79,9 +79,12 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, void *q, 
 //   L2 (pairs):   (2 * grp + slot) * 128 + [0, 128)         (two adjacent tiles)
 // so the two tiles one GEMM item multiplies are adjacent for every K tile.  A
 // pair slot past the last tile (odd tile count) is zero-filled padding.
+// Without bodies (the row-major layout) output block p is packet p's 512-byte
+// scale block alone, in the same order.
 __global__ void __launch_bounds__(128) transform_kernel(const uint8_t *__restrict__ w, const uint8_t *__restrict__ w_sf,
                                                         int rows_per_expert, int K, int groups, bool pairs,
-                                                        int half_rows, int64_t num_packets, uint8_t *__restrict__ out) {
+                                                        int half_rows, int64_t num_packets, uint8_t *__restrict__ out,
+                                                        bool with_body) {
     const int KB = K / kTileK;
     const int r = threadIdx.x;
     for (int64_t p = blockIdx.x; p < num_packets; p += gridDim.x) {
@@ -94,32 +97,37 @@ __global__ void __launch_bounds__(128) transform_kernel(const uint8_t *__restric
         const int64_t e = q / groups;
         const int64_t row_in_expert =
             pairs ? int64_t(2 * grp + slot) * kTileRows + r : int64_t(slot) * half_rows + int64_t(grp) * kTileRows + r;
-        uint8_t *pkt = out + p * kPacketBytes;
-        uint4 *dst = reinterpret_cast<uint4 *>(pkt + r * (kTileK / 2));
-        uint32_t *dsf = reinterpret_cast<uint32_t *>(pkt + kPacketBody + sf_block_offset(r, 0));
+        uint8_t *pkt = with_body ? out + p * kPacketBytes : nullptr;
+        uint4 *dst = with_body ? reinterpret_cast<uint4 *>(pkt + r * (kTileK / 2)) : nullptr;
+        uint32_t *dsf = reinterpret_cast<uint32_t *>((with_body ? pkt + kPacketBody : out + p * kPacketSf) +
+                                                     sf_block_offset(r, 0));
         if (row_in_expert >= rows_per_expert) {  // padding slot
+            if (with_body) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+            }
             *dsf = 0;
             continue;
         }
         const int64_t src_row = e * rows_per_expert + row_in_expert;
-        const uint4 *src = reinterpret_cast<const uint4 *>(w + src_row * (K / 2) + kb * (kTileK / 2));
+        if (with_body) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(w + src_row * (K / 2) + kb * (kTileK / 2));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
+            for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
+        }
         *dsf = __ldg(reinterpret_cast<const uint32_t *>(w_sf + src_row * (K / 32) + kb * 4));
     }
 }
 
 cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int groups,
-                             bool pairs, int half_rows, void *out, cudaStream_t stream) {
+                             bool pairs, int half_rows, void *out, bool with_body, cudaStream_t stream) {
     const int64_t num_packets = int64_t(E) * groups * (K / kTileK) * 2;
     if (num_packets == 0) return cudaSuccess;
     const int64_t grid = num_packets < 65536 ? num_packets : 65536;
     transform_kernel<<<unsigned(grid), 128, 0, stream>>>(static_cast<const uint8_t *>(w),
                                                          static_cast<const uint8_t *>(w_sf), rows_per_expert, K,
                                                          groups, pairs, half_rows, num_packets,
-                                                         static_cast<uint8_t *>(out));
+                                                         static_cast<uint8_t *>(out), with_body);
     return cudaGetLastError();
 }
 

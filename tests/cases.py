@@ -17,8 +17,9 @@ REL_L2_TOL = 1e-2
 MAX_ABS_TOL = 5e-2   # times max |row| of the oracle output
 
 
-def gpu_layer(w: W.Workload, routing=None, gen_device="cuda", device="cuda"):
-    """Inputs of the CUDA path: bf16 draws quantised and transformed by the library."""
+def gpu_layer(w: W.Workload, routing=None, gen_device="cuda", device="cuda", rowmajor=False):
+    """Inputs of the CUDA path: bf16 draws quantised and transformed by the library.
+    With rowmajor, also the same weights in the row-major layout ("rm")."""
     import moe_expert_layer_08_b200 as moe
     x = W.gen_x(w, gen_device).to(device)
     if routing is None:
@@ -29,12 +30,28 @@ def gpu_layer(w: W.Workload, routing=None, gen_device="cuda", device="cuda"):
     l1_t = torch.empty(n1, dtype=torch.uint8, device=device)
     l2_t = torch.empty(n2, dtype=torch.uint8, device=device)
     p1, p2 = n1 // w.E, n2 // w.E
+    if rowmajor:
+        u8 = dict(dtype=torch.uint8, device=device)
+        r1 = torch.empty((w.E, 2 * w.I, w.H // 2), **u8)
+        r2 = torch.empty((w.E, w.H, w.I // 2), **u8)
+        s1 = torch.empty((w.E, 2 * w.I, w.H // 32), **u8)
+        s2 = torch.empty((w.E, w.H, w.I // 32), **u8)
+        m1, m2 = moe.transformed_scale_bytes(w.E, w.H, w.I)
+        s1_t = torch.empty(m1, **u8)
+        s2_t = torch.empty(m2, **u8)
+        q1, q2 = m1 // w.E, m2 // w.E
     for e in range(w.E):
         a, b = moe.quantize_fp4(W.gen_l1(w, e, gen_device).to(device))
         c, d = moe.quantize_fp4(W.gen_l2(w, e, gen_device).to(device))
         moe.transform_weights(a[None], b[None], c[None], d[None],
                               out=(l1_t[e * p1:(e + 1) * p1], l2_t[e * p2:(e + 1) * p2]))
-    return dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw, l1_t=l1_t, l2_t=l2_t)
+        if rowmajor:
+            r1[e], s1[e], r2[e], s2[e] = a, b, c, d
+            moe.transform_scales(b[None], d[None], out=(s1_t[e * q1:(e + 1) * q1], s2_t[e * q2:(e + 1) * q2]))
+    g = dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw, l1_t=l1_t, l2_t=l2_t)
+    if rowmajor:
+        g["rm"] = moe.RowMajorWeights(r1, s1_t, r2, s2_t)
+    return g
 
 
 def oracle_side(w: W.Workload, x_bf16: torch.Tensor, idx: torch.Tensor, experts, gen_device="cuda"):

@@ -133,3 +133,25 @@ def test_forward_act_validates_activation_before_any_cuda_call(moelib):
     # a valid activation passes to the next check (workspace too small)
     a = m.activation("situ", 1.25, 1.5)
     assert f(p, p, p, p, p, p, p, 4, 8, 2, 256, 256, p, 16, None, None, ctypes.byref(a), None) == 3
+
+
+def test_layouts_and_scale_transform_validate_on_the_host(moelib):
+    """Row-major layout entry points: sizes, and every bad argument rejected
+    before any CUDA call."""
+    import moe_expert_layer_08_b200 as m
+    l1, l2 = m.transformed_weight_bytes(384, 7168, 3072)
+    s1, s2 = m.transformed_scale_bytes(384, 7168, 3072)
+    assert (s1 * 17, s2 * 17) == (l1, l2)           # one 512-byte block per 8704-byte packet
+    assert m.transformed_scale_bytes(2, 384, 128) == (2 * 1 * 3 * 2 * 512, 2 * 2 * 1 * 2 * 512)  # odd H tiles pad
+    n = ctypes.c_size_t()
+    assert moelib.moe_transformed_scale_bytes(8, 200, 256, ctypes.byref(n), ctypes.byref(n)) == 2
+    p = ctypes.c_void_p(256)
+    assert moelib.moe_transform_scales(None, p, 8, 256, 256, p, p, None) == 1
+    assert moelib.moe_transform_scales(p, p, 8, 256, 256, ctypes.c_void_p(260), p, None) == 1   # misaligned out
+    args = lambda wts: (p, p, p, p, wts, p, 4, 8, 2, 256, 256, p, 1 << 30, None, None, None, None)
+    assert moelib.moe_forward_weights(*args(None)) == 1
+    assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(7, 256, 0, 256, 0)))) == 1   # unknown layout
+    assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(0, 256, 256, 256, 0)))) == 1  # packets + scales
+    assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(1, 256, 0, 256, 256)))) == 1  # row-major, no l1_sf
+    assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(1, 256, 300, 256, 256)))) == 1  # misaligned
+    assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(1, 0, 256, 256, 256)))) == 1  # no body
