@@ -81,6 +81,18 @@ def _declare(lib):
                                            P, c.c_int, c.c_int, c.c_int,
                                            c.c_int, c.c_double, c.c_double,
                                            P, P, P, P, P, P]
+    lib.oracle_moe_forward_fmt.restype = c.c_int
+    lib.oracle_moe_forward_fmt.argtypes = [P, P, P, P, P, P, P, P,
+                                           c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
+                                           P, c.c_int, c.c_int, c.c_int,
+                                           c.c_int, c.c_double, c.c_double, c.c_int,
+                                           P, P, P, P, P, P]
+    lib.oracle_ue4m3_value.restype = c.c_double
+    lib.oracle_ue4m3_value.argtypes = [c.c_uint32]
+    lib.oracle_nvfp4_scale.restype = c.c_uint32
+    lib.oracle_nvfp4_scale.argtypes = [c.c_double]
+    lib.oracle_quantize_nvfp4.restype = None
+    lib.oracle_quantize_nvfp4.argtypes = [P, c.c_int64, c.c_int64, P, P]
     lib.oracle_moe_forward.restype = c.c_int
     lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, P, P,
                                        c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
@@ -167,6 +179,28 @@ def quantize_e2m1(src, lib=None):
     return packed, sf
 
 
+def ue4m3_value(b: int, lib=None) -> float:
+    return (lib or load()).oracle_ue4m3_value(b)
+
+
+def nvfp4_scale(amax: float, lib=None) -> int:
+    """UE4M3 scale code of a 16-element NVFP4 group with this amax."""
+    return (lib or load()).oracle_nvfp4_scale(amax)
+
+
+def quantize_nvfp4(src, lib=None):
+    """fp32 [rows, cols] -> (packed E2M1 u8 [rows, cols/2] (even element in the
+    low nibble), UE4M3 scale bytes u8 [rows, cols/16])."""
+    lib = lib or load()
+    src = _c(src, np.float32)
+    rows, cols = src.shape
+    assert cols % 16 == 0
+    packed = np.empty((rows, cols // 2), np.uint8)
+    sf = np.empty((rows, cols // 16), np.uint8)
+    lib.oracle_quantize_nvfp4(_ptr(src), rows, cols, _ptr(packed), _ptr(sf))
+    return packed, sf
+
+
 # ---------------------------------------------------------------- routing
 def route(topk_idx, E: int, lib=None):
     """Stable per-expert permutation.  Returns dict(count, offset, perm, inv,
@@ -187,7 +221,7 @@ def route(topk_idx, E: int, lib=None):
 def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: int,
             tokens=None, precision: str = "fp32", threads: int = 0,
             intermediates: bool = False, activation: str = "swiglu", beta: float = 1.0,
-            linear_beta=None, lib=None):
+            linear_beta=None, fmt: str = "mx", lib=None):
     """Evaluate the layer for the listed tokens (all when ``tokens`` is None).
 
     ``experts`` maps expert id -> (l1 [2I, H/2] u8, l1_sf [2I, H/32] u8,
@@ -196,7 +230,9 @@ def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: i
     ``out_f32``; with ``intermediates`` also ``h_pre`` [ntok, k, I] (the
     activation before requantisation), ``h_q``, ``h_sf`` and ``y`` [ntok, k, H].
     ``activation``: "swiglu" or "situ" (with ``beta`` and optional
-    ``linear_beta``).
+    ``linear_beta``).  ``fmt``: "mx" (the above) or "nvfp4": x packed E2M1
+    [T, H/2] with UE4M3 scales [T, H/16], the experts' scales [.., K/16]
+    UE4M3, h requantised to NVFP4 (``h_q`` [ntok, k, I/2], ``h_sf`` [.., I/16]).
     """
     lib = lib or load()
     x_codes = _c(x_codes, np.uint8)
@@ -204,7 +240,10 @@ def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: i
     idx = _c(topk_idx, np.int64)
     w = _c(topk_w, np.float32)
     T, k = idx.shape
-    assert x_codes.shape == (T, H) and x_sf.shape == (T, H // 32) and w.shape == (T, k)
+    nv = {"mx": 0, "nvfp4": 1}[fmt]
+    gs = 16 if nv else 32
+    xcols = H // 2 if nv else H
+    assert x_codes.shape == (T, xcols) and x_sf.shape == (T, H // gs) and w.shape == (T, k)
     if tokens is None:
         tok = None
         ntok = T
@@ -214,7 +253,7 @@ def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: i
     keep = []
     arrs = [(ctypes.c_void_p * E)() for _ in range(4)]
     for e, mats in experts.items():
-        shapes = [(2 * I, H // 2), (2 * I, H // 32), (H, I // 2), (H, I // 32)]
+        shapes = [(2 * I, H // 2), (2 * I, H // gs), (H, I // 2), (H, I // gs)]
         for a, m, shp in zip(arrs, mats, shapes):
             m = _c(m, np.uint8)
             assert m.shape == shp, (m.shape, shp)
@@ -223,16 +262,16 @@ def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: i
     out_bf16 = np.empty((ntok, H), np.uint16)
     out_f32 = np.empty((ntok, H), np.float32)
     h_pre = np.empty((ntok, k, I), np.float32) if intermediates else None
-    h_q = np.empty((ntok, k, I), np.uint8) if intermediates else None
-    h_sf = np.empty((ntok, k, I // 32), np.uint8) if intermediates else None
+    h_q = np.empty((ntok, k, I // 2 if nv else I), np.uint8) if intermediates else None
+    h_sf = np.empty((ntok, k, I // gs), np.uint8) if intermediates else None
     y = np.empty((ntok, k, H), np.float32) if intermediates else None
     act = {"swiglu": 0, "situ": 1}[activation]
-    rc = lib.oracle_moe_forward_act(
+    rc = lib.oracle_moe_forward_fmt(
         _ptr(x_codes), _ptr(x_sf), _ptr(idx), _ptr(w),
         ctypes.cast(arrs[0], ctypes.c_void_p), ctypes.cast(arrs[1], ctypes.c_void_p),
         ctypes.cast(arrs[2], ctypes.c_void_p), ctypes.cast(arrs[3], ctypes.c_void_p),
         T, E, k, H, I, _ptr(tok), ntok, 1 if precision == "double" else 0, threads,
-        act, float(beta), float(linear_beta or 0.0),
+        act, float(beta), float(linear_beta or 0.0), nv,
         _ptr(out_bf16), _ptr(out_f32), _ptr(h_pre), _ptr(h_q), _ptr(h_sf), _ptr(y))
     if rc == -1:
         raise KeyError("a listed token routes to an expert whose weights were not given")
@@ -254,13 +293,15 @@ def bf16_bits_to_f32(bits) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- inputs
-def quantize_inputs(x_bf16_f32, l1_f32: dict, l2_f32: dict, lib=None):
-    """Quantise fp32 copies of the bf16 draws: x -> E4M3, expert weights -> E2M1.
-    Returns (x_codes, x_sf, experts) in the layout ``forward`` takes."""
-    xq, xs = quantize_e4m3(x_bf16_f32, lib)
+def quantize_inputs(x_bf16_f32, l1_f32: dict, l2_f32: dict, fmt: str = "mx", lib=None):
+    """Quantise fp32 copies of the bf16 draws: x -> E4M3, expert weights -> E2M1
+    (fmt "mx"), or all to NVFP4 (fmt "nvfp4").  Returns (x_codes, x_sf,
+    experts) in the layout ``forward`` takes."""
+    qx, qw = (quantize_nvfp4, quantize_nvfp4) if fmt == "nvfp4" else (quantize_e4m3, quantize_e2m1)
+    xq, xs = qx(x_bf16_f32, lib)
     experts = {}
     for e in l1_f32:
-        a, b = quantize_e2m1(l1_f32[e], lib)
-        c, d = quantize_e2m1(l2_f32[e], lib)
+        a, b = qw(l1_f32[e], lib)
+        c, d = qw(l2_f32[e], lib)
         experts[e] = (a, b, c, d)
     return xq, xs, experts

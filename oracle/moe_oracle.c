@@ -34,8 +34,17 @@
  * scaled value; within an expert routed rows are in ascending t*k+j order;
  * out-of-range expert ids are dropped and counted.
  *
+ * NVFP4 variant (the "NVFP4 Mega MoE Kernel -- Mojo Rewrite" README, sections
+ * Key operations and NVFP4 specifics): activations, weights and the
+ * intermediate h are all FP4 E2M1 with one UE4M3 scale per 16 consecutive K
+ * elements.  The pages give no scale rule; the reading taken here mirrors the
+ * MX one: s = the smallest UE4M3 value with 6 * s >= amax (so no code
+ * saturates; amax = 0 gives s = 1), code = round-to-nearest-even onto the
+ * E2M1 grid of the fp32 quotient v / s.  No per-tensor scale (none is named).
+ *
  * Floating-point formats (OCP Microscaling Formats v1.0, the format the pages
- * name as FP8 E4M3 / FP4 E2M1 / UE8M0): decoded from their bit fields.
+ * name as FP8 E4M3 / FP4 E2M1 / UE8M0; UE4M3 = the E4M3 bit fields with the
+ * sign bit 0): decoded from their bit fields.
  *
  * Every function is written for a reader checking it against the definition,
  * not for speed: no blocking, no SIMD, no reordering of the sums.
@@ -92,6 +101,12 @@ double oracle_ue8m0_value(uint32_t b)
     if (b == 0xFFu)
         return NAN;
     return ldexp(1.0, (int)b - 127);
+}
+
+/* UE4M3: an E4M3 code with sign bit 0 (0x7F is NaN) */
+double oracle_ue4m3_value(uint32_t b)
+{
+    return oracle_e4m3_value(b & 0x7Fu);
 }
 
 /* ------------------------------------------------------------------ */
@@ -206,6 +221,42 @@ void oracle_quantize_e2m1(const float *src, int64_t rows, int64_t cols,
 }
 
 /* fp32 -> bf16 bits, round to nearest even (NaN -> canonical quiet NaN). */
+/* NVFP4 scale code of a 16-element group: the smallest UE4M3 value s with
+ * 6 * s >= amax (6 * s is exact in double), scanning the codebook upward;
+ * amax = 0 gives 1.0 (code 0x38); above 6 * 448 the largest finite code. */
+uint32_t oracle_nvfp4_scale(double amax)
+{
+    if (!(amax > 0.0))
+        return 0x38u;
+    for (uint32_t c = 1; c < 0x7Fu; c++)
+        if (6.0 * oracle_e4m3_value(c) >= amax)
+            return c;
+    return 0x7Eu;
+}
+
+/* FP4 E2M1 codes (two per byte, even column in the low nibble) and one UE4M3
+ * scale byte per 16 consecutive columns; cols % 16 == 0. */
+void oracle_quantize_nvfp4(const float *src, int64_t rows, int64_t cols,
+                           uint8_t *q, uint8_t *sf)
+{
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t g = 0; g < cols / 16; g++) {
+            const float *v = src + r * cols + g * 16;
+            double amax = 0.0;
+            for (int i = 0; i < 16; i++)
+                if (fabs((double)v[i]) > amax)
+                    amax = fabs((double)v[i]);
+            uint32_t c = oracle_nvfp4_scale(amax);
+            float s = (float)oracle_e4m3_value(c);
+            sf[r * (cols / 16) + g] = (uint8_t)c;
+            for (int i = 0; i < 16; i += 2) {
+                uint32_t lo = oracle_round_e2m1((double)(v[i] / s));
+                uint32_t hi = oracle_round_e2m1((double)(v[i + 1] / s));
+                q[(r * cols + g * 16 + i) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+}
+
 uint16_t oracle_f32_to_bf16(float f)
 {
     uint32_t u;
@@ -277,33 +328,39 @@ typedef struct {
     int use_double;                   /* 0: fp32 accumulation (the method); 1: double */
     int activation;                   /* 0: SwiGLU, 1: SiTU */
     double beta, linear_beta;         /* SiTU coefficients; linear_beta <= 0: absent */
+    int nv;                           /* 0: FP8 x FP4, UE8M0 / 32; 1: NVFP4 (FP4, UE4M3 / 16) */
+    int gs;                           /* scale group: 32 or 16 */
     /* outputs, indexed by position p in the token list */
     uint16_t *out_bf16;               /* [ntok, H] */
     float *out_f32;                   /* [ntok, H]       (nullable) */
     float *h_pre;                     /* [ntok, k, I]    (nullable) SwiGLU before requant */
-    uint8_t *h_q;                     /* [ntok, k, I]    (nullable) */
-    uint8_t *h_sf;                    /* [ntok, k, I/32] (nullable) */
+    uint8_t *h_q;                     /* [ntok, k, I] (NVFP4: [ntok, k, I/2]) (nullable) */
+    uint8_t *h_sf;                    /* [ntok, k, I/gs] (nullable) */
     float *y;                         /* [ntok, k, H]    (nullable) GEMM2 output */
     /* decode tables, each filled once from the bit-field decoders above */
-    double e4m3[256], e2m1[16], ue8m0[256];
+    double e4m3[256], e2m1[16], ue8m0[256], ue4m3[256];
     /* work distribution */
     int next;
     int missing_expert;
 } job_t;
 
-static double dq_x(const job_t *J, int t, int kk)
-{
-    return J->e4m3[J->x[(int64_t)t * J->H + kk]] *
-           J->ue8m0[J->x_sf[(int64_t)t * (J->H / 32) + kk / 32]];
-}
-
-/* element (row, col) of a packed FP4 matrix with `cols` columns */
+/* element (row, col) of a packed FP4 matrix with `cols` columns and one
+ * scale byte per J->gs columns */
 static double dq_w(const job_t *J, const uint8_t *w, const uint8_t *sf, int64_t row,
                    int cols, int col)
 {
     uint8_t byte = w[row * (cols / 2) + col / 2];
     uint32_t nib = (col % 2 == 0) ? (byte & 0xFu) : (byte >> 4);
-    return J->e2m1[nib] * J->ue8m0[sf[row * (cols / 32) + col / 32]];
+    uint8_t sb = sf[row * (cols / J->gs) + col / J->gs];
+    return J->e2m1[nib] * (J->nv ? J->ue4m3[sb] : J->ue8m0[sb]);
+}
+
+static double dq_x(const job_t *J, int t, int kk)
+{
+    if (J->nv)  /* packed FP4 [T, H/2] with UE4M3 per 16 */
+        return dq_w(J, J->x, J->x_sf, t, J->H, kk);
+    return J->e4m3[J->x[(int64_t)t * J->H + kk]] *
+           J->ue8m0[J->x_sf[(int64_t)t * (J->H / 32) + kk / 32]];
 }
 
 static void token_forward(job_t *J, int p, double *xd, double *c1, double *h,
@@ -313,6 +370,7 @@ static void token_forward(job_t *J, int p, double *xd, double *c1, double *h,
     const int H = J->H, I = J->I, k = J->k;
     const int t = J->tokens ? J->tokens[p] : p;
     uint8_t hq[32];
+    const int gs = J->gs;
 
     for (int kk = 0; kk < H; kk++)
         xd[kk] = dq_x(J, t, kk);
@@ -371,18 +429,37 @@ static void token_forward(job_t *J, int p, double *xd, double *c1, double *h,
         if (J->h_pre)
             for (int i = 0; i < I; i++)
                 J->h_pre[((int64_t)p * k + j) * I + i] = (float)h[i];
-        /* requantise h to FP8 E4M3 + UE8M0 per 32, then dequantise */
-        for (int g = 0; g < I / 32; g++) {
+        /* requantise h (FP8 E4M3 + UE8M0 per 32, or NVFP4), then dequantise */
+        for (int g = 0; g < I / gs; g++) {
             uint8_t sfb;
-            int ex = group_scale(&h[g * 32], 32, 448.0, &sfb);
-            for (int i = 0; i < 32; i++) {
-                hq[i] = (uint8_t)oracle_round_e4m3(ldexp(h[g * 32 + i], -ex));
-                hd[g * 32 + i] = J->e4m3[hq[i]] * J->ue8m0[sfb];
+            if (!J->nv) {
+                int ex = group_scale(&h[g * 32], 32, 448.0, &sfb);
+                for (int i = 0; i < 32; i++) {
+                    hq[i] = (uint8_t)oracle_round_e4m3(ldexp(h[g * 32 + i], -ex));
+                    hd[g * 32 + i] = J->e4m3[hq[i]] * J->ue8m0[sfb];
+                    if (J->h_q)
+                        J->h_q[((int64_t)p * k + j) * I + g * 32 + i] = hq[i];
+                }
+            } else {
+                double amax = 0.0;
+                for (int i = 0; i < 16; i++)
+                    if (fabs(h[g * 16 + i]) > amax)
+                        amax = fabs(h[g * 16 + i]);
+                sfb = (uint8_t)oracle_nvfp4_scale(amax);
+                for (int i = 0; i < 16; i++) {
+                    /* the fp32 quotient (fp32 mode); the double one in double mode */
+                    double qv = J->use_double ? h[g * 16 + i] / J->ue4m3[sfb]
+                                              : (double)((float)h[g * 16 + i] / (float)J->ue4m3[sfb]);
+                    hq[i] = (uint8_t)oracle_round_e2m1(qv);
+                    hd[g * 16 + i] = J->e2m1[hq[i]] * J->ue4m3[sfb];
+                }
                 if (J->h_q)
-                    J->h_q[((int64_t)p * k + j) * I + g * 32 + i] = hq[i];
+                    for (int i = 0; i < 16; i += 2)
+                        J->h_q[((int64_t)p * k + j) * (I / 2) + (g * 16 + i) / 2] =
+                            (uint8_t)(hq[i] | (hq[i + 1] << 4));
             }
             if (J->h_sf)
-                J->h_sf[((int64_t)p * k + j) * (I / 32) + g] = sfb;
+                J->h_sf[((int64_t)p * k + j) * (I / gs) + g] = sfb;
         }
         /* GEMM2: Y[c] = sum_i hd[i] * w2d[c, i], ascending i */
         for (int c = 0; c < H; c++) {
@@ -456,18 +533,23 @@ int oracle_num_threads(int requested)
  * Expert weight pointers are per expert (length E arrays); an expert that a
  * listed token uses must be present.  Returns 0, or -1 if a needed expert was
  * missing, or -2 on a bad argument.  Each token is evaluated by one thread in
- * a fixed order, so the result does not depend on the thread count. */
-int oracle_moe_forward_act(const uint8_t *x, const uint8_t *x_sf,
+ * a fixed order, so the result does not depend on the thread count.
+ * nvfp4 = 0: x is FP8 [T, H] with UE8M0 per 32 ([T, H/32]), weight scales
+ * UE8M0 per 32.  nvfp4 = 1: x is packed FP4 [T, H/2] with UE4M3 per 16
+ * ([T, H/16]), weight scales UE4M3 per 16, and h is requantised to NVFP4. */
+int oracle_moe_forward_fmt(const uint8_t *x, const uint8_t *x_sf,
                            const int64_t *topk_idx, const float *topk_w,
                            const uint8_t *const *l1, const uint8_t *const *l1_sf,
                            const uint8_t *const *l2, const uint8_t *const *l2_sf,
                            int T, int E, int k, int H, int I,
                            const int32_t *tokens, int ntok, int use_double, int nthreads,
-                           int activation, double beta, double linear_beta,
+                           int activation, double beta, double linear_beta, int nvfp4,
                            uint16_t *out_bf16, float *out_f32, float *h_pre,
                            uint8_t *h_q, uint8_t *h_sf, float *y)
 {
     if (H % 32 || I % 32 || H <= 0 || I <= 0 || k <= 0 || E <= 0 || T < 0 || ntok < 0)
+        return -2;
+    if (nvfp4 != 0 && nvfp4 != 1)
         return -2;
     if (activation != 0 && !(activation == 1 && beta > 0 && isfinite(beta) && isfinite(linear_beta)))
         return -2;
@@ -482,11 +564,13 @@ int oracle_moe_forward_act(const uint8_t *x, const uint8_t *x_sf,
     J.T = T; J.E = E; J.k = k; J.H = H; J.I = I;
     J.tokens = tokens; J.ntok = ntok; J.use_double = use_double;
     J.activation = activation; J.beta = beta; J.linear_beta = linear_beta;
+    J.nv = nvfp4; J.gs = nvfp4 ? 16 : 32;
     J.out_bf16 = out_bf16; J.out_f32 = out_f32; J.h_pre = h_pre;
     J.h_q = h_q; J.h_sf = h_sf; J.y = y;
     for (int c = 0; c < 256; c++) {
         J.e4m3[c] = oracle_e4m3_value((uint32_t)c);
         J.ue8m0[c] = oracle_ue8m0_value((uint32_t)c);
+        J.ue4m3[c] = oracle_ue4m3_value((uint32_t)c);
     }
     for (int c = 0; c < 16; c++)
         J.e2m1[c] = oracle_e2m1_value((uint32_t)c);
@@ -500,6 +584,22 @@ int oracle_moe_forward_act(const uint8_t *x, const uint8_t *x_sf,
         pthread_join(th[i], NULL);
     free(th);
     return J.missing_expert ? -1 : 0;
+}
+
+/* The FP8 x FP4 layer with a chosen activation (see oracle_moe_forward_fmt). */
+int oracle_moe_forward_act(const uint8_t *x, const uint8_t *x_sf,
+                           const int64_t *topk_idx, const float *topk_w,
+                           const uint8_t *const *l1, const uint8_t *const *l1_sf,
+                           const uint8_t *const *l2, const uint8_t *const *l2_sf,
+                           int T, int E, int k, int H, int I,
+                           const int32_t *tokens, int ntok, int use_double, int nthreads,
+                           int activation, double beta, double linear_beta,
+                           uint16_t *out_bf16, float *out_f32, float *h_pre,
+                           uint8_t *h_q, uint8_t *h_sf, float *y)
+{
+    return oracle_moe_forward_fmt(x, x_sf, topk_idx, topk_w, l1, l1_sf, l2, l2_sf, T, E, k, H, I,
+                                  tokens, ntok, use_double, nthreads, activation, beta, linear_beta, 0,
+                                  out_bf16, out_f32, h_pre, h_q, h_sf, y);
 }
 
 /* The layer with SwiGLU (see oracle_moe_forward_act). */
