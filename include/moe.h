@@ -265,6 +265,58 @@ moe_status_t moe_forward_weights(const void *x_fp8, const void *x_sf,
                                  const moe_activation_t *activation, moe_stream_t stream);
 
 /*
+ * NVFP4 variant ("NVFP4 Mega MoE Kernel -- Mojo Rewrite" README: Key
+ * operations, NVFP4 specifics): activations, weights and the intermediate h
+ * are all FP4 E2M1 with one UE4M3 scale per 16 consecutive K elements, and the
+ * GEMMs run tcgen05.mma.kind::mxf4nvf4.block_scale.scale_vec::4X.  Scale
+ * rule (the pages give none): s = the smallest UE4M3 value with 6*s >= amax
+ * (amax = 0 gives 1), code = E2M1 round-to-nearest-even of the fp32 quotient
+ * v / s.  H % 256 == 0 and I % 256 == 0.
+ */
+
+/*
+ * moe_quantize_nvfp4 -- bf16 [rows, cols] (16-byte aligned) -> packed E2M1 q
+ * [rows, cols/2] (even element in the low nibble, 8-byte aligned) and UE4M3
+ * sf [rows, cols/16].  cols % 16 == 0.
+ */
+moe_status_t moe_quantize_nvfp4(const void *x, int64_t rows, int64_t cols,
+                                void *q, void *sf, moe_stream_t stream);
+
+/*
+ * moe_transformed_weight_bytes_nvfp4 -- packet buffer sizes of the NVFP4
+ * weights (host-only): packets of 18432 bytes = 128 rows x 256 K of packed
+ * E2M1 (16384 B) + four 512-byte UE4M3 scale images (one per 64 K), in the
+ * same order as moe_transform_weights' packets with 256-K tiles.
+ */
+moe_status_t moe_transformed_weight_bytes_nvfp4(int E, int H, int I,
+                                                size_t *l1_bytes, size_t *l2_bytes);
+
+/*
+ * moe_transform_weights_nvfp4 -- l1 [E, 2I, H/2], l1_sf [E, 2I, H/16],
+ * l2 [E, H, I/2], l2_sf [E, H, I/16] as moe_quantize_nvfp4 wrote them ->
+ * packets in l1_t / l2_t (256-byte aligned).  Validation as
+ * moe_transform_weights.
+ */
+moe_status_t moe_transform_weights_nvfp4(const void *l1, const void *l1_sf,
+                                         const void *l2, const void *l2_sf,
+                                         int E, int H, int I,
+                                         void *l1_t, void *l2_t, moe_stream_t stream);
+
+/*
+ * moe_forward_nvfp4 -- the layer in NVFP4: x_fp4 [T, H/2] packed E2M1
+ * (16-byte aligned), x_sf [T, H/16] UE4M3 (4-byte aligned), l1_t / l2_t from
+ * moe_transform_weights_nvfp4; everything else as moe_forward_act (the same
+ * workspace size serves both formats).
+ */
+moe_status_t moe_forward_nvfp4(const void *x_fp4, const void *x_sf,
+                               const int64_t *topk_idx, const float *topk_w,
+                               const void *l1_t, const void *l2_t, void *out_bf16,
+                               int T, int E, int k, int H, int I,
+                               void *workspace, size_t ws_bytes,
+                               int32_t *expert_stats, void *const *stage_events,
+                               const moe_activation_t *activation, moe_stream_t stream);
+
+/*
  * moe_read_routing -- copies the routing metadata of the last moe_forward that
  * used `workspace` with these (T, E, k, H, I) into HOST arrays (test and
  * inspection hook; synchronises `stream`).  Any output may be NULL.

@@ -20,7 +20,8 @@ __all__ = [
     "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
     "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
-    "LAYOUT_ROW_MAJOR",
+    "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
+    "forward_nvfp4",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -95,6 +96,11 @@ def _declare(lib):
         "moe_forward_act": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P,
                                   c.POINTER(Activation), P]),
         "moe_transformed_scale_bytes": (I32, [I32, I32, I32, c.POINTER(SZ), c.POINTER(SZ)]),
+        "moe_quantize_nvfp4": (I32, [P, I64, I64, P, P, P]),
+        "moe_transformed_weight_bytes_nvfp4": (I32, [I32, I32, I32, c.POINTER(SZ), c.POINTER(SZ)]),
+        "moe_transform_weights_nvfp4": (I32, [P, P, P, P, I32, I32, I32, P, P, P]),
+        "moe_forward_nvfp4": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P,
+                                    c.POINTER(Activation), P]),
         "moe_transform_scales": (I32, [P, P, I32, I32, I32, P, P, P]),
         "moe_forward_weights": (I32, [P, P, P, P, c.POINTER(Weights), P, I32, I32, I32, I32, I32, P, SZ, P, P,
                                       c.POINTER(Activation), P]),
@@ -201,6 +207,45 @@ def transform_weights(l1, l1_sf, l2, l2_sf, out=None, stream=None):
     return l1_t, l2_t
 
 
+def quantize_nvfp4(x, stream=None):
+    """bf16 [rows, cols] -> (packed E2M1 u8 [rows, cols/2], UE4M3 scales u8 [rows, cols/16])."""
+    _need(x, torch.bfloat16, "x", 2)
+    rows, cols = x.shape
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
+    _check(load().moe_quantize_nvfp4(_ptr(x), rows, cols, _ptr(q), _ptr(sf), _stream(stream)), "moe_quantize_nvfp4")
+    return q, sf
+
+
+def transformed_weight_bytes_nvfp4(E: int, H: int, I: int):
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().moe_transformed_weight_bytes_nvfp4(E, H, I, ctypes.byref(a), ctypes.byref(b)),
+           "moe_transformed_weight_bytes_nvfp4")
+    return a.value, b.value
+
+
+def transform_weights_nvfp4(l1, l1_sf, l2, l2_sf, out=None, stream=None):
+    """[E, 2I, H/2], [E, 2I, H/16], [E, H, I/2], [E, H, I/16] (u8) -> (l1_t, l2_t)
+    NVFP4 packet buffers (u8, 1-D).  ``out`` may give the two destination views."""
+    for t, n in ((l1, "l1"), (l1_sf, "l1_sf"), (l2, "l2"), (l2_sf, "l2_sf")):
+        _need(t, torch.uint8, n, 3)
+    E, twoI, Hh = l1.shape
+    H, I = Hh * 2, twoI // 2
+    if l1_sf.shape != (E, 2 * I, H // 16) or l2.shape != (E, H, I // 2) or l2_sf.shape != (E, H, I // 16):
+        raise ValueError("inconsistent weight shapes")
+    n1, n2 = transformed_weight_bytes_nvfp4(E, H, I)
+    if out is None:
+        l1_t = torch.empty(n1, dtype=torch.uint8, device=l1.device)
+        l2_t = torch.empty(n2, dtype=torch.uint8, device=l1.device)
+    else:
+        l1_t, l2_t = out
+        if l1_t.numel() < n1 or l2_t.numel() < n2:
+            raise ValueError("output buffers too small")
+    _check(load().moe_transform_weights_nvfp4(_ptr(l1), _ptr(l1_sf), _ptr(l2), _ptr(l2_sf), E, H, I,
+                                              _ptr(l1_t), _ptr(l2_t), _stream(stream)), "moe_transform_weights_nvfp4")
+    return l1_t, l2_t
+
+
 def transformed_scale_bytes(E: int, H: int, I: int):
     """Byte sizes of the row-major layout's two scale arrays (host-only)."""
     a, b = ctypes.c_size_t(), ctypes.c_size_t()
@@ -301,6 +346,44 @@ def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
     return out
 
 
+def forward_nvfp4(x_fp4, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
+                  out=None, workspace=None, expert_stats=None, events=None, stream=None, act=None):
+    """One layer in NVFP4 (x packed E2M1 [T, H/2] with UE4M3 scales [T, H/16],
+    packets from transform_weights_nvfp4); returns out (bf16 [T, H])."""
+    _need(x_fp4, torch.uint8, "x_fp4", 2)
+    _need(x_sf, torch.uint8, "x_sf", 2)
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(l1_t, torch.uint8, "l1_t")
+    _need(l2_t, torch.uint8, "l2_t")
+    T, k = topk_idx.shape
+    if x_fp4.shape != (T, H // 2) or x_sf.shape != (T, H // 16) or topk_w.shape != (T, k):
+        raise ValueError("inconsistent activation / routing shapes")
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x_fp4.device)
+    else:
+        _need(out, torch.bfloat16, "out", 2)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(T, E, k, H, I), dtype=torch.uint8, device=x_fp4.device)
+    else:
+        _need(workspace, torch.uint8, "workspace")
+    if expert_stats is not None:
+        _need(expert_stats, torch.int32, "expert_stats", 1)
+    ev = None
+    if events is not None:
+        if len(events) != NUM_STAGE_EVENTS:
+            raise ValueError(f"events must hold {NUM_STAGE_EVENTS} torch.cuda.Event")
+        for e in events:
+            if e.cuda_event == 0:
+                e.record(stream if stream is not None else torch.cuda.current_stream())
+        ev = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[e.cuda_event for e in events])
+    st = load().moe_forward_nvfp4(_ptr(x_fp4), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t), _ptr(l2_t),
+                                  _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(), _ptr(expert_stats),
+                                  ev, ctypes.byref(act) if act is not None else None, _stream(stream))
+    _check(st, "moe_forward_nvfp4")
+    return out
+
+
 def forward_static(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
                    out=None, expert_stats=None, stream=None):
     """The layer for callers that cannot allocate device memory: the scratch is
@@ -351,8 +434,11 @@ def check_device_error(workspace, stream=None) -> int:
 class MoELayer:
     """Holds one layer's transformed weights and a workspace for up to T_max tokens."""
 
-    def __init__(self, l1_t, l2_t, E: int, k: int, H: int, I: int, T_max: int, device=None, weights=None):
-        self.l1_t, self.l2_t, self.weights = l1_t, l2_t, weights
+    def __init__(self, l1_t, l2_t, E: int, k: int, H: int, I: int, T_max: int, device=None, weights=None,
+                 fmt: str = "mx"):
+        if fmt not in ("mx", "nvfp4") or (fmt == "nvfp4" and weights is not None):
+            raise ValueError("fmt is 'mx' or 'nvfp4' (NVFP4 takes packet buffers)")
+        self.l1_t, self.l2_t, self.weights, self.fmt = l1_t, l2_t, weights, fmt
         self.E, self.k, self.H, self.I, self.T_max = E, k, H, I, T_max
         device = device or (l1_t.device if weights is None else weights.l1.device)
         self.workspace = torch.empty(workspace_bytes(T_max, E, k, H, I), dtype=torch.uint8, device=device)
@@ -361,6 +447,10 @@ class MoELayer:
                  act=None):
         if topk_idx.shape[0] > self.T_max:
             raise ValueError(f"T={topk_idx.shape[0]} exceeds T_max={self.T_max}")
+        if self.fmt == "nvfp4":
+            return forward_nvfp4(x_fp8, x_sf, topk_idx, topk_w, self.l1_t, self.l2_t, self.E, self.H, self.I,
+                                 out=out, workspace=self.workspace, expert_stats=expert_stats, events=events,
+                                 stream=stream, act=act)
         return forward(x_fp8, x_sf, topk_idx, topk_w, self.l1_t, self.l2_t, self.E, self.H, self.I,
                        out=out, workspace=self.workspace, expert_stats=expert_stats, events=events,
                        stream=stream, act=act, weights=self.weights)

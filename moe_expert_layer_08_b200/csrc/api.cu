@@ -48,9 +48,10 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     const size_t mc_large = size_t((L.R + kChunkRows - 1) / kChunkRows + (L.R < E ? L.R : E));
     const size_t sf_large = (mc_large > 0 ? mc_large : 1) * size_t(act_sf_bytes(kChunkRows));
     const size_t sf_per_kb = sf_small > sf_large ? sf_small : sf_large;
-    L.off_xg_sf = take(sf_per_kb * size_t(H / kTileK));
+    // twice that: NVFP4 operands have four images per 256 K, two per 128
+    L.off_xg_sf = take(2 * sf_per_kb * size_t(H / kTileK));
     L.off_hq = take(size_t(L.Rp) * size_t(L.kbi) * kTileK);
-    L.off_hq_sf = take(sf_per_kb * size_t(I / kTileK));
+    L.off_hq_sf = take(2 * sf_per_kb * size_t(I / kTileK));
     L.off_y = take(R * size_t(H) * 2);
     L.total = o;
     return L;
@@ -92,6 +93,33 @@ bool encode_weights4(CUtensorMap *m, const void *base, uint64_t rows, uint64_t r
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// NVFP4 packets: bodies as bytes (128 B, 128 rows, slot, K-tile pair), box
+// (128, 128, 2, 1) = both tiles of one 256-K block; their scale images as
+// words (128, image, packet) from the first image, box (128, 4, 2).
+bool encode_nv_packets(CUtensorMap *m, const void *base, int64_t num_packets) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[4] = {128, cuuint64_t(kTileRows), 2, cuuint64_t(num_packets / 2)};
+    const cuuint64_t strides[3] = {128, cuuint64_t(kNvPacketBytes), cuuint64_t(2 * kNvPacketBytes)};
+    const cuuint32_t box[4] = {128, cuuint32_t(kTileRows), 2, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool encode_nv_packet_sf(CUtensorMap *m, const void *base, int64_t num_packets) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const uint8_t *sf0 = static_cast<const uint8_t *>(base) + kNvPacketBody;
+    const cuuint64_t dims[3] = {cuuint64_t(kSfBlockBytes / 4), cuuint64_t(kNvImages), cuuint64_t(num_packets)};
+    const cuuint64_t strides[2] = {cuuint64_t(kSfBlockBytes), cuuint64_t(kNvPacketBytes)};
+    const cuuint32_t box[3] = {cuuint32_t(kSfBlockBytes / 4), cuuint32_t(kNvImages), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(sf0), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -173,19 +201,28 @@ moe_status_t use_device_of(const void *p) {
 moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
                        const moe_weights_t &w, void *out_bf16, int T, int E, int k, int H, int I,
                        uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream,
-                       const moe_activation_t &act) {
+                       const moe_activation_t &act, bool nvfp4) {
     const WsLayout L = ws_layout(T, E, k, H, I);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     size_t l1_bytes = 0, l2_bytes = 0;
-    moe_transformed_weight_bytes(E, H, I, &l1_bytes, &l2_bytes);
-
-    const int64_t np1 = int64_t(l1_bytes / kPacketBytes), np2 = int64_t(l2_bytes / kPacketBytes);
-    const int d1 = gemm_packets_per_stage(true, L.chunk_rows), d2 = gemm_packets_per_stage(false, L.chunk_rows);
-    const int dk = gemm_kblocks_per_stage(L.chunk_rows);
+    if (nvfp4)
+        moe_transformed_weight_bytes_nvfp4(E, H, I, &l1_bytes, &l2_bytes);
+    else
+        moe_transformed_weight_bytes(E, H, I, &l1_bytes, &l2_bytes);
+    const size_t pkt_bytes = nvfp4 ? kNvPacketBytes : kPacketBytes;
+    const int64_t np1 = int64_t(l1_bytes / pkt_bytes), np2 = int64_t(l2_bytes / pkt_bytes);
+    const int d1 = gemm_packets_per_stage(true, L.chunk_rows, nvfp4);
+    const int d2 = gemm_packets_per_stage(false, L.chunk_rows, nvfp4);
+    const int dk = gemm_kblocks_per_stage(L.chunk_rows, nvfp4);
+    // operand rows are stored in 128-byte column blocks (128 FP8 or 256 FP4 elements)
+    const int64_t kbh = nvfp4 ? H / kNvTileK : L.kbh, kbi = nvfp4 ? I / kNvTileK : L.kbi;
     CUtensorMap tm_w1, tm_w2, tm_s1, tm_s2, tm_xg, tm_hq, tm_xg_full, tm_hq_full;
     const bool rowmajor = w.layout == MOE_LAYOUT_ROW_MAJOR;
     bool ok;
-    if (rowmajor) {
+    if (nvfp4) {
+        ok = encode_nv_packets(&tm_w1, w.l1, np1) && encode_nv_packets(&tm_w2, w.l2, np2) &&
+             encode_nv_packet_sf(&tm_s1, w.l1, np1) && encode_nv_packet_sf(&tm_s2, w.l2, np2);
+    } else if (rowmajor) {
         const uint64_t e = uint64_t(E), h = uint64_t(H), i = uint64_t(I);
         ok = encode_weights4(&tm_w1, w.l1, e * 2 * i - i, h / 2, 2, i * h / 2, h / kTileK, kTileK / 2, kTileRows, 2,
                              d1 / 2) &&
@@ -202,10 +239,10 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
              encode_packet_sf(&tm_s2, w.l2, np2, d2, kPacketBytes / 4);
     }
     if (!ok ||
-        !encode_act(&tm_xg, ws + L.off_xg, L.Rp, L.kbh, dk, kActBoxRows) ||
-        !encode_act(&tm_hq, ws + L.off_hq, L.Rp, L.kbi, dk, kActBoxRows) ||
-        !encode_act(&tm_xg_full, ws + L.off_xg, L.Rp, L.kbh, dk, L.chunk_rows) ||
-        !encode_act(&tm_hq_full, ws + L.off_hq, L.Rp, L.kbi, dk, L.chunk_rows))
+        !encode_act(&tm_xg, ws + L.off_xg, L.Rp, kbh, dk, kActBoxRows) ||
+        !encode_act(&tm_hq, ws + L.off_hq, L.Rp, kbi, dk, kActBoxRows) ||
+        !encode_act(&tm_xg_full, ws + L.off_xg, L.Rp, kbh, dk, L.chunk_rows) ||
+        !encode_act(&tm_hq_full, ws + L.off_hq, L.Rp, kbi, dk, L.chunk_rows))
         return MOE_ERR_CUDA;
 
     auto record = [&](int i) -> cudaError_t {
@@ -221,13 +258,13 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
     cudaError_t e = record(0);
     if (e == cudaSuccess)
         e = launch_route(topk_idx, static_cast<const uint8_t *>(x_fp8), static_cast<const uint8_t *>(x_sf), T, k, E,
-                         H, ws, L, expert_stats, st);
+                         H, ws, L, expert_stats, nvfp4, st);
     if (e == cudaSuccess) e = record(1);
     if (e == cudaSuccess)
-        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, rowmajor, ws, L, H, I, grid1, st, act);
+        e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, rowmajor, ws, L, H, I, grid1, st, act, nvfp4);
     if (e == cudaSuccess) e = record(2);
     if (e == cudaSuccess)
-        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, rowmajor, ws, L, H, I, grid2, st, act);
+        e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, rowmajor, ws, L, H, I, grid2, st, act, nvfp4);
     if (e == cudaSuccess) e = record(3);
     if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
     if (e == cudaSuccess) e = record(4);
@@ -403,7 +440,83 @@ moe_status_t moe_forward_weights(const void *x_fp8, const void *x_sf, const int6
     s = use_device_of(workspace);
     if (s != MOE_OK) return s;
     return run_layer(x_fp8, x_sf, topk_idx, topk_w, w, out_bf16, T, E, k, H, I, static_cast<uint8_t *>(workspace),
-                     expert_stats, stage_events, stream, act);
+                     expert_stats, stage_events, stream, act, false);
+}
+
+// ---------------------------------------------------------------- NVFP4 variant
+static moe_status_t check_shape_nv(int E, int H, int I) {
+    const moe_status_t s = check_shape(E, H, I);
+    if (s != MOE_OK) return s;
+    return (H % kNvTileK || I % kNvTileK) ? MOE_ERR_UNSUPPORTED_SHAPE : MOE_OK;
+}
+
+moe_status_t moe_quantize_nvfp4(const void *x, int64_t rows, int64_t cols, void *q, void *sf, moe_stream_t stream) {
+    if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return MOE_OK;
+    if (!x || !q || !sf || !aligned(x, 16) || !aligned(q, 8)) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = use_device_of(q);
+    if (s != MOE_OK) return s;
+    return cuda_status(launch_quantize_nvfp4(x, rows, cols, q, sf, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_transformed_weight_bytes_nvfp4(int E, int H, int I, size_t *l1_bytes, size_t *l2_bytes) {
+    const moe_status_t s = check_shape_nv(E, H, I);
+    if (s != MOE_OK) return s;
+    // L1: (I/128 gate/up tile pairs) x (H/256 K tiles) x 2; L2: (H/256 tile pairs) x (I/256 K tiles) x 2
+    if (l1_bytes) *l1_bytes = size_t(E) * size_t(I / kTileRows) * size_t(H / kNvTileK) * 2 * kNvPacketBytes;
+    if (l2_bytes) *l2_bytes = size_t(E) * size_t(H / (2 * kTileRows)) * size_t(I / kNvTileK) * 2 * kNvPacketBytes;
+    return MOE_OK;
+}
+
+moe_status_t moe_transform_weights_nvfp4(const void *l1, const void *l1_sf, const void *l2, const void *l2_sf,
+                                         int E, int H, int I, void *l1_t, void *l2_t, moe_stream_t stream) {
+    const moe_status_t s = check_shape_nv(E, H, I);
+    if (s != MOE_OK) return s;
+    if (!l1 || !l1_sf || !l2 || !l2_sf || !l1_t || !l2_t) return MOE_ERR_INVALID_ARG;
+    if (!aligned(l1, 16) || !aligned(l2, 16) || !aligned(l1_sf, 4) || !aligned(l2_sf, 4) || !aligned(l1_t, 256) ||
+        !aligned(l2_t, 256))
+        return MOE_ERR_INVALID_ARG;
+    const moe_status_t d = use_device_of(l1_t);
+    if (d != MOE_OK) return d;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_transform_nv(l1, l1_sf, E, 2 * I, H, I / kTileRows, false, I, l1_t, st);
+    if (e == cudaSuccess) e = launch_transform_nv(l2, l2_sf, E, H, I, H / (2 * kTileRows), true, 0, l2_t, st);
+    return cuda_status(e);
+}
+
+moe_status_t moe_forward_nvfp4(const void *x_fp4, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
+                               const void *l1_t, const void *l2_t, void *out_bf16, int T, int E, int k, int H, int I,
+                               void *workspace, size_t ws_bytes, int32_t *expert_stats, void *const *stage_events,
+                               const moe_activation_t *activation, moe_stream_t stream) {
+    moe_activation_t act = {MOE_ACT_SWIGLU, 1.0f, 0.0f};
+    if (activation) {
+        act = *activation;
+        if (act.kind == MOE_ACT_SITU) {
+            if (!(act.beta > 0.0f) || !isfinite(act.beta) || !(act.linear_beta >= 0.0f) || !isfinite(act.linear_beta))
+                return MOE_ERR_INVALID_ARG;
+        } else if (act.kind != MOE_ACT_SWIGLU) {
+            return MOE_ERR_INVALID_ARG;
+        }
+    }
+    moe_status_t s = check_shape_nv(E, H, I);
+    if (s != MOE_OK) return s;
+    if (T < 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+    if (int64_t(T) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!x_fp4 || !x_sf || !topk_idx || !topk_w || !l1_t || !l2_t || !out_bf16 || !workspace)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_fp4, 16) || !aligned(x_sf, 4) || !aligned(topk_idx, 8) || !aligned(topk_w, 4) ||
+        !aligned(l1_t, 256) || !aligned(l2_t, 256) || !aligned(out_bf16, 16) || !aligned(workspace, 256) ||
+        (expert_stats && !aligned(expert_stats, 4)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, E, k, H, I);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    const moe_weights_t w = {MOE_LAYOUT_PACKETS, l1_t, nullptr, l2_t, nullptr};
+    return run_layer(x_fp4, x_sf, topk_idx, topk_w, w, out_bf16, T, E, k, H, I, static_cast<uint8_t *>(workspace),
+                     expert_stats, stage_events, stream, act, true);
 }
 
 moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H, int I, int32_t *count,

@@ -38,19 +38,27 @@ namespace moe {
 // tiles.  Each tile has its own accumulator and its own MMA-issuing warp, since
 // every tcgen05.mma / tcgen05.cp costs a fixed issue slot whatever its N.
 // Small-batch launches (kN = 32) take 256-K stages.
-template <bool kGemm1, int kN>
+//
+// kNv: the NVFP4 variant.  A "K block" is always 128 bytes of an operand row
+// in shared memory: 128 FP8 elements (or 128 FP4 expanded to bytes) in the
+// FP8 x FP4 path, 256 packed E2M1 elements in the NVFP4 path, so the tiles,
+// boxes and swizzle are the same; NVFP4 has four scale images per K block
+// (one per 64-K MMA step) instead of one, and 256-K stages throughout.
+template <bool kGemm1, int kN, bool kNv = false>
 struct GemmCfg {
     static constexpr bool kSmall = kN == kChunkRowsSmall;
     static constexpr int kNumA = 2;                     // weight tiles (accumulators, issuers) per item
-    static constexpr int kKB = kSmall ? 2 : 1;          // 128-K blocks per pipeline stage
+    static constexpr int kKB = kNv ? 1 : (kSmall ? 2 : 1);  // K blocks per pipeline stage
     static constexpr int kIssuers = 2;
-    static constexpr int kStages = kSmall ? 3 : 4;
-    static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 one-byte elements
+    static constexpr int kStages = kNv ? (kSmall ? 5 : 3) : (kSmall ? 3 : 4);
+    static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 bytes
     static constexpr int kBTile = kN * kTileK;          // token rows x 128 bytes, per K block
     static constexpr int kStageTiles = kNumA * kKB * kATile + kKB * kBTile;
-    static constexpr int kActSf = act_sf_bytes(kN);     // activation scale bytes per K block
+    static constexpr int kActSf = act_sf_bytes(kN);     // one activation scale image set (all rows)
     static constexpr int kSfbImages = kActSf / kSfBlockBytes;
-    static constexpr int kStageSf = kNumA * kKB * kSfBlockBytes + kKB * kActSf;
+    static constexpr int kImg = kNv ? kNvImages : 1;    // scale image sets per K block
+    static constexpr int kStageSf = kImg * (kNumA * kKB * kSfBlockBytes + kKB * kActSf);
+    static constexpr int kWTx = kNv ? kNvPacketBytes : kPacketBytes;  // copy bytes per weight packet
     static constexpr int kSmemTiles = kStages * kStageTiles;
     static constexpr int kSmemSf = kStages * kStageSf;
     static constexpr int kSmemMisc = 256;
@@ -62,9 +70,12 @@ struct GemmCfg {
     static constexpr int kEpiStage = kStaged ? kEpiWarpsC * 1024 : 0;
     static constexpr int kSmemBytes = 1024 + kSmemTiles + kSmemSf + kSmemMisc + kEpiStage;
     static constexpr int kAccCols = kNumA * kN;          // one accumulator buffer
-    // per issuer and stage: its weight tile's and the activations' scale images
-    static constexpr int kSfColsIssuer = kKB * (1 + kSfbImages) * 4;
-    static constexpr int kSfCols = kStages * kIssuers * kSfColsIssuer;
+    // per issuer and stage: its weight tile's and the activations' scale images;
+    // NVFP4 keeps two such regions per issuer (not one per stage) to fit TMEM,
+    // the issuer waiting for the MMAs two stages back before reusing one
+    static constexpr int kSfColsIssuer = kKB * kImg * (1 + kSfbImages) * 4;
+    static constexpr int kSfRegions = kNv ? 2 : kStages;
+    static constexpr int kSfCols = kSfRegions * kIssuers * kSfColsIssuer;
     static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
@@ -107,6 +118,29 @@ struct GemmArgs {
     float lbeta, inv_lbeta;
 };
 
+// After the call lane l holds, over the 16 lanes of its half-warp, the max of
+// a[l % 16] in ra and of a[16 + l % 16] in rb (the arrays are consumed): the
+// transposing butterfly below without its stage across half-warps, on the two
+// 16-token halves side by side.
+__device__ __forceinline__ void halfwarp_transpose_max(float (&a)[32], int lane, float &ra, float &rb) {
+#pragma unroll
+    for (int s = 8; s >= 1; s >>= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < s; ++i) {
+#pragma unroll
+            for (int h = 0; h < 32; h += 16) {
+                const float send = upper ? a[h + i] : a[h + i + s];
+                const float recv = __shfl_xor_sync(0xFFFFFFFFu, send, s);
+                const float keep = upper ? a[h + i + s] : a[h + i];
+                a[h + i] = fmaxf(keep, recv);
+            }
+        }
+    }
+    ra = a[0];
+    rb = a[16];
+}
+
 // After the call lane l holds max over the warp's lanes of a[l] (the input
 // arrays are consumed): 31 shuffles instead of 32 five-step all-reduces.
 __device__ __forceinline__ float warp_transpose_max(float (&a)[32], int lane) {
@@ -124,12 +158,12 @@ __device__ __forceinline__ float warp_transpose_max(float (&a)[32], int lane) {
     return a[0];
 }
 
-template <bool kGemm1, int kN>
-__global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
+template <bool kGemm1, int kN, bool kNv>
+__global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_wsf,
                     const __grid_constant__ CUtensorMap tmap_act, const __grid_constant__ CUtensorMap tmap_act_full,
                     const GemmArgs args) {
-    using C = GemmCfg<kGemm1, kN>;
+    using C = GemmCfg<kGemm1, kN, kNv>;
     constexpr int kNumA = C::kNumA, kKB = C::kKB, kStages = C::kStages, kBufs = C::kAccBufs;
     constexpr int kIssuers = C::kIssuers;
     extern __shared__ uint8_t smem_raw[];
@@ -182,7 +216,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
 
     const int n_tiles = args.n_tiles, n_items = args.n_items;
     const int num_items = __ldcg(args.hdr + kHdrNumChunks) * n_items;
-    const int KB = args.K / kTileK;
+    const int KB = args.K / (kNv ? kNvTileK : kTileK);  // K blocks of 128 operand bytes
     const int n_steps = (KB + kKB - 1) / kKB;  // pipeline stages per item
     int *err = args.hdr;
 
@@ -221,22 +255,29 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     if (weights) {
                         // a box always moves kBoxPackets packets (a last odd K
                         // block loads packets it then ignores)
-                        mbar_arrive_expect_tx(&full[stage], uint32_t(kNumA * kKB * (kPacketBody + kPacketSf)));
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(kNumA * kKB * C::kWTx));
                         // 4D box (128 K, 128 rows, tile a, K block b) lands as slots b * 2 + a
                         const int pkt = int((int64_t(ch.x) * groups + it) * KB * 2 + int64_t(kb0) * 2);
-                        if (args.w_rowmajor)
-                            tma_load_4d(st, &tmap_w, &full[stage], 0,
-                                        ch.x * args.w_rows_per_expert + it * args.w_item_rows, 0, kb0, pol);
-                        else
+                        if (kNv) {
+                            // packed E2M1 bodies as bytes; scale images (128 words, image, packet)
                             tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol);
-                        tma_load_2d(sf, &tmap_wsf, &full[stage], args.w_sf_x0, pkt, pol);
+                            tma_load_3d(sf, &tmap_wsf, &full[stage], 0, 0, pkt, pol);
+                        } else {
+                            if (args.w_rowmajor)
+                                tma_load_4d(st, &tmap_w, &full[stage], 0,
+                                            ch.x * args.w_rows_per_expert + it * args.w_item_rows, 0, kb0, pol);
+                            else
+                                tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol);
+                            tma_load_2d(sf, &tmap_wsf, &full[stage], args.w_sf_x0, pkt, pol);
+                        }
                     } else {
                         // the activation box always moves kKB K blocks (a K
                         // block past the end reads zeros); a nearly full large
                         // chunk takes one kN-row box instead of several 32-row ones
                         const bool one_box = !C::kSmall && ch.z > kN - 64;
                         const int rows_moved = one_box ? kN : nbox * kActBoxRows;
-                        mbar_arrive_expect_tx(&full[stage], uint32_t(rows_moved * kKB * kTileK + nkb * C::kActSf));
+                        mbar_arrive_expect_tx(&full[stage],
+                                              uint32_t(rows_moved * kKB * kTileK + nkb * C::kImg * C::kActSf));
                         uint8_t *bt = st + kNumA * kKB * C::kATile;
                         if (one_box) {
                             tma_load_3d(bt, &tmap_act_full, &full[stage], 0, ch.y, kb0, pol);
@@ -245,9 +286,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                                 tma_load_3d(bt + j * kActBoxRows * kTileK, &tmap_act, &full[stage], 0,
                                             ch.y + j * kActBoxRows, kb0, pol);
                         }
-                        bulk_load(sf + kNumA * kKB * kSfBlockBytes,
-                                  args.act_sf + (int64_t(c) * KB + kb0) * C::kActSf, nkb * C::kActSf,
-                                  &full[stage], pol);
+                        bulk_load(sf + C::kImg * kNumA * kKB * kSfBlockBytes,
+                                  args.act_sf + (int64_t(c) * KB + kb0) * C::kImg * C::kActSf,
+                                  nkb * C::kImg * C::kActSf, &full[stage], pol);
                     }
                     filled |= 1u << stage;
                     fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
@@ -274,7 +315,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
             const int a = issuer;
             int stage = 0;
             uint32_t phase = 0;
-            int li = 0;  // items handled by this CTA so far
+            int li = 0;        // items handled by this CTA so far
+            int gstage = 0;    // stages consumed so far (all items)
             bool ok = true;
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++li) {
                 const int4 ch = __ldcg(args.chunks + item / n_items);
@@ -294,7 +336,41 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    if (valid) {
+                    if (kNv && valid && gstage >= 2) {
+                        // this issuer's scale region was last read by the MMAs of stage
+                        // gstage - 2: their commit has completed that stage's `empty` phase
+                        const int g2 = gstage - 2;
+                        if (!mbar_wait(&empty[g2 % kStages], uint32_t(g2 / kStages) & 1u, abort_flag, err, 6)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    if (kNv && valid) {
+                        const uint8_t *st = tiles + stage * C::kStageTiles;
+                        const uint8_t *sfa = sfs + stage * C::kStageSf;           // [tile][image][512]
+                        const uint8_t *sfb = sfa + kNumA * kNvImages * kSfBlockBytes;  // [image][kActSf]
+                        const uint8_t *bt = st + kNumA * C::kATile;
+                        const uint32_t col = tmem + uint32_t(kBufs * C::kAccCols +
+                                                             ((gstage & 1) * kIssuers + a) * C::kSfColsIssuer);
+                        const uint32_t colb = col + kNvImages * 4;
+#pragma unroll
+                        for (int sI = 0; sI < kNvImages; ++sI) {
+                            tc_cp_sf(col + sI * 4, smem_desc_sf(smem_u32(sfa + (a * kNvImages + sI) * kSfBlockBytes)));
+#pragma unroll
+                            for (int im = 0; im < C::kSfbImages; ++im)
+                                tc_cp_sf(colb + (sI * C::kSfbImages + im) * 4,
+                                         smem_desc_sf(smem_u32(sfb + sI * C::kActSf + im * kSfBlockBytes)));
+                        }
+                        const uint64_t adesc = smem_desc_sw128(smem_u32(st + a * C::kATile));
+                        const uint64_t bdesc = smem_desc_sw128(smem_u32(bt));
+#pragma unroll
+                        for (int ks = 0; ks < kNvImages; ++ks)
+                            // 64 K (32 bytes) per step inside the 128-byte swizzled row, one image each
+                            tc_mma_nvf4(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks), idesc_nvf4(n),
+                                        col + ks * 4, colb + ks * C::kSfbImages * 4,
+                                        (kb0 == 0 && ks == 0) ? 0u : 1u);
+                    } else if (valid) {
                         const uint8_t *st = tiles + stage * C::kStageTiles;
                         const uint8_t *sfa = sfs + stage * C::kStageSf;
                         const uint8_t *sfb = sfa + kNumA * kKB * kSfBlockBytes;
@@ -323,6 +399,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         }
                     }
                     tc_commit(&empty[stage]);
+                    ++gstage;
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -383,6 +460,35 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                     }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
+                    if constexpr (kNv) {
+                        // NVFP4: groups of 16 rows of h = the two half-warps.  Lane l
+                        // gets the amax of tokens cb*32 + l%16 and cb*32 + 16 + l%16 over
+                        // its half-warp, and their UE4M3 scale codes.
+                        float amA, amB;
+                        halfwarp_transpose_max(amx, lane, amA, amB);
+                        const uint32_t cA = nvfp4_scale_code(amA), cB = nvfp4_scale_code(amB);
+                        const float sA = e4m3_mag_value(cA), sB = e4m3_mag_value(cB);
+                        // GEMM2 reads h in 256-K blocks: this item's 128 rows are half
+                        // `it % 2` of block it / 2; the warp's 32 rows are groups g4 =
+                        // (q % 2) * 2 + half-warp of image (it % 2) * 2 + q / 2
+                        const int img = (it & 1) * 2 + (q >> 1), g4 = (q & 1) * 2 + (lane >> 4);
+                        uint8_t *sfo = args.out_sf + ((int64_t(c) * (n_tiles / 2) + it / 2) * kNvImages + img) * C::kActSf;
+                        const int tA = cb * 32 + (lane & 15), tB = tA + 16;
+                        if (tA < ch.z) sfo[act_sf_offset(tA, g4)] = uint8_t(cA);
+                        if (tB < ch.z) sfo[act_sf_offset(tB, g4)] = uint8_t(cB);
+                        // codes: row (ch.y + token) of block it / 2 holds this warp's 32
+                        // values as bytes (it % 2) * 64 + q * 16 .. + 15, two per byte
+                        uint8_t *qbase = args.out_q + (int64_t(it >> 1) * args.rows + ch.y) * kTileK + (it & 1) * 64 +
+                                         q * 16 + (lane >> 1);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, (lane & 16) | (j & 15));
+                            const uint32_t code = to_e2m1(__fdiv_rn(h[j], sj));
+                            const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
+                            if (!(lane & 1) && cb * 32 + j < ch.z)
+                                qbase[int64_t(cb * 32 + j) * kTileK] = uint8_t(code | (partner << 4));
+                        }
+                    } else {
                     // lane l: amax of token cb*32+l over this warp's 32 rows of h
                     const float amax = warp_transpose_max(amx, lane);
                     const int e = scale_exponent<true>(amax);
@@ -400,6 +506,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
                         const float mj = __shfl_sync(0xFFFFFFFFu, mult, j);
                         const uint32_t code = to_e4m3(h[j] * mj);
                         if (cb * 32 + j < ch.z) qbase[int64_t(cb * 32 + j) * kTileK + lane] = uint8_t(code);
+                    }
                     }
                 } else {
 #pragma unroll
@@ -451,39 +558,57 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN>::kThreads, 1)
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <bool kGemm1, int kN>
+template <bool kGemm1, int kN, bool kNv>
 static cudaError_t launch_gemm_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf, const CUtensorMap &tmap_act,
                                  const CUtensorMap &tmap_act_full, const GemmArgs &args, int grid,
                                  cudaStream_t stream) {
-    using C = GemmCfg<kGemm1, kN>;
+    using C = GemmCfg<kGemm1, kN, kNv>;
     static int configured_for = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_for != dev) {
-        const cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kGemm1, kN>,
+        const cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kGemm1, kN, kNv>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (e != cudaSuccess) return e;
         configured_for = dev;
     }
-    return launch_pdl(moe_gemm_kernel<kGemm1, kN>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
+    return launch_pdl(moe_gemm_kernel<kGemm1, kN, kNv>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
                       tmap_w, tmap_wsf, tmap_act, tmap_act_full, args);
 }
 
-int gemm_kblocks_per_stage(int chunk_rows) {
-    return chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall>::kKB : GemmCfg<true, kChunkRows>::kKB;
+template <bool kNv>
+static int kblocks_per_stage(int chunk_rows) {
+    return chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall, kNv>::kKB
+                                         : GemmCfg<true, kChunkRows, kNv>::kKB;
 }
 
-int gemm_packets_per_stage(bool gemm1, int chunk_rows) {
-    return gemm1 ? (chunk_rows == kChunkRowsSmall ? GemmCfg<true, kChunkRowsSmall>::kBoxPackets
-                                                  : GemmCfg<true, kChunkRows>::kBoxPackets)
-                 : (chunk_rows == kChunkRowsSmall ? GemmCfg<false, kChunkRowsSmall>::kBoxPackets
-                                                  : GemmCfg<false, kChunkRows>::kBoxPackets);
+int gemm_kblocks_per_stage(int chunk_rows, bool nvfp4) {
+    return nvfp4 ? kblocks_per_stage<true>(chunk_rows) : kblocks_per_stage<false>(chunk_rows);
+}
+
+int gemm_packets_per_stage(bool gemm1, int chunk_rows, bool nvfp4) {
+    // every item owns two tiles; a stage moves both for each of its K blocks
+    (void)gemm1;
+    return 2 * gemm_kblocks_per_stage(chunk_rows, nvfp4);
+}
+
+template <bool kNv>
+static cudaError_t launch_gemm_fmt(bool gemm1, bool small, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
+                                   const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, const GemmArgs &a,
+                                   int grid, cudaStream_t stream) {
+    if (gemm1)
+        return small ? launch_gemm_t<true, kChunkRowsSmall, kNv>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid,
+                                                                 stream)
+                     : launch_gemm_t<true, kChunkRows, kNv>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
+    return small ? launch_gemm_t<false, kChunkRowsSmall, kNv>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid,
+                                                              stream)
+                 : launch_gemm_t<false, kChunkRows, kNv>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
 }
 
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
                         const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, bool w_rowmajor,
                         uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
-                        const moe_activation_t &act) {
+                        const moe_activation_t &act, bool nvfp4) {
     GemmArgs a{};
     a.w_rowmajor = w_rowmajor ? 1 : 0;
     a.w_rows_per_expert = gemm1 ? 2 * I : H;
@@ -496,7 +621,7 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
     a.inv_lbeta = (act.kind == MOE_ACT_SITU && act.linear_beta > 0.0f) ? 1.0f / act.linear_beta : 0.0f;
     a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
     a.hdr = reinterpret_cast<int *>(ws);
-    const bool small = L.chunk_rows == kChunkRowsSmall;
+    a.rows = int(L.Rp);
     if (gemm1) {
         a.act_sf = ws + L.off_xg_sf;
         a.out_q = ws + L.off_hq;
@@ -505,19 +630,17 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
         a.n_tiles = I / kTileRows;
         a.n_items = I / kTileRows;
         a.out_ld = I;
-        a.rows = int(L.Rp);
-        return small ? launch_gemm_t<true, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream)
-                     : launch_gemm_t<true, kChunkRows>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
+    } else {
+        a.act_sf = ws + L.off_hq_sf;
+        a.out_y = reinterpret_cast<__nv_bfloat16 *>(ws + L.off_y);
+        a.K = I;
+        a.n_tiles = H / kTileRows;
+        a.n_items = (H / kTileRows + 1) / 2;
+        a.out_ld = H;
     }
-    a.act_sf = ws + L.off_hq_sf;
-    a.out_y = reinterpret_cast<__nv_bfloat16 *>(ws + L.off_y);
-    a.K = I;
-    a.n_tiles = H / kTileRows;
-    a.n_items = (H / kTileRows + 1) / 2;
-    a.out_ld = H;
-    a.rows = int(L.Rp);
-    return small ? launch_gemm_t<false, kChunkRowsSmall>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream)
-                 : launch_gemm_t<false, kChunkRows>(tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
+    const bool small = L.chunk_rows == kChunkRowsSmall;
+    return nvfp4 ? launch_gemm_fmt<true>(gemm1, small, tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream)
+                 : launch_gemm_fmt<false>(gemm1, small, tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
 }
 
 }  // namespace moe

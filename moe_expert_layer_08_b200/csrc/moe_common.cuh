@@ -100,6 +100,35 @@ __device__ __forceinline__ uint32_t to_e2m1(float v) {
     return (uint32_t(m) & 0xFu) | ((__float_as_uint(v) >> 28) & 0x8u);
 }
 
+// ---------------------------------------------------------------- NVFP4
+// E2M1 values with one UE4M3 scale per 16 K elements.  A K block is 256
+// elements (128 bytes of packed FP4, one 128-byte swizzled shared-memory row),
+// and each of its four 64-K MMA steps takes one 512-byte scale image (4 groups
+// of 16 for 128 rows, the same image layout as above).
+constexpr int kNvTileK = 256;
+constexpr int kNvImages = 4;                                  // scale images per 256-K block
+constexpr int kNvPacketBody = kTileRows * kNvTileK / 2;       // 16384 B
+constexpr int kNvPacketSf = kNvImages * kSfBlockBytes;        // 2048 B
+constexpr int kNvPacketBytes = kNvPacketBody + kNvPacketSf;   // 18432 B
+
+// Value of an E4M3 magnitude code c in [0, 126], exactly.
+__device__ __forceinline__ float e4m3_mag_value(uint32_t c) {
+    const uint32_t e = c >> 3, m = c & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : float(m) * (1.0f / 512.0f);
+}
+
+// NVFP4 scale code of a 16-element group: the smallest UE4M3 value s with
+// 6 * s >= amax (6 * s is exact in fp32), found from a rounded estimate and
+// exact comparisons; amax = 0 gives 1.0 (code 0x38); at most 0x7E (448).
+__device__ __forceinline__ uint32_t nvfp4_scale_code(float amax) {
+    if (!(amax > 0.0f)) return 0x38u;
+    uint32_t c = uint32_t(__nv_cvt_float_to_fp8(amax * (1.0f / 6.0f), __NV_SATFINITE, __NV_E4M3)) & 0x7Fu;
+    if (c == 0u) c = 1u;
+    while (c < 0x7Eu && 6.0f * e4m3_mag_value(c) < amax) ++c;
+    while (c > 1u && 6.0f * e4m3_mag_value(c - 1u) >= amax) --c;
+    return c;
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -258,6 +287,20 @@ __device__ __forceinline__ void tc_mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc,
         : "memory");
 }
 
+// D[M=128, N] (+)= (A * SFA) . (B * SFB)^T with A and B both packed E2M1 and
+// UE4M3 scales per 16 K (K = 64 per instruction; sfa / sfb address the
+// 4-column scale image of this 64-K step).
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // 32 lanes x 32 columns of 32-bit words: thread l of the warp gets lane (base + l).
 __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -294,6 +337,16 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
     d |= uint64_t(128 >> 4) << 32;
     d |= uint64_t(1) << 46;
     return d;
+}
+// Instruction descriptor of kind::mxf4nvf4 block-scaled MMA with 16-element
+// scale vectors: A and B E2M1 (format 1), K-major, M = 128, N = n, UE4M3
+// scales (scale format 0), dense K = 64.
+__device__ __forceinline__ uint32_t idesc_nvf4(uint32_t n) {
+    return (1u << 7)             // A format: E2M1
+           | (1u << 10)          // B format: E2M1
+           | ((n >> 3) << 17)    // N / 8
+           | (0u << 23)          // scale format: UE4M3
+           | ((128u >> 4) << 24);// M / 16
 }
 // Instruction descriptor of kind::mxf8f6f4 block-scaled MMA: A = E2M1 weights,
 // B = E4M3 activations, both K-major, M = 128, N = n, UE8M0 scales, byte `id`

@@ -54,6 +54,9 @@ WsLayout ws_layout(int T, int E, int k, int H, int I);
 // Kernel launchers (all asynchronous on `stream`; return cudaGetLastError()).
 cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, void *q, void *sf, bool fp8,
                             cudaStream_t stream);
+cudaError_t launch_quantize_nvfp4(const void *x, int64_t rows, int64_t cols, void *q, void *sf, cudaStream_t stream);
+cudaError_t launch_transform_nv(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int groups,
+                                bool pairs, int half_rows, void *out, cudaStream_t stream);
 // Tile packets (body + scale block, kPacketBytes each) or, with out_body ==
 // nullptr, only the 512-byte scale blocks in the same order (row-major layout).
 cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_per_expert, int K, int groups,
@@ -63,15 +66,16 @@ cudaError_t launch_transform(const void *w, const void *w_sf, int E, int rows_pe
 // the gather)
 inline int route_kernel_launches(int64_t R) { return R <= kRouteSmallMax ? 2 : 5; }
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
-                         int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream);
+                         int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, bool nvfp4,
+                         cudaStream_t stream);
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
                         const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, bool w_rowmajor,
                         uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
-                        const moe_activation_t &act);
+                        const moe_activation_t &act, bool nvfp4);
 // Weight packets one pipeline stage of that GEMM variant moves (TMA box depth).
-int gemm_packets_per_stage(bool gemm1, int chunk_rows);
-// 128-K blocks one pipeline stage moves (the activation box depth).
-int gemm_kblocks_per_stage(int chunk_rows);
+int gemm_packets_per_stage(bool gemm1, int chunk_rows, bool nvfp4);
+// K blocks (128 operand bytes each) one pipeline stage moves (the activation box depth).
+int gemm_kblocks_per_stage(int chunk_rows, bool nvfp4);
 constexpr int kActBoxRows = 32;  // activation rows per TMA box
 cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
                            void *out, cudaStream_t stream);
@@ -86,6 +90,6 @@ moe_status_t use_device_of(const void *p);
 moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, const float *topk_w,
                        const moe_weights_t &w, void *out_bf16, int T, int E, int k, int H, int I,
                        uint8_t *ws, int32_t *expert_stats, void *const *stage_events, moe_stream_t stream,
-                       const moe_activation_t &act);
+                       const moe_activation_t &act, bool nvfp4);
 
 }  // namespace moe

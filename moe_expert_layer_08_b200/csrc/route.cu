@@ -246,16 +246,19 @@ __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
 // one routed row (the whole row for large batches; pieces of it when there are
 // few rows, so that enough warps run); warps stride over the tasks.  A task's
 // vectors move in batches of 32 lanes x kGatherVec, all loads of a batch issued
-// before its stores; each vector goes to its K block's plane of the K-block-
-// major destination [H/128][Rp][128] (8 lanes fill one 128-byte line).  The
-// first task of a row also copies the row's scale words into the chunk's scale
-// images.
+// before its stores; each vector goes to its column block's plane of the
+// block-major destination [row_bytes/128][Rp][128] (8 lanes fill one 128-byte
+// line).  The first task of a row also copies the row's scale words into the
+// chunk's scale images: FP8 rows (row_bytes = H) have one word (4 groups of
+// 32) per 128-byte block; NVFP4 rows (row_bytes = H/2) four (16 groups of 16),
+// word w of a block going to image w of that block's images.
 constexpr int kGatherThreads = 256;
 constexpr int kGatherVec = 8;
 
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__restrict__ rowinfo,
-                                                                const int *__restrict__ offset, int E, int H,
-                                                                int64_t Rp, int sf_bytes, int segs, int seg_vec,
+                                                                const int *__restrict__ offset, int E,
+                                                                int row_bytes, int sf_words, int64_t Rp, int sf_bytes,
+                                                                int segs, int seg_vec,
                                                                 const uint8_t *__restrict__ x,
                                                                 const uint8_t *__restrict__ x_sf,
                                                                 uint8_t *__restrict__ xg, uint8_t *__restrict__ xg_sf) {
@@ -265,13 +268,13 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__re
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = int64_t(gridDim.x) * kWarps;
     const int64_t nrows = __ldcg(offset + E);  // dropped slots leave no row
-    const int nvec = H / 16;
-    const int KB = H / kTileK;
+    const int nvec = row_bytes / 16;
+    const int KB = row_bytes / kTileK;  // 128-byte column blocks
     for (int64_t task = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); task < nrows * segs; task += nwarps) {
         const int64_t pos = task / segs;
         const int seg = int(task % segs);
         const int4 ri = __ldcg(rowinfo + pos);
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + int64_t(ri.x) * H);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + int64_t(ri.x) * row_bytes);
         const int vend = (seg + 1) * seg_vec < nvec ? (seg + 1) * seg_vec : nvec;
         for (int base = seg * seg_vec; base < vend; base += 32 * kGatherVec) {
             uint4 v[kGatherVec];
@@ -290,16 +293,18 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__re
             }
         }
         if (seg != 0) continue;
-        const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * (H / 32));
-        for (int kb = lane; kb < KB; kb += 32) {
-            uint8_t *blk = xg_sf + (int64_t(ri.y) * KB + kb) * sf_bytes;
-            *reinterpret_cast<uint32_t *>(blk + act_sf_offset(ri.z, 0)) = __ldcg(sfs + kb);
+        const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * KB * sf_words * 4);
+        for (int wi = lane; wi < KB * sf_words; wi += 32) {
+            const int kb = wi / sf_words, img = wi % sf_words;
+            uint8_t *blk = xg_sf + ((int64_t(ri.y) * KB + kb) * sf_words + img) * sf_bytes;
+            *reinterpret_cast<uint32_t *>(blk + act_sf_offset(ri.z, 0)) = __ldcg(sfs + wi);
         }
     }
 }
 
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
-                         int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, cudaStream_t stream) {
+                         int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, bool nvfp4,
+                         cudaStream_t stream) {
     const int R = int(L.R);
     int *hdr = reinterpret_cast<int *>(ws);
     int *hist = reinterpret_cast<int *>(ws + L.off_hist);
@@ -349,7 +354,8 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t warps = int64_t(sms) * 4 * (kGatherThreads / 32);
-    const int nvec = H / 16;
+    const int row_bytes = nvfp4 ? H / 2 : H;
+    const int nvec = row_bytes / 16;
     const int max_segs = (nvec + 31) / 32;
     int64_t segs = (warps + R - 1) / (R > 0 ? R : 1);
     if (segs > max_segs) segs = max_segs;
@@ -359,8 +365,9 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
     const int64_t want = (int64_t(R) * nseg + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
     const int grid = int(want < int64_t(sms) * 4 ? want : int64_t(sms) * 4);
     return launch_pdl(gather_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kGatherThreads), 0, stream,
-                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, H, int64_t(L.Rp),
-                      act_sf_bytes(L.chunk_rows), nseg, seg_vec, x, x_sf, ws + L.off_xg, ws + L.off_xg_sf);
+                      static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, row_bytes,
+                      nvfp4 ? kNvImages : 1, int64_t(L.Rp), act_sf_bytes(L.chunk_rows), nseg, seg_vec, x, x_sf,
+                      ws + L.off_xg, ws + L.off_xg_sf);
 }
 
 }  // namespace moe

@@ -81,5 +81,5 @@ extern "C" moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf, 
     const moe_activation_t swiglu = {MOE_ACT_SWIGLU, 1.0f, 0.0f};
     const moe_weights_t w = {MOE_LAYOUT_PACKETS, l1_t, nullptr, l2_t, nullptr};
     return run_layer(x_fp8, x_sf, topk_idx, topk_w, w, out_bf16, T, E, k, H, I, ws, expert_stats, stage_events,
-                     stream, swiglu);
+                     stream, swiglu, false);
 }

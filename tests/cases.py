@@ -101,3 +101,46 @@ def compare_rows(got: torch.Tensor, ref_bits: np.ndarray, what: str = ""):
     assert worst <= REL_L2_TOL, f"{what}: worst row rel L2 {worst:.3e}"
     assert (float(mabs.max()) if mabs.size else 0.0) <= MAX_ABS_TOL, f"{what}: max abs {mabs.max():.3e}"
     return worst
+
+
+def gpu_layer_nvfp4(w: W.Workload, routing=None, gen_device="cuda", device="cuda"):
+    """NVFP4 inputs of the CUDA path: the same bf16 draws quantised to E2M1 +
+    UE4M3 per 16 and packed by the library."""
+    import moe_expert_layer_08_b200 as moe
+    x = W.gen_x(w, gen_device).to(device)
+    if routing is None:
+        routing = W.gen_routing(w, gen_device)
+    idx, tw = routing[0].to(device).contiguous(), routing[1].to(device).contiguous()
+    xq, xs = moe.quantize_nvfp4(x)
+    n1, n2 = moe.transformed_weight_bytes_nvfp4(w.E, w.H, w.I)
+    l1_t = torch.empty(n1, dtype=torch.uint8, device=device)
+    l2_t = torch.empty(n2, dtype=torch.uint8, device=device)
+    p1, p2 = n1 // w.E, n2 // w.E
+    for e in range(w.E):
+        a, b = moe.quantize_nvfp4(W.gen_l1(w, e, gen_device).to(device))
+        c, d = moe.quantize_nvfp4(W.gen_l2(w, e, gen_device).to(device))
+        moe.transform_weights_nvfp4(a[None], b[None], c[None], d[None],
+                                    out=(l1_t[e * p1:(e + 1) * p1], l2_t[e * p2:(e + 1) * p2]))
+    return dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw, l1_t=l1_t, l2_t=l2_t)
+
+
+def oracle_side_nvfp4(w: W.Workload, x_bf16: torch.Tensor, experts, gen_device="cuda"):
+    """Oracle NVFP4 inputs from the same bf16 draws (listed experts only)."""
+    xq, xs = oracle.quantize_nvfp4(x_bf16.float().cpu().numpy())
+    experts = sorted(set(int(e) for e in experts))
+
+    def quant(item):
+        e, l1, l2 = item
+        a, b = oracle.quantize_nvfp4(l1)
+        c, d = oracle.quantize_nvfp4(l2)
+        return e, (a, b, c, d)
+
+    out = {}
+    workers = max(1, min(len(experts), os.cpu_count() or 1))
+    with ThreadPoolExecutor(workers) as pool:
+        futs = [pool.submit(quant, (e, W.gen_l1(w, e, gen_device).float().cpu().numpy(),
+                                    W.gen_l2(w, e, gen_device).float().cpu().numpy())) for e in experts]
+        for f in futs:
+            e, m = f.result()
+            out[e] = m
+    return xq, xs, out

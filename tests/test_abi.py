@@ -155,3 +155,22 @@ def test_layouts_and_scale_transform_validate_on_the_host(moelib):
     assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(1, 256, 0, 256, 256)))) == 1  # row-major, no l1_sf
     assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(1, 256, 300, 256, 256)))) == 1  # misaligned
     assert moelib.moe_forward_weights(*args(ctypes.byref(m.Weights(1, 0, 256, 256, 256)))) == 1  # no body
+
+
+def test_nvfp4_entry_points_validate_on_the_host(moelib):
+    import moe_expert_layer_08_b200 as m
+    a, b = m.transformed_weight_bytes_nvfp4(384, 7168, 3072)
+    assert (a, b) == (384 * 24 * 28 * 2 * 18432, 384 * 28 * 12 * 2 * 18432)
+    n = ctypes.c_size_t()
+    assert moelib.moe_transformed_weight_bytes_nvfp4(8, 384, 256, ctypes.byref(n), ctypes.byref(n)) == 2  # H % 256
+    assert moelib.moe_transformed_weight_bytes_nvfp4(8, 256, 384, ctypes.byref(n), ctypes.byref(n)) == 2  # I % 256
+    p = ctypes.c_void_p(256)
+    assert moelib.moe_quantize_nvfp4(p, 4, 40, p, p, None) == 2               # cols % 16
+    assert moelib.moe_quantize_nvfp4(None, 4, 32, p, p, None) == 1
+    assert moelib.moe_transform_weights_nvfp4(p, p, p, None, 2, 256, 256, p, p, None) == 1
+    args = lambda **kw: [kw.get("x", p), p, p, p, p, p, p, kw.get("T", 4), 8, kw.get("k", 2), kw.get("H", 256), 256,
+                         p, 1 << 30, None, None, None, None]
+    assert moelib.moe_forward_nvfp4(*args(H=384)) == 2
+    assert moelib.moe_forward_nvfp4(*args(k=9)) == 1
+    assert moelib.moe_forward_nvfp4(*args(x=ctypes.c_void_p(264))) == 1      # misaligned x
+    assert moelib.moe_forward_nvfp4(*args(T=0)) == 0
