@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=0, help="override T (with --experts: same rows per expert)")
     p.add_argument("--layout", default="packets", choices=["packets", "rowmajor"],
                    help="weight layout: tile packets, or row-major bodies with separate scale blocks")
+    p.add_argument("--format", default="mx", choices=["mx", "nvfp4"],
+                   help="mx: FP8 activations x FP4 weights, UE8M0 per 32; nvfp4: E2M1 x E2M1, UE4M3 per 16")
     return p.parse_args()
 
 
@@ -59,11 +61,11 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
-def expert_bytes(w):
-    """FP4 + UE8M0 bytes of one expert's L1 and L2 (0.5 + 1/32 byte per weight)."""
-    l1 = 2 * w.I * w.H * 17 // 32
-    l2 = w.H * w.I * 17 // 32
-    return l1, l2
+def expert_bytes(w, fmt="mx"):
+    """FP4 + scale bytes of one expert's L1 and L2: 0.5 + 1/32 byte per weight
+    (UE8M0 per 32), or 0.5 + 1/16 (NVFP4, UE4M3 per 16)."""
+    num, den = (17, 32) if fmt == "mx" else (9, 16)
+    return 2 * w.I * w.H * num // den, w.H * w.I * num // den
 
 
 class ClockSampler:
@@ -128,12 +130,12 @@ def kernel_source_hash() -> str:
     return hashlib.sha256(src).hexdigest()
 
 
-def measured_traffic(w, touched, gemm1: bool):
+def measured_traffic(w, touched, gemm1: bool, fmt="mx"):
     """DRAM bytes per launch of the dominant GEMM from the committed ncu
     capture (scaled by touched experts, which the traffic is proportional
     to), or None when the kernel changed since or another variant runs."""
     path = os.path.join(ROOT, "profiles", "gemm_decode_traffic.json")
-    if not os.path.exists(path) or w.T * w.k > 8 * w.E:
+    if not os.path.exists(path) or w.T * w.k > 8 * w.E or fmt != "mx":
         return None
     d = json.load(open(path))
     if d.get("kernel_source_sha256") != kernel_source_hash():
@@ -153,14 +155,27 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
-def build_layer(w, device, layout="packets"):
+def build_layer(w, device, layout="packets", fmt="mx"):
     """Seeded bf16 draws quantised and laid out by the CUDA library, resident in
-    HBM: tile packets (l1_t, l2_t) or row-major bodies + scale blocks (rm)."""
+    HBM: tile packets (l1_t, l2_t) or row-major bodies + scale blocks (rm);
+    fmt "nvfp4": NVFP4 activations and packets."""
     import moe_expert_layer_08_b200 as moe
     x = W.gen_x(w, device)
     idx, tw = W.gen_routing(w, device)
-    xq, xs = moe.quantize_fp8(x)
     u8 = dict(dtype=torch.uint8, device=device)
+    if fmt == "nvfp4":
+        xq, xs = moe.quantize_nvfp4(x)
+        n1, n2 = moe.transformed_weight_bytes_nvfp4(w.E, w.H, w.I)
+        l1_t, l2_t = torch.empty(n1, **u8), torch.empty(n2, **u8)
+        p1, p2 = n1 // w.E, n2 // w.E
+        for e in range(w.E):
+            a, b = moe.quantize_nvfp4(W.gen_l1(w, e, device))
+            c, d = moe.quantize_nvfp4(W.gen_l2(w, e, device))
+            moe.transform_weights_nvfp4(a[None], b[None], c[None], d[None],
+                                        out=(l1_t[e * p1:(e + 1) * p1], l2_t[e * p2:(e + 1) * p2]))
+        torch.cuda.synchronize()
+        return dict(x=x, xq=xq, xs=xs, idx=idx, tw=tw, l1_t=l1_t, l2_t=l2_t, rm=None)
+    xq, xs = moe.quantize_fp8(x)
     if layout == "packets":
         n1, n2 = moe.transformed_weight_bytes(w.E, w.H, w.I)
         l1_t, l2_t = torch.empty(n1, **u8), torch.empty(n2, **u8)
@@ -188,7 +203,7 @@ def build_layer(w, device, layout="packets"):
     return g
 
 
-def oracle_sample(w, ntok, device):
+def oracle_sample(w, ntok, device, fmt="mx"):
     """Host inputs of the oracle for the first ``ntok`` tokens (oracle-quantised)."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
@@ -196,18 +211,20 @@ def oracle_sample(w, ntok, device):
     idx, tw = W.gen_routing(w, device)
     idx, tw = idx.cpu().numpy(), tw.cpu().numpy()
     tokens = np.arange(min(ntok, w.T), dtype=np.int32)
-    xq, xs = oracle.quantize_e4m3(x.float().cpu().numpy())
+    qx, qw = (oracle.quantize_nvfp4, oracle.quantize_nvfp4) if fmt == "nvfp4" else \
+        (oracle.quantize_e4m3, oracle.quantize_e2m1)
+    xq, xs = qx(x.float().cpu().numpy())
     need = sorted(set(int(e) for e in idx[tokens].ravel()))
 
     def quant(item):
         e, a, b = item
-        return e, oracle.quantize_e2m1(a) + oracle.quantize_e2m1(b)
+        return e, qw(a) + qw(b)
 
     with ThreadPoolExecutor(max(1, min(len(need), os.cpu_count() or 1))) as pool:
         futs = [pool.submit(quant, (e, W.gen_l1(w, e, device).float().cpu().numpy(),
                                     W.gen_l2(w, e, device).float().cpu().numpy())) for e in need]
         experts = dict(f.result() for f in futs)
-    return dict(xq=xq, xs=xs, idx=idx, tw=tw, experts=experts, tokens=tokens)
+    return dict(xq=xq, xs=xs, idx=idx, tw=tw, experts=experts, tokens=tokens, fmt=fmt)
 
 
 def time_oracle(w, s, steps):
@@ -217,7 +234,7 @@ def time_oracle(w, s, steps):
     for _ in range(steps):
         t0 = time.perf_counter()
         oracle.forward(s["xq"], s["xs"], s["idx"], s["tw"], s["experts"], w.E, w.H, w.I,
-                       tokens=s["tokens"], threads=threads)
+                       tokens=s["tokens"], threads=threads, fmt=s["fmt"])
         times.append(time.perf_counter() - t0)
     flops = 2 * len(s["tokens"]) * w.k * 3 * w.H * w.I
     return flops, times, threads
@@ -227,7 +244,7 @@ def run_reference(args, w, rank, world):
     if rank != 0:
         return
     device = "cuda" if torch.cuda.is_available() else "cpu"
-    s = oracle_sample(w, args.cpu_tokens, device)
+    s = oracle_sample(w, args.cpu_tokens, device, args.format)
     flops, times, threads = time_oracle(w, s, args.warmup + args.steps)
     t = float(np.mean(times[args.warmup:])) if args.steps > 0 else float(np.mean(times))
     value = flops / t / 1e12
@@ -252,8 +269,11 @@ def run_b200(args, w, rank, world, local_rank):
         torch.distributed.barrier()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    g = build_layer(w, device, args.layout)
-    layer = moe.MoELayer(g["l1_t"], g["l2_t"], w.E, w.k, w.H, w.I, T_max=w.T, device=device, weights=g["rm"])
+    if args.format == "nvfp4" and args.layout != "packets":
+        raise SystemExit("the NVFP4 variant takes packet weights")
+    g = build_layer(w, device, args.layout, args.format)
+    layer = moe.MoELayer(g["l1_t"], g["l2_t"], w.E, w.k, w.H, w.I, T_max=w.T, device=device, weights=g["rm"],
+                         fmt=args.format)
     out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.NUM_STAGE_EVENTS)]
@@ -332,7 +352,7 @@ def run_b200(args, w, rank, world, local_rank):
         return
     # roofline of the dominant kernel (GEMM1 or GEMM2), timed by the stage events
     touched = len(W.touched_experts(g["idx"].cpu(), w.E))
-    b1, b2 = expert_bytes(w)
+    b1, b2 = expert_bytes(w, args.format)
     g1_ms, g2_ms = float(stage_ms[:, 1].mean()), float(stage_ms[:, 2].mean())
     pk = peaks()
     if g1_ms >= g2_ms:
@@ -340,7 +360,7 @@ def run_b200(args, w, rank, world, local_rank):
     else:
         kname, kms, kbytes = "moe_gemm_kernel<gemm2>", g2_ms, touched * b2
     achieved = kbytes / (kms * 1e-3) / 1e9
-    traffic = measured_traffic(w, touched, g1_ms >= g2_ms)
+    traffic = measured_traffic(w, touched, g1_ms >= g2_ms, args.format)
     roofline = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                 "frac": achieved / pk["hbm"], "peak_source": pk["source"], "algorithmic_bytes": kbytes,
                 "traffic": traffic}
@@ -349,19 +369,24 @@ def run_b200(args, w, rank, world, local_rank):
         # pipe binds as much as HBM; FP8 peak = 2 x measured bf16 (the nominal
         # dense FP8 / bf16 ratio), the block-scaled FP8 x FP4 MMA runs at it
         kflops = 2.0 * w.T * w.k * (2 * w.I if g1_ms >= g2_ms else w.H) * (w.H if g1_ms >= g2_ms else w.I)
-        fp8 = 2.0 * pk["bf16"]
+        # FP8 peak = 2 x measured bf16, FP4 (NVFP4) = 4 x (the nominal dense ratios)
+        fp8 = (2.0 if args.format == "mx" else 4.0) * pk["bf16"]
         tflops = kflops / (kms * 1e-3) / 1e12
         roofline = {"kernel": kname, "bound": "tensor", "achieved": tflops, "peak": fp8, "unit": "TFLOP/s",
-                    "frac": tflops / fp8, "peak_source": pk["source"] + " (2 x bf16)", "algorithmic_flops": kflops,
+                    "frac": tflops / fp8,
+                    "peak_source": pk["source"] + (" (2 x bf16)" if args.format == "mx" else " (4 x bf16)"),
+                    "algorithmic_flops": kflops,
                     "traffic": traffic, "hbm": {"achieved_GBps": achieved, "frac": achieved / pk["hbm"]}}
-    layer_bytes = touched * (b1 + b2) + w.T * w.H * 33 // 32 + w.T * w.k * 12 + w.T * w.H * 2
+    x_bytes = w.T * w.H * 33 // 32 if args.format == "mx" else w.T * w.H * 9 // 16
+    layer_bytes = touched * (b1 + b2) + x_bytes + w.T * w.k * 12 + w.T * w.H * 2
     flops = w.flops
     value = world * flops / (ms * 1e-3) / 1e12
     e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8xfp4 (fp32 accumulate)", "data": "synthetic",
+        "vs_baseline": None, "data": "synthetic",
+        "dtype": "fp8xfp4 (fp32 accumulate)" if args.format == "mx" else "nvfp4 e2m1xe2m1 (fp32 accumulate)",
         "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")},
                    "parallelism": f"replicas x{world}", "weight_layout": args.layout,
                    "l2": "inputs larger than L2 (touched expert weights per step >> 126 MB)"
@@ -376,14 +401,14 @@ def run_b200(args, w, rank, world, local_rank):
                                 "between kernels; the roofline's kernel duration comes from it",
                          "us_per_layer": staged_ms * 1e3},
         "roofline": roofline,
-        "layer_frac_of_fp8_peak": value / world / (2.0 * pk["bf16"]),
+        "layer_frac_of_tensor_peak": value / world / ((2.0 if args.format == "mx" else 4.0) * pk["bf16"]),
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * moe.forward_kernel_launches(w.T, w.E, w.k, w.H, w.I),
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:
-        s = oracle_sample(w, args.cpu_tokens, device)
+        s = oracle_sample(w, args.cpu_tokens, device, args.format)
         cflops, times, threads = time_oracle(w, s, 1)
         line["cpu_baseline"] = {"value": cflops / times[0] / 1e12, "unit": "TFLOP/s", "cores": threads,
                                 "kind": "oracle", "seconds": times[0],
