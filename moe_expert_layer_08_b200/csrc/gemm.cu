@@ -49,7 +49,11 @@ struct GemmCfg {
     static constexpr bool kSmall = kN == kChunkRowsSmall;
     static constexpr int kNumA = 2;                     // weight tiles (accumulators, issuers) per item
     static constexpr int kKB = kNv ? 1 : (kSmall ? 2 : 1);  // K blocks per pipeline stage
-    static constexpr int kIssuers = 2;
+    // issuers per tile: with 32-row chunks and two K blocks per stage, two
+    // threads split each tile's K blocks (even / odd) into two accumulators
+    // that the epilogue adds, halving the tcgen05 issue time per stage
+    static constexpr int kKSplit = (kSmall && kKB == 2) ? 2 : 1;
+    static constexpr int kIssuers = kNumA * kKSplit;
     static constexpr int kStages = kNv ? (kSmall ? 5 : 3) : (kSmall ? 3 : 4);
     static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 bytes
     static constexpr int kBTile = kN * kTileK;          // token rows x 128 bytes, per K block
@@ -65,23 +69,28 @@ struct GemmCfg {
     // GEMM2 with large chunks: each epilogue warp stages 1 KB of bf16 output in
     // shared memory and writes whole row pieces with 16-byte stores instead of
     // 32 two-byte stores per row block (no room with 32-row chunks)
-    static constexpr int kEpiWarpsC = 8;
+    // epilogue warps: two per TMEM lane quarter (alternating 32-token column
+    // blocks) for large chunks; one per quarter for 32-row chunks, which are a
+    // single column block
+    static constexpr int kEpiWarpsC = kSmall ? 4 : 8;
     static constexpr bool kStaged = !kSmall && !kGemm1;
     static constexpr int kEpiStage = kStaged ? kEpiWarpsC * 1024 : 0;
     static constexpr int kSmemBytes = 1024 + kSmemTiles + kSmemSf + kSmemMisc + kEpiStage;
-    static constexpr int kAccCols = kNumA * kN;          // one accumulator buffer
+    static constexpr int kAccCols = kNumA * kKSplit * kN;  // one accumulator buffer
     // per issuer and stage: its weight tile's and the activations' scale images;
     // NVFP4 keeps two such regions per issuer (not one per stage) to fit TMEM,
     // the issuer waiting for the MMAs two stages back before reusing one
-    static constexpr int kSfColsIssuer = kKB * kImg * (1 + kSfbImages) * 4;
+    static constexpr int kSfColsIssuer = (kKB / kKSplit) * kImg * (1 + kSfbImages) * 4;
     static constexpr int kSfRegions = kNv ? 2 : kStages;
     static constexpr int kSfCols = kSfRegions * kIssuers * kSfColsIssuer;
     static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
-    static constexpr int kEpiWarps = kEpiWarpsC;  // two per TMEM lane quarter, alternating 32-token column blocks
-    static constexpr int kThreads = 32 * (4 + kEpiWarps);  // producers (2), issuers (2), epilogue
+    static constexpr int kEpiWarps = kEpiWarpsC;
+    // warps: 0 weight producer, 6 activation producer, 1 / 7 / (8, 9) issuers,
+    // 2-5 / (8-11) epilogue
+    static constexpr int kThreads = 32 * (kEpiWarps == 8 ? 12 : (kIssuers == 4 ? 10 : 8));
     // weight packets one TMA box moves: an item's two tiles are adjacent for
     // every K tile (gate/up for GEMM1, a tile pair for GEMM2)
     static constexpr int kBoxPackets = kNumA * kKB;
@@ -89,6 +98,8 @@ struct GemmCfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kBTile % 1024 == 0, "swizzle atoms");
     static_assert(kKB == 1 || kN == kActBoxRows, "one activation box per stage when a stage spans K blocks");
+    static_assert(kEpiWarps == 8 || kN <= 32, "one epilogue warp per quarter covers one column block");
+    static_assert(!(kEpiWarps == 8 && kIssuers == 4), "warps 8-11 are either epilogue or issuers");
 };
 
 // Shared-memory slot of weight tile a (0, 1) of K block b within a stage:
@@ -175,7 +186,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     uint64_t *tmem_full = empty + kStages;   // [2]
     uint64_t *tmem_empty = tmem_full + 2;    // [2]
     uint64_t *mma_done = tmem_empty + 2;     // [kIssuers]
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 2);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     uint8_t *epi_stage = reinterpret_cast<uint8_t *>(full) + C::kSmemMisc;  // [kEpiWarps][1024] (large chunks)
 
@@ -189,7 +200,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             mbar_init(&tmem_full[b], kIssuers);
             mbar_init(&tmem_empty[b], C::kEpiWarps);
         }
-        for (int i = 0; i < 2; ++i) mbar_init(&mma_done[i], 1);
+        for (int i = 0; i < kIssuers; ++i) mbar_init(&mma_done[i], 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
@@ -221,7 +232,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     int *err = args.hdr;
 
     // which MMA issuer this warp is (-1: none)
-    const int issuer = warp == 1 ? 0 : warp == 7 ? 1 : -1;
+    const int issuer = warp == 1 ? 0 : warp == 7 ? 1 : (kIssuers == 4 && warp == 8) ? 2
+                     : (kIssuers == 4 && warp == 9) ? 3 : -1;
 
     if (warp == 0 || warp == 6) {
         if (lane == 0) {
@@ -311,8 +323,10 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     } else if (issuer >= 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ MMA issuer
-            // Issuer a owns weight tile a of every item and its accumulator.
-            const int a = issuer;
+            // Issuer (a, h) owns weight tile a of every item and, for K split
+            // h of kKSplit, its accumulator: the stage's K blocks b with
+            // b % kKSplit == h.
+            const int a = issuer % kNumA, h = issuer / kNumA;
             int stage = 0;
             uint32_t phase = 0;
             int li = 0;        // items handled by this CTA so far
@@ -327,7 +341,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 const uint32_t use = uint32_t(li / kBufs) & 1u;  // how often this buffer was used, mod 2
                 if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 2)) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + uint32_t(buf * C::kAccCols + a * kN);
+                const uint32_t acc = tmem + uint32_t(buf * C::kAccCols + (h * kNumA + a) * kN);
                 for (int step = 0; step < n_steps; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
@@ -352,7 +366,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         const uint8_t *sfb = sfa + kNumA * kNvImages * kSfBlockBytes;  // [image][kActSf]
                         const uint8_t *bt = st + kNumA * C::kATile;
                         const uint32_t col = tmem + uint32_t(kBufs * C::kAccCols +
-                                                             ((gstage & 1) * kIssuers + a) * C::kSfColsIssuer);
+                                                             ((gstage & 1) * kIssuers + issuer) * C::kSfColsIssuer);
                         const uint32_t colb = col + kNvImages * 4;
 #pragma unroll
                         for (int sI = 0; sI < kNvImages; ++sI) {
@@ -376,8 +390,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         const uint8_t *sfb = sfa + kNumA * kKB * kSfBlockBytes;
                         const uint8_t *bt = st + kNumA * kKB * C::kATile;
                         uint32_t col =
-                            tmem + uint32_t(kBufs * C::kAccCols + (stage * kIssuers + a) * C::kSfColsIssuer);
+                            tmem + uint32_t(kBufs * C::kAccCols + (stage * kIssuers + issuer) * C::kSfColsIssuer);
                         for (int b = 0; b < nkb; ++b) {
+                            if (b % C::kKSplit != h) continue;
                             const int slot = a_slot(a, b);
                             // scale images of this K block into TMEM: weight tile, then activations
                             tc_cp_sf(col, smem_desc_sf(smem_u32(sfa + slot * kSfBlockBytes)));
@@ -393,7 +408,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                                 // +32 bytes of K per step inside the 128-byte swizzled row
                                 tc_mma_mxf8f6f4(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks),
                                                 idesc_mxf8f6f4(n, uint32_t(ks)), col, sfb_col,
-                                                (kb0 + b == 0 && ks == 0) ? 0u : 1u);
+                                                (kb0 + b == h && ks == 0) ? 0u : 1u);
                             }
                             col += uint32_t((1 + C::kSfbImages) * 4);
                         }
@@ -409,16 +424,19 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 tc_commit(&tmem_full[buf]);
             }
             // All issued MMAs must be finished before TMEM is released.
-            tc_commit(&mma_done[a]);
+            tc_commit(&mma_done[issuer]);
             const unsigned long long t0 = global_timer_ns();
-            while (!mbar_try_wait(&mma_done[a], 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+            while (!mbar_try_wait(&mma_done[issuer], 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
             }
         }
         __syncwarp();
-    } else if ((warp >= 2 && warp <= 5) || warp >= 8) {
+    } else if ((warp >= 2 && warp <= 5) || (C::kEpiWarps == 8 && warp >= 8)) {
         // ---------------------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int half = warp >= 8 ? 1 : 0;     // which column blocks of the quarter it handles
+        constexpr int kCbStep = C::kEpiWarps / 4;
+        // with K split, accumulator h * kNumA + a holds tile a's K blocks of parity h
+        const bool add_split = C::kKSplit == 2 && KB > 1;
         uint8_t *my_stage = epi_stage + (warp < 8 ? warp - 2 : warp - 4) * 1024;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int li = 0;
@@ -431,12 +449,23 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             tc_fence_after();
             const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
             const int ncb = (ch.z + 31) / 32;
-            for (int cb = half; cb < ncb; cb += 2) {
+            for (int cb = half; cb < ncb; cb += kCbStep) {
                 if constexpr (kGemm1) {
                     uint32_t g[32], u[32];
                     tmem_ld_32x32(acc + uint32_t(cb * 32), g);
                     tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
                     tmem_ld_wait();
+                    if (add_split) {
+                        uint32_t g1[32], u1[32];
+                        tmem_ld_32x32(acc + uint32_t(2 * kN + cb * 32), g1);
+                        tmem_ld_32x32(acc + uint32_t(3 * kN + cb * 32), u1);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g1[j]));
+                            u[j] = __float_as_uint(__uint_as_float(u[j]) + __uint_as_float(u1[j]));
+                        }
+                    }
                     float h[32], amx[32];
                     if (args.act_kind == MOE_ACT_SWIGLU) {
 #pragma unroll
@@ -516,6 +545,14 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         uint32_t g[32];
                         tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), g);
                         tmem_ld_wait();
+                        if (add_split) {
+                            uint32_t g1[32];
+                            tmem_ld_32x32(acc + uint32_t((kNumA + a) * kN + cb * 32), g1);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g1[j]));
+                        }
                         __nv_bfloat16 *ybase = args.out_y + int64_t(ch.y + cb * 32) * args.out_ld + tile * kTileRows + q * 32;
                         if constexpr (C::kStaged) {
                             // two passes of 16 rows: stage [row][32 columns] bf16 (1 KB), then
