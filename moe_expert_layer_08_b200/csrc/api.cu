@@ -53,6 +53,7 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.off_hq = take(size_t(L.Rp) * size_t(L.kbi) * kTileK);
     L.off_hq_sf = take(2 * sf_per_kb * size_t(I / kTileK));
     L.off_y = take(R * size_t(H) * 2);
+    L.off_part = take(size_t(kMaxSplitUnits) * kPartUnitFloats * sizeof(float));
     L.total = o;
     return L;
 }

@@ -96,6 +96,8 @@ struct GemmCfg {
     static constexpr int kBoxPackets = kNumA * kKB;
     static_assert(kTmemUsed <= 512, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(8 * (2 * kStages + 10) + 12 <= kSmemMisc, "barriers and flags");
+    static_assert(!kSmall || kN * kNumA * kTileRows == kPartUnitFloats, "split-unit partial size");
     static_assert(kBTile % 1024 == 0, "swizzle atoms");
     static_assert(kKB == 1 || kN == kActBoxRows, "one activation box per stage when a stage spans K blocks");
     static_assert(kEpiWarps == 8 || kN <= 32, "one epilogue warp per quarter covers one column block");
@@ -124,6 +126,8 @@ struct GemmArgs {
     int n_items;               // items per chunk (GEMM1: I/128, GEMM2: tile pairs)
     int out_ld;                // row length of the output (I or H)
     int rows;                  // row extent of the K-block-major FP8 operands
+    float *part;               // 32-row chunks: fp32 partial accumulators of split units [unit][tile][32][128]
+    int *split_cnt;            // per leftover item: split units finished (reset by the last)
     int act_kind;              // GEMM1: MOE_ACT_SWIGLU or MOE_ACT_SITU
     float beta, inv_beta;      // SiTU coefficients (inv_lbeta = 0: no linear coefficient)
     float lbeta, inv_lbeta;
@@ -169,6 +173,55 @@ __device__ __forceinline__ float warp_transpose_max(float (&a)[32], int lane) {
     return a[0];
 }
 
+// Work of one CTA.  Items are dealt round-robin; with 32-row chunks the items
+// of an incomplete last round ("leftover" items) are instead cut along K into
+// `split` units of whole stages, one unit per CTA, so that the last round
+// keeps most SMs streaming weights.  Each unit writes its fp32 partial
+// accumulators; the last unit of an item to finish (a per-item counter) adds
+// all partials in unit order and runs the epilogue.  No CTA waits for another.
+struct WorkPlan {
+    int n_whole;     // whole items: blockIdx.x + k * gridDim.x for k < n_whole
+    int split;       // units per leftover item (0: no split)
+    int first_left;  // first leftover item
+    int unit;        // this CTA's unit (-1: none): item first_left + unit / split, part unit % split
+};
+
+__device__ __forceinline__ WorkPlan plan_work(int num_items, int n_steps, bool allow_split) {
+    WorkPlan P;
+    const int G = int(gridDim.x), b = int(blockIdx.x);
+    int whole_end = num_items, split = 0;
+    if (allow_split) {
+        const int rem = num_items % G;
+        if (rem > 0) {
+            int S = (G < kMaxSplitUnits ? G : kMaxSplitUnits) / rem;
+            if (S > n_steps) S = n_steps;
+            if (S >= 2) {
+                split = S;
+                whole_end = num_items - rem;
+            }
+        }
+    }
+    P.n_whole = b < whole_end ? (whole_end - b + G - 1) / G : 0;
+    P.split = split;
+    P.first_left = whole_end;
+    P.unit = (split && b < (num_items - whole_end) * split) ? b : -1;
+    return P;
+}
+
+// Work wk of the plan: item and stage range [s0, s1).
+__device__ __forceinline__ void work_of(const WorkPlan &P, int wk, int n_steps, int &item, int &s0, int &s1) {
+    if (wk < P.n_whole) {
+        item = int(blockIdx.x) + wk * int(gridDim.x);
+        s0 = 0;
+        s1 = n_steps;
+    } else {
+        const int part = P.unit % P.split;
+        item = P.first_left + P.unit / P.split;
+        s0 = part * n_steps / P.split;
+        s1 = (part + 1) * n_steps / P.split;
+    }
+}
+
 template <bool kGemm1, int kN, bool kNv>
 __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_wsf,
@@ -186,8 +239,11 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     uint64_t *tmem_full = empty + kStages;   // [2]
     uint64_t *tmem_empty = tmem_full + 2;    // [2]
     uint64_t *mma_done = tmem_empty + 2;     // [kIssuers]
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 4);
+    uint64_t *epi_bar = mma_done + 4;        // split unit: epilogue warps' partials written
+    uint64_t *epi_go = epi_bar + 1;          // split unit: the finishing decision taken
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(epi_go + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    volatile int *epi_last = abort_flag + 1;
     uint8_t *epi_stage = reinterpret_cast<uint8_t *>(full) + C::kSmemMisc;  // [kEpiWarps][1024] (large chunks)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -201,6 +257,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             mbar_init(&tmem_empty[b], C::kEpiWarps);
         }
         for (int i = 0; i < kIssuers; ++i) mbar_init(&mma_done[i], 1);
+        mbar_init(epi_bar, C::kEpiWarps);
+        mbar_init(epi_go, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
@@ -229,6 +287,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     const int num_items = __ldcg(args.hdr + kHdrNumChunks) * n_items;
     const int KB = args.K / (kNv ? kNvTileK : kTileK);  // K blocks of 128 operand bytes
     const int n_steps = (KB + kKB - 1) / kKB;  // pipeline stages per item
+    const WorkPlan P = plan_work(num_items, n_steps, C::kSmall);
+    const int n_works = P.n_whole + (P.unit >= 0 ? 1 : 0);
     int *err = args.hdr;
 
     // which MMA issuer this warp is (-1: none)
@@ -247,7 +307,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             uint32_t phase = 0;
             uint32_t filled = 0, fill_parity = 0;
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
+            for (int wk = 0; ok && wk < n_works; ++wk) {
+                int item, s0, s1;
+                work_of(P, wk, n_steps, item, s0, s1);
                 const int c = item / n_items, it = item % n_items;
                 const int4 ch = __ldcg(args.chunks + c);
                 const int nbox = (ch.z + kActBoxRows - 1) / kActBoxRows;
@@ -255,7 +317,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 // GEMM2: tiles 2*it and 2*it+1 (the second may not exist)
                 // packet group of the item: gate/up pair `it` (GEMM1) or tile pair `it` (GEMM2)
                 const int groups = kGemm1 ? n_tiles : n_items;
-                for (int step = 0; step < n_steps; ++step) {
+                for (int step = s0; step < s1; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, weights ? 1 : 5)) {
@@ -332,7 +394,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             int li = 0;        // items handled by this CTA so far
             int gstage = 0;    // stages consumed so far (all items)
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++li) {
+            for (int wk = 0; ok && wk < n_works; ++wk, ++li) {
+                int item, s0, s1;
+                work_of(P, wk, n_steps, item, s0, s1);
                 const int4 ch = __ldcg(args.chunks + item / n_items);
                 const int it = item % n_items;
                 const bool valid = kGemm1 || 2 * it + a < n_tiles;  // GEMM2's last pair may hold one tile
@@ -342,7 +406,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 2)) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + uint32_t(buf * C::kAccCols + (h * kNumA + a) * kN);
-                for (int step = 0; step < n_steps; ++step) {
+                for (int step = s0; step < s1; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
                     if (!mbar_wait(&full[stage], phase, abort_flag, err, 3)) {
@@ -383,7 +447,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                             // 64 K (32 bytes) per step inside the 128-byte swizzled row, one image each
                             tc_mma_nvf4(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks), idesc_nvf4(n),
                                         col + ks * 4, colb + ks * C::kSfbImages * 4,
-                                        (kb0 == 0 && ks == 0) ? 0u : 1u);
+                                        (step == s0 && ks == 0) ? 0u : 1u);
                     } else if (valid) {
                         const uint8_t *st = tiles + stage * C::kStageTiles;
                         const uint8_t *sfa = sfs + stage * C::kStageSf;
@@ -408,7 +472,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                                 // +32 bytes of K per step inside the 128-byte swizzled row
                                 tc_mma_mxf8f6f4(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks),
                                                 idesc_mxf8f6f4(n, uint32_t(ks)), col, sfb_col,
-                                                (kb0 + b == h && ks == 0) ? 0u : 1u);
+                                                (kb0 + b == s0 * kKB + h && ks == 0) ? 0u : 1u);
                             }
                             col += uint32_t((1 + C::kSfbImages) * 4);
                         }
@@ -435,12 +499,13 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int half = warp >= 8 ? 1 : 0;     // which column blocks of the quarter it handles
         constexpr int kCbStep = C::kEpiWarps / 4;
-        // with K split, accumulator h * kNumA + a holds tile a's K blocks of parity h
-        const bool add_split = C::kKSplit == 2 && KB > 1;
         uint8_t *my_stage = epi_stage + (warp < 8 ? warp - 2 : warp - 4) * 1024;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int li = 0;
-        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
+        for (int wk = 0; wk < n_works; ++wk, ++li) {
+            int item, s0, s1;
+            work_of(P, wk, n_steps, item, s0, s1);
+            const bool is_unit = wk >= P.n_whole;
             const int c = item / n_items, it = item % n_items;
             const int4 ch = __ldcg(args.chunks + c);
             const int buf = li % kBufs;
@@ -449,6 +514,133 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             tc_fence_after();
             const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
             const int ncb = (ch.z + 31) / 32;
+            // with K split, accumulator kNumA + a holds tile a's K blocks of
+            // odd index, written when the stage range holds one
+            const bool add_split = C::kKSplit == 2 && s0 * kKB + 1 < min(s1 * kKB, KB);
+            // GEMM2: fp32 words of token cb*32 + j of output tile 2 * it + a
+            auto load_tile = [&](int a, int cb, uint32_t (&v)[32]) {
+                tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), v);
+                tmem_ld_wait();
+                if (add_split) {
+                    uint32_t v1[32];
+                    tmem_ld_32x32(acc + uint32_t((kNumA + a) * kN + cb * 32), v1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(v1[j]));
+                }
+            };
+            // GEMM1 epilogue of 32 tokens: activation, scale, requantised h
+            auto finish1 = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], int cb) {
+            float h[32], amx[32];
+            if (args.act_kind == MOE_ACT_SWIGLU) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float gv = __uint_as_float(g[j]);
+                    const float uv = __uint_as_float(u[j]);
+                    // silu(g) * u with the fast exponential and division (within
+                    // the layer's tolerance; the division returns 0 where 1 + e^-g
+                    // overflows, the limit of silu)
+                    h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float gv = __uint_as_float(g[j]);
+                    const float uv = __uint_as_float(u[j]);
+                    // SiTU: sigmoid(g) * beta*tanh(g/beta) * lbeta*tanh(u/lbeta)
+                    const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
+                    h[j] = __fdividef(args.beta * tanhf(gv * args.inv_beta), 1.0f + __expf(-gv)) * up;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
+            if constexpr (kNv) {
+                // NVFP4: groups of 16 rows of h = the two half-warps.  Lane l
+                // gets the amax of tokens cb*32 + l%16 and cb*32 + 16 + l%16 over
+                // its half-warp, and their UE4M3 scale codes.
+                float amA, amB;
+                halfwarp_transpose_max(amx, lane, amA, amB);
+                const uint32_t cA = nvfp4_scale_code(amA), cB = nvfp4_scale_code(amB);
+                const float sA = e4m3_mag_value(cA), sB = e4m3_mag_value(cB);
+                // GEMM2 reads h in 256-K blocks: this item's 128 rows are half
+                // `it % 2` of block it / 2; the warp's 32 rows are groups g4 =
+                // (q % 2) * 2 + half-warp of image (it % 2) * 2 + q / 2
+                const int img = (it & 1) * 2 + (q >> 1), g4 = (q & 1) * 2 + (lane >> 4);
+                uint8_t *sfo = args.out_sf + ((int64_t(c) * (n_tiles / 2) + it / 2) * kNvImages + img) * C::kActSf;
+                const int tA = cb * 32 + (lane & 15), tB = tA + 16;
+                if (tA < ch.z) sfo[act_sf_offset(tA, g4)] = uint8_t(cA);
+                if (tB < ch.z) sfo[act_sf_offset(tB, g4)] = uint8_t(cB);
+                // codes: row (ch.y + token) of block it / 2 holds this warp's 32
+                // values as bytes (it % 2) * 64 + q * 16 .. + 15, two per byte
+                uint8_t *qbase = args.out_q + (int64_t(it >> 1) * args.rows + ch.y) * kTileK + (it & 1) * 64 +
+                                 q * 16 + (lane >> 1);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, (lane & 16) | (j & 15));
+                    const uint32_t code = to_e2m1(__fdiv_rn(h[j], sj));
+                    const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
+                    if (!(lane & 1) && cb * 32 + j < ch.z)
+                        qbase[int64_t(cb * 32 + j) * kTileK] = uint8_t(code | (partner << 4));
+                }
+            } else {
+            // lane l: amax of token cb*32+l over this warp's 32 rows of h
+            const float amax = warp_transpose_max(amx, lane);
+            const int e = scale_exponent<true>(amax);
+            const float mult = exp2_neg(e);
+            const int tok = cb * 32 + lane;
+            if (tok < ch.z)
+                args.out_sf[(int64_t(c) * n_tiles + it) * C::kActSf + act_sf_offset(tok, q)] =
+                    uint8_t(e + 127);
+            // K-block-major [I/128][rows][128]: this warp's 32 codes of a row are
+            // bytes q*32 .. q*32+31 of row (ch.y + token) in K block `it`
+            uint8_t *qbase = args.out_q + (int64_t(it) * args.rows + ch.y) * kTileK + q * 32;
+            // one store per token: the warp's 32 lanes write 32 contiguous bytes
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float mj = __shfl_sync(0xFFFFFFFFu, mult, j);
+                const uint32_t code = to_e4m3(h[j] * mj);
+                if (cb * 32 + j < ch.z) qbase[int64_t(cb * 32 + j) * kTileK + lane] = uint8_t(code);
+            }
+            }
+            };
+            // GEMM2 epilogue of 32 tokens of output tile 2 * it + a: bf16 Y rows
+            auto finish2 = [&](const uint32_t (&g)[32], int a, int cb) {
+                const int tile = 2 * it + a;
+            __nv_bfloat16 *ybase = args.out_y + int64_t(ch.y + cb * 32) * args.out_ld + tile * kTileRows + q * 32;
+            if constexpr (C::kStaged) {
+                // two passes of 16 rows: stage [row][32 columns] bf16 (1 KB), then
+                // 16-byte stores, four lanes per 64-byte row piece
+                __nv_bfloat16 *sb = reinterpret_cast<__nv_bfloat16 *>(my_stage);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        sb[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[hh * 16 + j]));
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int cidx = i * 32 + lane;  // row hh*16 + cidx / 4, columns (cidx % 4) * 8 ..
+                        const int r = hh * 16 + (cidx >> 2);
+                        if (cb * 32 + r < ch.z)
+                            *reinterpret_cast<uint4 *>(ybase + int64_t(r) * args.out_ld + (cidx & 3) * 8) =
+                                *reinterpret_cast<const uint4 *>(my_stage + cidx * 16);
+                    }
+                    __syncwarp();
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (cb * 32 + j < ch.z)
+                        ybase[int64_t(j) * args.out_ld + lane] = __float2bfloat16_rn(__uint_as_float(g[j]));
+            }
+            };
+            // a split unit's partial: [tile][kN columns][128 rows] fp32
+            float *part = is_unit ? args.part + size_t(P.unit) * kPartUnitFloats : nullptr;
+            auto put_part = [&](int a, int cb, const uint32_t (&v)[32]) {
+                float *p = part + size_t(a * kN + cb * 32) * kTileRows + q * 32 + lane;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) p[j * kTileRows] = __uint_as_float(v[j]);
+            };
             for (int cb = half; cb < ncb; cb += kCbStep) {
                 if constexpr (kGemm1) {
                     uint32_t g[32], u[32];
@@ -466,126 +658,76 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                             u[j] = __float_as_uint(__uint_as_float(u[j]) + __uint_as_float(u1[j]));
                         }
                     }
-                    float h[32], amx[32];
-                    if (args.act_kind == MOE_ACT_SWIGLU) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float gv = __uint_as_float(g[j]);
-                            const float uv = __uint_as_float(u[j]);
-                            // silu(g) * u with the fast exponential and division (within
-                            // the layer's tolerance; the division returns 0 where 1 + e^-g
-                            // overflows, the limit of silu)
-                            h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
-                        }
+                    if (is_unit) {
+                        put_part(0, cb, g);
+                        put_part(1, cb, u);
                     } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float gv = __uint_as_float(g[j]);
-                            const float uv = __uint_as_float(u[j]);
-                            // SiTU: sigmoid(g) * beta*tanh(g/beta) * lbeta*tanh(u/lbeta)
-                            const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
-                            h[j] = __fdividef(args.beta * tanhf(gv * args.inv_beta), 1.0f + __expf(-gv)) * up;
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
-                    if constexpr (kNv) {
-                        // NVFP4: groups of 16 rows of h = the two half-warps.  Lane l
-                        // gets the amax of tokens cb*32 + l%16 and cb*32 + 16 + l%16 over
-                        // its half-warp, and their UE4M3 scale codes.
-                        float amA, amB;
-                        halfwarp_transpose_max(amx, lane, amA, amB);
-                        const uint32_t cA = nvfp4_scale_code(amA), cB = nvfp4_scale_code(amB);
-                        const float sA = e4m3_mag_value(cA), sB = e4m3_mag_value(cB);
-                        // GEMM2 reads h in 256-K blocks: this item's 128 rows are half
-                        // `it % 2` of block it / 2; the warp's 32 rows are groups g4 =
-                        // (q % 2) * 2 + half-warp of image (it % 2) * 2 + q / 2
-                        const int img = (it & 1) * 2 + (q >> 1), g4 = (q & 1) * 2 + (lane >> 4);
-                        uint8_t *sfo = args.out_sf + ((int64_t(c) * (n_tiles / 2) + it / 2) * kNvImages + img) * C::kActSf;
-                        const int tA = cb * 32 + (lane & 15), tB = tA + 16;
-                        if (tA < ch.z) sfo[act_sf_offset(tA, g4)] = uint8_t(cA);
-                        if (tB < ch.z) sfo[act_sf_offset(tB, g4)] = uint8_t(cB);
-                        // codes: row (ch.y + token) of block it / 2 holds this warp's 32
-                        // values as bytes (it % 2) * 64 + q * 16 .. + 15, two per byte
-                        uint8_t *qbase = args.out_q + (int64_t(it >> 1) * args.rows + ch.y) * kTileK + (it & 1) * 64 +
-                                         q * 16 + (lane >> 1);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, (lane & 16) | (j & 15));
-                            const uint32_t code = to_e2m1(__fdiv_rn(h[j], sj));
-                            const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
-                            if (!(lane & 1) && cb * 32 + j < ch.z)
-                                qbase[int64_t(cb * 32 + j) * kTileK] = uint8_t(code | (partner << 4));
-                        }
-                    } else {
-                    // lane l: amax of token cb*32+l over this warp's 32 rows of h
-                    const float amax = warp_transpose_max(amx, lane);
-                    const int e = scale_exponent<true>(amax);
-                    const float mult = exp2_neg(e);
-                    const int tok = cb * 32 + lane;
-                    if (tok < ch.z)
-                        args.out_sf[(int64_t(c) * n_tiles + it) * C::kActSf + act_sf_offset(tok, q)] =
-                            uint8_t(e + 127);
-                    // K-block-major [I/128][rows][128]: this warp's 32 codes of a row are
-                    // bytes q*32 .. q*32+31 of row (ch.y + token) in K block `it`
-                    uint8_t *qbase = args.out_q + (int64_t(it) * args.rows + ch.y) * kTileK + q * 32;
-                    // one store per token: the warp's 32 lanes write 32 contiguous bytes
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float mj = __shfl_sync(0xFFFFFFFFu, mult, j);
-                        const uint32_t code = to_e4m3(h[j] * mj);
-                        if (cb * 32 + j < ch.z) qbase[int64_t(cb * 32 + j) * kTileK + lane] = uint8_t(code);
-                    }
+                        finish1(g, u, cb);
                     }
                 } else {
-#pragma unroll
+#pragma unroll 1
                     for (int a = 0; a < kNumA; ++a) {
-                        const int tile = 2 * it + a;
-                        if (tile >= n_tiles) break;
+                        if (2 * it + a >= n_tiles) break;
                         uint32_t g[32];
-                        tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), g);
-                        tmem_ld_wait();
-                        if (add_split) {
-                            uint32_t g1[32];
-                            tmem_ld_32x32(acc + uint32_t((kNumA + a) * kN + cb * 32), g1);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g1[j]));
-                        }
-                        __nv_bfloat16 *ybase = args.out_y + int64_t(ch.y + cb * 32) * args.out_ld + tile * kTileRows + q * 32;
-                        if constexpr (C::kStaged) {
-                            // two passes of 16 rows: stage [row][32 columns] bf16 (1 KB), then
-                            // 16-byte stores, four lanes per 64-byte row piece
-                            __nv_bfloat16 *sb = reinterpret_cast<__nv_bfloat16 *>(my_stage);
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                                for (int j = 0; j < 16; ++j)
-                                    sb[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(g[hh * 16 + j]));
-                                __syncwarp();
-#pragma unroll
-                                for (int i = 0; i < 2; ++i) {
-                                    const int cidx = i * 32 + lane;  // row hh*16 + cidx / 4, columns (cidx % 4) * 8 ..
-                                    const int r = hh * 16 + (cidx >> 2);
-                                    if (cb * 32 + r < ch.z)
-                                        *reinterpret_cast<uint4 *>(ybase + int64_t(r) * args.out_ld + (cidx & 3) * 8) =
-                                            *reinterpret_cast<const uint4 *>(my_stage + cidx * 16);
-                                }
-                                __syncwarp();
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (cb * 32 + j < ch.z)
-                                    ybase[int64_t(j) * args.out_ld + lane] = __float2bfloat16_rn(__uint_as_float(g[j]));
-                        }
+                        load_tile(a, cb, g);
+                        if (is_unit)
+                            put_part(a, cb, g);
+                        else
+                            finish2(g, a, cb);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+            if (!is_unit) continue;
+            // split unit: count it in; the item's last unit adds the partials of
+            // units 0 .. split-1 in that order and finishes the item
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_bar);
+            if (warp == 2 && lane == 0) {
+                int last = 0;
+                if (mbar_wait(epi_bar, 0, abort_flag, err, 7)) {
+                    __threadfence();
+                    last = atomicAdd(args.split_cnt + P.unit / P.split, 1) == P.split - 1;
+                    __threadfence();
+                }
+                *epi_last = last;
+                mbar_arrive(epi_go);
+            }
+            if (!mbar_wait(epi_go, 0, abort_flag, err, 8)) break;
+            if (!*epi_last) continue;
+            const float *p0 = args.part + size_t(P.unit / P.split) * P.split * kPartUnitFloats;
+            auto sum_part = [&](int a, int cb, uint32_t (&v)[32]) {
+                float acc_v[32];
+                const float *p = p0 + size_t(a * kN + cb * 32) * kTileRows + q * 32 + lane;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc_v[j] = __ldcg(p + j * kTileRows);
+                for (int sp = 1; sp < P.split; ++sp) {
+                    p += kPartUnitFloats;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc_v[j] += __ldcg(p + j * kTileRows);
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(acc_v[j]);
+            };
+            for (int cb = half; cb < ncb; cb += kCbStep) {
+                if constexpr (kGemm1) {
+                    uint32_t g[32], u[32];
+                    sum_part(0, cb, g);
+                    sum_part(1, cb, u);
+                    finish1(g, u, cb);
+                } else {
+#pragma unroll 1
+                    for (int a = 0; a < kNumA; ++a) {
+                        if (2 * it + a >= n_tiles) break;
+                        uint32_t g[32];
+                        sum_part(a, cb, g);
+                        finish2(g, a, cb);
+                    }
+                }
+            }
         }
     }
 
@@ -658,6 +800,8 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
     a.inv_lbeta = (act.kind == MOE_ACT_SITU && act.linear_beta > 0.0f) ? 1.0f / act.linear_beta : 0.0f;
     a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
     a.hdr = reinterpret_cast<int *>(ws);
+    a.part = reinterpret_cast<float *>(ws + L.off_part);
+    a.split_cnt = a.hdr + (gemm1 ? kHdrSplitCnt1 : kHdrSplitCnt2);
     a.rows = int(L.Rp);
     if (gemm1) {
         a.act_sf = ws + L.off_xg_sf;

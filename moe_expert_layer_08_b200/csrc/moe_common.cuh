@@ -40,7 +40,16 @@ constexpr int kHdrError = 0;
 constexpr int kHdrNumChunks = 1;
 constexpr int kHdrDropped = 2;
 constexpr int kHdrTimeoutWhere = 3;
-constexpr int kHdrBytes = 256;
+// Split-unit counters of the 32-row GEMMs (zeroed by routing on every forward):
+// GEMM1 at words kHdrSplitCnt1.., GEMM2 at kHdrSplitCnt2.., one per leftover item.
+constexpr int kMaxSplitUnits = 256;  // units per launch (leftover items x split)
+constexpr int kHdrSplitWords = kMaxSplitUnits / 2;
+constexpr int kHdrSplitCnt1 = 64;
+constexpr int kHdrSplitCnt2 = kHdrSplitCnt1 + kHdrSplitWords;
+constexpr int kHdrBytes = 2048;
+static_assert(4 * (kHdrSplitCnt2 + kHdrSplitWords) <= kHdrBytes, "workspace header");
+// fp32 partial accumulators of one split unit: two 128-row tiles x 32 tokens
+constexpr int kPartUnitFloats = 2 * 32 * 128;
 
 // Bounded waits: a device-side wait gives up after this many nanoseconds.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;

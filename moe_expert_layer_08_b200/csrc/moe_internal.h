@@ -46,6 +46,7 @@ struct WsLayout {
     size_t off_count = 0, off_offset = 0, off_chunk_base = 0, off_chunks = 0;
     size_t off_hist = 0, off_bad = 0, off_lrank = 0, off_perm = 0, off_inv = 0, off_rowinfo = 0;
     size_t off_xg = 0, off_xg_sf = 0, off_hq = 0, off_hq_sf = 0, off_y = 0;
+    size_t off_part = 0;    // split-unit partial accumulators of the 32-row GEMMs
     size_t total = 0;
 };
 

@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const int64_t *__rest
         hdr[kHdrError] = nbad ? kDevErrBadRouting : 0;
         hdr[kHdrTimeoutWhere] = 0;
     }
+    for (int i = tid; i < 2 * kHdrSplitWords; i += blockDim.x) hdr[kHdrSplitCnt1 + i] = 0;
 }
 
 // ------------------------------------------------------------------ large batches
@@ -219,6 +220,7 @@ __global__ void __launch_bounds__(1024) route_meta_kernel(const int *__restrict_
         hdr[kHdrError] = s_bad ? kDevErrBadRouting : 0;
         hdr[kHdrTimeoutWhere] = 0;
     }
+    for (int i = threadIdx.x; i < 2 * kHdrSplitWords; i += blockDim.x) hdr[kHdrSplitCnt1 + i] = 0;
 }
 
 __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(

@@ -93,6 +93,56 @@ def test_layer_duplicate_and_dropped_slots(moe):
     assert status == 5  # MOE_ERR_BAD_ROUTING is reported, the rest is computed
 
 
+def split_of(idx, w, gemm1, mx=True):
+    """Units per leftover item the 32-row GEMMs cut their incomplete last round
+    into (0: none), for asserting that a case exercises that path: grid =
+    min(item bound, SMs), leftover = items % grid, split = min(min(grid, 256) //
+    leftover, stages per item) when at least 2."""
+    R = idx.size
+    counts = np.bincount(idx[idx >= 0].ravel(), minlength=w.E)
+    chunks = int(sum((c + 31) // 32 for c in counts))
+    per_chunk = w.I // 128 if gemm1 else (w.H // 128 + 1) // 2
+    max_chunks = (R + 31) // 32 + min(R, w.E)
+    grid = min(max_chunks * per_chunk, torch.cuda.get_device_properties(0).multi_processor_count)
+    K = w.H if gemm1 else w.I
+    n_steps = K // 256 if not mx else (K // 128 + 1) // 2
+    rem = chunks * per_chunk % grid
+    if rem == 0:
+        return 0
+    S = min(min(grid, 256) // rem, n_steps)
+    return S if S >= 2 else 0
+
+
+def one_expert_routing(w, experts):
+    """Slot j of every token goes to experts[j]; positive normalised weights."""
+    idx = torch.tensor([experts] * w.T, dtype=torch.int64)
+    tw = torch.rand((w.T, w.k), generator=torch.Generator().manual_seed(w.seed)) + 0.1
+    return idx, (tw / tw.sum(1, keepdim=True)).float()
+
+
+SPLIT = [
+    # one chunk: every item is cut along K (4 units of one stage each)
+    (W.custom("split_even", T=32, E=64, k=1, H=1024, I=1024, seed=47), [5]),
+    # two chunks; an odd number of K blocks leaves a last unit with one block,
+    # and GEMM2's last item holds one tile
+    (W.custom("split_odd_kb", T=20, E=64, k=2, H=640, I=384, seed=48), [3, 9]),
+    # whole rounds first, then the leftover items cut into units
+    (W.custom("split_mixed", T=32, E=64, k=2, H=1024, I=1024, seed=49), None),
+]
+
+
+@pytest.mark.parametrize("w,experts", SPLIT, ids=lambda c: getattr(c, "name", ""))
+def test_layer_split_units(moe, w, experts):
+    """Items of an incomplete last round split along K across CTAs, their
+    partial accumulators added by the last unit: same results as the oracle,
+    and deterministic."""
+    routing = one_expert_routing(w, experts) if experts else W.gen_routing(w)
+    ic = routing[0].numpy()
+    assert split_of(ic, w, True) >= 2 and split_of(ic, w, False) >= 2, "case does not split"
+    status, _ = run_and_compare(moe, w, routing=routing)
+    assert status == 0
+
+
 def test_layer_decode_full(moe):
     w = W.WORKLOADS[1]            # T=8, E=384, k=6, H=7168, I=3072: every token
     status, _ = run_and_compare(moe, w)

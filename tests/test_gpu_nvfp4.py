@@ -110,6 +110,17 @@ def test_nvfp4_layer_small(moe, w):
     assert run_and_compare_nv(moe, w) == 0
 
 
+def test_nvfp4_layer_split_units(moe):
+    """One chunk: every item of both GEMMs is cut along K into units whose
+    partial accumulators the last unit adds (GEMM2 with three 256-K stages)."""
+    from test_gpu_layer import one_expert_routing, split_of
+    w = W.custom("nv_split", T=32, E=64, k=1, H=1024, I=768, seed=86)
+    idx, tw = one_expert_routing(w, [7])
+    ic = idx.numpy()
+    assert split_of(ic, w, True, mx=False) >= 2 and split_of(ic, w, False, mx=False) >= 2
+    assert run_and_compare_nv(moe, w, routing=(idx, tw)) == 0
+
+
 def test_nvfp4_layer_situ(moe):
     assert run_and_compare_nv(moe, W.custom("nv_situ", T=40, E=6, k=2, H=256, I=256, seed=85), situ=(1.25, 1.5)) == 0
 
