@@ -641,8 +641,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) p[j * kTileRows] = __uint_as_float(v[j]);
             };
-            for (int cb = half; cb < ncb; cb += kCbStep) {
-                if constexpr (kGemm1) {
+            if constexpr (kGemm1) {
+                for (int cb = half; cb < ncb; cb += kCbStep) {
                     uint32_t g[32], u[32];
                     tmem_ld_32x32(acc + uint32_t(cb * 32), g);
                     tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
@@ -664,17 +664,20 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                     } else {
                         finish1(g, u, cb);
                     }
-                } else {
+                }
+            } else {
+                // units (column block cb, tile a) = u / kNumA, u % kNumA: with two
+                // warps per lane quarter each takes one tile's column blocks
 #pragma unroll 1
-                    for (int a = 0; a < kNumA; ++a) {
-                        if (2 * it + a >= n_tiles) break;
-                        uint32_t g[32];
-                        load_tile(a, cb, g);
-                        if (is_unit)
-                            put_part(a, cb, g);
-                        else
-                            finish2(g, a, cb);
-                    }
+                for (int u = half; u < kNumA * ncb; u += kCbStep) {
+                    const int a = u % kNumA, cb = u / kNumA;
+                    if (2 * it + a >= n_tiles) continue;
+                    uint32_t g[32];
+                    load_tile(a, cb, g);
+                    if (is_unit)
+                        put_part(a, cb, g);
+                    else
+                        finish2(g, a, cb);
                 }
             }
             tc_fence_before();
