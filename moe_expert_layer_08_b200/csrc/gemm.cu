@@ -52,7 +52,8 @@ struct GemmCfg {
     // issuers per tile: with 32-row chunks and two K blocks per stage, two
     // threads split each tile's K blocks (even / odd) into two accumulators
     // that the epilogue adds, halving the tcgen05 issue time per stage
-    static constexpr int kKSplit = (kSmall && kKB == 2) ? 2 : 1;
+    // (NVFP4 with 32-row chunks: the stage's four 64-K MMA steps, two per issuer)
+    static constexpr int kKSplit = (kSmall && (kKB == 2 || kNv)) ? 2 : 1;
     static constexpr int kIssuers = kNumA * kKSplit;
     static constexpr int kStages = kNv ? (kSmall ? 5 : 3) : (kSmall ? 3 : 4);
     static constexpr int kATile = kTileRows * kTileK;   // 16 KB: 128 rows x 128 bytes
@@ -80,7 +81,8 @@ struct GemmCfg {
     // per issuer and stage: its weight tile's and the activations' scale images;
     // NVFP4 keeps two such regions per issuer (not one per stage) to fit TMEM,
     // the issuer waiting for the MMAs two stages back before reusing one
-    static constexpr int kSfColsIssuer = (kKB / kKSplit) * kImg * (1 + kSfbImages) * 4;
+    static constexpr int kSfColsIssuer = kNv ? (kImg / kKSplit) * (1 + kSfbImages) * 4
+                                             : (kKB / kKSplit) * kImg * (1 + kSfbImages) * 4;
     static constexpr int kSfRegions = kNv ? 2 : kStages;
     static constexpr int kSfCols = kSfRegions * kIssuers * kSfColsIssuer;
     static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             // ------------------------------------------------------------ MMA issuer
             // Issuer (a, h) owns weight tile a of every item and, for K split
             // h of kKSplit, its accumulator: the stage's K blocks b with
-            // b % kKSplit == h.
+            // b % kKSplit == h (NVFP4: the stage's 64-K steps 2h and 2h + 1).
             const int a = issuer % kNumA, h = issuer / kNumA;
             int stage = 0;
             uint32_t phase = 0;
@@ -425,29 +427,35 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         tc_fence_after();
                     }
                     if (kNv && valid) {
+                        // this issuer's MMA steps ks = h * kSteps .. (h + 1) * kSteps - 1
+                        // of the four, each with its weight and activation scale image
+                        constexpr int kSteps = kNvImages / C::kKSplit;
                         const uint8_t *st = tiles + stage * C::kStageTiles;
                         const uint8_t *sfa = sfs + stage * C::kStageSf;           // [tile][image][512]
                         const uint8_t *sfb = sfa + kNumA * kNvImages * kSfBlockBytes;  // [image][kActSf]
                         const uint8_t *bt = st + kNumA * C::kATile;
                         const uint32_t col = tmem + uint32_t(kBufs * C::kAccCols +
                                                              ((gstage & 1) * kIssuers + issuer) * C::kSfColsIssuer);
-                        const uint32_t colb = col + kNvImages * 4;
+                        const uint32_t colb = col + kSteps * 4;
 #pragma unroll
-                        for (int sI = 0; sI < kNvImages; ++sI) {
-                            tc_cp_sf(col + sI * 4, smem_desc_sf(smem_u32(sfa + (a * kNvImages + sI) * kSfBlockBytes)));
+                        for (int j = 0; j < kSteps; ++j) {
+                            const int sI = h * kSteps + j;
+                            tc_cp_sf(col + j * 4, smem_desc_sf(smem_u32(sfa + (a * kNvImages + sI) * kSfBlockBytes)));
 #pragma unroll
                             for (int im = 0; im < C::kSfbImages; ++im)
-                                tc_cp_sf(colb + (sI * C::kSfbImages + im) * 4,
+                                tc_cp_sf(colb + (j * C::kSfbImages + im) * 4,
                                          smem_desc_sf(smem_u32(sfb + sI * C::kActSf + im * kSfBlockBytes)));
                         }
                         const uint64_t adesc = smem_desc_sw128(smem_u32(st + a * C::kATile));
                         const uint64_t bdesc = smem_desc_sw128(smem_u32(bt));
 #pragma unroll
-                        for (int ks = 0; ks < kNvImages; ++ks)
+                        for (int j = 0; j < kSteps; ++j) {
                             // 64 K (32 bytes) per step inside the 128-byte swizzled row, one image each
+                            const int ks = h * kSteps + j;
                             tc_mma_nvf4(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks), idesc_nvf4(n),
-                                        col + ks * 4, colb + ks * C::kSfbImages * 4,
-                                        (step == s0 && ks == 0) ? 0u : 1u);
+                                        col + j * 4, colb + j * C::kSfbImages * 4,
+                                        (step == s0 && j == 0) ? 0u : 1u);
+                        }
                     } else if (valid) {
                         const uint8_t *st = tiles + stage * C::kStageTiles;
                         const uint8_t *sfa = sfs + stage * C::kStageSf;
@@ -515,8 +523,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
             const int ncb = (ch.z + 31) / 32;
             // with K split, accumulator kNumA + a holds tile a's K blocks of
-            // odd index, written when the stage range holds one
-            const bool add_split = C::kKSplit == 2 && s0 * kKB + 1 < min(s1 * kKB, KB);
+            // odd index, written when the stage range holds one (NVFP4: the
+            // last two 64-K steps of every stage)
+            const bool add_split = C::kKSplit == 2 && (kNv || s0 * kKB + 1 < min(s1 * kKB, KB));
             // GEMM2: fp32 words of token cb*32 + j of output tile 2 * it + a
             auto load_tile = [&](int a, int cb, uint32_t (&v)[32]) {
                 tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), v);
