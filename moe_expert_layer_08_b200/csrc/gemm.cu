@@ -4,27 +4,33 @@
 // to the tensor cores undequantised and the accumulator is fp32, as its Key
 // design points state).
 //
-// One persistent kernel per GEMM over work items (chunk, output tile): a chunk
-// is up to 128 consecutive routed rows of one expert, an output tile is 128
-// weight rows.  The operands are swapped so that the weight tile is the
-// MMA's M = 128 side and the chunk's tokens are the N side (N = rows rounded up
-// to 16), which keeps decode-sized chunks (1-2 tokens per expert) from padding
-// to 128.  Per CTA, warp-specialised:
-//   warp 0 (one thread): TMA producer.  Per 128-K stage: the weight packet
-//     body(s) via a 3D tensor map whose 4-bit element type expands FP4 into
-//     the 1-byte-per-element shared-memory form the f8f6f4 MMA reads, the
-//     packet's 512 scale bytes and the chunk's activation scale block via bulk
-//     copies, the chunk's FP8 rows via 16-row 2D boxes.  Weights are one-use
-//     (L2 evict-first), activations are re-read by every tile (evict-last).
-//   warp 1 (one thread): tcgen05.cp of the stage's scale blocks into TMEM,
-//     then 4 tcgen05.mma.kind::mxf8f6f4.block_scale (K = 32 each) per
-//     accumulator; tcgen05.commit releases the stage and, after the last
-//     stage, hands the accumulator to the epilogue.
-//   warps 2-5: epilogue, TMEM -> registers (thread = weight row, registers =
-//     tokens).  GEMM1: h = silu(gate) * up, per-token amax over each 32-row
-//     group (a warp) by a transposing butterfly, UE8M0 scale, FP8 codes
-//     written row-major plus the scale block of the chunk in the layout GEMM2's
-//     tcgen05.cp consumes.  GEMM2: Y rows as bf16.
+// One persistent kernel per GEMM over work items (chunk, pair of 128-row
+// weight tiles): a chunk is up to kN consecutive routed rows of one expert
+// (32 for small batches, 160 for large ones).  The operands are swapped so
+// that the weight tile is the MMA's M = 128 side and the chunk's tokens are
+// the N side (N = rows rounded up to 16), which keeps decode-sized chunks (1-2
+// tokens per expert) from padding to 128.  Per CTA, warp-specialised:
+//   warp 0 (one thread): weight producer.  Per stage one 4D TMA box of the
+//     item's two tiles (a 4-bit element type that expands FP4 into the
+//     1-byte-per-element shared-memory form the f8f6f4 MMA reads) and one 2D
+//     box of their 512-byte scale blocks; weights are one-use (L2 evict-first).
+//   warp 6 (one thread): activation producer.  The chunk's FP8 rows, stored
+//     K-block-major, as 3D boxes (32-row boxes, or one kN-row box for a nearly
+//     full large chunk) and the chunk's scale images by a bulk copy; they are
+//     re-read by every tile of the chunk (evict-last).
+//   warps 1 and 7 (and 8, 9 with K split; one thread each): MMA issuers, one
+//     per tile (and K half): tcgen05.cp of the stage's scale images into TMEM,
+//     then tcgen05.mma.kind::mxf8f6f4.block_scale (K = 32 each) or
+//     kind::mxf4nvf4 (K = 64); tcgen05.commit releases the stage and, after
+//     the item's last stage, hands the accumulator to the epilogue.
+//   warps 2-5 (and 8-11 for large chunks): epilogue, TMEM -> registers (thread
+//     = weight row, registers = 32 tokens).  GEMM1: h = silu(gate) * up (or
+//     SiTU), per-token amax over each 32-row group (a warp) by a transposing
+//     butterfly, the scale, FP8 (or NVFP4) codes written K-block-major plus the
+//     chunk's scale images in the layout GEMM2's tcgen05.cp consumes.  GEMM2:
+//     Y rows as bf16.
+// Items are dealt round-robin; with 32-row chunks the items of an incomplete
+// last round are split along K over the idle CTAs (plan_work below).
 // Every mbarrier wait is bounded; on timeout the kernel records the failure in
 // the workspace error word and all roles leave their loops.
 #include "moe_common.cuh"
