@@ -133,8 +133,10 @@ moe_status_t moe_workspace_bytes(int T_max, int E, int k, int H, int I, size_t *
  * graph builder, know the layer's launch structure).  Routing takes two
  * kernels when T * k <= 1024 (one block does histogram, scan and placement,
  * then the gather) and five otherwise (histogram, per-expert scan, metadata,
- * placement, gather); GEMM1, GEMM2 and the combine add three.  T = 0 enqueues
- * nothing.  Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE for sizes
+ * placement, gather); GEMM1, GEMM2 and the combine add three.  When
+ * T * k > 8 * E (160-row chunks) GEMM1 and GEMM2 run a second time, as the
+ * 32-row kernels over the experts with at most 32 routed rows (two more).
+ * T = 0 enqueues nothing.  Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE for sizes
  * moe_forward would reject.
  */
 moe_status_t moe_forward_kernel_launches(int T, int E, int k, int H, int I, int *launches);

@@ -54,6 +54,14 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.off_hq_sf = take(2 * sf_per_kb * size_t(I / kTileK));
     L.off_y = take(R * size_t(H) * 2);
     L.off_part = take(size_t(kMaxSplitUnits) * kPartUnitFloats * sizeof(float));
+    // side list (large batches): one 32-row chunk per lightly loaded expert;
+    // allocated at every size so that the workspace grows monotonically with T
+    L.side = L.chunk_rows == kChunkRows;
+    L.max_side = L.R < E ? L.R : E;
+    const size_t MS = size_t(L.max_side > 0 ? L.max_side : 1);
+    L.off_chunks_s = take(sizeof(int4) * MS);
+    L.off_xg_sf_s = take(2 * MS * size_t(act_sf_bytes(kChunkRowsSmall)) * size_t(H / kTileK));
+    L.off_hq_sf_s = take(2 * MS * size_t(act_sf_bytes(kChunkRowsSmall)) * size_t(I / kTileK));
     L.total = o;
     return L;
 }
@@ -219,32 +227,44 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
     const int64_t kbh = nvfp4 ? H / kNvTileK : L.kbh, kbi = nvfp4 ? I / kNvTileK : L.kbi;
     CUtensorMap tm_w1, tm_w2, tm_s1, tm_s2, tm_xg, tm_hq, tm_xg_full, tm_hq_full;
     const bool rowmajor = w.layout == MOE_LAYOUT_ROW_MAJOR;
-    bool ok;
-    if (nvfp4) {
-        ok = encode_nv_packets(&tm_w1, w.l1, np1) && encode_nv_packets(&tm_w2, w.l2, np2) &&
-             encode_nv_packet_sf(&tm_s1, w.l1, np1) && encode_nv_packet_sf(&tm_s2, w.l2, np2);
-    } else if (rowmajor) {
-        const uint64_t e = uint64_t(E), h = uint64_t(H), i = uint64_t(I);
-        ok = encode_weights4(&tm_w1, w.l1, e * 2 * i - i, h / 2, 2, i * h / 2, h / kTileK, kTileK / 2, kTileRows, 2,
-                             d1 / 2) &&
-             encode_weights4(&tm_w2, w.l2, e * h, i / 2, 1, e * h * i / 2, i / kTileK, kTileK / 2, 2 * kTileRows, 1,
-                             d2 / 2) &&
-             encode_packet_sf(&tm_s1, w.l1_sf, np1, d1, kPacketSf / 4) &&
-             encode_packet_sf(&tm_s2, w.l2_sf, np2, d2, kPacketSf / 4);
-    } else {
-        ok = encode_weights4(&tm_w1, w.l1, kTileRows, kTileK / 2, 2, kPacketBytes, uint64_t(np1 / 2),
-                             2 * kPacketBytes, kTileRows, 2, d1 / 2) &&
-             encode_weights4(&tm_w2, w.l2, kTileRows, kTileK / 2, 2, kPacketBytes, uint64_t(np2 / 2),
-                             2 * kPacketBytes, kTileRows, 2, d2 / 2) &&
-             encode_packet_sf(&tm_s1, w.l1, np1, d1, kPacketBytes / 4) &&
-             encode_packet_sf(&tm_s2, w.l2, np2, d2, kPacketBytes / 4);
-    }
+    // weight maps whose boxes move b1 / b2 packets (a stage of that GEMM variant)
+    auto encode_w = [&](int b1, int b2, CUtensorMap *w1, CUtensorMap *w2, CUtensorMap *s1, CUtensorMap *s2) {
+        if (nvfp4)
+            return encode_nv_packets(w1, w.l1, np1) && encode_nv_packets(w2, w.l2, np2) &&
+                   encode_nv_packet_sf(s1, w.l1, np1) && encode_nv_packet_sf(s2, w.l2, np2);
+        if (rowmajor) {
+            const uint64_t e = uint64_t(E), h = uint64_t(H), i = uint64_t(I);
+            return encode_weights4(w1, w.l1, e * 2 * i - i, h / 2, 2, i * h / 2, h / kTileK, kTileK / 2, kTileRows, 2,
+                                   b1 / 2) &&
+                   encode_weights4(w2, w.l2, e * h, i / 2, 1, e * h * i / 2, i / kTileK, kTileK / 2, 2 * kTileRows, 1,
+                                   b2 / 2) &&
+                   encode_packet_sf(s1, w.l1_sf, np1, b1, kPacketSf / 4) &&
+                   encode_packet_sf(s2, w.l2_sf, np2, b2, kPacketSf / 4);
+        }
+        return encode_weights4(w1, w.l1, kTileRows, kTileK / 2, 2, kPacketBytes, uint64_t(np1 / 2), 2 * kPacketBytes,
+                               kTileRows, 2, b1 / 2) &&
+               encode_weights4(w2, w.l2, kTileRows, kTileK / 2, 2, kPacketBytes, uint64_t(np2 / 2), 2 * kPacketBytes,
+                               kTileRows, 2, b2 / 2) &&
+               encode_packet_sf(s1, w.l1, np1, b1, kPacketBytes / 4) &&
+               encode_packet_sf(s2, w.l2, np2, b2, kPacketBytes / 4);
+    };
+    bool ok = encode_w(d1, d2, &tm_w1, &tm_w2, &tm_s1, &tm_s2);
     if (!ok ||
         !encode_act(&tm_xg, ws + L.off_xg, L.Rp, kbh, dk, kActBoxRows) ||
         !encode_act(&tm_hq, ws + L.off_hq, L.Rp, kbi, dk, kActBoxRows) ||
         !encode_act(&tm_xg_full, ws + L.off_xg, L.Rp, kbh, dk, L.chunk_rows) ||
         !encode_act(&tm_hq_full, ws + L.off_hq, L.Rp, kbi, dk, L.chunk_rows))
         return MOE_ERR_CUDA;
+    // the side list's 32-row kernels: their own box depths
+    CUtensorMap tm_w1s, tm_w2s, tm_s1s, tm_s2s, tm_xgs, tm_hqs;
+    if (L.side) {
+        const int dks = gemm_kblocks_per_stage(kChunkRowsSmall, nvfp4);
+        if (!encode_w(gemm_packets_per_stage(true, kChunkRowsSmall, nvfp4),
+                      gemm_packets_per_stage(false, kChunkRowsSmall, nvfp4), &tm_w1s, &tm_w2s, &tm_s1s, &tm_s2s) ||
+            !encode_act(&tm_xgs, ws + L.off_xg, L.Rp, kbh, dks, kActBoxRows) ||
+            !encode_act(&tm_hqs, ws + L.off_hq, L.Rp, kbi, dks, kActBoxRows))
+            return MOE_ERR_CUDA;
+    }
 
     auto record = [&](int i) -> cudaError_t {
         if (!stage_events || !stage_events[i]) return cudaSuccess;
@@ -255,6 +275,8 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
     const int64_t items2 = L.max_chunks * (H / kTileRows);
     const int grid1 = int(items1 < sms ? items1 : sms);
     const int grid2 = int(items2 < sms ? items2 : sms);
+    const int64_t items1s = L.max_side * (I / kTileRows), items2s = L.max_side * ((H / kTileRows + 1) / 2);
+    const int grid1s = int(items1s < sms ? items1s : sms), grid2s = int(items2s < sms ? items2s : sms);
 
     cudaError_t e = record(0);
     if (e == cudaSuccess)
@@ -263,9 +285,15 @@ moe_status_t run_layer(const void *x_fp8, const void *x_sf, const int64_t *topk_
     if (e == cudaSuccess) e = record(1);
     if (e == cudaSuccess)
         e = launch_gemm(true, tm_w1, tm_s1, tm_xg, tm_xg_full, rowmajor, ws, L, H, I, grid1, st, act, nvfp4);
+    if (e == cudaSuccess && L.side)
+        e = launch_gemm(true, tm_w1s, tm_s1s, tm_xgs, tm_xgs, rowmajor, ws, L, H, I, grid1s > 0 ? grid1s : 1, st, act,
+                        nvfp4, true);
     if (e == cudaSuccess) e = record(2);
     if (e == cudaSuccess)
         e = launch_gemm(false, tm_w2, tm_s2, tm_hq, tm_hq_full, rowmajor, ws, L, H, I, grid2, st, act, nvfp4);
+    if (e == cudaSuccess && L.side)
+        e = launch_gemm(false, tm_w2s, tm_s2s, tm_hqs, tm_hqs, rowmajor, ws, L, H, I, grid2s > 0 ? grid2s : 1, st, act,
+                        nvfp4, true);
     if (e == cudaSuccess) e = record(3);
     if (e == cudaSuccess) e = launch_combine(ws, L, topk_w, T, k, H, out_bf16, st);
     if (e == cudaSuccess) e = record(4);
@@ -380,7 +408,9 @@ moe_status_t moe_forward_kernel_launches(int T, int E, int k, int H, int I, int 
     if (s != MOE_OK) return s;
     if (T < 0 || k <= 0 || k > E || !launches) return MOE_ERR_INVALID_ARG;
     if (int64_t(T) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
-    *launches = T == 0 ? 0 : route_kernel_launches(T * k) + 3;
+    // route + gather, GEMM1, GEMM2 (each twice with a side list: T*k > 8E), combine
+    const bool side = int64_t(T) * k > int64_t(8) * E;
+    *launches = T == 0 ? 0 : route_kernel_launches(T * k) + (side ? 5 : 3);
     return MOE_OK;
 }
 

@@ -125,7 +125,8 @@ struct GemmArgs {
     int w_sf_x0;               // word offset of a scale block within a row of the scale map
     const uint8_t *act_sf;     // activation scale blocks [chunk][K/128][512]
     const int4 *chunks;        // (expert, first row, rows, -)
-    int *hdr;                  // workspace header (chunk count, error word)
+    int *hdr;                  // workspace header (chunk counts, error word)
+    int chunks_word;           // header word holding this list's chunk count
     uint8_t *out_q;            // GEMM1: h codes [R, I]
     uint8_t *out_sf;           // GEMM1: h scale blocks [chunk][I/128][512]
     __nv_bfloat16 *out_y;      // GEMM2: Y [R, H]
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     if (threadIdx.x == 32) pdl_trigger();
 
     const int n_tiles = args.n_tiles, n_items = args.n_items;
-    const int num_items = __ldcg(args.hdr + kHdrNumChunks) * n_items;
+    const int num_items = __ldcg(args.hdr + args.chunks_word) * n_items;
     const int KB = args.K / (kNv ? kNvTileK : kTileK);  // K blocks of 128 operand bytes
     const int n_steps = (KB + kKB - 1) / kKB;  // pipeline stages per item
     const WorkPlan P = plan_work(num_items, n_steps, C::kSmall);
@@ -805,7 +806,7 @@ static cudaError_t launch_gemm_fmt(bool gemm1, bool small, const CUtensorMap &tm
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
                         const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, bool w_rowmajor,
                         uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
-                        const moe_activation_t &act, bool nvfp4) {
+                        const moe_activation_t &act, bool nvfp4, bool side) {
     GemmArgs a{};
     a.w_rowmajor = w_rowmajor ? 1 : 0;
     a.w_rows_per_expert = gemm1 ? 2 * I : H;
@@ -816,28 +817,30 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
     a.inv_beta = act.kind == MOE_ACT_SITU ? 1.0f / act.beta : 0.0f;
     a.lbeta = act.linear_beta;
     a.inv_lbeta = (act.kind == MOE_ACT_SITU && act.linear_beta > 0.0f) ? 1.0f / act.linear_beta : 0.0f;
-    a.chunks = reinterpret_cast<const int4 *>(ws + L.off_chunks);
+    a.chunks = reinterpret_cast<const int4 *>(ws + (side ? L.off_chunks_s : L.off_chunks));
     a.hdr = reinterpret_cast<int *>(ws);
+    a.chunks_word = side ? kHdrNumChunksSide : kHdrNumChunks;
     a.part = reinterpret_cast<float *>(ws + L.off_part);
     a.split_cnt = a.hdr + (gemm1 ? kHdrSplitCnt1 : kHdrSplitCnt2);
     a.rows = int(L.Rp);
+    const size_t xg_sf = side ? L.off_xg_sf_s : L.off_xg_sf, hq_sf = side ? L.off_hq_sf_s : L.off_hq_sf;
     if (gemm1) {
-        a.act_sf = ws + L.off_xg_sf;
+        a.act_sf = ws + xg_sf;
         a.out_q = ws + L.off_hq;
-        a.out_sf = ws + L.off_hq_sf;
+        a.out_sf = ws + hq_sf;
         a.K = H;
         a.n_tiles = I / kTileRows;
         a.n_items = I / kTileRows;
         a.out_ld = I;
     } else {
-        a.act_sf = ws + L.off_hq_sf;
+        a.act_sf = ws + hq_sf;
         a.out_y = reinterpret_cast<__nv_bfloat16 *>(ws + L.off_y);
         a.K = I;
         a.n_tiles = H / kTileRows;
         a.n_items = (H / kTileRows + 1) / 2;
         a.out_ld = H;
     }
-    const bool small = L.chunk_rows == kChunkRowsSmall;
+    const bool small = side || L.chunk_rows == kChunkRowsSmall;
     return nvfp4 ? launch_gemm_fmt<true>(gemm1, small, tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream)
                  : launch_gemm_fmt<false>(gemm1, small, tmap_w, tmap_wsf, tmap_act, tmap_act_full, a, grid, stream);
 }

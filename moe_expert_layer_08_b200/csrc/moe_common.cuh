@@ -40,6 +40,9 @@ constexpr int kHdrError = 0;
 constexpr int kHdrNumChunks = 1;
 constexpr int kHdrDropped = 2;
 constexpr int kHdrTimeoutWhere = 3;
+constexpr int kHdrNumChunksSide = 4;  // chunks of the side list (large batches: lightly loaded experts)
+// A per-expert chunk base with this bit set indexes the side list.
+constexpr int kSideChunkBit = 1 << 30;
 // Split-unit counters of the 32-row GEMMs (zeroed by routing on every forward):
 // GEMM1 at words kHdrSplitCnt1.., GEMM2 at kHdrSplitCnt2.., one per leftover item.
 constexpr int kMaxSplitUnits = 256;  // units per launch (leftover items x split)

@@ -40,13 +40,19 @@ struct WsLayout {
     int64_t R = 0;          // routed slots T*k
     int64_t max_chunks = 0; // upper bound of (expert, <=128-row) work chunks
     int nb = 0;             // routing blocks
-    int chunk_rows = 0;     // routed rows per chunk (32 or 128)
+    int chunk_rows = 0;     // routed rows per chunk of the main list (32 or 160)
+    // Large batches (chunk_rows = 160) also keep a side list: experts with at
+    // most kChunkRowsSmall rows get one 32-row chunk there, which the 32-row
+    // kernels process (they stream weights faster than the 160-row ones).
+    bool side = false;
+    int64_t max_side = 0;   // side-list chunks, at most (one per expert)
     int64_t Rp = 0;         // rows of the K-block-major FP8 operands (R, at least one TMA box)
     int kbh = 0, kbi = 0;   // K blocks of those operands (H/128, I/128, at least 2)
     size_t off_count = 0, off_offset = 0, off_chunk_base = 0, off_chunks = 0;
     size_t off_hist = 0, off_bad = 0, off_lrank = 0, off_perm = 0, off_inv = 0, off_rowinfo = 0;
     size_t off_xg = 0, off_xg_sf = 0, off_hq = 0, off_hq_sf = 0, off_y = 0;
     size_t off_part = 0;    // split-unit partial accumulators of the 32-row GEMMs
+    size_t off_chunks_s = 0, off_xg_sf_s = 0, off_hq_sf_s = 0;  // side list and its scale images
     size_t total = 0;
 };
 
@@ -69,10 +75,13 @@ inline int route_kernel_launches(int64_t R) { return R <= kRouteSmallMax ? 2 : 5
 cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
                          int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, bool nvfp4,
                          cudaStream_t stream);
+// GEMM1 / GEMM2 over the main chunk list (side = false: chunks of
+// L.chunk_rows rows) or the side list (32-row chunks of lightly loaded
+// experts); the tensor maps are those of that chunk size.
 cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_wsf,
                         const CUtensorMap &tmap_act, const CUtensorMap &tmap_act_full, bool w_rowmajor,
                         uint8_t *ws, const WsLayout &L, int H, int I, int grid, cudaStream_t stream,
-                        const moe_activation_t &act, bool nvfp4);
+                        const moe_activation_t &act, bool nvfp4, bool side = false);
 // Weight packets one pipeline stage of that GEMM variant moves (TMA box depth).
 int gemm_packets_per_stage(bool gemm1, int chunk_rows, bool nvfp4);
 // K blocks (128 operand bytes each) one pipeline stage moves (the activation box depth).

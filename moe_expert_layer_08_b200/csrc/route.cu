@@ -49,32 +49,50 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *s_warp) {
     return r;
 }
 
-// Per expert e (one thread each): count c, offset, chunk base, chunk list
-// entries, statistics.  Shared by both routing paths.
-__device__ __forceinline__ void write_expert_meta(int e, int E, int c, int off, int cbase, int chunk_rows,
-                                                 int *count, int *offset, int *chunk_base, int4 *chunks, int *hdr,
-                                                 int32_t *expert_stats) {
-    const int nch = (c + chunk_rows - 1) / chunk_rows;
+// Whether expert e with c rows goes to the side list (one 32-row chunk;
+// only with `side` lists, i.e. 160-row main chunks).
+__device__ __forceinline__ bool on_side(bool side, int c) { return side && c <= kChunkRowsSmall; }
+
+// Per expert e (one thread each): count c, offset, chunk base (main-list
+// index, or side-list index | kSideChunkBit), chunk list entries, statistics.
+// cbase / sbase: the expert's first chunk in the main / side list (exclusive
+// scans over experts).  Shared by both routing paths.
+__device__ __forceinline__ void write_expert_meta(int e, int E, int c, int off, int cbase, int sbase, bool side,
+                                                 int chunk_rows, int *count, int *offset, int *chunk_base,
+                                                 int4 *chunks, int4 *chunks_s, int *hdr, int32_t *expert_stats) {
+    const bool s = on_side(side, c);
+    const int nch = s ? 0 : (c + chunk_rows - 1) / chunk_rows;
+    const int nside = (s && c > 0) ? 1 : 0;
     count[e] = c;
     offset[e] = off;
-    chunk_base[e] = cbase;
+    chunk_base[e] = s ? (kSideChunkBit | sbase) : cbase;
     for (int q = 0; q < nch; ++q)
         chunks[cbase + q] = make_int4(e, off + q * chunk_rows, min(chunk_rows, c - q * chunk_rows), 0);
+    if (nside) chunks_s[sbase] = make_int4(e, off, c, 0);
     if (expert_stats) expert_stats[e] += c;
     if (e == E - 1) {
         offset[E] = off + c;
         chunk_base[E] = cbase + nch;
         hdr[kHdrNumChunks] = cbase + nch;
+        hdr[kHdrNumChunksSide] = sbase + nside;
     }
+}
+
+// Gather descriptor of a routed row: token, chunk (in its list), row within
+// the chunk, list (0 main, 1 side).
+__device__ __forceinline__ int4 row_info(int token, int cb, int local, int chunk_rows) {
+    return (cb & kSideChunkBit) ? make_int4(token, cb & ~kSideChunkBit, local, 1)
+                                : make_int4(token, cb + local / chunk_rows, local % chunk_rows, 0);
 }
 
 // ------------------------------------------------------------------ small batches
 // One 1024-thread block, one slot per thread (R <= 1024).  Shared memory:
 // cnt[32 warps][E] per-warp per-expert counts, turned into per-warp bases.
 __global__ void __launch_bounds__(1024) route_small_kernel(const int64_t *__restrict__ topk_idx, int R, int k, int E,
-                                                           int chunk_rows, int *__restrict__ count,
+                                                           int chunk_rows, int side, int *__restrict__ count,
                                                            int *__restrict__ offset, int *__restrict__ chunk_base,
-                                                           int4 *__restrict__ chunks, int *__restrict__ perm,
+                                                           int4 *__restrict__ chunks, int4 *__restrict__ chunks_s,
+                                                           int *__restrict__ perm,
                                                            int *__restrict__ inv, int4 *__restrict__ rowinfo,
                                                            int *__restrict__ hdr, int32_t *__restrict__ expert_stats) {
     extern __shared__ int cnt[];
@@ -104,12 +122,15 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const int64_t *__rest
             cnt[w * E + tid] = c;
             c += x;
         }
+    const bool s = tid < E && on_side(side, c);
     const int off = block_exclusive_scan(tid < E ? c : 0, s_warp);
-    const int cbase = block_exclusive_scan(tid < E ? (c + chunk_rows - 1) / chunk_rows : 0, s_warp);
+    const int cbase = block_exclusive_scan(tid < E && !s ? (c + chunk_rows - 1) / chunk_rows : 0, s_warp);
+    const int sbase = block_exclusive_scan(s && c > 0 ? 1 : 0, s_warp);
     if (tid < E) {
         s_off[tid] = off;
-        s_cbase[tid] = cbase;
-        write_expert_meta(tid, E, c, off, cbase, chunk_rows, count, offset, chunk_base, chunks, hdr, expert_stats);
+        s_cbase[tid] = s ? (kSideChunkBit | sbase) : cbase;
+        write_expert_meta(tid, E, c, off, cbase, sbase, side, chunk_rows, count, offset, chunk_base, chunks,
+                          chunks_s, hdr, expert_stats);
     }
     __syncthreads();
     if (tid < R) {
@@ -118,7 +139,7 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const int64_t *__rest
             const int pos = s_off[e] + local;
             perm[pos] = tid;
             inv[tid] = pos;
-            rowinfo[pos] = make_int4(tid / k, s_cbase[e] + local / chunk_rows, local % chunk_rows, 0);
+            rowinfo[pos] = row_info(tid / k, s_cbase[e], local, chunk_rows);
         } else {
             inv[tid] = -1;
         }
@@ -197,18 +218,23 @@ __global__ void __launch_bounds__(1024) route_colscan_kernel(int *__restrict__ h
 // One block: offsets and chunk bases (scans over experts), chunk list,
 // statistics, dropped count and error word.
 __global__ void __launch_bounds__(1024) route_meta_kernel(const int *__restrict__ bad, int nb, int E, int chunk_rows,
-                                                          int *__restrict__ count, int *__restrict__ offset,
+                                                          int side, int *__restrict__ count, int *__restrict__ offset,
                                                           int *__restrict__ chunk_base, int4 *__restrict__ chunks,
-                                                          int *__restrict__ hdr, int32_t *__restrict__ expert_stats) {
+                                                          int4 *__restrict__ chunks_s, int *__restrict__ hdr,
+                                                          int32_t *__restrict__ expert_stats) {
     __shared__ int s_warp[32];
     __shared__ int s_bad;
     const int e = threadIdx.x;
     pdl_wait();
     pdl_trigger();
     const int c = e < E ? __ldcg(count + e) : 0;
+    const bool s = e < E && on_side(side, c);
     const int off = block_exclusive_scan(c, s_warp);
-    const int cbase = block_exclusive_scan((c + chunk_rows - 1) / chunk_rows, s_warp);
-    if (e < E) write_expert_meta(e, E, c, off, cbase, chunk_rows, count, offset, chunk_base, chunks, hdr, expert_stats);
+    const int cbase = block_exclusive_scan(s ? 0 : (c + chunk_rows - 1) / chunk_rows, s_warp);
+    const int sbase = block_exclusive_scan(s && c > 0 ? 1 : 0, s_warp);
+    if (e < E)
+        write_expert_meta(e, E, c, off, cbase, sbase, side, chunk_rows, count, offset, chunk_base, chunks, chunks_s,
+                          hdr, expert_stats);
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
     int d = 0;
@@ -241,7 +267,7 @@ __global__ void __launch_bounds__(kRouteBlock) route_place_kernel(
     perm[pos] = int(s);
     inv[s] = pos;
     const int local = pos - __ldcg(offset + e);
-    rowinfo[pos] = make_int4(int(s / k), __ldcg(chunk_base + e) + local / chunk_rows, local % chunk_rows, 0);
+    rowinfo[pos] = row_info(int(s / k), __ldcg(chunk_base + e), local, chunk_rows);
 }
 
 // gather_kernel: one warp per task, a task being `seg_vec` 16-byte vectors of
@@ -260,10 +286,11 @@ constexpr int kGatherVec = 8;
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__restrict__ rowinfo,
                                                                 const int *__restrict__ offset, int E,
                                                                 int row_bytes, int sf_words, int64_t Rp, int sf_bytes,
-                                                                int segs, int seg_vec,
+                                                                int sf_bytes_s, int segs, int seg_vec,
                                                                 const uint8_t *__restrict__ x,
                                                                 const uint8_t *__restrict__ x_sf,
-                                                                uint8_t *__restrict__ xg, uint8_t *__restrict__ xg_sf) {
+                                                                uint8_t *__restrict__ xg, uint8_t *__restrict__ xg_sf,
+                                                                uint8_t *__restrict__ xg_sf_s) {
     pdl_wait();
     pdl_trigger();
     constexpr int kWarps = kGatherThreads / 32;
@@ -296,9 +323,12 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__re
         }
         if (seg != 0) continue;
         const uint32_t *sfs = reinterpret_cast<const uint32_t *>(x_sf + int64_t(ri.x) * KB * sf_words * 4);
+        // the chunk's images in its list's region (side-list chunks: 32 rows)
+        uint8_t *const sf_dst = ri.w ? xg_sf_s : xg_sf;
+        const int img_bytes = ri.w ? sf_bytes_s : sf_bytes;
         for (int wi = lane; wi < KB * sf_words; wi += 32) {
             const int kb = wi / sf_words, img = wi % sf_words;
-            uint8_t *blk = xg_sf + ((int64_t(ri.y) * KB + kb) * sf_words + img) * sf_bytes;
+            uint8_t *blk = sf_dst + ((int64_t(ri.y) * KB + kb) * sf_words + img) * img_bytes;
             *reinterpret_cast<uint32_t *>(blk + act_sf_offset(ri.z, 0)) = __ldcg(sfs + wi);
         }
     }
@@ -316,6 +346,8 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
     int *offset = reinterpret_cast<int *>(ws + L.off_offset);
     int *chunk_base = reinterpret_cast<int *>(ws + L.off_chunk_base);
     int4 *chunks = reinterpret_cast<int4 *>(ws + L.off_chunks);
+    int4 *chunks_s = reinterpret_cast<int4 *>(ws + L.off_chunks_s);
+    const int side = L.side ? 1 : 0;
     int *perm = reinterpret_cast<int *>(ws + L.off_perm);
     int *inv = reinterpret_cast<int *>(ws + L.off_inv);
     int4 *rowinfo = reinterpret_cast<int4 *>(ws + L.off_rowinfo);
@@ -332,8 +364,8 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
             if (e != cudaSuccess) return e;
             configured_for = dev;
         }
-        e = launch_pdl(route_small_kernel, dim3(1), dim3(1024), smem, stream, topk_idx, R, k, E, cr, count, offset,
-                       chunk_base, chunks, perm, inv, rowinfo, hdr, expert_stats);
+        e = launch_pdl(route_small_kernel, dim3(1), dim3(1024), smem, stream, topk_idx, R, k, E, cr, side, count,
+                       offset, chunk_base, chunks, chunks_s, perm, inv, rowinfo, hdr, expert_stats);
     } else {
         const size_t cnt_smem = size_t(kRouteBlock / 32) * E * sizeof(int);
         e = launch_pdl(route_count_kernel, dim3(L.nb), dim3(kRouteBlock), cnt_smem, stream, topk_idx, R, E, hist,
@@ -343,7 +375,7 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
             e = launch_pdl(route_colscan_kernel, dim3(E), dim3(cs_threads), 0, stream, hist, L.nb, count);
         if (e == cudaSuccess)
             e = launch_pdl(route_meta_kernel, dim3(1), dim3(1024), 0, stream, static_cast<const int *>(bad), L.nb, E,
-                           cr, count, offset, chunk_base, chunks, hdr, expert_stats);
+                           cr, side, count, offset, chunk_base, chunks, chunks_s, hdr, expert_stats);
         if (e == cudaSuccess)
             e = launch_pdl(route_place_kernel, dim3(L.nb), dim3(kRouteBlock), 0, stream, topk_idx, R, k, E, cr, hist,
                            lrank, offset, chunk_base, perm, inv, rowinfo);
@@ -368,8 +400,9 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
     const int grid = int(want < int64_t(sms) * 4 ? want : int64_t(sms) * 4);
     return launch_pdl(gather_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kGatherThreads), 0, stream,
                       static_cast<const int4 *>(rowinfo), static_cast<const int *>(offset), E, row_bytes,
-                      nvfp4 ? kNvImages : 1, int64_t(L.Rp), act_sf_bytes(L.chunk_rows), nseg, seg_vec, x, x_sf,
-                      ws + L.off_xg, ws + L.off_xg_sf);
+                      nvfp4 ? kNvImages : 1, int64_t(L.Rp), act_sf_bytes(L.chunk_rows),
+                      act_sf_bytes(kChunkRowsSmall), nseg, seg_vec, x, x_sf, ws + L.off_xg, ws + L.off_xg_sf,
+                      ws + L.off_xg_sf_s);
 }
 
 }  // namespace moe

@@ -52,12 +52,17 @@ def test_sizes_are_host_only_and_consistent(moelib):
 
 def test_forward_kernel_launches(moelib):
     """One-block routing up to T*k = 1024 routed rows (2 kernels), block-scan
-    routing above (5), plus GEMM1, GEMM2 and the combine; nothing for T = 0."""
+    routing above (5), plus GEMM1, GEMM2 and the combine; above T*k = 8E
+    (160-row chunks) GEMM1 and GEMM2 run once more over the side list of
+    lightly loaded experts; nothing for T = 0."""
     import moe_expert_layer_08_b200 as m
     assert m.forward_kernel_launches(8, 384, 6, 7168, 3072) == 5
     assert m.forward_kernel_launches(170, 384, 6, 7168, 3072) == 5     # 1020 rows
     assert m.forward_kernel_launches(171, 384, 6, 7168, 3072) == 8     # 1026 rows
-    assert m.forward_kernel_launches(8192, 384, 6, 7168, 3072) == 8
+    assert m.forward_kernel_launches(512, 384, 6, 7168, 3072) == 8     # 3072 rows = 8E: 32-row chunks
+    assert m.forward_kernel_launches(513, 384, 6, 7168, 3072) == 10    # side list
+    assert m.forward_kernel_launches(8192, 384, 6, 7168, 3072) == 10
+    assert m.forward_kernel_launches(64, 8, 2, 256, 256) == 7          # one-block routing, side list
     assert m.forward_kernel_launches(0, 8, 2, 256, 256) == 0
     with pytest.raises(m.MoEError):
         m.forward_kernel_launches(4, 8, 9, 256, 256)                   # k > E

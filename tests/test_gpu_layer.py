@@ -143,6 +143,29 @@ def test_layer_split_units(moe, w, experts):
     assert status == 0
 
 
+def side_list_routing(w, counts, seed):
+    """Routing with the given rows per expert (T*k in total), slots shuffled."""
+    ids = np.repeat(np.arange(len(counts)), counts)
+    assert ids.size == w.T * w.k
+    np.random.default_rng(seed).shuffle(ids)
+    idx = torch.as_tensor(ids.reshape(w.T, w.k), dtype=torch.int64)
+    tw = torch.rand((w.T, w.k), generator=torch.Generator().manual_seed(seed)) + 0.1
+    return idx, (tw / tw.sum(1, keepdim=True)).float()
+
+
+# T*k > 8E: 160-row chunks for the main list; experts with at most 32 rows
+# (here 32, 31 and 1; two experts get none) go to the side list of 32-row chunks
+SIDE_COUNTS = [32, 33, 1, 0, 31, 60, 43, 0]
+
+
+def test_layer_side_list(moe):
+    """Both chunk lists in one forward: the boundary loads (32 rows: side; 33:
+    main), an expert with one row and experts with none."""
+    w = W.custom("side_list", T=100, E=8, k=2, H=384, I=256, seed=61)
+    status, _ = run_and_compare(moe, w, routing=side_list_routing(w, SIDE_COUNTS, 61))
+    assert status == 0
+
+
 def test_layer_decode_full(moe):
     w = W.WORKLOADS[1]            # T=8, E=384, k=6, H=7168, I=3072: every token
     status, _ = run_and_compare(moe, w)

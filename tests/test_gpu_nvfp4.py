@@ -121,6 +121,13 @@ def test_nvfp4_layer_split_units(moe):
     assert run_and_compare_nv(moe, w, routing=(idx, tw)) == 0
 
 
+def test_nvfp4_layer_side_list(moe):
+    """NVFP4 with both chunk lists (160-row main chunks, 32-row side chunks)."""
+    from test_gpu_layer import SIDE_COUNTS, side_list_routing
+    w = W.custom("nv_side_list", T=100, E=8, k=2, H=512, I=256, seed=87)
+    assert run_and_compare_nv(moe, w, routing=side_list_routing(w, SIDE_COUNTS, 87)) == 0
+
+
 def test_nvfp4_layer_situ(moe):
     assert run_and_compare_nv(moe, W.custom("nv_situ", T=40, E=6, k=2, H=256, I=256, seed=85), situ=(1.25, 1.5)) == 0
 
