@@ -162,6 +162,10 @@ bool encode_act(CUtensorMap *m, const void *base, int64_t rows, int64_t kblocks,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
 int num_sms() {
     static std::mutex mu;
     static int cache[64] = {0};
@@ -176,10 +180,6 @@ int num_sms() {
     }
     return cache[dev];
 }
-
-moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
-
-}  // namespace
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

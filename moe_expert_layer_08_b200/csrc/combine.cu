@@ -15,63 +15,70 @@ constexpr int kCombineBatch = 8;                   // top-k up to this many: loa
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfloat16 *__restrict__ y,
                                                                   const int *__restrict__ inv,
                                                                   const float *__restrict__ topk_w, int k, int H,
-                                                                  int col_blocks, __nv_bfloat16 *__restrict__ out) {
+                                                                  int col_blocks, int T,
+                                                                  __nv_bfloat16 *__restrict__ out) {
     pdl_wait();
     pdl_trigger();
-    const int64_t t = blockIdx.x / col_blocks;
-    const int col = (blockIdx.x % col_blocks) * kCombineCols + threadIdx.x * 8;
-    if (col >= H) return;
-    float acc[8];
+    // blocks stride over (token, 1024-column block) tasks
+    for (int64_t task = blockIdx.x; task < int64_t(T) * col_blocks; task += gridDim.x) {
+        const int64_t t = task / col_blocks;
+        const int col = int(task % col_blocks) * kCombineCols + threadIdx.x * 8;
+        if (col >= H) continue;
+        float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    auto add = [&](const uint4 &v, float wv) {
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        auto add = [&](const uint4 &v, float wv) {
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] += wv * __uint_as_float(u[i] << 16);
+                acc[2 * i + 1] += wv * __uint_as_float(u[i] & 0xFFFF0000u);
+            }
+        };
+        if (k <= kCombineBatch) {
+            // all of the token's row indices, then all row loads in flight at once;
+            // the sum still runs over j ascending
+            int r[kCombineBatch];
+            float wv[kCombineBatch];
+            uint4 v[kCombineBatch];
+#pragma unroll
+            for (int j = 0; j < kCombineBatch; ++j) {
+                r[j] = j < k ? __ldcg(inv + t * k + j) : -1;
+                wv[j] = j < k ? __ldg(topk_w + t * k + j) : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < kCombineBatch; ++j)
+                if (r[j] >= 0) v[j] = __ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r[j]) * H + col));
+#pragma unroll
+            for (int j = 0; j < kCombineBatch; ++j)
+                if (r[j] >= 0) add(v[j], wv[j]);  // r < 0: dropped slot
+        } else {
+            for (int j = 0; j < k; ++j) {
+                const int r = __ldcg(inv + t * k + j);
+                if (r < 0) continue;  // dropped slot
+                add(__ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col)), __ldg(topk_w + t * k + j));
+            }
+        }
+        uint32_t o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            acc[2 * i] += wv * __uint_as_float(u[i] << 16);
-            acc[2 * i + 1] += wv * __uint_as_float(u[i] & 0xFFFF0000u);
+            const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+            o[i] = *reinterpret_cast<const uint32_t *>(&b);
         }
-    };
-    if (k <= kCombineBatch) {
-        // all of the token's row indices, then all row loads in flight at once;
-        // the sum still runs over j ascending
-        int r[kCombineBatch];
-        float wv[kCombineBatch];
-        uint4 v[kCombineBatch];
-#pragma unroll
-        for (int j = 0; j < kCombineBatch; ++j) {
-            r[j] = j < k ? __ldcg(inv + t * k + j) : -1;
-            wv[j] = j < k ? __ldg(topk_w + t * k + j) : 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < kCombineBatch; ++j)
-            if (r[j] >= 0) v[j] = __ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r[j]) * H + col));
-#pragma unroll
-        for (int j = 0; j < kCombineBatch; ++j)
-            if (r[j] >= 0) add(v[j], wv[j]);  // r < 0: dropped slot
-    } else {
-        for (int j = 0; j < k; ++j) {
-            const int r = __ldcg(inv + t * k + j);
-            if (r < 0) continue;  // dropped slot
-            add(__ldcg(reinterpret_cast<const uint4 *>(y + int64_t(r) * H + col)), __ldg(topk_w + t * k + j));
-        }
+        *reinterpret_cast<uint4 *>(out + t * H + col) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        o[i] = *reinterpret_cast<const uint32_t *>(&b);
-    }
-    *reinterpret_cast<uint4 *>(out + t * H + col) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
                            void *out, cudaStream_t stream) {
     const int col_blocks = (H + kCombineCols - 1) / kCombineCols;
-    const int64_t grid = int64_t(T) * col_blocks;
+    // at most 16 blocks (2048 threads) per SM, each looping over tasks: fewer,
+    // longer-lived blocks than one per task keep more loads in flight
+    const int64_t tasks = int64_t(T) * col_blocks, cap = int64_t(num_sms()) * 16;
+    const int64_t grid = tasks < cap ? tasks : cap;
     return launch_pdl(combine_kernel, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
                       reinterpret_cast<const __nv_bfloat16 *>(ws + L.off_y),
-                      reinterpret_cast<const int *>(ws + L.off_inv), topk_w, k, H, col_blocks,
+                      reinterpret_cast<const int *>(ws + L.off_inv), topk_w, k, H, col_blocks, T,
                       static_cast<__nv_bfloat16 *>(out));
 }
 

@@ -90,6 +90,9 @@ constexpr int kActBoxRows = 32;  // activation rows per TMA box
 cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
                            void *out, cudaStream_t stream);
 
+// Multiprocessors of the current device (cached per device).
+int num_sms();
+
 // Argument checks shared by the entry points.
 bool aligned(const void *p, uintptr_t a);
 moe_status_t check_shape(int E, int H, int I);
