@@ -18,6 +18,9 @@ Parity status of each function (the pins are the ``-m "not gpu"`` tests in
 * ``forward``: pinned against a float64 numpy evaluation of every selected
   expert on tiny inputs, the dense single-expert special case and layer
   invariants (token-permutation equivariance, identical experts, determinism).
+* ``shared_forward`` (the BF16 shared expert): pinned against a float64 numpy
+  evaluation with torch's bf16 rounding between the steps, the dense identity
+  special case and token-permutation equivariance.
 """
 from __future__ import annotations
 
@@ -93,6 +96,9 @@ def _declare(lib):
     lib.oracle_nvfp4_scale.argtypes = [c.c_double]
     lib.oracle_quantize_nvfp4.restype = None
     lib.oracle_quantize_nvfp4.argtypes = [P, c.c_int64, c.c_int64, P, P]
+    lib.oracle_shared_forward.restype = c.c_int
+    lib.oracle_shared_forward.argtypes = [P, P, P, c.c_int, c.c_int, c.c_int, P, c.c_int, c.c_int,
+                                          c.c_int, c.c_double, c.c_double, P, P]
     lib.oracle_moe_forward.restype = c.c_int
     lib.oracle_moe_forward.argtypes = [P, P, P, P, P, P, P, P,
                                        c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
@@ -280,6 +286,37 @@ def forward(x_codes, x_sf, topk_idx, topk_w, experts: dict, E: int, H: int, I: i
     res = dict(out_bf16=out_bf16, out_f32=out_f32)
     if intermediates:
         res.update(h_pre=h_pre, h_q=h_q, h_sf=h_sf, y=y)
+    return res
+
+
+def shared_forward(x_bits, l1_bits, l2_bits, tokens=None, activation: str = "swiglu", beta: float = 1.0,
+                   linear_beta=None, threads: int = 0, intermediates: bool = False, lib=None):
+    """The BF16 shared expert (bf16 bit patterns as uint16): x [T, SH], l1
+    [2 SI, SH] (gate rows first), l2 [SH, SI].  Returns dict with ``y`` [ntok,
+    SH] (bf16 bits) and, with ``intermediates``, ``h`` [ntok, SI] (the rounded
+    activation)."""
+    lib = lib or load()
+    x = _c(x_bits, np.uint16)
+    l1 = _c(l1_bits, np.uint16)
+    l2 = _c(l2_bits, np.uint16)
+    T, SH = x.shape
+    SI = l1.shape[0] // 2
+    assert l1.shape == (2 * SI, SH) and l2.shape == (SH, SI)
+    if tokens is None:
+        tok, ntok = None, T
+    else:
+        tok = _c(tokens, np.int32)
+        ntok = int(tok.size)
+    y = np.empty((ntok, SH), np.uint16)
+    h = np.empty((ntok, SI), np.uint16) if intermediates else None
+    act = {"swiglu": 0, "situ": 1}[activation]
+    rc = lib.oracle_shared_forward(_ptr(x), _ptr(l1), _ptr(l2), T, SH, SI, _ptr(tok), ntok, threads, act,
+                                   float(beta), float(linear_beta or 0.0), _ptr(y), _ptr(h))
+    if rc != 0:
+        raise ValueError(f"oracle_shared_forward rejected its arguments (rc={rc})")
+    res = dict(y=y)
+    if intermediates:
+        res["h"] = h
     return res
 
 

@@ -616,3 +616,120 @@ int oracle_moe_forward(const uint8_t *x, const uint8_t *x_sf,
                                   tokens, ntok, use_double, nthreads, 0, 1.0, 0.0,
                                   out_bf16, out_f32, h_pre, h_q, h_sf, y);
 }
+
+/* ------------------------------------------------------------------ */
+/* BF16 shared expert                                                  */
+/* ------------------------------------------------------------------ */
+
+/* The optional dense expert of DeepGEMM PR #416 (its BF16 shared-expert test
+ * body defines it), run on every token beside the routed experts and written
+ * to its own output.  With bf16 values x [T, SH], L1 [2 SI, SH] (gate rows
+ * 0..SI-1, up rows SI..2 SI-1) and L2 [SH, SI]:
+ *   gate, up = bf16_rne(x . L1^T)          (the linear layer's bf16 output)
+ *   h        = bf16_rne(act(gate, up))     (SwiGLU or SiTU, as above)
+ *   y        = bf16_rne(h . L2^T)
+ * The dot products are exact sums in double, ascending k (the test body
+ * leaves the accumulation to its bf16 linear layer; any order of a sum of
+ * bf16 products rounds to the same bf16 value except near ties). */
+
+static double bf16_value(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+static double bf16_round(double v)
+{
+    return bf16_value(oracle_f32_to_bf16((float)v));
+}
+
+typedef struct {
+    const uint16_t *x, *l1, *l2;
+    int SH, SI, activation;
+    double beta, linear_beta;
+    const int32_t *tokens;
+    int ntok;
+    uint16_t *y;   /* [ntok, SH] */
+    uint16_t *h;   /* [ntok, SI] or NULL */
+    int next;
+} shared_job_t;
+
+static void shared_token(shared_job_t *J, int p, double *xd, double *hd)
+{
+    const int SH = J->SH, SI = J->SI;
+    const int t = J->tokens ? J->tokens[p] : p;
+    for (int kk = 0; kk < SH; kk++)
+        xd[kk] = bf16_value(J->x[(int64_t)t * SH + kk]);
+    for (int i = 0; i < SI; i++) {
+        double g = 0.0, u = 0.0;
+        for (int kk = 0; kk < SH; kk++) {
+            g += xd[kk] * bf16_value(J->l1[(int64_t)i * SH + kk]);
+            u += xd[kk] * bf16_value(J->l1[(int64_t)(SI + i) * SH + kk]);
+        }
+        g = bf16_round(g);
+        u = bf16_round(u);
+        double a;
+        if (J->activation == 0) {
+            a = g / (1.0 + exp(-g)) * u;
+        } else {
+            double up = J->linear_beta > 0 ? J->linear_beta * tanh(u / J->linear_beta) : u;
+            a = (1.0 / (1.0 + exp(-g))) * (J->beta * tanh(g / J->beta)) * up;
+        }
+        hd[i] = bf16_round(a);
+        if (J->h)
+            J->h[(int64_t)p * SI + i] = oracle_f32_to_bf16((float)hd[i]);
+    }
+    for (int c = 0; c < SH; c++) {
+        double s = 0.0;
+        for (int i = 0; i < SI; i++)
+            s += hd[i] * bf16_value(J->l2[(int64_t)c * SI + i]);
+        J->y[(int64_t)p * SH + c] = oracle_f32_to_bf16((float)s);
+    }
+}
+
+static void *shared_worker(void *arg)
+{
+    shared_job_t *J = (shared_job_t *)arg;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)J->SH);
+    double *hd = (double *)malloc(sizeof(double) * (size_t)J->SI);
+    for (;;) {
+        int p = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (p >= J->ntok)
+            break;
+        shared_token(J, p, xd, hd);
+    }
+    free(xd);
+    free(hd);
+    return NULL;
+}
+
+/* The shared expert for `ntok` tokens (tokens == NULL: 0..ntok-1); all arrays
+ * bf16 bit patterns.  activation 0: SwiGLU, 1: SiTU(beta, linear_beta; 0 =
+ * none).  y: [ntok, SH]; h: [ntok, SI] (the rounded intermediate) or NULL.
+ * Returns 0, or -2 on a bad argument.  One thread per token. */
+int oracle_shared_forward(const uint16_t *x, const uint16_t *l1, const uint16_t *l2, int T, int SH, int SI,
+                          const int32_t *tokens, int ntok, int nthreads, int activation, double beta,
+                          double linear_beta, uint16_t *y, uint16_t *h)
+{
+    if (!x || !l1 || !l2 || !y || T < 0 || SH <= 0 || SI <= 0 || ntok < 0)
+        return -2;
+    if (activation == 1 && !(beta > 0))
+        return -2;
+    for (int p = 0; p < ntok; p++)
+        if (tokens && (tokens[p] < 0 || tokens[p] >= T))
+            return -2;
+    shared_job_t J = {x, l1, l2, SH, SI, activation, beta, linear_beta, tokens, ntok, y, h, 0};
+    int n = oracle_num_threads(nthreads);
+    if (n > ntok)
+        n = ntok > 0 ? ntok : 1;
+    pthread_t th[256];
+    if (n > 256)
+        n = 256;
+    for (int i = 0; i < n; i++)
+        pthread_create(&th[i], NULL, shared_worker, &J);
+    for (int i = 0; i < n; i++)
+        pthread_join(th[i], NULL);
+    return 0;
+}
