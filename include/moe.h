@@ -383,6 +383,39 @@ moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf,
                                 int32_t *expert_stats, void *const *stage_events,
                                 moe_stream_t stream);
 
+/*
+ * BF16 shared expert (DeepGEMM PR #416, "BF16 shared expert" test body: an
+ * optional dense expert that runs on every token beside the routed experts,
+ * with bf16 input, weights and its own bf16 output).  With x [T, SH],
+ * L1 [2 SI, SH] (rows 0..SI-1 gate, SI..2 SI-1 up) and L2 [SH, SI]:
+ *   gate, up = bf16_rne(x . L1^T);  h = bf16_rne(act(gate, up));
+ *   y = bf16_rne(h . L2^T)
+ * with fp32 accumulation on the tensor cores (tcgen05 kind::f16) and act
+ * SwiGLU or SiTU (moe_activation_t, as for the routed layer).
+ *
+ * moe_shared_workspace_bytes -- bytes of device workspace moe_shared_forward
+ *   needs for up to T_max tokens (a 2 KiB header with the device error word,
+ *   then h [T, SI] bf16).  MOE_ERR_UNSUPPORTED_SHAPE unless SH and SI are
+ *   multiples of 128.
+ *
+ * moe_shared_forward -- y for T tokens.  All pointers are device pointers on
+ *   one device, row-major and contiguous: x_bf16 [T, SH], l1_bf16 [2 SI, SH],
+ *   l2_bf16 [SH, SI], out_bf16 [T, SH] (fully overwritten), all 16-byte
+ *   aligned; workspace 256-byte aligned, ws_bytes >= moe_shared_workspace_bytes
+ *   (T, SH, SI) (else MOE_ERR_WORKSPACE_TOO_SMALL).  activation NULL means
+ *   SwiGLU.  The caller owns every buffer; the call allocates nothing,
+ *   enqueues a 2 KiB memset of the workspace header and two kernels on
+ *   `stream`, and does not synchronise.  T = 0 enqueues nothing.  Argument
+ *   errors (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE) are returned
+ *   before any CUDA call; a device-side wait that times out is reported by
+ *   moe_check_device_error(workspace) as MOE_ERR_DEVICE_TIMEOUT.
+ */
+moe_status_t moe_shared_workspace_bytes(int T_max, int SH, int SI, size_t *bytes);
+moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const void *l2_bf16,
+                                void *out_bf16, int T, int SH, int SI,
+                                const moe_activation_t *activation, void *workspace, size_t ws_bytes,
+                                moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

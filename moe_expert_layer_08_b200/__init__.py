@@ -21,7 +21,7 @@ __all__ = [
     "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
-    "forward_nvfp4",
+    "forward_nvfp4", "shared_workspace_bytes", "shared_forward",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -104,6 +104,8 @@ def _declare(lib):
         "moe_transform_scales": (I32, [P, P, I32, I32, I32, P, P, P]),
         "moe_forward_weights": (I32, [P, P, P, P, c.POINTER(Weights), P, I32, I32, I32, I32, I32, P, SZ, P, P,
                                       c.POINTER(Activation), P]),
+        "moe_shared_workspace_bytes": (I32, [I32, I32, I32, c.POINTER(SZ)]),
+        "moe_shared_forward": (I32, [P, P, P, P, I32, I32, I32, c.POINTER(Activation), P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -381,6 +383,39 @@ def forward_nvfp4(x_fp4, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: 
                                   _ptr(out), T, E, k, H, I, _ptr(workspace), workspace.numel(), _ptr(expert_stats),
                                   ev, ctypes.byref(act) if act is not None else None, _stream(stream))
     _check(st, "moe_forward_nvfp4")
+    return out
+
+
+def shared_workspace_bytes(T_max: int, SH: int, SI: int) -> int:
+    """Device workspace bytes of shared_forward for up to T_max tokens."""
+    n = ctypes.c_size_t()
+    _check(load().moe_shared_workspace_bytes(T_max, SH, SI, ctypes.byref(n)), "moe_shared_workspace_bytes")
+    return n.value
+
+
+def shared_forward(x, l1, l2, out=None, workspace=None, act=None, stream=None):
+    """The BF16 shared expert: x [T, SH], l1 [2 SI, SH] (gate rows first), l2
+    [SH, SI], all bf16; returns y (bf16 [T, SH]).  ``act``: an Activation, None
+    = SwiGLU."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(l1, torch.bfloat16, "l1", 2)
+    _need(l2, torch.bfloat16, "l2", 2)
+    T, SH = x.shape
+    SI = l1.shape[0] // 2
+    if l1.shape != (2 * SI, SH) or l2.shape != (SH, SI):
+        raise ValueError("inconsistent shared-expert shapes")
+    if out is None:
+        out = torch.empty((T, SH), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, torch.bfloat16, "out", 2)
+    if workspace is None:
+        workspace = torch.empty(shared_workspace_bytes(T, SH, SI), dtype=torch.uint8, device=x.device)
+    else:
+        _need(workspace, torch.uint8, "workspace")
+    st = load().moe_shared_forward(_ptr(x), _ptr(l1), _ptr(l2), _ptr(out), T, SH, SI,
+                                   ctypes.byref(act) if act is not None else None, _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _check(st, "moe_shared_forward")
     return out
 
 

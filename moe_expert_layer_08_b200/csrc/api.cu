@@ -166,6 +166,18 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
 
 }  // namespace
 
+bool encode_bf16_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, int box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(cols * 2)};
+    const cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int num_sms() {
     static std::mutex mu;
     static int cache[64] = {0};
@@ -569,6 +581,56 @@ moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H,
     if (e == cudaSuccess && inv && L.R > 0)
         e = cudaMemcpyAsync(inv, ws + L.off_inv, sizeof(int32_t) * L.R, cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e);
+}
+
+// ---------------------------------------------------------------- BF16 shared expert
+static size_t shared_ws_bytes(int T, int SI) { return kHdrBytes + align_up(size_t(T) * size_t(SI) * 2, 256); }
+
+moe_status_t moe_shared_workspace_bytes(int T_max, int SH, int SI, size_t *bytes) {
+    if (!bytes || T_max < 0 || SH <= 0 || SI <= 0) return MOE_ERR_INVALID_ARG;
+    if (SH % kTileRows || SI % kTileRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+    *bytes = shared_ws_bytes(T_max, SI);
+    return MOE_OK;
+}
+
+moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const void *l2_bf16, void *out_bf16, int T,
+                                int SH, int SI, const moe_activation_t *activation, void *workspace,
+                                size_t ws_bytes, moe_stream_t stream) {
+    moe_activation_t act = {MOE_ACT_SWIGLU, 1.0f, 0.0f};
+    if (activation) {
+        act = *activation;
+        if (act.kind == MOE_ACT_SITU) {
+            if (!(act.beta > 0.0f) || !isfinite(act.beta) || !(act.linear_beta >= 0.0f) || !isfinite(act.linear_beta))
+                return MOE_ERR_INVALID_ARG;
+        } else if (act.kind != MOE_ACT_SWIGLU) {
+            return MOE_ERR_INVALID_ARG;
+        }
+    }
+    if (T < 0 || SH <= 0 || SI <= 0) return MOE_ERR_INVALID_ARG;
+    if (SH % kTileRows || SI % kTileRows) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!x_bf16 || !l1_bf16 || !l2_bf16 || !out_bf16 || !workspace) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(l1_bf16, 16) || !aligned(l2_bf16, 16) || !aligned(out_bf16, 16) ||
+        !aligned(workspace, 256))
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < shared_ws_bytes(T, SI)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    moe_status_t s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *h = ws + kHdrBytes;
+    const int kn = shared_block_rows(T);
+    CUtensorMap tm_l1, tm_x, tm_l2, tm_h;
+    if (!encode_bf16_rows(&tm_l1, l1_bf16, uint64_t(SH), uint64_t(2) * SI, kTileRows) ||
+        !encode_bf16_rows(&tm_x, x_bf16, uint64_t(SH), uint64_t(T), kn) ||
+        !encode_bf16_rows(&tm_l2, l2_bf16, uint64_t(SI), uint64_t(SH), kTileRows) ||
+        !encode_bf16_rows(&tm_h, h, uint64_t(SI), uint64_t(T), kn))
+        return MOE_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int *hdr = reinterpret_cast<int *>(ws);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHdrBytes, st);  // error word of this call
+    if (e == cudaSuccess) e = launch_shared(true, tm_l1, tm_x, T, SH, SI, h, hdr, act, st);
+    if (e == cudaSuccess) e = launch_shared(false, tm_l2, tm_h, T, SH, SI, out_bf16, hdr, act, st);
     return cuda_status(e);
 }
 

@@ -313,6 +313,18 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uin
         : "memory");
 }
 
+// D[M=128, N] (+)= A . B^T with A and B both bf16 (K = 16 per instruction,
+// 32 bytes of each operand row), fp32 accumulator in TMEM.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // 32 lanes x 32 columns of 32-bit words: thread l of the warp gets lane (base + l).
 __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -349,6 +361,15 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
     d |= uint64_t(128 >> 4) << 32;
     d |= uint64_t(1) << 46;
     return d;
+}
+// Instruction descriptor of kind::f16 MMA: fp32 accumulator, A and B both
+// bf16 (format 1), K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_bf16(uint32_t n) {
+    return (1u << 4)             // D format: F32
+           | (1u << 7)           // A format: BF16
+           | (1u << 10)          // B format: BF16
+           | ((n >> 3) << 17)    // N / 8
+           | ((128u >> 4) << 24);// M / 16
 }
 // Instruction descriptor of kind::mxf4nvf4 block-scaled MMA with 16-element
 // scale vectors: A and B E2M1 (format 1), K-major, M = 128, N = n, UE4M3

@@ -1,0 +1,325 @@
+// shared.cu -- the BF16 shared expert (DeepGEMM PR #416: an optional dense
+// expert that runs on every token beside the routed experts, bf16 input,
+// weights and output; its test body defines the computation):
+//   gate, up = bf16(x . L1^T)   (L1 rows 0..SI-1 gate, SI..2SI-1 up)
+//   h        = bf16(act(gate, up))           (SwiGLU or SiTU)
+//   y        = bf16(h . L2^T)
+// Two persistent kernels, GEMM1 (+ activation) and GEMM2, on sm_100a tensor
+// cores (tcgen05.mma.kind::f16, bf16 x bf16 -> fp32 in TMEM).  A work item is
+// (block of kN tokens, pair of 128-row weight tiles); items are token-block
+// major, so the CTAs working at one time share a token block (L2-resident) and
+// every weight tile is re-read from L2 by later blocks.  Operands come by TMA
+// straight from the row-major bf16 tensors (64 elements = one 128-byte
+// swizzled row per K block): no gather and no layout transform.  Per CTA:
+// warp 0 loads the two weight tiles, warp 6 the token tile, warps 1 and 7
+// issue the MMAs of tile 0 and 1, and warps 2-5 (and 8-11 with 128-token
+// blocks) drain the double-buffered TMEM accumulators.  Every wait is bounded
+// (workspace error word, as in the routed layer).
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+template <int kN>
+struct SharedCfg {
+    static constexpr int kStages = kN == 128 ? 4 : 6;
+    static constexpr int kATile = kTileRows * kTileK;  // 16 KB: 128 rows x 64 bf16
+    static constexpr int kBTile = kN * kTileK;
+    static constexpr int kStageBytes = 2 * kATile + kBTile;
+    static constexpr int kSmemMisc = 256;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kSmemMisc;
+    static constexpr int kAccCols = 2 * kN;  // one accumulator buffer: tile 0, tile 1
+    static constexpr int kTmemCols = 4 * kN <= 128 ? 128 : 512;
+    static constexpr int kEpiWarps = kN == 128 ? 8 : 4;
+    static constexpr int kThreads = 32 * (kEpiWarps == 8 ? 12 : 8);
+    static_assert(4 * kN <= kTmemCols, "two accumulator buffers");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kBTile % 1024 == 0, "swizzle atoms");
+    static_assert(8 * (2 * kStages + 6) + 8 <= kSmemMisc, "barriers and flags");
+};
+
+struct SharedArgs {
+    int T;             // tokens
+    int K;             // reduction length (SH for GEMM1, SI for GEMM2)
+    int n_tiles;       // 128-row output tiles (GEMM1: SI / 128 per half, GEMM2: SH / 128)
+    int n_items;       // tile pairs per token block
+    int second_row;    // GEMM1: row of the up tile relative to the gate tile (SI); GEMM2: 128
+    int out_ld;        // row length of the output (SI or SH)
+    __nv_bfloat16 *out;
+    int *hdr;          // workspace header (error word)
+    int act_kind;      // GEMM1: MOE_ACT_SWIGLU or MOE_ACT_SITU
+    float beta, inv_beta, lbeta, inv_lbeta;
+};
+
+__device__ __forceinline__ float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+
+template <bool kGemm1, int kN>
+__global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
+    shared_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_act,
+                       const SharedArgs args) {
+    using C = SharedCfg<kN>;
+    constexpr int kStages = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(tiles + kStages * C::kStageBytes);
+    uint64_t *empty = full + kStages;
+    uint64_t *tmem_full = empty + kStages;   // [2]
+    uint64_t *tmem_empty = tmem_full + 2;    // [2]
+    uint64_t *mma_done = tmem_empty + 2;     // [2]
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 2);   // weight producer + token producer
+            mbar_init(&empty[s], 2);  // both issuers
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], 2);
+            mbar_init(&tmem_empty[b], C::kEpiWarps);
+            mbar_init(&mma_done[b], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmap_w);
+        prefetch_tmap(&tmap_act);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    pdl_wait();
+    if (threadIdx.x == 32) pdl_trigger();
+
+    const int n_items = args.n_items, n_tiles = args.n_tiles;
+    const int n_blocks = (args.T + kN - 1) / kN;
+    const int num_items = n_blocks * n_items;
+    const int KB = args.K / 64;  // K blocks of 64 bf16 (128 bytes)
+    int *err = args.hdr;
+    // rows of weight tile a of tile pair `it`
+    auto tile_row = [&](int it, int a) {
+        return kGemm1 ? it * kTileRows + a * args.second_row : (2 * it + a) * kTileRows;
+    };
+
+    if (warp == 0 || warp == 6) {
+        if (lane == 0) {
+            // -------------------------------------------------------- producers
+            const bool weights = warp == 0;
+            // weights are re-read by every token block (keep them in L2); a token
+            // block is read by the CTAs of its items at about the same time
+            const uint64_t pol = weights ? policy_evict_last() : policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0, filled = 0, fill_parity = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
+                const int blk = item / n_items, it = item % n_items;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = tiles + stage * C::kStageBytes;
+                    if (weights) {
+                        // rows past the tensor (GEMM2's padded last pair) read as zeros
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(2 * C::kATile));
+                        tma_load_2d(st, &tmap_w, &full[stage], kb * 64, tile_row(it, 0), pol);
+                        tma_load_2d(st + C::kATile, &tmap_w, &full[stage], kb * 64, tile_row(it, 1), pol);
+                    } else {
+                        // tokens past T read as zeros
+                        mbar_arrive_expect_tx(&full[stage], uint32_t(C::kBTile));
+                        tma_load_2d(st + 2 * C::kATile, &tmap_act, &full[stage], kb * 64, blk * kN, pol);
+                    }
+                    filled |= 1u << stage;
+                    fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // every issued copy must have landed before the CTA may exit
+            for (int s = 0; s < kStages; ++s) {
+                if (!(filled >> s & 1u)) continue;
+                const uint32_t par = (fill_parity >> s) & 1u;
+                const unsigned long long t0 = global_timer_ns();
+                while (!mbar_try_wait(&full[s], par) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1 || warp == 7) {
+        if (lane == 0) {
+            // -------------------------------------------------------- MMA issuer of tile a
+            const int a = warp == 1 ? 0 : 1;
+            int stage = 0, li = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++li) {
+                const int blk = item / n_items, it = item % n_items;
+                const int rows = min(kN, args.T - blk * kN);
+                const uint32_t n = uint32_t((rows + 15) / 16 * 16);
+                const bool valid = kGemm1 || 2 * it + a < n_tiles;
+                const int buf = li & 1;
+                const uint32_t use = uint32_t(li >> 1) & 1u;
+                if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 12)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + uint32_t(buf * C::kAccCols + a * kN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, err, 13)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (valid) {
+                        const uint8_t *st = tiles + stage * C::kStageBytes;
+                        const uint64_t adesc = smem_desc_sw128(smem_u32(st + a * C::kATile));
+                        const uint64_t bdesc = smem_desc_sw128(smem_u32(st + 2 * C::kATile));
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            // 16 bf16 (32 bytes) of K per step inside the 128-byte swizzled row
+                            tc_mma_bf16(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks), idesc_bf16(n),
+                                        (kb == 0 && ks == 0) ? 0u : 1u);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&tmem_full[buf]);
+            }
+            // all issued MMAs must be finished before TMEM is released
+            tc_commit(&mma_done[a]);
+            const unsigned long long t0 = global_timer_ns();
+            while (!mbar_try_wait(&mma_done[a], 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+            }
+        }
+        __syncwarp();
+    } else if ((warp >= 2 && warp <= 5) || (C::kEpiWarps == 8 && warp >= 8)) {
+        // ------------------------------------------------------------ epilogue
+        // thread = output column (weight row) q * 32 + lane of a tile,
+        // registers = 32 consecutive tokens
+        const int q = warp & 3;
+        const int half = warp >= 8 ? 1 : 0;
+        constexpr int kCbStep = C::kEpiWarps / 4;
+        const uint32_t lane_base = uint32_t(q * 32) << 16;
+        int li = 0;
+        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
+            const int blk = item / n_items, it = item % n_items;
+            const int rows = min(kN, args.T - blk * kN);
+            const int buf = li & 1;
+            const uint32_t use = uint32_t(li >> 1) & 1u;
+            if (!mbar_wait(&tmem_full[buf], use, abort_flag, err, 14)) break;
+            tc_fence_after();
+            const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
+            const int ncb = (rows + 31) / 32;
+            for (int cb = half; cb < ncb; cb += kCbStep) {
+                const int tok0 = blk * kN + cb * 32;
+                if constexpr (kGemm1) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32(acc + uint32_t(cb * 32), g);
+                    tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
+                    tmem_ld_wait();
+                    __nv_bfloat16 *hb = args.out + int64_t(tok0) * args.out_ld + it * kTileRows + q * 32 + lane;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        // the linear layer's bf16 output, then the activation in fp32
+                        const float gv = bf16_round_f(__uint_as_float(g[j]));
+                        const float uv = bf16_round_f(__uint_as_float(u[j]));
+                        float hv;
+                        if (args.act_kind == MOE_ACT_SWIGLU) {
+                            hv = gv / (1.0f + expf(-gv)) * uv;
+                        } else {
+                            const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
+                            hv = (1.0f / (1.0f + expf(-gv))) * (args.beta * tanhf(gv * args.inv_beta)) * up;
+                        }
+                        if (cb * 32 + j < rows) hb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(hv);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int a = 0; a < 2; ++a) {
+                        const int tile = 2 * it + a;
+                        if (tile >= n_tiles) break;
+                        uint32_t v[32];
+                        tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), v);
+                        tmem_ld_wait();
+                        __nv_bfloat16 *yb = args.out + int64_t(tok0) * args.out_ld + tile * kTileRows + q * 32 + lane;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (cb * 32 + j < rows) yb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(__uint_as_float(v[j]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+template <bool kGemm1, int kN>
+static cudaError_t launch_shared_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, const SharedArgs &a,
+                                   int items, cudaStream_t stream) {
+    using C = SharedCfg<kN>;
+    static int configured_for = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_for != dev) {
+        const cudaError_t e = cudaFuncSetAttribute(shared_gemm_kernel<kGemm1, kN>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured_for = dev;
+    }
+    const int sms = num_sms();
+    const int grid = items < sms ? (items > 0 ? items : 1) : sms;
+    return launch_pdl(shared_gemm_kernel<kGemm1, kN>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
+                      tmap_w, tmap_act, a);
+}
+
+int shared_block_rows(int T) { return T <= kSharedSmallT ? 32 : 128; }
+
+cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, int T, int SH, int SI,
+                          void *out, int *hdr, const moe_activation_t &act, cudaStream_t stream) {
+    SharedArgs a{};
+    a.T = T;
+    a.hdr = hdr;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.act_kind = act.kind;
+    a.beta = act.beta;
+    a.inv_beta = act.kind == MOE_ACT_SITU ? 1.0f / act.beta : 0.0f;
+    a.lbeta = act.linear_beta;
+    a.inv_lbeta = (act.kind == MOE_ACT_SITU && act.linear_beta > 0.0f) ? 1.0f / act.linear_beta : 0.0f;
+    if (gemm1) {
+        a.K = SH;
+        a.n_tiles = SI / kTileRows;
+        a.n_items = SI / kTileRows;
+        a.second_row = SI;
+        a.out_ld = SI;
+    } else {
+        a.K = SI;
+        a.n_tiles = SH / kTileRows;
+        a.n_items = (SH / kTileRows + 1) / 2;
+        a.second_row = kTileRows;
+        a.out_ld = SH;
+    }
+    const int kn = shared_block_rows(T);
+    const int items = (T + kn - 1) / kn * a.n_items;
+    if (kn == 32)
+        return gemm1 ? launch_shared_t<true, 32>(tmap_w, tmap_act, a, items, stream)
+                     : launch_shared_t<false, 32>(tmap_w, tmap_act, a, items, stream);
+    return gemm1 ? launch_shared_t<true, 128>(tmap_w, tmap_act, a, items, stream)
+                 : launch_shared_t<false, 128>(tmap_w, tmap_act, a, items, stream);
+}
+
+}  // namespace moe

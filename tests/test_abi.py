@@ -179,3 +179,27 @@ def test_nvfp4_entry_points_validate_on_the_host(moelib):
     assert moelib.moe_forward_nvfp4(*args(k=9)) == 1
     assert moelib.moe_forward_nvfp4(*args(x=ctypes.c_void_p(264))) == 1      # misaligned x
     assert moelib.moe_forward_nvfp4(*args(T=0)) == 0
+
+
+def test_shared_expert_entry_points_validate_on_the_host(moelib):
+    """Workspace size = 2 KiB header + h [T, SI] bf16 (256-aligned); shapes,
+    token counts, activations and sizes are checked before any CUDA call."""
+    import ctypes
+    import moe_expert_layer_08_b200 as m
+    lib = m.load()
+    assert m.shared_workspace_bytes(8192, 7168, 2048) == 2048 + 8192 * 2048 * 2
+    assert m.shared_workspace_bytes(3, 256, 128) == 2048 + 768
+    assert m.shared_workspace_bytes(0, 256, 128) == 2048
+    n = ctypes.c_size_t()
+    assert lib.moe_shared_workspace_bytes(8, 200, 128, ctypes.byref(n)) == 2   # SH % 128
+    assert lib.moe_shared_workspace_bytes(8, 256, 100, ctypes.byref(n)) == 2   # SI % 128
+    assert lib.moe_shared_workspace_bytes(-1, 256, 128, ctypes.byref(n)) == 1
+    f = lib.moe_shared_forward
+    assert f(None, None, None, None, 0, 256, 128, None, None, 0, None) == 0     # T = 0: nothing to do
+    assert f(None, None, None, None, 4, 256, 128, None, None, 0, None) == 1     # null pointers
+    assert f(None, None, None, None, 4, 200, 128, None, None, 0, None) == 2     # SH % 128
+    assert f(None, None, None, None, -1, 256, 128, None, None, 0, None) == 1
+    bad = m.Activation(1, 0.0, 0.0)                                             # SiTU needs beta > 0
+    assert f(None, None, None, None, 4, 256, 128, ctypes.byref(bad), None, 0, None) == 1
+    fake = ctypes.c_void_p(1 << 20)                                            # never dereferenced
+    assert f(fake, fake, fake, fake, 4, 256, 128, None, fake, 16, None) == 3   # workspace too small

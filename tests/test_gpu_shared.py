@@ -1,0 +1,69 @@
+"""GPU parity of the BF16 shared expert (moe_shared_forward through the C ABI)
+against the oracle, per token row: rel L2 <= 1e-2 and max abs <= 5e-2 *
+max|row| (the DeepGEMM PR #416 test body bounds the shared output's relative
+L2 by 1e-2).  Small cases on every token, with both token-block sizes (32 up
+to 256 tokens, else 128), ragged token counts and an odd output-tile count;
+the full-size case on sampled tokens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from cases import compare_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe(moelib):
+    import moe_expert_layer_08_b200 as m
+    return m
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def run_and_compare(moe, T, SH, SI, seed, tokens=None, situ=None, repeat=True):
+    x, l1, l2 = W.gen_shared(T, SH, SI, seed, "cuda")
+    act = None if situ is None else moe.activation("situ", situ[0], situ[1])
+    ws = torch.empty(moe.shared_workspace_bytes(T, SH, SI), dtype=torch.uint8, device="cuda")
+    y = moe.shared_forward(x, l1, l2, workspace=ws, act=act)
+    assert moe.check_device_error(ws) == 0
+    if repeat:
+        y2 = moe.shared_forward(x, l1, l2, workspace=ws, act=act)
+        assert torch.equal(y.view(torch.int16), y2.view(torch.int16)), "not deterministic"
+    kw = {} if situ is None else dict(activation="situ", beta=situ[0], linear_beta=situ[1])
+    tok = None if tokens is None else np.asarray(tokens, np.int32)
+    ref = oracle.shared_forward(bits(x), bits(l1), bits(l2), tokens=tok, **kw)["y"]
+    got = y if tokens is None else y[torch.as_tensor(tok, device="cuda", dtype=torch.int64)]
+    return compare_rows(got, ref, f"shared T={T} SH={SH} SI={SI}")
+
+
+@pytest.mark.parametrize("T,SH,SI,seed", [
+    (1, 256, 128, 1),        # one token
+    (37, 512, 256, 2),       # ragged 32-token blocks
+    (300, 384, 256, 3),      # odd output-tile count: GEMM2's last pair holds one tile
+    (1100, 256, 128, 4),     # 128-token blocks, ragged last block
+    (250, 256, 256, 8),      # 32-token blocks at the largest such T
+])
+def test_shared_small(moe, T, SH, SI, seed):
+    run_and_compare(moe, T, SH, SI, seed)
+
+
+def test_shared_situ(moe):
+    run_and_compare(moe, 70, 256, 256, 5, situ=(1.25, 1.5))
+
+
+def test_shared_full_size_sampled(moe):
+    """T = 8192 tokens, SH = 7168, SI = 2048, 8 sampled tokens (incl. the first
+    and the last)."""
+    T = 8192
+    tokens = sorted(set(np.random.default_rng(6).choice(T, 6, replace=False).tolist()) | {0, T - 1})
+    run_and_compare(moe, T, 7168, 2048, 6, tokens=tokens, repeat=False)
+
+
+def test_shared_decode_size(moe):
+    """T = 8 tokens (32-token blocks, most SMs idle), SH = 7168, SI = 2048."""
+    run_and_compare(moe, 8, 7168, 2048, 7)

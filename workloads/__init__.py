@@ -99,6 +99,14 @@ def gen_l2(w: Workload, e: int, device="cpu") -> torch.Tensor:
     return _randn_bf16((w.H, w.I), 0.04, device, w.seed, "l2", e)
 
 
+def gen_shared(T: int, SH: int, SI: int, seed: int, device="cpu"):
+    """BF16 shared-expert inputs as the DeepGEMM PR #416 test body draws them:
+    x [T, SH] ~ N(0, 0.25^2), L1 [2 SI, SH] and L2 [SH, SI] ~ N(0, 0.02^2)."""
+    return (_randn_bf16((T, SH), 0.25, device, seed, "shared_x"),
+            _randn_bf16((2 * SI, SH), 0.02, device, seed, "shared_l1"),
+            _randn_bf16((SH, SI), 0.02, device, seed, "shared_l2"))
+
+
 def gen_routing(w: Workload, device="cpu"):
     """(topk_idx int64 [T, k], topk_w fp32 [T, k]) as the recipe above states."""
     g = _generator(device, w.seed, "route")
