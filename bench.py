@@ -53,7 +53,84 @@ def parse():
                    help="weight layout: tile packets, or row-major bodies with separate scale blocks")
     p.add_argument("--format", default="mx", choices=["mx", "nvfp4"],
                    help="mx: FP8 activations x FP4 weights, UE8M0 per 32; nvfp4: E2M1 x E2M1, UE4M3 per 16")
+    p.add_argument("--shared-expert", type=int, default=0, metavar="T",
+                   help="time the BF16 shared expert (moe_shared_forward) on T tokens instead of the layer")
+    p.add_argument("--shared-dims", default="7168,2048", help="SH,SI of the shared expert")
     return p.parse_args()
+
+
+SPEC_BF16_TFLOPS = 2250.0
+
+
+def run_shared(args, rank, world, local_rank):
+    """The BF16 shared expert alone: T tokens through moe_shared_forward, inputs
+    resident in HBM, CUDA events on the launch stream around K calls; beside
+    it the same computation as torch operators (cuBLAS GEMMs + elementwise
+    activation) for context."""
+    import moe_expert_layer_08_b200 as moe
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    T = args.shared_expert
+    SH, SI = (int(v) for v in args.shared_dims.split(","))
+    x, l1, l2 = W.gen_shared(T, SH, SI, 1, device)
+    ws = torch.empty(moe.shared_workspace_bytes(T, SH, SI), dtype=torch.uint8, device=device)
+    out = torch.empty((T, SH), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        barrier()
+        start.record(stream)
+        for _ in range(args.steps):
+            fn()
+        stop.record(stream)
+        barrier()
+        return max_over_ranks(start.elapsed_time(stop) / args.steps, device)
+
+    with ClockSampler(device.index) as clocks:
+        ms = timed(lambda: moe.shared_forward(x, l1, l2, out=out, workspace=ws))
+    st = moe.check_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {moe.STATUS.get(st, st)}")
+
+    def torch_ops():
+        g, u = torch.nn.functional.linear(x, l1).chunk(2, dim=-1)
+        h = (torch.nn.functional.silu(g.float()) * u.float()).to(torch.bfloat16)
+        return torch.nn.functional.linear(h, l2)
+
+    torch_ms = timed(torch_ops)
+    if rank != 0:
+        return
+    pk = peaks()
+    flops = 2.0 * T * 3 * SH * SI
+    tf = flops / (ms * 1e-3) / 1e12
+    wbytes = 3 * SH * SI * 2
+    line = {
+        "metric": f"BF16 shared expert TFLOP/s (SH={SH}, SI={SI})", "value": world * tf, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+        "dtype": "bf16 (fp32 accumulate)",
+        "config": {"workload": f"shared_expert_T{T}", "T": T, "SH": SH, "SI": SI, "activation": "swiglu",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "weights (88 MB at SH=7168, SI=2048) fit in L2; not flushed"},
+        "us_per_call": ms * 1e3,
+        "roofline": {"kernel": "shared_gemm_kernel (GEMM1 + GEMM2)", "bound": "tensor", "achieved": tf,
+                     "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": tf / pk["bf16_sustained"],
+                     "peak_source": pk["source"] + " sustained bf16", "frac_of_burst": tf / pk["bf16"],
+                     "spec": {"peak": SPEC_BF16_TFLOPS, "frac": tf / SPEC_BF16_TFLOPS},
+                     "weight_GBps": wbytes / (ms * 1e-3) / 1e9, "traffic": None},
+        "torch_ops_us": torch_ms * 1e3,
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def peaks():
@@ -447,7 +524,9 @@ def main():
         w = W.custom(f"{w.name}_T{T}_E{E}", T=T, E=E, k=w.k, H=w.H, I=w.I, seed=w.seed,
                      routing=w.routing, zipf_s=w.zipf_s)
     try:
-        if args.impl == "reference":
+        if args.shared_expert:
+            run_shared(args, rank, world, local_rank)
+        elif args.impl == "reference":
             run_reference(args, w, rank, world)
         else:
             run_b200(args, w, rank, world, local_rank)

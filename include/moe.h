@@ -395,7 +395,8 @@ moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf,
  *
  * moe_shared_workspace_bytes -- bytes of device workspace moe_shared_forward
  *   needs for up to T_max tokens (a 2 KiB header with the device error word,
- *   then h [T, SI] bf16).  MOE_ERR_UNSUPPORTED_SHAPE unless SH and SI are
+ *   then h [T, SI] bf16, then 8 MiB of fp32 partial sums for the K split that
+ *   small token counts use).  MOE_ERR_UNSUPPORTED_SHAPE unless SH and SI are
  *   multiples of 128.
  *
  * moe_shared_forward -- y for T tokens.  All pointers are device pointers on

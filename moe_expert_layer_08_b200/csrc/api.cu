@@ -585,7 +585,11 @@ moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H,
 }
 
 // ---------------------------------------------------------------- BF16 shared expert
-static size_t shared_ws_bytes(int T, int SI) { return kHdrBytes + align_up(size_t(T) * size_t(SI) * 2, 256); }
+// header (error word, split counters), h [T][SI] bf16, K-split partial sums
+static size_t shared_h_bytes(int T, int SI) { return align_up(size_t(T) * size_t(SI) * 2, 256); }
+static size_t shared_ws_bytes(int T, int SI) {
+    return kHdrBytes + shared_h_bytes(T, SI) + size_t(kMaxSplitUnits) * kPartUnitFloats * sizeof(float);
+}
 
 moe_status_t moe_shared_workspace_bytes(int T_max, int SH, int SI, size_t *bytes) {
     if (!bytes || T_max < 0 || SH <= 0 || SI <= 0) return MOE_ERR_INVALID_ARG;
@@ -629,8 +633,9 @@ moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const v
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int *hdr = reinterpret_cast<int *>(ws);
     cudaError_t e = cudaMemsetAsync(ws, 0, kHdrBytes, st);  // error word of this call
-    if (e == cudaSuccess) e = launch_shared(true, tm_l1, tm_x, T, SH, SI, h, hdr, act, st);
-    if (e == cudaSuccess) e = launch_shared(false, tm_l2, tm_h, T, SH, SI, out_bf16, hdr, act, st);
+    float *part = reinterpret_cast<float *>(ws + kHdrBytes + shared_h_bytes(T, SI));
+    if (e == cudaSuccess) e = launch_shared(true, tm_l1, tm_x, T, SH, SI, h, hdr, part, act, st);
+    if (e == cudaSuccess) e = launch_shared(false, tm_l2, tm_h, T, SH, SI, out_bf16, hdr, part, act, st);
     return cuda_status(e);
 }
 

@@ -35,7 +35,7 @@ struct SharedCfg {
     static_assert(4 * kN <= kTmemCols, "two accumulator buffers");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kBTile % 1024 == 0, "swizzle atoms");
-    static_assert(8 * (2 * kStages + 6) + 8 <= kSmemMisc, "barriers and flags");
+    static_assert(8 * (2 * kStages + 8) + 12 <= kSmemMisc, "barriers and flags");
 };
 
 struct SharedArgs {
@@ -47,6 +47,9 @@ struct SharedArgs {
     int out_ld;        // row length of the output (SI or SH)
     __nv_bfloat16 *out;
     int *hdr;          // workspace header (error word)
+    int split;         // K parts per item (1: none); parts > 1 only with 32-token blocks
+    float *part;       // split: fp32 partial accumulators [unit][tile][32 tokens][128 rows]
+    int *cnt;          // split: per item, parts finished (the last resets it)
     int act_kind;      // GEMM1: MOE_ACT_SWIGLU or MOE_ACT_SITU
     float beta, inv_beta, lbeta, inv_lbeta;
 };
@@ -66,8 +69,11 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     uint64_t *tmem_full = empty + kStages;   // [2]
     uint64_t *tmem_empty = tmem_full + 2;    // [2]
     uint64_t *mma_done = tmem_empty + 2;     // [2]
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 2);
+    uint64_t *epi_bar = mma_done + 2;        // split: the epilogue warps' partials written
+    uint64_t *epi_go = epi_bar + 1;          // split: the finishing decision taken
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(epi_go + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    volatile int *epi_last = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -80,6 +86,8 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
             mbar_init(&tmem_empty[b], C::kEpiWarps);
             mbar_init(&mma_done[b], 1);
         }
+        mbar_init(epi_bar, C::kEpiWarps);
+        mbar_init(epi_go, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_w);
@@ -100,6 +108,11 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     const int n_blocks = (args.T + kN - 1) / kN;
     const int num_items = n_blocks * n_items;
     const int KB = args.K / 64;  // K blocks of 64 bf16 (128 bytes)
+    // work units: item u / split, K blocks [kb_lo(u), kb_hi(u)) of its K
+    const int split = kN == 32 ? args.split : 1;
+    const int num_units = num_items * split;
+    auto kb_lo = [&](int u) { return (u % split) * KB / split; };
+    auto kb_hi = [&](int u) { return (u % split + 1) * KB / split; };
     int *err = args.hdr;
     // rows of weight tile a of tile pair `it`
     auto tile_row = [&](int it, int a) {
@@ -116,9 +129,9 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_parity = 0;
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
-                const int blk = item / n_items, it = item % n_items;
-                for (int kb = 0; kb < KB; ++kb) {
+            for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+                const int item = u / split, blk = item / n_items, it = item % n_items;
+                for (int kb = kb_lo(u); kb < kb_hi(u); ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, 11)) {
                         ok = false;
                         break;
@@ -159,8 +172,9 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
             int stage = 0, li = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++li) {
-                const int blk = item / n_items, it = item % n_items;
+            for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x, ++li) {
+                const int item = u / split, blk = item / n_items, it = item % n_items;
+                const int k0 = kb_lo(u);
                 const int rows = min(kN, args.T - blk * kN);
                 const uint32_t n = uint32_t((rows + 15) / 16 * 16);
                 const bool valid = kGemm1 || 2 * it + a < n_tiles;
@@ -169,7 +183,7 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 12)) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + uint32_t(buf * C::kAccCols + a * kN);
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = k0; kb < kb_hi(u); ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag, err, 13)) {
                         ok = false;
                         break;
@@ -183,7 +197,7 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                         for (int ks = 0; ks < 4; ++ks)
                             // 16 bf16 (32 bytes) of K per step inside the 128-byte swizzled row
                             tc_mma_bf16(acc, adesc + uint64_t(2 * ks), bdesc + uint64_t(2 * ks), idesc_bf16(n),
-                                        (kb == 0 && ks == 0) ? 0u : 1u);
+                                        (kb == k0 && ks == 0) ? 0u : 1u);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -209,56 +223,129 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
         const int half = warp >= 8 ? 1 : 0;
         constexpr int kCbStep = C::kEpiWarps / 4;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        int li = 0;
-        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++li) {
-            const int blk = item / n_items, it = item % n_items;
+        // GEMM1: h of 32 tokens of intermediate tile `it` from gate g and up u
+        auto finish1 = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], int tok0, int nrows, int it) {
+            __nv_bfloat16 *hb = args.out + int64_t(tok0) * args.out_ld + it * kTileRows + q * 32 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                // the linear layer's bf16 output, then the activation in fp32
+                const float gv = bf16_round_f(__uint_as_float(g[j]));
+                const float uv = bf16_round_f(__uint_as_float(u[j]));
+                float hv;
+                if (args.act_kind == MOE_ACT_SWIGLU) {
+                    hv = gv / (1.0f + expf(-gv)) * uv;
+                } else {
+                    const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
+                    hv = (1.0f / (1.0f + expf(-gv))) * (args.beta * tanhf(gv * args.inv_beta)) * up;
+                }
+                if (j < nrows) hb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(hv);
+            }
+        };
+        // GEMM2: y of 32 tokens of output tile `tile`
+        auto finish2 = [&](const uint32_t (&v)[32], int tok0, int nrows, int tile) {
+            __nv_bfloat16 *yb = args.out + int64_t(tok0) * args.out_ld + tile * kTileRows + q * 32 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j < nrows) yb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        };
+        int li = 0, nsplit = 0;
+        for (int uu = blockIdx.x; uu < num_units; uu += gridDim.x, ++li) {
+            const int item = uu / split, blk = item / n_items, it = item % n_items;
             const int rows = min(kN, args.T - blk * kN);
             const int buf = li & 1;
             const uint32_t use = uint32_t(li >> 1) & 1u;
             if (!mbar_wait(&tmem_full[buf], use, abort_flag, err, 14)) break;
             tc_fence_after();
             const uint32_t acc = tmem + lane_base + uint32_t(buf * C::kAccCols);
-            const int ncb = (rows + 31) / 32;
-            for (int cb = half; cb < ncb; cb += kCbStep) {
-                const int tok0 = blk * kN + cb * 32;
+            if (split == 1) {
+                const int ncb = (rows + 31) / 32;
+                for (int cb = half; cb < ncb; cb += kCbStep) {
+                    const int tok0 = blk * kN + cb * 32;
+                    if constexpr (kGemm1) {
+                        uint32_t g[32], u[32];
+                        tmem_ld_32x32(acc + uint32_t(cb * 32), g);
+                        tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
+                        tmem_ld_wait();
+                        finish1(g, u, tok0, rows - cb * 32, it);
+                    } else {
+#pragma unroll 1
+                        for (int a = 0; a < 2; ++a) {
+                            if (2 * it + a >= n_tiles) break;
+                            uint32_t v[32];
+                            tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), v);
+                            tmem_ld_wait();
+                            finish2(v, tok0, rows - cb * 32, 2 * it + a);
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+                continue;
+            }
+            // K part of an item (32-token blocks: one column block): write this
+            // part's fp32 accumulators; the item's last part to finish adds the
+            // parts 0 .. split-1 in that order and runs the epilogue, so the
+            // result does not depend on which part ends last
+            if constexpr (kN == 32) {
+                float *pu = args.part + size_t(uu) * kPartUnitFloats + q * 32 + lane;
+#pragma unroll 1
+                for (int a = 0; a < 2; ++a) {
+                    uint32_t v[32];
+                    tmem_ld_32x32(acc + uint32_t(a * kN), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pu[(a * 32 + j) * kTileRows] = __uint_as_float(v[j]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(epi_bar);
+                if (warp == 2 && lane == 0) {
+                    int last = 0;
+                    if (mbar_wait(epi_bar, uint32_t(nsplit & 1), abort_flag, err, 15)) {
+                        __threadfence();
+                        last = atomicAdd(args.cnt + item, 1) == split - 1;
+                        if (last) args.cnt[item] = 0;  // ready for the next launch
+                        __threadfence();
+                    }
+                    *epi_last = last;
+                    mbar_arrive(epi_go);
+                }
+                if (!mbar_wait(epi_go, uint32_t(nsplit & 1), abort_flag, err, 16)) break;
+                ++nsplit;
+                if (!*epi_last) continue;
+                const float *p0 = args.part + size_t(item) * split * kPartUnitFloats + q * 32 + lane;
+                auto sum_part = [&](int a, uint32_t (&v)[32]) {
+                    float s_[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s_[j] = __ldcg(p0 + (a * 32 + j) * kTileRows);
+                    for (int sp = 1; sp < split; ++sp) {
+                        const float *p = p0 + size_t(sp) * kPartUnitFloats;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) s_[j] += __ldcg(p + (a * 32 + j) * kTileRows);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(s_[j]);
+                };
+                const int tok0 = blk * kN;
                 if constexpr (kGemm1) {
                     uint32_t g[32], u[32];
-                    tmem_ld_32x32(acc + uint32_t(cb * 32), g);
-                    tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
-                    tmem_ld_wait();
-                    __nv_bfloat16 *hb = args.out + int64_t(tok0) * args.out_ld + it * kTileRows + q * 32 + lane;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        // the linear layer's bf16 output, then the activation in fp32
-                        const float gv = bf16_round_f(__uint_as_float(g[j]));
-                        const float uv = bf16_round_f(__uint_as_float(u[j]));
-                        float hv;
-                        if (args.act_kind == MOE_ACT_SWIGLU) {
-                            hv = gv / (1.0f + expf(-gv)) * uv;
-                        } else {
-                            const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
-                            hv = (1.0f / (1.0f + expf(-gv))) * (args.beta * tanhf(gv * args.inv_beta)) * up;
-                        }
-                        if (cb * 32 + j < rows) hb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(hv);
-                    }
+                    sum_part(0, g);
+                    sum_part(1, u);
+                    finish1(g, u, tok0, rows, it);
                 } else {
 #pragma unroll 1
                     for (int a = 0; a < 2; ++a) {
-                        const int tile = 2 * it + a;
-                        if (tile >= n_tiles) break;
+                        if (2 * it + a >= n_tiles) break;
                         uint32_t v[32];
-                        tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), v);
-                        tmem_ld_wait();
-                        __nv_bfloat16 *yb = args.out + int64_t(tok0) * args.out_ld + tile * kTileRows + q * 32 + lane;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (cb * 32 + j < rows) yb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(__uint_as_float(v[j]));
+                        sum_part(a, v);
+                        finish2(v, tok0, rows, 2 * it + a);
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty[buf]);
         }
     }
 
@@ -290,10 +377,12 @@ static cudaError_t launch_shared_t(const CUtensorMap &tmap_w, const CUtensorMap 
 int shared_block_rows(int T) { return T <= kSharedSmallT ? 32 : 128; }
 
 cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, int T, int SH, int SI,
-                          void *out, int *hdr, const moe_activation_t &act, cudaStream_t stream) {
+                          void *out, int *hdr, float *part, const moe_activation_t &act, cudaStream_t stream) {
     SharedArgs a{};
     a.T = T;
     a.hdr = hdr;
+    a.part = part;
+    a.cnt = hdr + kHdrSplitCnt1;  // per item; zeroed with the header, reset by each item's last part
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.act_kind = act.kind;
     a.beta = act.beta;
@@ -315,9 +404,20 @@ cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorM
     }
     const int kn = shared_block_rows(T);
     const int items = (T + kn - 1) / kn * a.n_items;
+    // 32-token blocks with fewer items than SMs: cut each item's K into parts
+    // (at least four 64-element K blocks each) so that about every SM works
+    const int sms = num_sms();
+    a.split = 1;
+    if (kn == 32 && items < sms) {
+        int s = sms / items;
+        if (s > (a.K / 64) / 4) s = (a.K / 64) / 4;
+        if (s > kMaxSplitUnits / items) s = kMaxSplitUnits / items;
+        a.split = s > 1 ? s : 1;
+    }
+    const int units = items * a.split;
     if (kn == 32)
-        return gemm1 ? launch_shared_t<true, 32>(tmap_w, tmap_act, a, items, stream)
-                     : launch_shared_t<false, 32>(tmap_w, tmap_act, a, items, stream);
+        return gemm1 ? launch_shared_t<true, 32>(tmap_w, tmap_act, a, units, stream)
+                     : launch_shared_t<false, 32>(tmap_w, tmap_act, a, units, stream);
     return gemm1 ? launch_shared_t<true, 128>(tmap_w, tmap_act, a, items, stream)
                  : launch_shared_t<false, 128>(tmap_w, tmap_act, a, items, stream);
 }

@@ -182,14 +182,16 @@ def test_nvfp4_entry_points_validate_on_the_host(moelib):
 
 
 def test_shared_expert_entry_points_validate_on_the_host(moelib):
-    """Workspace size = 2 KiB header + h [T, SI] bf16 (256-aligned); shapes,
-    token counts, activations and sizes are checked before any CUDA call."""
+    """Workspace size = 2 KiB header + h [T, SI] bf16 (256-aligned) + 8 MiB of
+    K-split partial sums; shapes, token counts, activations and sizes are
+    checked before any CUDA call."""
     import ctypes
     import moe_expert_layer_08_b200 as m
     lib = m.load()
-    assert m.shared_workspace_bytes(8192, 7168, 2048) == 2048 + 8192 * 2048 * 2
-    assert m.shared_workspace_bytes(3, 256, 128) == 2048 + 768
-    assert m.shared_workspace_bytes(0, 256, 128) == 2048
+    scratch = 256 * 2 * 32 * 128 * 4
+    assert m.shared_workspace_bytes(8192, 7168, 2048) == 2048 + 8192 * 2048 * 2 + scratch
+    assert m.shared_workspace_bytes(3, 256, 128) == 2048 + 768 + scratch
+    assert m.shared_workspace_bytes(0, 256, 128) == 2048 + scratch
     n = ctypes.c_size_t()
     assert lib.moe_shared_workspace_bytes(8, 200, 128, ctypes.byref(n)) == 2   # SH % 128
     assert lib.moe_shared_workspace_bytes(8, 256, 100, ctypes.byref(n)) == 2   # SI % 128
