@@ -342,6 +342,39 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_shared_reference(args, rank):
+    """The oracle's shared expert on the host cores, on the first
+    ``--cpu-tokens`` of the T tokens per step (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    T = args.shared_expert
+    SH, SI = (int(v) for v in args.shared_dims.split(","))
+    x, l1, l2 = W.gen_shared(T, SH, SI, 1, "cuda" if torch.cuda.is_available() else "cpu")
+    u16 = lambda t: t.cpu().view(torch.int16).numpy().view(np.uint16)
+    xb, l1b, l2b = u16(x), u16(l1), u16(l2)
+    n = min(args.cpu_tokens, T)
+    tok = np.arange(n, dtype=np.int32)
+    times = []
+    for _ in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.shared_forward(xb, l1b, l2b, tokens=tok)
+        times.append(time.perf_counter() - t0)
+    t = float(np.mean(times[args.warmup:])) if args.steps > 0 else float(np.mean(times))
+    value = 2.0 * n * 3 * SH * SI / t / 1e12
+    threads = min(oracle.num_threads(), n)
+    line = {
+        "metric": f"BF16 shared expert TFLOP/s (SH={SH}, SI={SI})", "impl": "reference", "value": value,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"shared_expert_T{T}", "T": T, "SH": SH, "SI": SI, "activation": "swiglu"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {n} of {T} tokens per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_b200(args, w, rank, world, local_rank):
     import moe_expert_layer_08_b200 as moe
     from moe_expert_layer_08_b200 import build as mbuild
@@ -524,7 +557,9 @@ def main():
         w = W.custom(f"{w.name}_T{T}_E{E}", T=T, E=E, k=w.k, H=w.H, I=w.I, seed=w.seed,
                      routing=w.routing, zipf_s=w.zipf_s)
     try:
-        if args.shared_expert:
+        if args.shared_expert and args.impl == "reference":
+            run_shared_reference(args, rank)
+        elif args.shared_expert:
             run_shared(args, rank, world, local_rank)
         elif args.impl == "reference":
             run_reference(args, w, rank, world)

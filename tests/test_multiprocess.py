@@ -65,3 +65,19 @@ def test_reference_arm_under_torchrun_world2():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_shared_expert_reference_arm_on_cpu():
+    """bench.py --shared-expert with --impl reference times the oracle's shared
+    expert on a bounded token sample and prints one reference line."""
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--shared-expert", "16", "--shared-dims", "256,128",
+           "--steps", "1", "--warmup", "0", "--cpu-tokens", "4"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600,
+                       env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    import json
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["config"]["SH"] == 256
+    assert d["cpu_baseline"]["sample"] == "first 4 of 16 tokens per step"
