@@ -16,9 +16,12 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.R = int64_t(T) * k;
     L.nb = int((L.R + kRouteBlock - 1) / kRouteBlock);
     if (L.nb < 1) L.nb = 1;
-    // Small per-expert loads (decode) use 32-row chunks and the kN = 32 GEMMs;
-    // the chunk bound is taken for 32-row chunks either way, so the workspace
-    // size grows monotonically with T.
+    // Small per-expert loads (decode) use 32-row chunks and the kN = 32 GEMMs,
+    // large ones 160-row chunks (plus the side list).  The chunk-count bound is
+    // taken for 32-row chunks either way; the scale regions are sized for the
+    // chunking in use, which still grows monotonically with T (at the switch
+    // the 160-row bound, (R/160 + E) x 1 KB per K block, exceeds the 32-row one,
+    // (R/32 + E) x 512 B with R = 8E).
     L.chunk_rows = L.R <= int64_t(8) * E ? kChunkRowsSmall : kChunkRows;
     L.max_chunks = (L.R + kChunkRowsSmall - 1) / kChunkRowsSmall + (L.R < E ? L.R : E);
     const size_t R = size_t(L.R > 0 ? L.R : 1);
@@ -43,22 +46,21 @@ WsLayout ws_layout(int T, int E, int k, int H, int I) {
     L.kbh = H / kTileK > 2 ? H / kTileK : 2;
     L.kbi = I / kTileK > 2 ? I / kTileK : 2;
     L.off_xg = take(size_t(L.Rp) * size_t(L.kbh) * kTileK);
-    // scale blocks per (chunk, K block): the larger of the two chunkings' needs
+    // scale blocks per K block: (chunk bound) x (image bytes) of the chunking in use
     const size_t sf_small = MC * size_t(act_sf_bytes(kChunkRowsSmall));
     const size_t mc_large = size_t((L.R + kChunkRows - 1) / kChunkRows + (L.R < E ? L.R : E));
     const size_t sf_large = (mc_large > 0 ? mc_large : 1) * size_t(act_sf_bytes(kChunkRows));
-    const size_t sf_per_kb = sf_small > sf_large ? sf_small : sf_large;
+    const size_t sf_per_kb = L.chunk_rows == kChunkRowsSmall ? sf_small : sf_large;
     // twice that: NVFP4 operands have four images per 256 K, two per 128
     L.off_xg_sf = take(2 * sf_per_kb * size_t(H / kTileK));
     L.off_hq = take(size_t(L.Rp) * size_t(L.kbi) * kTileK);
     L.off_hq_sf = take(2 * sf_per_kb * size_t(I / kTileK));
     L.off_y = take(R * size_t(H) * 2);
     L.off_part = take(size_t(kMaxSplitUnits) * kPartUnitFloats * sizeof(float));
-    // side list (large batches): one 32-row chunk per lightly loaded expert;
-    // allocated at every size so that the workspace grows monotonically with T
+    // side list (large batches only): one 32-row chunk per lightly loaded expert
     L.side = L.chunk_rows == kChunkRows;
-    L.max_side = L.R < E ? L.R : E;
-    const size_t MS = size_t(L.max_side > 0 ? L.max_side : 1);
+    L.max_side = L.side ? (L.R < E ? L.R : E) : 0;
+    const size_t MS = size_t(L.max_side);
     L.off_chunks_s = take(sizeof(int4) * MS);
     L.off_xg_sf_s = take(2 * MS * size_t(act_sf_bytes(kChunkRowsSmall)) * size_t(H / kTileK));
     L.off_hq_sf_s = take(2 * MS * size_t(act_sf_bytes(kChunkRowsSmall)) * size_t(I / kTileK));

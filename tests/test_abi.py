@@ -205,3 +205,19 @@ def test_shared_expert_entry_points_validate_on_the_host(moelib):
     assert f(None, None, None, None, 4, 256, 128, ctypes.byref(bad), None, 0, None) == 1
     fake = ctypes.c_void_p(1 << 20)                                            # never dereferenced
     assert f(fake, fake, fake, fake, 4, 256, 128, None, fake, 16, None) == 3   # workspace too small
+
+
+def test_workspace_grows_monotonically_with_T(moelib):
+    """A workspace sized for T_max serves every T <= T_max, across the switch
+    from 32-row to 160-row chunks (T*k > 8E) and the side list's regions."""
+    import moe_expert_layer_08_b200 as m
+    for E, k, H, I in ((8, 2, 256, 256), (64, 6, 1024, 512), (384, 6, 7168, 3072)):
+        sizes = [m.workspace_bytes(T, E, k, H, I) for T in range(0, 1200, 7)]
+        assert all(a <= b for a, b in zip(sizes, sizes[1:])), (E, k, H, I)
+
+
+def test_static_workspace_holds_decode_batches(moelib):
+    """The fixed scratch of moe_forward_static holds T = 128 tokens at E = 384,
+    top-6, H = 7168, I = 3072 (the sizes its documentation names)."""
+    import moe_expert_layer_08_b200 as m
+    assert m.workspace_bytes(128, 384, 6, 7168, 3072) <= m.STATIC_WORKSPACE_BYTES
