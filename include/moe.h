@@ -384,6 +384,19 @@ moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf,
                                 moe_stream_t stream);
 
 /*
+ * moe_probe_wait_timeout -- diagnostic (no counterpart on the pages): runs one
+ * thread through the library's bounded device-side wait on a barrier that
+ * nothing completes, with a limit of timeout_us microseconds (1 .. 1e6)
+ * instead of the kernels' 2 s.  The wait gives up and records the timeout in
+ * the workspace's error word, after which moe_check_device_error(workspace)
+ * returns MOE_ERR_DEVICE_TIMEOUT and the context stays usable.  Enqueues a
+ * 2 KiB memset of the workspace header and one kernel; workspace 256-byte
+ * aligned, ws_bytes >= 2048.  Exercises the failure path without a fault.
+ */
+moe_status_t moe_probe_wait_timeout(void *workspace, size_t ws_bytes, unsigned timeout_us,
+                                    moe_stream_t stream);
+
+/*
  * BF16 shared expert (DeepGEMM PR #416, "BF16 shared expert" test body: an
  * optional dense expert that runs on every token beside the routed experts,
  * with bf16 input, weights and its own bf16 output).  With x [T, SH],

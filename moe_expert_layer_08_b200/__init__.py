@@ -21,7 +21,7 @@ __all__ = [
     "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
-    "forward_nvfp4", "shared_workspace_bytes", "shared_forward",
+    "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -105,6 +105,7 @@ def _declare(lib):
         "moe_forward_weights": (I32, [P, P, P, P, c.POINTER(Weights), P, I32, I32, I32, I32, I32, P, SZ, P, P,
                                       c.POINTER(Activation), P]),
         "moe_shared_workspace_bytes": (I32, [I32, I32, I32, c.POINTER(SZ)]),
+        "moe_probe_wait_timeout": (I32, [P, SZ, c.c_uint, P]),
         "moe_shared_forward": (I32, [P, P, P, P, I32, I32, I32, c.POINTER(Activation), P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -384,6 +385,14 @@ def forward_nvfp4(x_fp4, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: 
                                   ev, ctypes.byref(act) if act is not None else None, _stream(stream))
     _check(st, "moe_forward_nvfp4")
     return out
+
+
+def probe_wait_timeout(workspace, timeout_us: int = 1000, stream=None):
+    """Diagnostic: a bounded device-side wait that times out (see
+    moe_probe_wait_timeout); check_device_error(workspace) then reports it."""
+    _need(workspace, torch.uint8, "workspace")
+    _check(load().moe_probe_wait_timeout(_ptr(workspace), workspace.numel(), timeout_us, _stream(stream)),
+           "moe_probe_wait_timeout")
 
 
 def shared_workspace_bytes(T_max: int, SH: int, SI: int) -> int:

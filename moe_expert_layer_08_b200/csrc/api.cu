@@ -586,6 +586,36 @@ moe_status_t moe_read_routing(const void *workspace, int T, int E, int k, int H,
     return cuda_status(e);
 }
 
+// ---------------------------------------------------------------- bounded-wait probe
+// One thread waits on a barrier that nothing completes, through the same
+// bounded wait every kernel of the library uses, with a short limit: the wait
+// gives up, records the timeout in the workspace error word (and `where`) and
+// the kernel returns.
+__global__ void wait_probe_kernel(int *hdr, unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag, hdr, kProbeWhere, timeout_ns);
+}
+
+moe_status_t moe_probe_wait_timeout(void *workspace, size_t ws_bytes, unsigned timeout_us, moe_stream_t stream) {
+    if (!workspace || !aligned(workspace, 256) || timeout_us == 0 || timeout_us > 1000000u)
+        return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < size_t(kHdrBytes)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    moe_status_t s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kHdrBytes, st);
+    if (e == cudaSuccess) {
+        wait_probe_kernel<<<1, 32, 0, st>>>(static_cast<int *>(workspace), 1000ull * timeout_us);
+        e = cudaGetLastError();
+    }
+    return cuda_status(e);
+}
+
 // ---------------------------------------------------------------- BF16 shared expert
 // header (error word, split counters), h [T][SI] bf16, K-split partial sums
 static size_t shared_h_bytes(int T, int SI) { return align_up(size_t(T) * size_t(SI) * 2, 256); }

@@ -40,7 +40,8 @@ constexpr int kHdrError = 0;
 constexpr int kHdrNumChunks = 1;
 constexpr int kHdrDropped = 2;
 constexpr int kHdrTimeoutWhere = 3;
-constexpr int kHdrNumChunksSide = 4;  // chunks of the side list (large batches: lightly loaded experts)
+constexpr int kHdrNumChunksSide = 4;
+constexpr int kProbeWhere = 99;       // kHdrTimeoutWhere value the bounded-wait probe records  // chunks of the side list (large batches: lightly loaded experts)
 // A per-expert chunk base with this bit set indexes the side list.
 constexpr int kSideChunkBit = 1 << 30;
 // Split-unit counters of the 32-row GEMMs (zeroed by routing on every forward):
@@ -182,13 +183,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // another role has raised `abort` or after kWaitTimeoutNs, in which case it
 // raises `abort`, records `where` and the timeout bit in the error word.
 static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                       int *err_word, int where) {
+                                       int *err_word, int where,
+                                       unsigned long long timeout_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        if (global_timer_ns() - t0 > timeout_ns) {
             *abort = 1;
             atomicOr(err_word + kHdrError, kDevErrTimeout);
             atomicExch(err_word + kHdrTimeoutWhere, where);
