@@ -189,7 +189,11 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = threading.Thread(target=self._run, daemon=True)
         self._t.start()
-        time.sleep(0.02)
+        # the timed region starts once sampling runs (NVML's handle lookup can
+        # take longer than a short region)
+        t0 = time.time()
+        while not self.sm and time.time() - t0 < 2.0:
+            time.sleep(0.001)
         return self
 
     def __exit__(self, *a):
