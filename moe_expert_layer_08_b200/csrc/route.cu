@@ -11,8 +11,15 @@
 // bases and its count), route_meta (one block: offsets, chunk list,
 // statistics, error word), route_place (perm, inv, per-row gather
 // descriptor).  Then gather_kernel copies the FP8 rows of x into permuted
-// order (stored K-block-major, [H/128][R][128]) and the UE8M0 scales into per-chunk blocks of 512-byte images laid out as the
-// image tcgen05.cp copies into TMEM.
+// order (stored K-block-major, [H/128][R][128]) and the UE8M0 scales into
+// per-chunk blocks of 512-byte images laid out as the image tcgen05.cp copies
+// into TMEM.
+//
+// Chunks: an expert's rows are cut into chunks of chunk_rows (32 for small
+// batches, 160 for large ones) in the main list.  With 160-row chunks the
+// experts with at most 32 rows instead get one 32-row chunk in a side list,
+// which the 32-row GEMM kernels process; their per-expert chunk base carries
+// kSideChunkBit.
 //
 // Within an expert, routed rows keep ascending slot order t*k+j (a stable
 // counting sort), so the metadata is unique and compared bit-exactly.
