@@ -1,0 +1,57 @@
+"""Host logic of bench.py (no GPU): the peak denominators, the per-expert
+byte counts, and the ncu-traffic lookup that reports `roofline.traffic` only
+for the kernel sources it was captured from."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+import workloads as W  # noqa: E402
+
+
+def fake_root(tmp_path, peaks=None):
+    csrc = tmp_path / "moe_expert_layer_08_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("gemm.cu", "moe_common.cuh", "moe_internal.h"):
+        (csrc / f).write_text(f"// {f}\n")
+    (tmp_path / "profiles").mkdir()
+    if peaks is not None:
+        (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(peaks))
+    return tmp_path
+
+
+def test_peaks_measured_and_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(fake_root(tmp_path / "a", {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0,
+                                                                       "bf16_tflops_sustained": 1300.0})))
+    assert bench.peaks() == dict(hbm=6000.0, bf16=1600.0, bf16_sustained=1300.0, source="measured")
+    monkeypatch.setattr(bench, "ROOT", str(fake_root(tmp_path / "b")))
+    assert bench.peaks()["source"] == "fallback"
+
+
+def test_expert_bytes():
+    w = W.WORKLOADS[1]
+    b1, b2 = bench.expert_bytes(w, "mx")
+    assert (b1, b2) == (2 * 3072 * 7168 * 17 // 32, 7168 * 3072 * 17 // 32) == (23396352, 11698176)
+    n1, n2 = bench.expert_bytes(w, "nvfp4")
+    assert (n1, n2) == (2 * 3072 * 7168 * 9 // 16, 7168 * 3072 * 9 // 16)
+
+
+def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
+    root = fake_root(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    decode, prefill = W.WORKLOADS[1], W.WORKLOADS[3]
+    for regime, g1, g2 in (("decode", 100.0, 50.0), ("prefill", 110.0, 60.0)):
+        (root / "profiles" / f"gemm_{regime}_traffic.json").write_text(json.dumps(
+            {"kernel_source_sha256": bench.kernel_source_hash(),
+             "gemm1_bytes_per_touched_expert": g1, "gemm2_bytes_per_touched_expert": g2}))
+    assert bench.measured_traffic(decode, 10, True) == 1000.0
+    assert bench.measured_traffic(decode, 10, False) == 500.0
+    assert bench.measured_traffic(prefill, 10, True) == 1100.0      # T*k > 8E: the prefill capture
+    assert bench.measured_traffic(decode, 10, True, "nvfp4") is None
+    # any edit to the GEMM sources retires the capture
+    (root / "moe_expert_layer_08_b200" / "csrc" / "gemm.cu").write_text("// changed\n")
+    assert bench.measured_traffic(decode, 10, True) is None
