@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--shared-expert", type=int, default=0, metavar="T",
                    help="time the BF16 shared expert (moe_shared_forward) on T tokens instead of the layer")
     p.add_argument("--shared-dims", default="7168,2048", help="SH,SI of the shared expert")
+    p.add_argument("--fp8-peak", action="store_true",
+                   help="measure cuBLAS FP8 (per-tensor scaled) 8192^3 matmul throughput, burst and sustained")
     return p.parse_args()
 
 
@@ -140,6 +142,17 @@ def peaks():
         return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
                     bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def cublas_fp8():
+    """The measured cuBLAS FP8 matmul figures committed beside the ncu
+    summaries (`--fp8-peak` writes them), or None: context for the FP8 tensor
+    roofline, whose denominator stays 2 x the measured bf16 peak."""
+    path = os.path.join(ROOT, "profiles", "cublas_fp8_matmul_8192.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    return dict(burst=float(d["burst_tflops"]), sustained=float(d["sustained_tflops"]))
 
 
 def expert_bytes(w, fmt="mx"):
@@ -346,6 +359,44 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8_peak(args):
+    """A library FP8 reference figure for the tensor roofline: an 8192^3 E4M3
+    x E4M3 matmul with per-tensor scales (torch._scaled_mm -> cuBLAS), best
+    of 10 timed calls (burst) and back to back for ~4 s (sustained)."""
+    device = torch.device("cuda", 0)
+    n = 8192
+    g = torch.Generator(device=device).manual_seed(0)
+    a = torch.randn((n, n), device=device, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn((n, n), device=device, generator=g).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=device)
+    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(5):
+        mm()
+    flops = 2.0 * n ** 3
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 0.0
+    for _ in range(10):
+        s0.record()
+        mm()
+        s1.record()
+        torch.cuda.synchronize()
+        best = max(best, flops / (s0.elapsed_time(s1) * 1e-3) / 1e12)
+    with ClockSampler(device.index) as clocks:
+        reps, t_end, done = 0, time.time() + 4.0, 0.0
+        s0.record()
+        while time.time() < t_end:
+            for _ in range(20):
+                mm()
+            reps += 20
+            torch.cuda.synchronize()
+        s1.record()
+        torch.cuda.synchronize()
+        done = s0.elapsed_time(s1)
+    print(json.dumps({"metric": "cuBLAS FP8 E4M3 8192^3 matmul (per-tensor scales)", "unit": "TFLOP/s",
+                      "burst": best, "sustained": flops * reps / (done * 1e-3) / 1e12,
+                      "clocks": clocks.summary()}), flush=True)
+
+
 def run_shared_reference(args, rank):
     """The oracle's shared expert on the host cores, on the first
     ``--cpu-tokens`` of the T tokens per step (rank 0 only)."""
@@ -514,11 +565,20 @@ def run_b200(args, w, rank, world, local_rank):
                     "spec": {"peak": spec_tc, "frac": tflops / spec_tc},
                     "algorithmic_flops": kflops,
                     "traffic": traffic, "hbm": {"achieved_GBps": achieved, "frac": achieved / pk["hbm"]}}
+        if cublas_fp8() and args.format == "mx":
+            c8 = cublas_fp8()
+            roofline["cublas_fp8"] = {"sustained": c8["sustained"], "frac": tflops / c8["sustained"],
+                                      "burst": c8["burst"], "frac_of_burst": tflops / c8["burst"]}
     x_bytes = w.T * w.H * 33 // 32 if args.format == "mx" else w.T * w.H * 9 // 16
     layer_bytes = touched * (b1 + b2) + x_bytes + w.T * w.k * 12 + w.T * w.H * 2
     flops = w.flops
     value = world * flops / (ms * 1e-3) / 1e12
     e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+    layer_tc = {"sustained": value / world / (ratio * pk["bf16_sustained"]),
+                "burst": value / world / (ratio * pk["bf16"]),
+                "spec": value / world / spec_tc}
+    if cublas_fp8() and args.format == "mx":
+        layer_tc["cublas_fp8_sustained"] = value / world / cublas_fp8()["sustained"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -538,9 +598,7 @@ def run_b200(args, w, rank, world, local_rank):
                                 "between kernels; the roofline's kernel duration comes from it",
                          "us_per_layer": staged_ms * 1e3},
         "roofline": roofline,
-        "layer_frac_of_tensor_peak": {"sustained": value / world / (ratio * pk["bf16_sustained"]),
-                                      "burst": value / world / (ratio * pk["bf16"]),
-                                      "spec": value / world / spec_tc},
+        "layer_frac_of_tensor_peak": layer_tc,
         "layer_frac_of_hbm_spec": layer_bytes / (ms * 1e-3) / 1e9 / SPEC_HBM_GBPS,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
@@ -571,7 +629,9 @@ def main():
         w = W.custom(f"{w.name}_T{T}_E{E}", T=T, E=E, k=w.k, H=w.H, I=w.I, seed=w.seed,
                      routing=w.routing, zipf_s=w.zipf_s)
     try:
-        if args.shared_expert and args.impl == "reference":
+        if args.fp8_peak:
+            run_fp8_peak(args)
+        elif args.shared_expert and args.impl == "reference":
             run_shared_reference(args, rank)
         elif args.shared_expert:
             run_shared(args, rank, world, local_rank)

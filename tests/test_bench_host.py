@@ -55,3 +55,21 @@ def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
     # any edit to the GEMM sources retires the capture
     (root / "moe_expert_layer_08_b200" / "csrc" / "gemm.cu").write_text("// changed\n")
     assert bench.measured_traffic(decode, 10, True) is None
+
+
+def test_cublas_fp8_context(tmp_path, monkeypatch):
+    root = fake_root(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.cublas_fp8() is None
+    (root / "profiles" / "cublas_fp8_matmul_8192.json").write_text(json.dumps(
+        {"burst_tflops": 3000.0, "sustained_tflops": 2500.0}))
+    assert bench.cublas_fp8() == dict(burst=3000.0, sustained=2500.0)
+
+
+def test_committed_cublas_fp8_figure_is_below_the_derived_denominator():
+    # the measured FP8 figure is context: the reported roofline keeps the
+    # stricter 2 x bf16 sustained denominator while it is the larger one
+    c8, pk = bench.cublas_fp8(), bench.peaks()
+    assert c8 is not None and 0 < c8["sustained"] <= c8["burst"]
+    if pk["source"] == "measured":
+        assert c8["sustained"] <= 2.0 * pk["bf16_sustained"]
