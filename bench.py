@@ -57,7 +57,8 @@ def parse():
                    help="time the BF16 shared expert (moe_shared_forward) on T tokens instead of the layer")
     p.add_argument("--shared-dims", default="7168,2048", help="SH,SI of the shared expert")
     p.add_argument("--fp8-peak", action="store_true",
-                   help="measure cuBLAS FP8 (per-tensor scaled) 8192^3 matmul throughput, burst and sustained")
+                   help="measure cuBLAS FP8 8192^3 matmul throughput (MX block-scaled and per-tensor scaled), "
+                        "burst and sustained")
     return p.parse_args()
 
 
@@ -152,7 +153,8 @@ def cublas_fp8():
     if not os.path.exists(path):
         return None
     d = json.load(open(path))
-    return dict(burst=float(d["burst_tflops"]), sustained=float(d["sustained_tflops"]))
+    return {arm: dict(burst=float(d[arm]["burst_tflops"]), sustained=float(d[arm]["sustained_tflops"]))
+            for arm in ("mx_blockwise_1x32", "per_tensor") if arm in d}
 
 
 def expert_bytes(w, fmt="mx"):
@@ -360,41 +362,58 @@ def run_reference(args, w, rank, world):
 
 
 def run_fp8_peak(args):
-    """A library FP8 reference figure for the tensor roofline: an 8192^3 E4M3
-    x E4M3 matmul with per-tensor scales (torch._scaled_mm -> cuBLAS), best
-    of 10 timed calls (burst) and back to back for ~4 s (sustained)."""
+    """Library FP8 reference figures for the tensor roofline, 8192^3 E4M3 x
+    E4M3 matmuls with bf16 output: MX block scaling (UE8M0 per 32 along K,
+    F.scaled_mm -> cuBLAS) and per-tensor scales (torch._scaled_mm), each as
+    the best of 10 timed calls (burst) and back to back for ~4 s
+    (sustained)."""
+    import torch.nn.functional as F
     device = torch.device("cuda", 0)
     n = 8192
     g = torch.Generator(device=device).manual_seed(0)
     a = torch.randn((n, n), device=device, generator=g).to(torch.float8_e4m3fn)
     b = torch.randn((n, n), device=device, generator=g).to(torch.float8_e4m3fn).t()
     one = torch.ones((), device=device)
-    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
-    for _ in range(5):
-        mm()
+    # scale 2^0 everywhere: the swizzled image of a constant is the constant
+    sf = torch.full((n * (n // 32),), 127, dtype=torch.uint8, device=device).view(torch.float8_e8m0fnu)
+    blk, swz = F.ScalingType.BlockWise1x32, F.SwizzleType.SWIZZLE_32_4_4
+    arms = {
+        "mx_blockwise_1x32": lambda: F.scaled_mm(a, b, sf, blk, sf, blk, swizzle_a=swz, swizzle_b=swz,
+                                                 output_dtype=torch.bfloat16),
+        "per_tensor": lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+    }
     flops = 2.0 * n ** 3
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    best = 0.0
-    for _ in range(10):
-        s0.record()
-        mm()
-        s1.record()
-        torch.cuda.synchronize()
-        best = max(best, flops / (s0.elapsed_time(s1) * 1e-3) / 1e12)
-    with ClockSampler(device.index) as clocks:
-        reps, t_end, done = 0, time.time() + 4.0, 0.0
-        s0.record()
-        while time.time() < t_end:
-            for _ in range(20):
-                mm()
-            reps += 20
+    out = {"metric": "cuBLAS FP8 E4M3 8192^3 matmul, bf16 out", "unit": "TFLOP/s"}
+    for name, mm in arms.items():
+        try:
+            mm()
             torch.cuda.synchronize()
-        s1.record()
-        torch.cuda.synchronize()
-        done = s0.elapsed_time(s1)
-    print(json.dumps({"metric": "cuBLAS FP8 E4M3 8192^3 matmul (per-tensor scales)", "unit": "TFLOP/s",
-                      "burst": best, "sustained": flops * reps / (done * 1e-3) / 1e12,
-                      "clocks": clocks.summary()}), flush=True)
+        except (RuntimeError, TypeError, ValueError) as e:
+            out[name] = {"unavailable": str(e).splitlines()[0][:200]}
+            continue
+        for _ in range(5):
+            mm()
+        best = 0.0
+        for _ in range(10):
+            s0.record()
+            mm()
+            s1.record()
+            torch.cuda.synchronize()
+            best = max(best, flops / (s0.elapsed_time(s1) * 1e-3) / 1e12)
+        with ClockSampler(device.index) as clocks:
+            reps, t_end = 0, time.time() + 4.0
+            s0.record()
+            while time.time() < t_end:
+                for _ in range(20):
+                    mm()
+                reps += 20
+                torch.cuda.synchronize()
+            s1.record()
+            torch.cuda.synchronize()
+        out[name] = {"burst": best, "sustained": flops * reps / (s0.elapsed_time(s1) * 1e-3) / 1e12,
+                     "clocks": clocks.summary()}
+    print(json.dumps(out), flush=True)
 
 
 def run_shared_reference(args, rank):
@@ -566,9 +585,9 @@ def run_b200(args, w, rank, world, local_rank):
                     "algorithmic_flops": kflops,
                     "traffic": traffic, "hbm": {"achieved_GBps": achieved, "frac": achieved / pk["hbm"]}}
         if cublas_fp8() and args.format == "mx":
-            c8 = cublas_fp8()
-            roofline["cublas_fp8"] = {"sustained": c8["sustained"], "frac": tflops / c8["sustained"],
-                                      "burst": c8["burst"], "frac_of_burst": tflops / c8["burst"]}
+            roofline["cublas_fp8"] = {arm: {"sustained": c["sustained"], "frac": tflops / c["sustained"],
+                                            "burst": c["burst"], "frac_of_burst": tflops / c["burst"]}
+                                      for arm, c in cublas_fp8().items()}
     x_bytes = w.T * w.H * 33 // 32 if args.format == "mx" else w.T * w.H * 9 // 16
     layer_bytes = touched * (b1 + b2) + x_bytes + w.T * w.k * 12 + w.T * w.H * 2
     flops = w.flops
@@ -578,7 +597,8 @@ def run_b200(args, w, rank, world, local_rank):
                 "burst": value / world / (ratio * pk["bf16"]),
                 "spec": value / world / spec_tc}
     if cublas_fp8() and args.format == "mx":
-        layer_tc["cublas_fp8_sustained"] = value / world / cublas_fp8()["sustained"]
+        layer_tc["cublas_fp8_sustained"] = {arm: value / world / c["sustained"]
+                                            for arm, c in cublas_fp8().items()}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

@@ -62,14 +62,18 @@ def test_cublas_fp8_context(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(root))
     assert bench.cublas_fp8() is None
     (root / "profiles" / "cublas_fp8_matmul_8192.json").write_text(json.dumps(
-        {"burst_tflops": 3000.0, "sustained_tflops": 2500.0}))
-    assert bench.cublas_fp8() == dict(burst=3000.0, sustained=2500.0)
+        {"per_tensor": {"burst_tflops": 3000.0, "sustained_tflops": 2500.0},
+         "mx_blockwise_1x32": {"burst_tflops": 2700.0, "sustained_tflops": 2200.0}}))
+    assert bench.cublas_fp8() == {"per_tensor": dict(burst=3000.0, sustained=2500.0),
+                                  "mx_blockwise_1x32": dict(burst=2700.0, sustained=2200.0)}
 
 
 def test_committed_cublas_fp8_figure_is_below_the_derived_denominator():
     # the measured FP8 figure is context: the reported roofline keeps the
     # stricter 2 x bf16 sustained denominator while it is the larger one
     c8, pk = bench.cublas_fp8(), bench.peaks()
-    assert c8 is not None and 0 < c8["sustained"] <= c8["burst"]
-    if pk["source"] == "measured":
-        assert c8["sustained"] <= 2.0 * pk["bf16_sustained"]
+    assert c8 is not None and set(c8) == {"mx_blockwise_1x32", "per_tensor"}
+    for c in c8.values():
+        assert 0 < c["sustained"] <= c["burst"]
+        if pk["source"] == "measured":
+            assert c["sustained"] <= 2.0 * pk["bf16_sustained"]
