@@ -40,8 +40,8 @@ constexpr int kHdrError = 0;
 constexpr int kHdrNumChunks = 1;
 constexpr int kHdrDropped = 2;
 constexpr int kHdrTimeoutWhere = 3;
-constexpr int kHdrNumChunksSide = 4;
-constexpr int kProbeWhere = 99;       // kHdrTimeoutWhere value the bounded-wait probe records  // chunks of the side list (large batches: lightly loaded experts)
+constexpr int kHdrNumChunksSide = 4;  // chunks of the side list (large batches: lightly loaded experts)
+constexpr int kProbeWhere = 99;       // kHdrTimeoutWhere value the bounded-wait probe records
 // A per-expert chunk base with this bit set indexes the side list.
 constexpr int kSideChunkBit = 1 << 30;
 // Split-unit counters of the 32-row GEMMs (zeroed by routing on every forward):
