@@ -430,6 +430,57 @@ moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const v
                                 const moe_activation_t *activation, void *workspace, size_t ws_bytes,
                                 moe_stream_t stream);
 
+/*
+ * Expert parallelism: the per-rank ends of the dispatch and combine phases of
+ * "Mega moe fusion with symmetric memory" (Procedure, step 5, phases 1 and 5;
+ * MATE "Mega MoE" API page, Typical Flow), with the exchange between ranks
+ * left to the caller (an all-to-all-v, e.g. NCCL through torch.distributed).
+ * Rank r of R holds experts [r E/R, (r+1) E/R) (E % R == 0).  One step:
+ *   1. moe_ep_dispatch on every rank: its T tokens' routed rows, grouped by
+ *      destination rank, and the per-rank row counts;
+ *   2. exchange the counts, then the rows (x, scales, local expert ids);
+ *   3. on every rank, moe_forward over the received rows with E/R experts,
+ *      k = 1, topk_idx = the received local ids and topk_w = 1, which yields
+ *      each received row's bf16 expert output Y unchanged;
+ *   4. send those outputs back (the reverse all-to-all-v);
+ *   5. moe_ep_combine on every rank: out = the top-k-weighted sum, as
+ *      moe_forward's own combine forms it.
+ * With R = 1 (no exchange) the result equals moe_forward's bit for bit.
+ *
+ * moe_ep_workspace_bytes -- bytes of the dispatch workspace for up to T_max
+ *   tokens (the routing metadata only: a 2 KiB header with the device error
+ *   word, counts, offsets, permutation and its inverse, ...).
+ *
+ * moe_ep_dispatch -- routing plus the send buffers, in routing order (by
+ *   expert, then by slot t*k+j; a dropped slot, id outside [0, E), has no row
+ *   and is reported by moe_check_device_error(workspace)):
+ *   x_fp8 u8 [T, H] (16-byte aligned), x_sf u8 [T, H/32] (4-byte aligned),
+ *   topk_idx i64 [T, k] as for moe_forward;
+ *   send_x u8 [T k, H] (16-byte aligned), send_sf u8 [T k, H/32] (4-byte
+ *   aligned), send_eid i64 [T k] (the row's expert id minus its rank's first
+ *   expert): the first n = sum(send_counts) rows are written;
+ *   send_counts i64 [ranks] (rows for each destination rank, device memory).
+ *   workspace 256-byte aligned, ws_bytes >= moe_ep_workspace_bytes(T, E, k, H);
+ *   it must stay untouched until the matching moe_ep_combine.  H must be a
+ *   multiple of 128.  T = 0 only zeroes send_counts.  Asynchronous on `stream`.
+ *
+ * moe_ep_combine -- out_bf16 [T, H] (16-byte aligned, fully overwritten) =
+ *   bf16_rne(sum_{j ascending} topk_w[t, j] * y_bf16[inv[t k + j]]), fp32 sum,
+ *   no atomics; y_bf16 [n, H] holds the rows returned for the dispatched rows,
+ *   in send order; inv is the inverse permutation the dispatch with the same
+ *   T, E, k, H left in the workspace.  T = 0 enqueues nothing.
+ *
+ * Argument errors (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE /
+ * MOE_ERR_WORKSPACE_TOO_SMALL) are returned before any CUDA call; a launch
+ * failure is MOE_ERR_CUDA.  The caller owns every buffer.
+ */
+moe_status_t moe_ep_workspace_bytes(int T_max, int E, int k, int H, size_t *bytes);
+moe_status_t moe_ep_dispatch(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, int T, int E, int k,
+                             int H, int ranks, void *workspace, size_t ws_bytes, void *send_x, void *send_sf,
+                             int64_t *send_eid, int64_t *send_counts, moe_stream_t stream);
+moe_status_t moe_ep_combine(const void *y_bf16, const float *topk_w, int T, int E, int k, int H,
+                            const void *workspace, size_t ws_bytes, void *out_bf16, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,6 +22,7 @@ __all__ = [
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
     "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
+    "ep_workspace_bytes", "ep_dispatch", "ep_combine",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -107,6 +108,9 @@ def _declare(lib):
         "moe_shared_workspace_bytes": (I32, [I32, I32, I32, c.POINTER(SZ)]),
         "moe_probe_wait_timeout": (I32, [P, SZ, c.c_uint, P]),
         "moe_shared_forward": (I32, [P, P, P, P, I32, I32, I32, c.POINTER(Activation), P, SZ, P]),
+        "moe_ep_workspace_bytes": (I32, [I32, I32, I32, I32, c.POINTER(SZ)]),
+        "moe_ep_dispatch": (I32, [P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P, P, P]),
+        "moe_ep_combine": (I32, [P, P, I32, I32, I32, I32, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -498,3 +502,67 @@ class MoELayer:
         return forward(x_fp8, x_sf, topk_idx, topk_w, self.l1_t, self.l2_t, self.E, self.H, self.I,
                        out=out, workspace=self.workspace, expert_stats=expert_stats, events=events,
                        stream=stream, act=act, weights=self.weights)
+
+
+# ------------------------------------------------------------ expert parallelism
+def ep_workspace_bytes(T: int, E: int, k: int, H: int) -> int:
+    """Bytes of the dispatch workspace for up to T tokens (host-only)."""
+    n = ctypes.c_size_t()
+    _check(load().moe_ep_workspace_bytes(T, E, k, H, ctypes.byref(n)), "moe_ep_workspace_bytes")
+    return n.value
+
+
+def ep_dispatch(x_fp8, x_sf, topk_idx, E: int, ranks: int, workspace, send_x=None, send_sf=None, send_eid=None,
+                send_counts=None, stream=None):
+    """Routing and the send buffers of expert parallelism: returns (send_x u8
+    [T*k, H], send_sf u8 [T*k, H/32], send_eid i64 [T*k], send_counts i64
+    [ranks]); the first sum(send_counts) rows, grouped by destination rank,
+    are written.  ``workspace`` (u8, ep_workspace_bytes) must stay untouched
+    until the matching ep_combine."""
+    _need(x_fp8, torch.uint8, "x_fp8", 2)
+    _need(x_sf, torch.uint8, "x_sf", 2)
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(workspace, torch.uint8, "workspace")
+    T, H = x_fp8.shape
+    k = topk_idx.shape[1]
+    if x_sf.shape != (T, H // 32) or topk_idx.shape[0] != T:
+        raise ValueError("inconsistent input shapes")
+    dev = x_fp8.device
+    if send_x is None:
+        send_x = torch.empty((T * k, H), dtype=torch.uint8, device=dev)
+    if send_sf is None:
+        send_sf = torch.empty((T * k, H // 32), dtype=torch.uint8, device=dev)
+    if send_eid is None:
+        send_eid = torch.empty(T * k, dtype=torch.int64, device=dev)
+    if send_counts is None:
+        send_counts = torch.empty(ranks, dtype=torch.int64, device=dev)
+    _need(send_x, torch.uint8, "send_x", 2)
+    _need(send_sf, torch.uint8, "send_sf", 2)
+    _need(send_eid, torch.int64, "send_eid", 1)
+    _need(send_counts, torch.int64, "send_counts", 1)
+    if (send_x.shape[0] < T * k or send_x.shape[1] != H or send_sf.shape[0] < T * k or send_sf.shape[1] != H // 32
+            or send_eid.numel() < T * k or send_counts.numel() != ranks):
+        raise ValueError("send buffers too small")
+    _check(load().moe_ep_dispatch(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), T, E, k, H, ranks, _ptr(workspace),
+                                  workspace.numel(), _ptr(send_x), _ptr(send_sf), _ptr(send_eid), _ptr(send_counts),
+                                  _stream(stream)), "moe_ep_dispatch")
+    return send_x, send_sf, send_eid, send_counts
+
+
+def ep_combine(y, topk_w, E: int, workspace, out=None, stream=None):
+    """out (bf16 [T, H]) = the top-k-weighted sum of the returned rows y (bf16
+    [n, H], in send order) through the inverse permutation of the ep_dispatch
+    that used ``workspace`` with the same T, E, k, H."""
+    _need(y, torch.bfloat16, "y", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(workspace, torch.uint8, "workspace")
+    T, k = topk_w.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=topk_w.device)
+    _need(out, torch.bfloat16, "out", 2)
+    if out.shape != (T, H):
+        raise ValueError("out must be [T, H]")
+    _check(load().moe_ep_combine(_ptr(y), _ptr(topk_w), T, E, k, H, _ptr(workspace), workspace.numel(), _ptr(out),
+                                 _stream(stream)), "moe_ep_combine")
+    return out

@@ -3,6 +3,7 @@
 // local gather through the inverse permutation instead of cross-rank stores).
 // out[t] = bf16_rne(sum_{j ascending} topk_w[t, j] * Y[inv[t*k + j]]), fp32
 // sum, no atomics, so the result is deterministic.
+#include "ep_internal.h"
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -69,17 +70,22 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfl
     }
 }
 
-cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
-                           void *out, cudaStream_t stream) {
+cudaError_t launch_combine_rows(const void *y, const int *inv, const float *topk_w, int T, int k, int H, void *out,
+                                cudaStream_t stream) {
     const int col_blocks = (H + kCombineCols - 1) / kCombineCols;
     // at most 16 blocks (2048 threads) per SM, each looping over tasks: fewer,
     // longer-lived blocks than one per task keep more loads in flight
     const int64_t tasks = int64_t(T) * col_blocks, cap = int64_t(num_sms()) * 16;
     const int64_t grid = tasks < cap ? tasks : cap;
     return launch_pdl(combine_kernel, dim3(unsigned(grid)), dim3(kCombineThreads), 0, stream,
-                      reinterpret_cast<const __nv_bfloat16 *>(ws + L.off_y),
-                      reinterpret_cast<const int *>(ws + L.off_inv), topk_w, k, H, col_blocks, T,
+                      static_cast<const __nv_bfloat16 *>(y), inv, topk_w, k, H, col_blocks, T,
                       static_cast<__nv_bfloat16 *>(out));
+}
+
+cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
+                           void *out, cudaStream_t stream) {
+    return launch_combine_rows(ws + L.off_y, reinterpret_cast<const int *>(ws + L.off_inv), topk_w, T, k, H, out,
+                               stream);
 }
 
 }  // namespace moe

@@ -1,0 +1,146 @@
+// ep.cu -- the per-rank ends of expert parallelism: the dispatch and combine
+// phases of "Mega moe fusion with symmetric memory" (Procedure, step 5,
+// phases 1 and 5) with the cross-rank exchange left to the caller (an
+// all-to-all-v over NCCL between the two calls and after the expert layer).
+//
+// Ranks own contiguous expert ranges: rank r holds experts [r*E/R, (r+1)*E/R).
+// Dispatch runs the layer's routing (the stable counting sort by expert), so
+// the routed rows in permutation order are already grouped by destination
+// rank; it copies each routed slot's FP8 row, its UE8M0 scales and its local
+// expert id into send buffers in that order and writes the per-rank row
+// counts.  The receiving rank runs the expert layer over its E/R experts with
+// k = 1 and weight 1 (the layer's output for such a row is its bf16 Y row
+// unchanged).  Combine takes the returned rows, still in send order, and
+// forms out[t] = bf16(sum_j w[t, j] * Y[inv[t*k + j]]) with the layer's own
+// combine kernel through the inverse permutation the dispatch left in the
+// workspace.
+#include "ep_internal.h"
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kPackThreads = 256;
+
+// Workspace of the dispatch: the layer's routing regions only (header,
+// counts, offsets, chunk lists, histograms, permutation, inverse, gather
+// descriptors), with the side chunk list moved down to where the layer's
+// gathered activations would start.
+WsLayout ep_layout(int T, int E, int k, int H) {
+    WsLayout L = ws_layout(T, E, k, H, kTileK);
+    L.off_chunks_s = L.off_xg;
+    L.total = L.off_chunks_s + align_up(sizeof(int4) * size_t(L.max_side > 0 ? L.max_side : 1), 256);
+    return L;
+}
+
+// One warp per routed row (rows in permutation order, nrows = offset[E]):
+// send row pos <- token perm[pos] / k (row_vec 16-byte vectors, sf_words
+// 4-byte scale words), send_eid[pos] = the slot's expert id modulo e_loc.
+// Block 0 also writes send_counts[r] = rows for experts [r*e_loc, (r+1)*e_loc).
+__global__ void __launch_bounds__(kPackThreads) ep_pack_kernel(const int *__restrict__ perm,
+                                                               const int *__restrict__ offset,
+                                                               const int64_t *__restrict__ topk_idx, int E, int k,
+                                                               int e_loc, int ranks, int row_vec, int sf_words,
+                                                               const uint4 *__restrict__ x,
+                                                               const uint32_t *__restrict__ x_sf,
+                                                               uint4 *__restrict__ send_x,
+                                                               uint32_t *__restrict__ send_sf,
+                                                               int64_t *__restrict__ send_eid,
+                                                               int64_t *__restrict__ send_counts) {
+    pdl_wait();
+    pdl_trigger();
+    if (blockIdx.x == 0)
+        for (int r = threadIdx.x; r < ranks; r += blockDim.x)
+            send_counts[r] = int64_t(__ldcg(offset + (r + 1) * e_loc)) - __ldcg(offset + r * e_loc);
+    constexpr int kWarps = kPackThreads / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t nrows = __ldcg(offset + E);  // dropped slots leave no row
+    const int64_t nwarps = int64_t(gridDim.x) * kWarps;
+    for (int64_t pos = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); pos < nrows; pos += nwarps) {
+        const int s = __ldcg(perm + pos);
+        const int64_t t = s / k;
+        const uint4 *src = x + t * row_vec;
+        uint4 *dst = send_x + pos * row_vec;
+        for (int v = lane; v < row_vec; v += 32) dst[v] = __ldg(src + v);
+        for (int w = lane; w < sf_words; w += 32) send_sf[pos * sf_words + w] = __ldg(x_sf + t * sf_words + w);
+        if (lane == 0) send_eid[pos] = __ldg(topk_idx + s) % e_loc;  // routed: the id is in [0, E)
+    }
+}
+
+moe_status_t check_ep_args(int T, int E, int k, int H) {
+    if (T < 0 || E <= 0 || k <= 0 || k > E || H <= 0) return MOE_ERR_INVALID_ARG;
+    if (H % kTileK != 0 || E > kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (int64_t(T) * k > int64_t(0x7FFFFFFF) / 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status_t moe_ep_workspace_bytes(int T_max, int E, int k, int H, size_t *bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const moe_status_t s = check_ep_args(T_max, E, k, H);
+    if (s != MOE_OK) return s;
+    *bytes = ep_layout(T_max, E, k, H).total;
+    return MOE_OK;
+}
+
+moe_status_t moe_ep_dispatch(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, int T, int E, int k,
+                             int H, int ranks, void *workspace, size_t ws_bytes, void *send_x, void *send_sf,
+                             int64_t *send_eid, int64_t *send_counts, moe_stream_t stream) {
+    moe_status_t s = check_ep_args(T, E, k, H);
+    if (s != MOE_OK) return s;
+    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
+    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!workspace || !send_counts || !aligned(workspace, 256) || !aligned(send_counts, 8))
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x_fp8 || !x_sf || !topk_idx || !send_x || !send_sf || !send_eid || !aligned(x_fp8, 16) ||
+                  !aligned(x_sf, 4) || !aligned(topk_idx, 8) || !aligned(send_x, 16) || !aligned(send_sf, 4) ||
+                  !aligned(send_eid, 8)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ep_layout(T, E, k, H);
+    if (T > 0 && ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0)
+        return cudaMemsetAsync(send_counts, 0, sizeof(int64_t) * size_t(ranks), st) == cudaSuccess ? MOE_OK
+                                                                                                     : MOE_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    cudaError_t e = launch_routing(topk_idx, k, E, ws, L, nullptr, st);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    const int64_t want = (L.R + kPackThreads / 32 - 1) / (kPackThreads / 32);
+    const int64_t cap = int64_t(num_sms()) * 8;
+    const int grid = int(want < cap ? want : cap);
+    e = launch_pdl(ep_pack_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kPackThreads), 0, st,
+                   reinterpret_cast<const int *>(ws + L.off_perm), reinterpret_cast<const int *>(ws + L.off_offset),
+                   topk_idx, E, k, E / ranks, ranks, H / 16, H / 128, static_cast<const uint4 *>(x_fp8),
+                   static_cast<const uint32_t *>(x_sf), static_cast<uint4 *>(send_x), static_cast<uint32_t *>(send_sf),
+                   send_eid, send_counts);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_ep_combine(const void *y_bf16, const float *topk_w, int T, int E, int k, int H,
+                            const void *workspace, size_t ws_bytes, void *out_bf16, moe_stream_t stream) {
+    moe_status_t s = check_ep_args(T, E, k, H);
+    if (s != MOE_OK) return s;
+    if (T == 0) return MOE_OK;
+    if (!y_bf16 || !topk_w || !workspace || !out_bf16 || !aligned(y_bf16, 16) || !aligned(topk_w, 4) ||
+        !aligned(workspace, 256) || !aligned(out_bf16, 16))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ep_layout(T, E, k, H);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    const cudaError_t e = launch_combine_rows(y_bf16, reinterpret_cast<const int *>(ws + L.off_inv), topk_w, T, k, H,
+                                              out_bf16, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -23,6 +23,7 @@
 //
 // Within an expert, routed rows keep ascending slot order t*k+j (a stable
 // counting sort), so the metadata is unique and compared bit-exactly.
+#include "ep_internal.h"
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -341,9 +342,8 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const int4 *__re
     }
 }
 
-cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
-                         int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, bool nvfp4,
-                         cudaStream_t stream) {
+cudaError_t launch_routing(const int64_t *topk_idx, int k, int E, uint8_t *ws, const WsLayout &L,
+                           int32_t *expert_stats, cudaStream_t stream) {
     const int R = int(L.R);
     int *hdr = reinterpret_cast<int *>(ws);
     int *hist = reinterpret_cast<int *>(ws + L.off_hist);
@@ -387,7 +387,17 @@ cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_
             e = launch_pdl(route_place_kernel, dim3(L.nb), dim3(kRouteBlock), 0, stream, topk_idx, R, k, E, cr, hist,
                            lrank, offset, chunk_base, perm, inv, rowinfo);
     }
+    return e;
+}
+
+cudaError_t launch_route(const int64_t *topk_idx, const uint8_t *x, const uint8_t *x_sf, int T, int k, int E,
+                         int H, uint8_t *ws, const WsLayout &L, int32_t *expert_stats, bool nvfp4,
+                         cudaStream_t stream) {
+    cudaError_t e = launch_routing(topk_idx, k, E, ws, L, expert_stats, stream);
     if (e != cudaSuccess) return e;
+    const int R = int(L.R);
+    const int *offset = reinterpret_cast<const int *>(ws + L.off_offset);
+    const int4 *rowinfo = reinterpret_cast<const int4 *>(ws + L.off_rowinfo);
     // up to 4 blocks per SM, striding over (row, piece) tasks; rows are cut
     // into pieces of a multiple of 32 vectors until there are about that many
     // warps' worth of tasks

@@ -1,0 +1,148 @@
+"""Expert parallelism across ranks, one process per GPU: the dispatch, expert
+layer and combine of "Mega moe fusion with symmetric memory" (Procedure,
+step 5) with the cross-rank exchange as all-to-all-v collectives of
+torch.distributed (NCCL over NVLink between GPUs).
+
+Rank r of R holds experts [r E/R, (r+1) E/R) in the packet layout.  A step
+on each rank:
+
+1. ``dispatch``: the library's routing packs the rank's routed rows (FP8 row,
+   UE8M0 scales, local expert id), grouped by destination rank, and counts
+   them per rank;
+2. the counts (all_gather), then the rows (all_to_all_single) cross ranks;
+3. ``expert``: the expert layer over the received rows with E/R experts, k = 1
+   and weight 1, whose output is each row's bf16 expert output Y unchanged;
+4. the outputs go back (the reverse all_to_all_single);
+5. ``combine``: the library's top-k-weighted sum through the inverse
+   permutation of step 1.
+
+Every step of the computation runs in the CUDA library; this module sizes the
+buffers and issues the collectives.  Every rank takes the same collective
+steps in the same order, whatever its row counts.  The row counts are needed
+on the host for the split sizes, so ``forward`` synchronises once per step
+after the count exchange (an all-gather of every rank's per-destination
+counts).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import ep_combine, ep_dispatch, ep_workspace_bytes, forward, workspace_bytes
+
+__all__ = ["ExpertParallelLayer"]
+
+
+class ExpertParallelLayer:
+    """One rank's share of an expert-parallel MoE layer.
+
+    l1_t, l2_t: the packet buffers (``transform_weights``) of this rank's E/R
+    experts; E, k, H, I: the layer's sizes (E counts all ranks' experts);
+    T_max: tokens per step on this rank; recv_max: rows this rank can receive
+    per step (default R * T_max * k, every slot of every rank); rank, ranks:
+    this rank and the rank count (default: from the initialised default
+    process group, else 0 and 1); group: the process group of the exchange.
+    """
+
+    def __init__(self, l1_t, l2_t, E: int, k: int, H: int, I: int, T_max: int, recv_max: int | None = None,
+                 rank: int | None = None, ranks: int | None = None, group=None, device=None):
+        import torch.distributed as dist
+        live = dist.is_available() and dist.is_initialized()
+        self.group = group
+        self.ranks = ranks if ranks is not None else (dist.get_world_size(group) if live else 1)
+        self.rank = rank if rank is not None else (dist.get_rank(group) if live else 0)
+        if E % self.ranks != 0:
+            raise ValueError(f"E = {E} is not a multiple of the rank count {self.ranks}")
+        if not 0 <= self.rank < self.ranks:
+            raise ValueError("rank out of range")
+        self.l1_t, self.l2_t = l1_t, l2_t
+        self.E, self.k, self.H, self.I, self.T_max = E, k, H, I, T_max
+        self.E_loc = E // self.ranks
+        self.recv_max = recv_max if recv_max is not None else self.ranks * T_max * k
+        dev = torch.device(device) if device is not None else (l1_t.device if l1_t is not None else None)
+        u8, i64 = torch.uint8, torch.int64
+        n = max(T_max * k, 1)
+        self.ws = torch.empty(ep_workspace_bytes(T_max, E, k, H), dtype=u8, device=dev)
+        self.send_x = torch.empty((n, H), dtype=u8, device=dev)
+        self.send_sf = torch.empty((n, H // 32), dtype=u8, device=dev)
+        self.send_eid = torch.empty(n, dtype=i64, device=dev)
+        self.send_counts = torch.empty(self.ranks, dtype=i64, device=dev)
+        m = max(self.recv_max, 1)
+        self.recv_x = torch.empty((m, H), dtype=u8, device=dev)
+        self.recv_sf = torch.empty((m, H // 32), dtype=u8, device=dev)
+        self.recv_eid = torch.empty((m, 1), dtype=i64, device=dev)
+        self.ones = torch.ones((m, 1), dtype=torch.float32, device=dev)
+        self.y_loc = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
+        self.y_back = torch.empty((n, H), dtype=torch.bfloat16, device=dev)
+        self.ws_loc = torch.empty(workspace_bytes(self.recv_max, self.E_loc, 1, H, I), dtype=u8, device=dev)
+
+    # ---------------------------------------------------------------- phases
+    def dispatch(self, x_fp8, x_sf, topk_idx, stream=None):
+        """Step 1: fills send_x / send_sf / send_eid (rows grouped by destination
+        rank) and returns send_counts (i64 [ranks], device)."""
+        if x_fp8.shape[0] > self.T_max:
+            raise ValueError(f"{x_fp8.shape[0]} tokens > T_max = {self.T_max}")
+        ep_dispatch(x_fp8, x_sf, topk_idx, self.E, self.ranks, self.ws, self.send_x, self.send_sf, self.send_eid,
+                    self.send_counts, stream=stream)
+        return self.send_counts
+
+    def expert(self, n: int, x=None, sf=None, eid=None, out=None, stream=None):
+        """Step 3: the expert layer over n rows (default: the first n received
+        rows; x u8 [>=n, H], sf u8 [>=n, H/32], eid i64 [>=n] local expert
+        ids); returns their bf16 outputs ([n, H], a view of ``out``, default
+        y_loc)."""
+        n = int(n)
+        if n > self.recv_max:
+            raise ValueError(f"{n} rows > recv_max = {self.recv_max}")
+        x = self.recv_x if x is None else x
+        sf = self.recv_sf if sf is None else sf
+        eid = self.recv_eid[:, 0] if eid is None else eid
+        out = self.y_loc if out is None else out
+        if n == 0:
+            return out[:0]
+        return forward(x[:n], sf[:n], eid[:n].view(n, 1), self.ones[:n], self.l1_t, self.l2_t, self.E_loc, self.H,
+                       self.I, out=out[:n], workspace=self.ws_loc, stream=stream)
+
+    def combine(self, topk_w, out=None, stream=None):
+        """Step 5: out (bf16 [T, H]) from the returned rows in y_back."""
+        return ep_combine(self.y_back, topk_w, self.E, self.ws, out=out, stream=stream)
+
+    # ------------------------------------------------------------- one step
+    def _exchange(self, dst, src, out_splits, in_splits):
+        import torch.distributed as dist
+        dist.all_to_all_single(dst, src, output_split_sizes=out_splits, input_split_sizes=in_splits,
+                               group=self.group)
+
+    def forward(self, x_fp8, x_sf, topk_idx, topk_w, out=None):
+        """One layer step on this rank's tokens; returns out (bf16 [T, H])."""
+        for t, dt, name in ((x_fp8, torch.uint8, "x_fp8"), (x_sf, torch.uint8, "x_sf"),
+                            (topk_idx, torch.int64, "topk_idx"), (topk_w, torch.float32, "topk_w")):
+            if not isinstance(t, torch.Tensor) or t.dtype != dt or not t.is_contiguous():
+                raise TypeError(f"{name} must be a contiguous {dt} tensor")
+        counts = self.dispatch(x_fp8, x_sf, topk_idx)
+        if self.ranks == 1:
+            # no exchange: the expert layer reads the send buffers and writes
+            # the rows combine reads
+            self.expert(int(counts[0].item()), self.send_x, self.send_sf, self.send_eid, out=self.y_back)
+            return self.combine(topk_w, out=out)
+        import torch.distributed as dist
+        # every rank gets the whole [ranks, ranks] count matrix (row = source),
+        # so that all ranks see an overflow of any rank's receive buffers and
+        # stop together (recv_max must be the same on every rank)
+        rows = [torch.empty_like(counts) for _ in range(self.ranks)]
+        dist.all_gather(rows, counts, group=self.group)
+        matrix = torch.stack(rows).tolist()
+        send_splits = matrix[self.rank]
+        recv_splits = [matrix[src][self.rank] for src in range(self.ranks)]
+        n_send, n_recv = sum(send_splits), sum(recv_splits)
+        most = max(sum(matrix[src][dst] for src in range(self.ranks)) for dst in range(self.ranks))
+        if most > self.recv_max:
+            raise ValueError(f"a rank would receive {most} rows > recv_max = {self.recv_max}")
+        self._exchange(self.recv_x[:n_recv], self.send_x[:n_send], recv_splits, send_splits)
+        self._exchange(self.recv_sf[:n_recv], self.send_sf[:n_send], recv_splits, send_splits)
+        self._exchange(self.recv_eid[:n_recv, 0], self.send_eid[:n_send], recv_splits, send_splits)
+        y = self.expert(n_recv)
+        # bf16 rows travel as bytes (2H per row), which every backend moves
+        self._exchange(self.y_back[:n_send].view(torch.uint8), y.view(torch.uint8), send_splits, recv_splits)
+        return self.combine(topk_w, out=out)
+
+    __call__ = forward

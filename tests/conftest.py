@@ -12,6 +12,14 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_collection_modifyitems(config, items):
+    # The expert-parallel tests run the single-GPU layer inside every rank, so
+    # they come after every test of the layer's own entry points (a layer
+    # failure is reported as such first).
+    rank = {"test_gpu_ep": 1}
+    items.sort(key=lambda it: rank.get(getattr(it.module, "__name__", ""), 0))
+
+
 @pytest.fixture(scope="session")
 def olib():
     import oracle

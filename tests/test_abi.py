@@ -221,3 +221,43 @@ def test_static_workspace_holds_decode_batches(moelib):
     top-6, H = 7168, I = 3072 (the sizes its documentation names)."""
     import moe_expert_layer_08_b200 as m
     assert m.workspace_bytes(128, 384, 6, 7168, 3072) <= m.STATIC_WORKSPACE_BYTES
+
+
+def test_expert_parallel_entry_points_validate_on_the_host(moelib):
+    """The dispatch workspace holds the routing metadata only (monotone in T,
+    a small fraction of the layer's); shapes, rank counts, pointers,
+    alignment and sizes are checked before any CUDA call."""
+    import moe_expert_layer_08_b200 as m
+    lib = m.load()
+    sizes = [m.ep_workspace_bytes(T, 384, 6, 7168) for T in range(0, 9000, 97)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+    assert m.ep_workspace_bytes(8192, 384, 6, 7168) < m.workspace_bytes(8192, 384, 6, 7168, 3072) // 100
+    n = ctypes.c_size_t()
+    assert lib.moe_ep_workspace_bytes(8, 384, 6, 200, ctypes.byref(n)) == 2    # H % 128
+    assert lib.moe_ep_workspace_bytes(8, 4, 6, 256, ctypes.byref(n)) == 1      # k > E
+    assert lib.moe_ep_workspace_bytes(8, 4, 2, 256, None) == 1
+    p = ctypes.c_void_p(1 << 20)                                               # never dereferenced
+
+    def dispatch(**kw):
+        return lib.moe_ep_dispatch(kw.get("x", p), p, p, kw.get("T", 4), 8, 2, kw.get("H", 256),
+                                   kw.get("ranks", 2), kw.get("ws", p), kw.get("ws_bytes", 1 << 30), p, p, p,
+                                   kw.get("counts", p), None)
+
+    assert dispatch(ranks=0) == 1
+    assert dispatch(ranks=9) == 1                                  # more ranks than experts
+    assert dispatch(ranks=3) == 2                                  # E % ranks
+    assert dispatch(H=200) == 2
+    assert dispatch(T=-1) == 1
+    assert dispatch(ws=None) == 1
+    assert dispatch(counts=None) == 1
+    assert dispatch(x=ctypes.c_void_p((1 << 20) + 8)) == 1         # x not 16-byte aligned
+    assert dispatch(ws_bytes=16) == 3
+
+    def combine(**kw):
+        return lib.moe_ep_combine(kw.get("y", p), p, kw.get("T", 4), 8, 2, 256, kw.get("ws", p),
+                                  kw.get("ws_bytes", 1 << 30), p, None)
+
+    assert combine(T=0) == 0                                       # nothing to do
+    assert combine(T=-1) == 1
+    assert combine(y=None) == 1
+    assert combine(ws_bytes=16) == 3
