@@ -56,6 +56,9 @@ def parse():
     p.add_argument("--shared-expert", type=int, default=0, metavar="T",
                    help="time the BF16 shared expert (moe_shared_forward) on T tokens instead of the layer")
     p.add_argument("--shared-dims", default="7168,2048", help="SH,SI of the shared expert")
+    p.add_argument("--ep", action="store_true",
+                   help="expert parallelism: rank r of N holds experts [r E/N, (r+1) E/N) and T tokens of its own; "
+                        "NCCL all-to-alls around the library's dispatch and combine")
     p.add_argument("--fp8-peak", action="store_true",
                    help="measure cuBLAS FP8 8192^3 matmul throughput (MX block-scaled and per-tensor scaled), "
                         "burst and sustained")
@@ -416,6 +419,87 @@ def run_fp8_peak(args):
     print(json.dumps(out), flush=True)
 
 
+def run_ep(args, w, rank, world, local_rank):
+    """Expert-parallel steps (moe_expert_layer_08_b200.ep): every rank routes
+    its own T tokens over all E experts and holds E / N of them; a step is
+    the dispatch, the count all-gather and row all-to-alls, the layer over the
+    received rows, the all-to-all back and the combine.  Timed like the main
+    arm (barrier + CUDA events around K steps, max over ranks); the step
+    includes its one host synchronisation (the split sizes)."""
+    import moe_expert_layer_08_b200 as moe
+    from moe_expert_layer_08_b200 import build as mbuild
+    from moe_expert_layer_08_b200.ep import ExpertParallelLayer
+    if rank == 0:
+        mbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    if w.E % world:
+        raise SystemExit(f"E = {w.E} is not a multiple of {world} ranks")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    e_loc = w.E // world
+    mine = W.custom(f"{w.name}_rank{rank}", T=w.T, E=w.E, k=w.k, H=w.H, I=w.I, seed=w.seed + 7919 * rank,
+                    routing=w.routing, zipf_s=w.zipf_s)
+    x = W.gen_x(mine, device)
+    idx, tw = W.gen_routing(mine, device)
+    xq, xs = moe.quantize_fp8(x)
+    n1, n2 = moe.transformed_weight_bytes(w.E, w.H, w.I)
+    p1, p2 = n1 // w.E, n2 // w.E
+    l1_t = torch.empty(e_loc * p1, dtype=torch.uint8, device=device)
+    l2_t = torch.empty(e_loc * p2, dtype=torch.uint8, device=device)
+    for i, e in enumerate(range(rank * e_loc, (rank + 1) * e_loc)):   # the experts' draws depend on w.seed only
+        a, b = moe.quantize_fp4(W.gen_l1(w, e, device))
+        c, d = moe.quantize_fp4(W.gen_l2(w, e, device))
+        moe.transform_weights(a[None], b[None], c[None], d[None],
+                              out=(l1_t[i * p1:(i + 1) * p1], l2_t[i * p2:(i + 1) * p2]))
+    torch.cuda.synchronize(device)
+    layer = ExpertParallelLayer(l1_t, l2_t, w.E, w.k, w.H, w.I, T_max=w.T)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        layer(xq, xs, idx, tw, out=out)
+
+    for _ in range(args.warmup):
+        step()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clocks:
+        barrier()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        barrier()
+    ms = max_over_ranks(start.elapsed_time(stop) / args.steps, device)
+    st = moe.check_device_error(layer.ws)
+    if st != 0:
+        raise RuntimeError(f"device error: {moe.STATUS.get(st, st)}")
+    # kernels of this library per step: routing (one block up to 1024 rows,
+    # else four kernels) + pack, the layer over the received rows, the combine
+    route = 1 if w.T * w.k <= 1024 else 4
+    launches = route + 1 + moe.forward_kernel_launches(layer.last_n_recv, e_loc, 1, w.H, w.I) + 1
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * w.flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "data": "synthetic", "dtype": "fp8xfp4 (fp32 accumulate)",
+            "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "routing")},
+                       "tokens_per_rank": w.T, "experts_per_rank": e_loc, "parallelism": f"ep{world}",
+                       "exchange": "NCCL all_gather (counts) + all_to_all_single (rows out, outputs back)"
+                       if world > 1 else "none (one rank)"},
+            "us_per_layer": ms * 1e3,
+            "gpu_launches": args.steps * launches,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def run_shared_reference(args, rank):
     """The oracle's shared expert on the host cores, on the first
     ``--cpu-tokens`` of the T tokens per step (rank 0 only)."""
@@ -651,6 +735,8 @@ def main():
     try:
         if args.fp8_peak:
             run_fp8_peak(args)
+        elif args.ep and args.impl == "b200":
+            run_ep(args, w, rank, world, local_rank)
         elif args.shared_expert and args.impl == "reference":
             run_shared_reference(args, rank)
         elif args.shared_expert:

@@ -74,6 +74,7 @@ class ExpertParallelLayer:
         self.y_loc = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
         self.y_back = torch.empty((n, H), dtype=torch.bfloat16, device=dev)
         self.ws_loc = torch.empty(workspace_bytes(self.recv_max, self.E_loc, 1, H, I), dtype=u8, device=dev)
+        self.last_n_recv = 0  # rows the expert layer ran over in the last step
 
     # ---------------------------------------------------------------- phases
     def dispatch(self, x_fp8, x_sf, topk_idx, stream=None):
@@ -122,7 +123,8 @@ class ExpertParallelLayer:
         if self.ranks == 1:
             # no exchange: the expert layer reads the send buffers and writes
             # the rows combine reads
-            self.expert(int(counts[0].item()), self.send_x, self.send_sf, self.send_eid, out=self.y_back)
+            self.last_n_recv = int(counts[0].item())
+            self.expert(self.last_n_recv, self.send_x, self.send_sf, self.send_eid, out=self.y_back)
             return self.combine(topk_w, out=out)
         import torch.distributed as dist
         # every rank gets the whole [ranks, ranks] count matrix (row = source),
@@ -137,6 +139,7 @@ class ExpertParallelLayer:
         most = max(sum(matrix[src][dst] for src in range(self.ranks)) for dst in range(self.ranks))
         if most > self.recv_max:
             raise ValueError(f"a rank would receive {most} rows > recv_max = {self.recv_max}")
+        self.last_n_recv = n_recv
         self._exchange(self.recv_x[:n_recv], self.send_x[:n_send], recv_splits, send_splits)
         self._exchange(self.recv_sf[:n_recv], self.send_sf[:n_send], recv_splits, send_splits)
         self._exchange(self.recv_eid[:n_recv, 0], self.send_eid[:n_send], recv_splits, send_splits)
