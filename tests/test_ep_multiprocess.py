@@ -46,13 +46,17 @@ def _fake_layer_class():
             return self.send_counts
 
         def expert(self, n, x=None, sf=None, eid=None, out=None, stream=None):
+            x = self.recv_x if x is None else x
+            sf = self.recv_sf if sf is None else sf
+            eid = self.recv_eid[:, 0] if eid is None else eid
+            out = self.y_loc if out is None else out
             if n == 0:
-                return self.y_loc[:0]
-            ids = self.recv_eid[:n, 0].numpy() + self.rank * self.E_loc
-            res = oracle.forward(self.recv_x[:n].numpy(), self.recv_sf[:n].numpy(), ids[:, None],
-                                 np.ones((n, 1), np.float32), self.experts, self.E, self.H, self.I)
-            self.y_loc[:n].view(torch.int16).copy_(torch.from_numpy(res["out_bf16"].view(np.int16)))
-            return self.y_loc[:n]
+                return out[:0]
+            ids = eid[:n].numpy() + self.rank * self.E_loc
+            res = oracle.forward(x[:n].numpy(), sf[:n].numpy(), ids[:, None], np.ones((n, 1), np.float32),
+                                 self.experts, self.E, self.H, self.I)
+            out[:n].view(torch.int16).copy_(torch.from_numpy(res["out_bf16"].view(np.int16)))
+            return out[:n]
 
         def combine(self, topk_w, out=None, stream=None):
             n = int(self.send_counts.sum())
@@ -80,6 +84,19 @@ def _inputs(rank, T):
     return xq, xs, idx, tw, experts
 
 
+def _expected(xq, xs, idx, tw, experts, ranks):
+    """The combine of the bf16-rounded expert outputs the oracle computes for
+    these tokens with every expert at hand."""
+    import ep_definition as D
+    import oracle
+    if idx.shape[0] == 0:
+        return torch.empty((0, H), dtype=torch.bfloat16)
+    y = oracle.forward(xq, xs, idx.numpy(), tw.numpy(), experts, E, H, I, intermediates=True)["y"]
+    order, _, _, inv = D.dispatch_plan(idx.numpy(), E, ranks)
+    rows = torch.from_numpy(y[order // K, order % K]).to(torch.bfloat16).float().numpy()
+    return D.combine(rows, inv, tw.numpy(), K)
+
+
 def _worker(rank, world, port, q, tokens, recv_max):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -88,8 +105,6 @@ def _worker(rank, world, port, q, tokens, recv_max):
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        import ep_definition as D
-        import oracle
         T = tokens[rank]
         xq, xs, idx, tw, experts = _inputs(rank, T)
         layer = _fake_layer_class()(None, None, E, K, H, I, T_max=max(tokens), recv_max=recv_max, device="cpu")
@@ -100,13 +115,7 @@ def _worker(rank, world, port, q, tokens, recv_max):
         except ValueError as err:
             q.put((rank, "ValueError", str(err)))
             return
-        if T > 0:
-            y = oracle.forward(xq, xs, idx.numpy(), tw.numpy(), experts, E, H, I, intermediates=True)["y"]
-            order, _, _, inv = D.dispatch_plan(idx.numpy(), E, world)
-            rows = torch.from_numpy(y[order // K, order % K]).to(torch.bfloat16).float().numpy()
-            want = D.combine(rows, inv, tw.numpy(), K)
-        else:
-            want = torch.empty((0, H), dtype=torch.bfloat16)
+        want = _expected(xq, xs, idx, tw, experts, world)
         same = out.shape == want.shape and torch.equal(out.view(torch.int16), want.view(torch.int16))
         q.put((rank, "ok", bool(same)))
     finally:
@@ -135,3 +144,18 @@ def test_exchange_matches_single_rank_definition(tokens):
 def test_receive_overflow_stops_every_rank():
     res = _run((12, 7), recv_max=3)
     assert {r: kind for r, (kind, _) in res.items()} == {0: "ValueError", 1: "ValueError"}, res
+
+
+def test_one_rank_runs_without_exchange():
+    """Without a process group the layer is one rank: no collective, the
+    expert phase reads the send buffers and writes the rows combine reads."""
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    xq, xs, idx, tw, experts = _inputs(0, 11)
+    layer = _fake_layer_class()(None, None, E, K, H, I, T_max=11, device="cpu")
+    assert layer.ranks == 1 and layer.E_loc == E
+    layer.experts = experts
+    out = layer.forward(torch.from_numpy(xq), torch.from_numpy(xs), idx, tw)
+    want = _expected(xq, xs, idx, tw, experts, 1)
+    assert torch.equal(out.view(torch.int16), want.view(torch.int16))
+    assert layer.last_n_recv == int((idx.numpy() < E).sum())
