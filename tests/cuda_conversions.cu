@@ -9,6 +9,7 @@
 // entries) or -1 for a bad argument.  Device entries take device pointers and
 // a cudaStream_t (NULL = the legacy default stream) and return once the
 // kernel is queued; the caller synchronises.
+#include <cuda_bf16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -97,6 +98,39 @@ int cvt_host_round_e2m1(const float *in, uint8_t *out, int n)
         return -1;
     for (int i = 0; i < n; ++i)
         out[i] = round_e2m1(in[i]);
+    return 0;
+}
+
+// host path: out[i] = the UE8M0 byte of the smallest power of two >= |in[i]|
+// (rounding toward +infinity, clipped to 2^-127 .. 2^127), i < n
+int cvt_host_e8m0_ceil(const double *in, uint8_t *out, int n)
+{
+    if (n < 0 || (n > 0 && (!in || !out)))
+        return -1;
+    for (int i = 0; i < n; ++i)
+        out[i] = (uint8_t)__nv_cvt_double_to_e8m0(in[i], __NV_SATFINITE, cudaRoundPosInf);
+    return 0;
+}
+
+// host path: out[b] = the value of UE8M0 byte b, b < 256
+int cvt_host_decode_e8m0(float *out)
+{
+    if (!out)
+        return -1;
+    for (uint32_t b = 0; b < 256; ++b)
+        out[b] = __bfloat162float(__nv_bfloat16(__nv_cvt_e8m0_to_bf16raw((__nv_fp8_storage_t)b)));
+    return 0;
+}
+
+// host path: out[i] = the bf16 bits of in[i] rounded to nearest even, i < n
+int cvt_host_f32_to_bf16(const float *in, uint16_t *out, int n)
+{
+    if (n < 0 || (n > 0 && (!in || !out)))
+        return -1;
+    for (int i = 0; i < n; ++i) {
+        const __nv_bfloat16 b = __float2bfloat16_rn(in[i]);
+        out[i] = __nv_bfloat16_raw(b).x;
+    }
     return 0;
 }
 

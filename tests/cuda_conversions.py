@@ -37,5 +37,8 @@ def load():
             getattr(lib, name).argtypes = [vp, vp]
         for name in ("cvt_dev_round_e4m3", "cvt_dev_round_e2m1"):
             getattr(lib, name).argtypes = [vp, vp, ctypes.c_int, vp]
+        lib.cvt_host_e8m0_ceil.argtypes = [ctypes.POINTER(ctypes.c_double), u8p, ctypes.c_int]
+        lib.cvt_host_decode_e8m0.argtypes = [f32p]
+        lib.cvt_host_f32_to_bf16.argtypes = [f32p, ctypes.POINTER(ctypes.c_uint16), ctypes.c_int]
         _lib = lib
     return _lib
