@@ -470,6 +470,19 @@ moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const v
  *   in send order; inv is the inverse permutation the dispatch with the same
  *   T, E, k, H left in the workspace.  T = 0 enqueues nothing.
  *
+ * moe_ep_combine_peers -- steps 4 and 5 in one kernel, for ranks whose
+ *   expert-layer outputs are mapped into this rank's address space (CUDA IPC
+ *   or symmetric memory over NVLink): each returned row is read where rank d
+ *   left it instead of being sent back first.  peer_y: device array [ranks]
+ *   of device pointers, rank d's bf16 [rows, H] output of step 3 (16-byte
+ *   aligned; an entry may be NULL only for a rank that holds none of this
+ *   rank's rows); recv_base: i64 [ranks] device, the row at which this rank's
+ *   block starts in rank d's received rows (the sum of what ranks 0..r-1
+ *   sent to d); topk_idx and topk_w as for the dispatch.  The result equals
+ *   moe_ep_combine's for the same rows bit for bit.  The caller orders the
+ *   call after every rank's step 3 (e.g. a stream-ordered barrier) and keeps
+ *   the peers' outputs until it completes.
+ *
  * Argument errors (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE /
  * MOE_ERR_WORKSPACE_TOO_SMALL) are returned before any CUDA call; a launch
  * failure is MOE_ERR_CUDA.  The caller owns every buffer.
@@ -480,6 +493,9 @@ moe_status_t moe_ep_dispatch(const void *x_fp8, const void *x_sf, const int64_t 
                              int64_t *send_eid, int64_t *send_counts, moe_stream_t stream);
 moe_status_t moe_ep_combine(const void *y_bf16, const float *topk_w, int T, int E, int k, int H,
                             const void *workspace, size_t ws_bytes, void *out_bf16, moe_stream_t stream);
+moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv_base, const int64_t *topk_idx,
+                                  const float *topk_w, int T, int E, int k, int H, int ranks, const void *workspace,
+                                  size_t ws_bytes, void *out_bf16, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

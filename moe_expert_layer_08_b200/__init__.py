@@ -22,7 +22,7 @@ __all__ = [
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
     "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
-    "ep_workspace_bytes", "ep_dispatch", "ep_combine",
+    "ep_workspace_bytes", "ep_dispatch", "ep_combine", "ep_combine_peers",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -111,6 +111,7 @@ def _declare(lib):
         "moe_ep_workspace_bytes": (I32, [I32, I32, I32, I32, c.POINTER(SZ)]),
         "moe_ep_dispatch": (I32, [P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P, P, P]),
         "moe_ep_combine": (I32, [P, P, I32, I32, I32, I32, P, SZ, P, P]),
+        "moe_ep_combine_peers": (I32, [P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -565,4 +566,30 @@ def ep_combine(y, topk_w, E: int, workspace, out=None, stream=None):
         raise ValueError("out must be [T, H]")
     _check(load().moe_ep_combine(_ptr(y), _ptr(topk_w), T, E, k, H, _ptr(workspace), workspace.numel(), _ptr(out),
                                  _stream(stream)), "moe_ep_combine")
+    return out
+
+
+def ep_combine_peers(peer_y, recv_base, topk_idx, topk_w, E: int, H: int, workspace, out=None, stream=None):
+    """The combine reading each returned row from the rank that computed it:
+    ``peer_y`` i64 [ranks] device tensor of the ranks' output addresses (bf16
+    [rows, H] each, mapped into this process), ``recv_base`` i64 [ranks]
+    device tensor (where this rank's rows start in each rank's received
+    rows); returns out (bf16 [T, H])."""
+    _need(peer_y, torch.int64, "peer_y", 1)
+    _need(recv_base, torch.int64, "recv_base", 1)
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(topk_w, torch.float32, "topk_w", 2)
+    _need(workspace, torch.uint8, "workspace")
+    T, k = topk_w.shape
+    ranks = peer_y.numel()
+    if recv_base.numel() != ranks or topk_idx.shape != (T, k):
+        raise ValueError("inconsistent shapes")
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=topk_w.device)
+    _need(out, torch.bfloat16, "out", 2)
+    if out.shape != (T, H):
+        raise ValueError("out must be [T, H]")
+    _check(load().moe_ep_combine_peers(_ptr(peer_y), _ptr(recv_base), _ptr(topk_idx), _ptr(topk_w), T, E, k, H,
+                                       ranks, _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)),
+           "moe_ep_combine_peers")
     return out

@@ -68,6 +68,54 @@ __global__ void __launch_bounds__(kPackThreads) ep_pack_kernel(const int *__rest
     }
 }
 
+// The combine over peer memory: out[t] = bf16_rne(sum_{j ascending} w[t, j] *
+// Y_j) with Y_j read where the expert layer of the row's rank left it: rank
+// d = e / e_loc, row recv_base[d] + (pos - offset[d * e_loc]) of peer_y[d]
+// (pos = inv[t*k + j], the row's place in this rank's send order).  Blocks
+// stride over (token, 1024-column block) tasks; each thread sums 8 columns
+// with the arithmetic of the layer's combine.
+constexpr int kPeerThreads = 128;
+constexpr int kPeerCols = kPeerThreads * 8;
+
+__global__ void __launch_bounds__(kPeerThreads) ep_combine_peers_kernel(
+    const __nv_bfloat16 *const *__restrict__ peer_y, const int64_t *__restrict__ recv_base,
+    const int *__restrict__ inv, const int *__restrict__ offset, const int64_t *__restrict__ topk_idx,
+    const float *__restrict__ topk_w, int k, int H, int e_loc, int col_blocks, int T, __nv_bfloat16 *__restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t task = blockIdx.x; task < int64_t(T) * col_blocks; task += gridDim.x) {
+        const int64_t t = task / col_blocks;
+        const int col = int(task % col_blocks) * kPeerCols + threadIdx.x * 8;
+        if (col >= H) continue;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int pos = __ldcg(inv + t * k + j);
+            if (pos < 0) continue;  // dropped slot
+            const int d = int(__ldg(topk_idx + t * k + j) / e_loc);
+            const int64_t row = __ldcg(recv_base + d) + (pos - __ldcg(offset + d * e_loc));
+            const __nv_bfloat16 *src = peer_y[d];
+            if (!src) continue;  // no buffer given for that rank (its rows contribute nothing)
+            const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(src + row * H + col));
+            const float wv = __ldg(topk_w + t * k + j);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] += wv * __uint_as_float(u[i] << 16);
+                acc[2 * i + 1] += wv * __uint_as_float(u[i] & 0xFFFF0000u);
+            }
+        }
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+            o[i] = *reinterpret_cast<const uint32_t *>(&b);
+        }
+        *reinterpret_cast<uint4 *>(out + t * H + col) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 moe_status_t check_ep_args(int T, int E, int k, int H) {
     if (T < 0 || E <= 0 || k <= 0 || k > E || H <= 0) return MOE_ERR_INVALID_ARG;
     if (H % kTileK != 0 || E > kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -140,6 +188,35 @@ moe_status_t moe_ep_combine(const void *y_bf16, const float *topk_w, int T, int 
     const uint8_t *ws = static_cast<const uint8_t *>(workspace);
     const cudaError_t e = launch_combine_rows(y_bf16, reinterpret_cast<const int *>(ws + L.off_inv), topk_w, T, k, H,
                                               out_bf16, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv_base, const int64_t *topk_idx,
+                                  const float *topk_w, int T, int E, int k, int H, int ranks, const void *workspace,
+                                  size_t ws_bytes, void *out_bf16, moe_stream_t stream) {
+    moe_status_t s = check_ep_args(T, E, k, H);
+    if (s != MOE_OK) return s;
+    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
+    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!peer_y || !recv_base || !topk_idx || !topk_w || !workspace || !out_bf16 || !aligned(peer_y, 8) ||
+        !aligned(recv_base, 8) || !aligned(topk_idx, 8) || !aligned(topk_w, 4) || !aligned(workspace, 256) ||
+        !aligned(out_bf16, 16))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ep_layout(T, E, k, H);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    const int col_blocks = (H + kPeerCols - 1) / kPeerCols;
+    const int64_t tasks = int64_t(T) * col_blocks, cap = int64_t(num_sms()) * 16;
+    const int64_t grid = tasks < cap ? tasks : cap;
+    const cudaError_t e = launch_pdl(ep_combine_peers_kernel, dim3(unsigned(grid)), dim3(kPeerThreads), 0,
+                                     reinterpret_cast<cudaStream_t>(stream),
+                                     reinterpret_cast<const __nv_bfloat16 *const *>(peer_y), recv_base,
+                                     reinterpret_cast<const int *>(ws + L.off_inv),
+                                     reinterpret_cast<const int *>(ws + L.off_offset), topk_idx, topk_w, k, H,
+                                     E / ranks, col_blocks, T, static_cast<__nv_bfloat16 *>(out_bf16));
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -261,3 +261,15 @@ def test_expert_parallel_entry_points_validate_on_the_host(moelib):
     assert combine(T=-1) == 1
     assert combine(y=None) == 1
     assert combine(ws_bytes=16) == 3
+
+    def peers(**kw):
+        return lib.moe_ep_combine_peers(kw.get("peer_y", p), kw.get("base", p), p, p, kw.get("T", 4), 8, 2, 256,
+                                        kw.get("ranks", 2), p, kw.get("ws_bytes", 1 << 30), kw.get("out", p), None)
+
+    assert peers(T=0) == 0
+    assert peers(ranks=3) == 2
+    assert peers(ranks=0) == 1
+    assert peers(peer_y=None) == 1
+    assert peers(base=ctypes.c_void_p((1 << 20) + 4)) == 1                  # recv_base not 8-byte aligned
+    assert peers(out=ctypes.c_void_p((1 << 20) + 8)) == 1                   # out not 16-byte aligned
+    assert peers(ws_bytes=16) == 3

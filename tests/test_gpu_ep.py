@@ -8,7 +8,10 @@ layer with k = 1 over each rank's experts, moe_ep_combine).
 * Two and four ranks emulated in one process: every rank's dispatch, then
   the exchange done by the test as copies between the ranks' buffers (no
   collective, no kernel that waits on another rank), every rank's expert
-  layer, the copies back, every rank's combine.  The dispatch outputs (row
+  layer, the copies back, every rank's combine; and the combine over peer
+  memory (moe_ep_combine_peers), reading each row from the buffer of the
+  rank that computed it, equal to the combine of the returned rows bit for
+  bit.  The dispatch outputs (row
   counts per rank, local expert ids, rows and scales in routing order) are
   compared bit for bit with the definition; each rank's output with the
   oracle within the layer's tolerance and with moe_forward over all experts.
@@ -103,13 +106,20 @@ def run_emulated(moe, n_ranks, tokens, w_weights, drop=True):
             rk["layer"].y_back[a:b] = ys[d][start:start + b - a]
         outs.append(rk["layer"].combine(rk["tw"]))
     torch.cuda.synchronize()
-    return g, ranks, outs
+    return g, ranks, outs, C
 
 
 @pytest.mark.parametrize("n_ranks,tokens", [(2, (37, 20)), (4, (64, 0, 9, 33))], ids=["R2", "R4_idle_rank"])
 def test_emulated_ranks_match_oracle(moe, n_ranks, tokens):
     ww = W.custom("ep_weights", T=1, E=8, k=2, H=256, I=256, seed=80)
-    g, ranks, outs = run_emulated(moe, n_ranks, tokens, ww)
+    g, ranks, outs, C = run_emulated(moe, n_ranks, tokens, ww)
+    # the combine over peer memory: every rank reads its rows where the ranks'
+    # expert layers left them (here other buffers of the same GPU)
+    peer_y = torch.tensor([rk["layer"].y_loc.data_ptr() for rk in ranks], dtype=torch.int64, device=DEVICE)
+    for r, (rk, out) in enumerate(zip(ranks, outs)):
+        base = torch.tensor([int(C[:r, d].sum()) for d in range(n_ranks)], dtype=torch.int64, device=DEVICE)
+        fused = moe.ep_combine_peers(peer_y, base, rk["idx"], rk["tw"], ww.E, ww.H, rk["layer"].ws)
+        assert torch.equal(fused.view(torch.int16), out.view(torch.int16)), f"rank {r}"
     for r, (rk, out) in enumerate(zip(ranks, outs)):
         T = rk["x"].shape[0]
         assert out.shape == (T, ww.H)
