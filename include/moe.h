@@ -470,6 +470,25 @@ moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const v
  *   in send order; inv is the inverse permutation the dispatch with the same
  *   T, E, k, H left in the workspace.  T = 0 enqueues nothing.
  *
+ * moe_ep_route -- step 1 without the copies, for moe_ep_dispatch_peers: the
+ *   routing into the workspace and send_counts (i64 [ranks], device); the
+ *   same arguments and rules as moe_ep_dispatch.
+ *
+ * moe_ep_dispatch_peers -- steps 1 and 2 for rows: after moe_ep_route with the
+ *   same T, E, k, H, ranks and workspace, and once every rank's counts are
+ *   known, writes each routed row (x_fp8 row, its UE8M0 scales, its local
+ *   expert id) straight into the receive buffers of the rank that holds its
+ *   expert, mapped into this rank's address space (CUDA IPC or symmetric
+ *   memory over NVLink).  peer_x / peer_sf / peer_eid: device arrays [ranks]
+ *   of device pointers to rank d's u8 [rows, H] (16-byte aligned), u8
+ *   [rows, H/32] (4-byte aligned) and i64 [rows] receive buffers (an entry
+ *   may be NULL only for a rank this rank sends nothing to); recv_base: i64
+ *   [ranks] device, the row at which this rank's block starts in rank d's
+ *   buffers (the sum of what ranks 0..r-1 send to d).  The rows land as the
+ *   all-to-all of moe_ep_dispatch's send buffers would place them (source
+ *   rank major, then send order).  The caller orders rank d's step 3 after
+ *   every rank's call (e.g. a stream-ordered barrier).
+ *
  * moe_ep_combine_peers -- steps 4 and 5 in one kernel, for ranks whose
  *   expert-layer outputs are mapped into this rank's address space (CUDA IPC
  *   or symmetric memory over NVLink): each returned row is read where rank d
@@ -493,6 +512,12 @@ moe_status_t moe_ep_dispatch(const void *x_fp8, const void *x_sf, const int64_t 
                              int64_t *send_eid, int64_t *send_counts, moe_stream_t stream);
 moe_status_t moe_ep_combine(const void *y_bf16, const float *topk_w, int T, int E, int k, int H,
                             const void *workspace, size_t ws_bytes, void *out_bf16, moe_stream_t stream);
+moe_status_t moe_ep_route(const int64_t *topk_idx, int T, int E, int k, int H, int ranks, void *workspace,
+                          size_t ws_bytes, int64_t *send_counts, moe_stream_t stream);
+moe_status_t moe_ep_dispatch_peers(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, int T, int E, int k,
+                                   int H, int ranks, const void *workspace, size_t ws_bytes,
+                                   void *const *peer_x, void *const *peer_sf, int64_t *const *peer_eid,
+                                   const int64_t *recv_base, moe_stream_t stream);
 moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv_base, const int64_t *topk_idx,
                                   const float *topk_w, int T, int E, int k, int H, int ranks, const void *workspace,
                                   size_t ws_bytes, void *out_bf16, moe_stream_t stream);

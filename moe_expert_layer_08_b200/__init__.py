@@ -22,7 +22,7 @@ __all__ = [
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
     "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
-    "ep_workspace_bytes", "ep_dispatch", "ep_combine", "ep_combine_peers",
+    "ep_workspace_bytes", "ep_dispatch", "ep_combine", "ep_combine_peers", "ep_route", "ep_dispatch_peers",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
@@ -112,6 +112,8 @@ def _declare(lib):
         "moe_ep_dispatch": (I32, [P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P, P, P]),
         "moe_ep_combine": (I32, [P, P, I32, I32, I32, I32, P, SZ, P, P]),
         "moe_ep_combine_peers": (I32, [P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P]),
+        "moe_ep_route": (I32, [P, I32, I32, I32, I32, I32, P, SZ, P, P]),
+        "moe_ep_dispatch_peers": (I32, [P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -593,3 +595,41 @@ def ep_combine_peers(peer_y, recv_base, topk_idx, topk_w, E: int, H: int, worksp
                                        ranks, _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)),
            "moe_ep_combine_peers")
     return out
+
+
+def ep_route(topk_idx, E: int, H: int, ranks: int, workspace, send_counts=None, stream=None):
+    """The dispatch's routing and per-rank row counts without copying rows
+    (for ep_dispatch_peers); returns send_counts (i64 [ranks], device)."""
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(workspace, torch.uint8, "workspace")
+    T, k = topk_idx.shape
+    if send_counts is None:
+        send_counts = torch.empty(ranks, dtype=torch.int64, device=workspace.device)
+    _need(send_counts, torch.int64, "send_counts", 1)
+    if send_counts.numel() != ranks:
+        raise ValueError("send_counts must hold one count per rank")
+    _check(load().moe_ep_route(_ptr(topk_idx), T, E, k, H, ranks, _ptr(workspace), workspace.numel(),
+                               _ptr(send_counts), _stream(stream)), "moe_ep_route")
+    return send_counts
+
+
+def ep_dispatch_peers(x_fp8, x_sf, topk_idx, E: int, workspace, peer_x, peer_sf, peer_eid, recv_base, stream=None):
+    """Writes this rank's routed rows into the ranks' receive buffers (after
+    ep_route on the same workspace): ``peer_x`` / ``peer_sf`` / ``peer_eid``
+    i64 [ranks] device tensors of the buffers' addresses, ``recv_base`` i64
+    [ranks] device tensor of this rank's first row in each of them."""
+    _need(x_fp8, torch.uint8, "x_fp8", 2)
+    _need(x_sf, torch.uint8, "x_sf", 2)
+    _need(topk_idx, torch.int64, "topk_idx", 2)
+    _need(workspace, torch.uint8, "workspace")
+    for t, n in ((peer_x, "peer_x"), (peer_sf, "peer_sf"), (peer_eid, "peer_eid"), (recv_base, "recv_base")):
+        _need(t, torch.int64, n, 1)
+    T, H = x_fp8.shape
+    k = topk_idx.shape[1]
+    ranks = peer_x.numel()
+    if x_sf.shape != (T, H // 32) or topk_idx.shape[0] != T or not (
+            peer_sf.numel() == peer_eid.numel() == recv_base.numel() == ranks):
+        raise ValueError("inconsistent shapes")
+    _check(load().moe_ep_dispatch_peers(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), T, E, k, H, ranks, _ptr(workspace),
+                                        workspace.numel(), _ptr(peer_x), _ptr(peer_sf), _ptr(peer_eid),
+                                        _ptr(recv_base), _stream(stream)), "moe_ep_dispatch_peers")

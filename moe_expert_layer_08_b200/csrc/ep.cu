@@ -68,6 +68,55 @@ __global__ void __launch_bounds__(kPackThreads) ep_pack_kernel(const int *__rest
     }
 }
 
+// The dispatch over peer memory: one warp per routed row (permutation order)
+// writes the row, its scale words and its local expert id straight into the
+// receive buffers of the rank d = e / e_loc that holds its expert, at row
+// recv_base[d] + (pos - offset[d * e_loc]).  Block 0 also writes the per-rank
+// counts (as ep_pack_kernel does), which the caller has already exchanged
+// when it computes recv_base; a NULL peer entry skips that rank's rows.
+__global__ void __launch_bounds__(kPackThreads) ep_push_kernel(const int *__restrict__ perm,
+                                                               const int *__restrict__ offset,
+                                                               const int64_t *__restrict__ topk_idx, int E, int k,
+                                                               int e_loc, int row_vec, int sf_words,
+                                                               const uint4 *__restrict__ x,
+                                                               const uint32_t *__restrict__ x_sf,
+                                                               uint4 *const *__restrict__ peer_x,
+                                                               uint32_t *const *__restrict__ peer_sf,
+                                                               int64_t *const *__restrict__ peer_eid,
+                                                               const int64_t *__restrict__ recv_base) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int kWarps = kPackThreads / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t nrows = __ldcg(offset + E);
+    const int64_t nwarps = int64_t(gridDim.x) * kWarps;
+    for (int64_t pos = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); pos < nrows; pos += nwarps) {
+        const int s = __ldcg(perm + pos);
+        const int64_t t = s / k;
+        const int64_t e = __ldg(topk_idx + s);  // routed: in [0, E)
+        const int d = int(e / e_loc);
+        uint4 *dx = peer_x[d];
+        uint32_t *dsf = peer_sf[d];
+        int64_t *deid = peer_eid[d];
+        if (!dx || !dsf || !deid) continue;
+        const int64_t row = __ldcg(recv_base + d) + (pos - __ldcg(offset + d * e_loc));
+        const uint4 *src = x + t * row_vec;
+        for (int v = lane; v < row_vec; v += 32) dx[row * row_vec + v] = __ldg(src + v);
+        for (int w = lane; w < sf_words; w += 32) dsf[row * sf_words + w] = __ldg(x_sf + t * sf_words + w);
+        if (lane == 0) deid[row] = e % e_loc;
+    }
+}
+
+// Per-rank row counts of a finished routing: counts[r] = rows for experts
+// [r*e_loc, (r+1)*e_loc).
+__global__ void ep_counts_kernel(const int *__restrict__ offset, int e_loc, int ranks,
+                                 int64_t *__restrict__ counts) {
+    pdl_wait();
+    pdl_trigger();
+    for (int r = threadIdx.x; r < ranks; r += blockDim.x)
+        counts[r] = int64_t(__ldcg(offset + (r + 1) * e_loc)) - __ldcg(offset + r * e_loc);
+}
+
 // The combine over peer memory: out[t] = bf16_rne(sum_{j ascending} w[t, j] *
 // Y_j) with Y_j read where the expert layer of the row's rank left it: rank
 // d = e / e_loc, row recv_base[d] + (pos - offset[d * e_loc]) of peer_y[d]
@@ -217,6 +266,61 @@ moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv
                                      reinterpret_cast<const int *>(ws + L.off_inv),
                                      reinterpret_cast<const int *>(ws + L.off_offset), topk_idx, topk_w, k, H,
                                      E / ranks, col_blocks, T, static_cast<__nv_bfloat16 *>(out_bf16));
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_ep_route(const int64_t *topk_idx, int T, int E, int k, int H, int ranks, void *workspace,
+                          size_t ws_bytes, int64_t *send_counts, moe_stream_t stream) {
+    moe_status_t s = check_ep_args(T, E, k, H);
+    if (s != MOE_OK) return s;
+    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
+    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!workspace || !send_counts || !aligned(workspace, 256) || !aligned(send_counts, 8) ||
+        (T > 0 && (!topk_idx || !aligned(topk_idx, 8))))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ep_layout(T, E, k, H);
+    if (T > 0 && ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0)
+        return cudaMemsetAsync(send_counts, 0, sizeof(int64_t) * size_t(ranks), st) == cudaSuccess ? MOE_OK
+                                                                                                     : MOE_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    cudaError_t e = launch_routing(topk_idx, k, E, ws, L, nullptr, st);
+    if (e == cudaSuccess)
+        e = launch_pdl(ep_counts_kernel, dim3(1), dim3(256), 0, st, reinterpret_cast<const int *>(ws + L.off_offset),
+                       E / ranks, ranks, send_counts);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_ep_dispatch_peers(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, int T, int E, int k,
+                                   int H, int ranks, const void *workspace, size_t ws_bytes,
+                                   void *const *peer_x, void *const *peer_sf, int64_t *const *peer_eid,
+                                   const int64_t *recv_base, moe_stream_t stream) {
+    moe_status_t s = check_ep_args(T, E, k, H);
+    if (s != MOE_OK) return s;
+    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
+    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MOE_OK;
+    if (!x_fp8 || !x_sf || !topk_idx || !workspace || !peer_x || !peer_sf || !peer_eid || !recv_base ||
+        !aligned(x_fp8, 16) || !aligned(x_sf, 4) || !aligned(topk_idx, 8) || !aligned(workspace, 256) ||
+        !aligned(peer_x, 8) || !aligned(peer_sf, 8) || !aligned(peer_eid, 8) || !aligned(recv_base, 8))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ep_layout(T, E, k, H);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    s = use_device_of(workspace);
+    if (s != MOE_OK) return s;
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    const int64_t want = (L.R + kPackThreads / 32 - 1) / (kPackThreads / 32);
+    const int64_t cap = int64_t(num_sms()) * 8;
+    const int grid = int(want < cap ? want : cap);
+    const cudaError_t e = launch_pdl(
+        ep_push_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kPackThreads), 0,
+        reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const int *>(ws + L.off_perm),
+        reinterpret_cast<const int *>(ws + L.off_offset), topk_idx, E, k, E / ranks, H / 16, H / 128,
+        static_cast<const uint4 *>(x_fp8), static_cast<const uint32_t *>(x_sf),
+        reinterpret_cast<uint4 *const *>(peer_x), reinterpret_cast<uint32_t *const *>(peer_sf), peer_eid, recv_base);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -273,3 +273,22 @@ def test_expert_parallel_entry_points_validate_on_the_host(moelib):
     assert peers(base=ctypes.c_void_p((1 << 20) + 4)) == 1                  # recv_base not 8-byte aligned
     assert peers(out=ctypes.c_void_p((1 << 20) + 8)) == 1                   # out not 16-byte aligned
     assert peers(ws_bytes=16) == 3
+
+    def route(**kw):
+        return lib.moe_ep_route(kw.get("idx", p), kw.get("T", 4), 8, 2, 256, kw.get("ranks", 2), kw.get("ws", p),
+                                kw.get("ws_bytes", 1 << 30), kw.get("counts", p), None)
+
+    assert route(ranks=3) == 2
+    assert route(idx=None) == 1
+    assert route(counts=None) == 1
+    assert route(ws_bytes=16) == 3
+
+    def push(**kw):
+        return lib.moe_ep_dispatch_peers(p, p, p, kw.get("T", 4), 8, 2, 256, kw.get("ranks", 2), p,
+                                         kw.get("ws_bytes", 1 << 30), kw.get("px", p), p, p, p, None)
+
+    assert push(T=0) == 0
+    assert push(ranks=3) == 2
+    assert push(px=None) == 1
+    assert push(px=ctypes.c_void_p((1 << 20) + 4)) == 1                     # pointer table not 8-byte aligned
+    assert push(ws_bytes=16) == 3

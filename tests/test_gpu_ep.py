@@ -11,7 +11,9 @@ layer with k = 1 over each rank's experts, moe_ep_combine).
   layer, the copies back, every rank's combine; and the combine over peer
   memory (moe_ep_combine_peers), reading each row from the buffer of the
   rank that computed it, equal to the combine of the returned rows bit for
-  bit.  The dispatch outputs (row
+  bit; and the dispatch over peer memory (moe_ep_route, then
+  moe_ep_dispatch_peers writing into every rank's receive buffers), equal to
+  what the exchange of the send buffers delivered.  The dispatch outputs (row
   counts per rank, local expert ids, rows and scales in routing order) are
   compared bit for bit with the definition; each rank's output with the
   oracle within the layer's tolerance and with moe_forward over all experts.
@@ -120,6 +122,27 @@ def test_emulated_ranks_match_oracle(moe, n_ranks, tokens):
         base = torch.tensor([int(C[:r, d].sum()) for d in range(n_ranks)], dtype=torch.int64, device=DEVICE)
         fused = moe.ep_combine_peers(peer_y, base, rk["idx"], rk["tw"], ww.E, ww.H, rk["layer"].ws)
         assert torch.equal(fused.view(torch.int16), out.view(torch.int16)), f"rank {r}"
+    # the dispatch over peer memory: routing and counts, then every rank
+    # writes its rows into the ranks' receive buffers (fresh ones here), which
+    # must then hold what the exchange of the send buffers delivered
+    n_recv = C.sum(axis=0)
+    u8 = dict(dtype=torch.uint8, device=DEVICE)
+    bufs = [dict(x=torch.zeros((max(int(n), 1), ww.H), **u8), sf=torch.zeros((max(int(n), 1), ww.H // 32), **u8),
+                 eid=torch.full((max(int(n), 1),), -1, dtype=torch.int64, device=DEVICE)) for n in n_recv]
+    table = {key: torch.tensor([b[key].data_ptr() for b in bufs], dtype=torch.int64, device=DEVICE)
+             for key in ("x", "sf", "eid")}
+    for r, rk in enumerate(ranks):
+        ws = torch.empty(moe.ep_workspace_bytes(rk["layer"].T_max, ww.E, ww.k, ww.H), **u8)
+        counts = moe.ep_route(rk["idx"], ww.E, ww.H, n_ranks, ws)
+        assert np.array_equal(counts.cpu().numpy(), C[r])
+        base = torch.tensor([int(C[:r, d].sum()) for d in range(n_ranks)], dtype=torch.int64, device=DEVICE)
+        moe.ep_dispatch_peers(rk["xq"], rk["xs"], rk["idx"], ww.E, ws, table["x"], table["sf"], table["eid"], base)
+    torch.cuda.synchronize()
+    for d, rk in enumerate(ranks):
+        n, L = int(n_recv[d]), rk["layer"]
+        assert torch.equal(bufs[d]["x"][:n], L.recv_x[:n]), f"rank {d} rows"
+        assert torch.equal(bufs[d]["sf"][:n], L.recv_sf[:n]), f"rank {d} scales"
+        assert torch.equal(bufs[d]["eid"][:n], L.recv_eid[:n, 0]), f"rank {d} expert ids"
     for r, (rk, out) in enumerate(zip(ranks, outs)):
         T = rk["x"].shape[0]
         assert out.shape == (T, ww.H)
