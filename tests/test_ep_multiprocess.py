@@ -1,5 +1,5 @@
 """The exchange of the expert-parallel layer (ExpertParallelLayer.forward) on
-CPU with gloo at world size 2: the count all-gather, the row all-to-alls in
+CPU with gloo at world sizes 2 and 4: the count all-gather, the row all-to-alls in
 both directions and their split sizes, every rank taking the same collective
 steps whatever its token count, and an overflow of the receive buffers
 stopping both ranks.  The three CUDA phases (dispatch, expert layer, combine)
@@ -123,22 +123,23 @@ def _worker(rank, world, port, q, tokens, recv_max):
 
 
 def _run(tokens, recv_max=None):
+    world = len(tokens)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, tokens, recv_max)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, tokens, recv_max)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(timeout=180)
         assert p.exitcode == 0
-    return {r: (kind, val) for r, kind, val in (q.get(timeout=5) for _ in range(2))}
+    return {r: (kind, val) for r, kind, val in (q.get(timeout=5) for _ in range(world))}
 
 
-@pytest.mark.parametrize("tokens", [(12, 7), (9, 0)], ids=["uneven", "one_rank_idle"])
+@pytest.mark.parametrize("tokens", [(12, 7), (9, 0), (5, 0, 12, 3)], ids=["uneven", "one_rank_idle", "four_ranks"])
 def test_exchange_matches_single_rank_definition(tokens):
     res = _run(tokens)
-    assert res == {0: ("ok", True), 1: ("ok", True)}, res
+    assert res == {r: ("ok", True) for r in range(len(tokens))}, res
 
 
 def test_receive_overflow_stops_every_rank():
