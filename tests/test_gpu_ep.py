@@ -111,20 +111,18 @@ def run_emulated(moe, n_ranks, tokens, w_weights, drop=True):
     return g, ranks, outs, C
 
 
-@pytest.mark.parametrize("n_ranks,tokens", [(2, (37, 20)), (4, (64, 0, 9, 33))], ids=["R2", "R4_idle_rank"])
-def test_emulated_ranks_match_oracle(moe, n_ranks, tokens):
-    ww = W.custom("ep_weights", T=1, E=8, k=2, H=256, I=256, seed=80)
-    g, ranks, outs, C = run_emulated(moe, n_ranks, tokens, ww)
-    # the combine over peer memory: every rank reads its rows where the ranks'
-    # expert layers left them (here other buffers of the same GPU)
+def check_peer_paths(moe, ranks, outs, C, ww):
+    """The combine over peer memory (each rank reads its rows where the ranks'
+    expert layers left them, here other buffers of the same GPU) equals the
+    combine of the returned rows; the dispatch over peer memory (routing and
+    counts, then every rank writing its rows into fresh receive buffers)
+    delivers what the exchange of the send buffers delivered."""
+    n_ranks = len(ranks)
     peer_y = torch.tensor([rk["layer"].y_loc.data_ptr() for rk in ranks], dtype=torch.int64, device=DEVICE)
     for r, (rk, out) in enumerate(zip(ranks, outs)):
         base = torch.tensor([int(C[:r, d].sum()) for d in range(n_ranks)], dtype=torch.int64, device=DEVICE)
         fused = moe.ep_combine_peers(peer_y, base, rk["idx"], rk["tw"], ww.E, ww.H, rk["layer"].ws)
         assert torch.equal(fused.view(torch.int16), out.view(torch.int16)), f"rank {r}"
-    # the dispatch over peer memory: routing and counts, then every rank
-    # writes its rows into the ranks' receive buffers (fresh ones here), which
-    # must then hold what the exchange of the send buffers delivered
     n_recv = C.sum(axis=0)
     u8 = dict(dtype=torch.uint8, device=DEVICE)
     bufs = [dict(x=torch.zeros((max(int(n), 1), ww.H), **u8), sf=torch.zeros((max(int(n), 1), ww.H // 32), **u8),
@@ -143,6 +141,13 @@ def test_emulated_ranks_match_oracle(moe, n_ranks, tokens):
         assert torch.equal(bufs[d]["x"][:n], L.recv_x[:n]), f"rank {d} rows"
         assert torch.equal(bufs[d]["sf"][:n], L.recv_sf[:n]), f"rank {d} scales"
         assert torch.equal(bufs[d]["eid"][:n], L.recv_eid[:n, 0]), f"rank {d} expert ids"
+
+
+@pytest.mark.parametrize("n_ranks,tokens", [(2, (37, 20)), (4, (64, 0, 9, 33))], ids=["R2", "R4_idle_rank"])
+def test_emulated_ranks_match_oracle(moe, n_ranks, tokens):
+    ww = W.custom("ep_weights", T=1, E=8, k=2, H=256, I=256, seed=80)
+    g, ranks, outs, C = run_emulated(moe, n_ranks, tokens, ww)
+    check_peer_paths(moe, ranks, outs, C, ww)
     for r, (rk, out) in enumerate(zip(ranks, outs)):
         T = rk["x"].shape[0]
         assert out.shape == (T, ww.H)
@@ -154,3 +159,21 @@ def test_emulated_ranks_match_oracle(moe, n_ranks, tokens):
         compare_rows(out, ref["out_bf16"], f"rank {r}")
         full = moe.forward(rk["xq"], rk["xs"], rk["idx"], rk["tw"], g["l1_t"], g["l2_t"], ww.E, ww.H, ww.I)
         compare_rows(out, oracle.f32_to_bf16(full.float().cpu().numpy()), f"rank {r} vs one GPU")
+
+
+def test_emulated_ranks_decode_sizes(moe):
+    """Eight ranks at the decode workload's sizes: 384 experts (48 per rank),
+    8 tokens per rank, top-6, H = 7168, I = 3072.  Every rank against
+    moe_forward over all experts, rank 0 against the oracle, and the
+    peer-memory paths."""
+    ww = W.custom("ep_decode", T=1, E=384, k=6, H=7168, I=3072, seed=90)
+    g, ranks, outs, C = run_emulated(moe, 8, (8,) * 8, ww, drop=False)
+    check_peer_paths(moe, ranks, outs, C, ww)
+    for r, (rk, out) in enumerate(zip(ranks, outs)):
+        full = moe.forward(rk["xq"], rk["xs"], rk["idx"], rk["tw"], g["l1_t"], g["l2_t"], ww.E, ww.H, ww.I)
+        compare_rows(out, oracle.f32_to_bf16(full.float().cpu().numpy()), f"rank {r} vs one GPU")
+    rk = ranks[0]
+    idx = rk["idx"].cpu().numpy()
+    xq, xs, ex = oracle_side(ww, rk["x"], rk["idx"], experts_of(idx, np.arange(8), ww.E), gen_device=DEVICE)
+    ref = oracle.forward(xq, xs, idx, rk["tw"].cpu().numpy(), ex, ww.E, ww.H, ww.I)
+    compare_rows(outs[0], ref["out_bf16"], "rank 0")
