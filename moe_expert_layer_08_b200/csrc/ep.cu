@@ -172,6 +172,23 @@ moe_status_t check_ep_args(int T, int E, int k, int H) {
     return MOE_OK;
 }
 
+// The sizes plus a rank count: 1 <= ranks <= E, E a multiple of ranks.
+moe_status_t check_ep_args(int T, int E, int k, int H, int ranks) {
+    const moe_status_t s = check_ep_args(T, E, k, H);
+    if (s != MOE_OK) return s;
+    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
+    return E % ranks == 0 ? MOE_OK : MOE_ERR_UNSUPPORTED_SHAPE;
+}
+
+// Blocks of the one-warp-per-row kernels for R routed rows: one warp per row
+// up to 8 blocks per SM, the warps striding over the rest.
+int row_grid(int64_t R) {
+    const int64_t want = (R + kPackThreads / 32 - 1) / (kPackThreads / 32);
+    const int64_t cap = int64_t(num_sms()) * 8;
+    const int64_t g = want < cap ? want : cap;
+    return int(g > 0 ? g : 1);
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -190,10 +207,8 @@ moe_status_t moe_ep_workspace_bytes(int T_max, int E, int k, int H, size_t *byte
 moe_status_t moe_ep_dispatch(const void *x_fp8, const void *x_sf, const int64_t *topk_idx, int T, int E, int k,
                              int H, int ranks, void *workspace, size_t ws_bytes, void *send_x, void *send_sf,
                              int64_t *send_eid, int64_t *send_counts, moe_stream_t stream) {
-    moe_status_t s = check_ep_args(T, E, k, H);
+    moe_status_t s = check_ep_args(T, E, k, H, ranks);
     if (s != MOE_OK) return s;
-    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
-    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!workspace || !send_counts || !aligned(workspace, 256) || !aligned(send_counts, 8))
         return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x_fp8 || !x_sf || !topk_idx || !send_x || !send_sf || !send_eid || !aligned(x_fp8, 16) ||
@@ -211,10 +226,8 @@ moe_status_t moe_ep_dispatch(const void *x_fp8, const void *x_sf, const int64_t 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaError_t e = launch_routing(topk_idx, k, E, ws, L, nullptr, st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    const int64_t want = (L.R + kPackThreads / 32 - 1) / (kPackThreads / 32);
-    const int64_t cap = int64_t(num_sms()) * 8;
-    const int grid = int(want < cap ? want : cap);
-    e = launch_pdl(ep_pack_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kPackThreads), 0, st,
+    const int grid = row_grid(L.R);
+    e = launch_pdl(ep_pack_kernel, dim3(unsigned(grid)), dim3(kPackThreads), 0, st,
                    reinterpret_cast<const int *>(ws + L.off_perm), reinterpret_cast<const int *>(ws + L.off_offset),
                    topk_idx, E, k, E / ranks, ranks, H / 16, H / 128, static_cast<const uint4 *>(x_fp8),
                    static_cast<const uint32_t *>(x_sf), static_cast<uint4 *>(send_x), static_cast<uint32_t *>(send_sf),
@@ -243,10 +256,8 @@ moe_status_t moe_ep_combine(const void *y_bf16, const float *topk_w, int T, int 
 moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv_base, const int64_t *topk_idx,
                                   const float *topk_w, int T, int E, int k, int H, int ranks, const void *workspace,
                                   size_t ws_bytes, void *out_bf16, moe_stream_t stream) {
-    moe_status_t s = check_ep_args(T, E, k, H);
+    moe_status_t s = check_ep_args(T, E, k, H, ranks);
     if (s != MOE_OK) return s;
-    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
-    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (T == 0) return MOE_OK;
     if (!peer_y || !recv_base || !topk_idx || !topk_w || !workspace || !out_bf16 || !aligned(peer_y, 8) ||
         !aligned(recv_base, 8) || !aligned(topk_idx, 8) || !aligned(topk_w, 4) || !aligned(workspace, 256) ||
@@ -271,10 +282,8 @@ moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv
 
 moe_status_t moe_ep_route(const int64_t *topk_idx, int T, int E, int k, int H, int ranks, void *workspace,
                           size_t ws_bytes, int64_t *send_counts, moe_stream_t stream) {
-    moe_status_t s = check_ep_args(T, E, k, H);
+    moe_status_t s = check_ep_args(T, E, k, H, ranks);
     if (s != MOE_OK) return s;
-    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
-    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!workspace || !send_counts || !aligned(workspace, 256) || !aligned(send_counts, 8) ||
         (T > 0 && (!topk_idx || !aligned(topk_idx, 8))))
         return MOE_ERR_INVALID_ARG;
@@ -298,10 +307,8 @@ moe_status_t moe_ep_dispatch_peers(const void *x_fp8, const void *x_sf, const in
                                    int H, int ranks, const void *workspace, size_t ws_bytes,
                                    void *const *peer_x, void *const *peer_sf, int64_t *const *peer_eid,
                                    const int64_t *recv_base, moe_stream_t stream) {
-    moe_status_t s = check_ep_args(T, E, k, H);
+    moe_status_t s = check_ep_args(T, E, k, H, ranks);
     if (s != MOE_OK) return s;
-    if (ranks <= 0 || ranks > E) return MOE_ERR_INVALID_ARG;
-    if (E % ranks != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (T == 0) return MOE_OK;
     if (!x_fp8 || !x_sf || !topk_idx || !workspace || !peer_x || !peer_sf || !peer_eid || !recv_base ||
         !aligned(x_fp8, 16) || !aligned(x_sf, 4) || !aligned(topk_idx, 8) || !aligned(workspace, 256) ||
@@ -312,11 +319,9 @@ moe_status_t moe_ep_dispatch_peers(const void *x_fp8, const void *x_sf, const in
     s = use_device_of(workspace);
     if (s != MOE_OK) return s;
     const uint8_t *ws = static_cast<const uint8_t *>(workspace);
-    const int64_t want = (L.R + kPackThreads / 32 - 1) / (kPackThreads / 32);
-    const int64_t cap = int64_t(num_sms()) * 8;
-    const int grid = int(want < cap ? want : cap);
+    const int grid = row_grid(L.R);
     const cudaError_t e = launch_pdl(
-        ep_push_kernel, dim3(unsigned(grid > 0 ? grid : 1)), dim3(kPackThreads), 0,
+        ep_push_kernel, dim3(unsigned(grid)), dim3(kPackThreads), 0,
         reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const int *>(ws + L.off_perm),
         reinterpret_cast<const int *>(ws + L.off_offset), topk_idx, E, k, E / ranks, H / 16, H / 128,
         static_cast<const uint4 *>(x_fp8), static_cast<const uint32_t *>(x_sf),
