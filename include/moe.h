@@ -364,15 +364,15 @@ moe_status_t moe_check_device_error(const void *workspace, moe_stream_t stream);
  *  - A (T, E, k, H, I) whose moe_workspace_bytes exceeds
  *    MOE_STATIC_WORKSPACE_BYTES is rejected with MOE_ERR_WORKSPACE_TOO_SMALL
  *    before any device work (decode-sized batches fit: T = 128 tokens at
- *    E = 384, top-6, H = 7168, I = 3072 needs 34 MiB).
+ *    E = 384, top-6, H = 7168, I = 3072 needs 57.9 MiB).
  *  - All calls on a device share the one array, which keeps the last call's
  *    contents; nothing in it needs to start at zero.  Calls that overlap on
  *    the GPU (different streams, or threads without ordering between their
  *    streams) race on it and give undefined results: issue them in order on
  *    one stream.
- *  - Out-of-range expert ids are dropped as in moe_forward, but the device
- *    error word lives in the shared array, so moe_check_device_error cannot
- *    report it for this entry point.
+ *  - Out-of-range expert ids are dropped as in moe_forward.  The device
+ *    error word of the last call lives in the shared array; read it with
+ *    moe_check_device_error_static on that device.
  */
 #define MOE_STATIC_WORKSPACE_BYTES (64u * 1024u * 1024u)
 
@@ -382,6 +382,18 @@ moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf,
                                 int T, int E, int k, int H, int I,
                                 int32_t *expert_stats, void *const *stage_events,
                                 moe_stream_t stream);
+
+/*
+ * moe_check_device_error_static -- moe_check_device_error for the fixed array
+ * of moe_forward_static on CUDA device `device`: synchronises `stream`, then
+ * returns the status the last moe_forward_static on that device left in the
+ * array's error word (MOE_OK, MOE_ERR_BAD_ROUTING or MOE_ERR_DEVICE_TIMEOUT).
+ * The first kernel of every moe_forward_static rewrites the word, so the
+ * result belongs to the last call enqueued before `stream` was synchronised
+ * (call it on the stream the forward ran on).  MOE_ERR_INVALID_ARG for a
+ * device index outside [0, 64); allocates nothing.
+ */
+moe_status_t moe_check_device_error_static(int device, moe_stream_t stream);
 
 /*
  * moe_probe_wait_timeout -- diagnostic (no counterpart on the pages): runs one

@@ -18,7 +18,7 @@ __all__ = [
     "MoEError", "load", "status_string", "abi_version", "quantize_fp8", "quantize_fp4",
     "transformed_weight_bytes", "transform_weights", "workspace_bytes", "forward",
     "read_routing", "check_device_error", "MoELayer", "NUM_STAGE_EVENTS", "STATUS",
-    "forward_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
+    "forward_static", "check_device_error_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
     "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
@@ -94,6 +94,7 @@ def _declare(lib):
         "moe_read_routing": (I32, [P, I32, I32, I32, I32, I32, P, P, P, P, P]),
         "moe_check_device_error": (I32, [P, P]),
         "moe_forward_static": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, P, P]),
+        "moe_check_device_error_static": (I32, [I32, P]),
         "moe_forward_act": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P,
                                   c.POINTER(Activation), P]),
         "moe_transformed_scale_bytes": (I32, [I32, I32, I32, c.POINTER(SZ), c.POINTER(SZ)]),
@@ -322,6 +323,8 @@ def forward(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: int,
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x_fp8.device)
     else:
         _need(out, torch.bfloat16, "out", 2)
+        if out.shape != (T, H) or out.device != x_fp8.device:
+            raise ValueError("out must be bf16 [T, H] on the device of x_fp8")
     if workspace is None:
         workspace = torch.empty(workspace_bytes(T, E, k, H, I), dtype=torch.uint8, device=x_fp8.device)
     else:
@@ -373,6 +376,8 @@ def forward_nvfp4(x_fp4, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I: 
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x_fp4.device)
     else:
         _need(out, torch.bfloat16, "out", 2)
+        if out.shape != (T, H) or out.device != x_fp4.device:
+            raise ValueError("out must be bf16 [T, H] on the device of x_fp4")
     if workspace is None:
         workspace = torch.empty(workspace_bytes(T, E, k, H, I), dtype=torch.uint8, device=x_fp4.device)
     else:
@@ -455,6 +460,8 @@ def forward_static(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=x_fp8.device)
     else:
         _need(out, torch.bfloat16, "out", 2)
+        if out.shape != (T, H) or out.device != x_fp8.device:
+            raise ValueError("out must be bf16 [T, H] on the device of x_fp8")
     if expert_stats is not None:
         _need(expert_stats, torch.int32, "expert_stats", 1)
     st = load().moe_forward_static(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(l1_t),
@@ -462,6 +469,19 @@ def forward_static(x_fp8, x_sf, topk_idx, topk_w, l1_t, l2_t, E: int, H: int, I:
                                    _stream(stream))
     _check(st, "moe_forward_static")
     return out
+
+
+def check_device_error_static(device=None, stream=None) -> int:
+    """Synchronises the stream and returns the status the last forward_static
+    on ``device`` (a CUDA device or index; default: the current one) left in the
+    library's fixed array (0, MOE_ERR_BAD_ROUTING or MOE_ERR_DEVICE_TIMEOUT)."""
+    if isinstance(device, int):
+        index = device
+    else:
+        index = None if device is None else torch.device(device).index
+        if index is None:
+            index = torch.cuda.current_device()
+    return load().moe_check_device_error_static(int(index), _stream(stream))
 
 
 def read_routing(workspace, T: int, E: int, k: int, H: int, I: int, stream=None):
@@ -561,6 +581,9 @@ def ep_combine(y, topk_w, E: int, workspace, out=None, stream=None):
     _need(workspace, torch.uint8, "workspace")
     T, k = topk_w.shape
     H = y.shape[1]
+    if y.shape[0] < T * k:
+        # the combine reads row inv[t*k + j] of y, and inv reaches T*k - 1
+        raise ValueError("y must hold at least T*k rows (the dispatch's routed rows)")
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=topk_w.device)
     _need(out, torch.bfloat16, "out", 2)
@@ -576,7 +599,9 @@ def ep_combine_peers(peer_y, recv_base, topk_idx, topk_w, E: int, H: int, worksp
     ``peer_y`` i64 [ranks] device tensor of the ranks' output addresses (bf16
     [rows, H] each, mapped into this process), ``recv_base`` i64 [ranks]
     device tensor (where this rank's rows start in each rank's received
-    rows); returns out (bf16 [T, H])."""
+    rows); returns out (bf16 [T, H]).  The peers' buffers are raw addresses
+    that this function cannot size-check: rank r's must hold at least
+    recv_base[r] + (rows this rank sent to r) rows."""
     _need(peer_y, torch.int64, "peer_y", 1)
     _need(recv_base, torch.int64, "recv_base", 1)
     _need(topk_idx, torch.int64, "topk_idx", 2)

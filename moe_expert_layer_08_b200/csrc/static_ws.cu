@@ -83,3 +83,15 @@ extern "C" moe_status_t moe_forward_static(const void *x_fp8, const void *x_sf, 
     return run_layer(x_fp8, x_sf, topk_idx, topk_w, w, out_bf16, T, E, k, H, I, ws, expert_stats, stage_events,
                      stream, swiglu, false);
 }
+
+extern "C" moe_status_t moe_check_device_error_static(int device, moe_stream_t stream) {
+    if (device < 0 || device >= kMaxDevices) return MOE_ERR_INVALID_ARG;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cur != device && cudaSetDevice(device) != cudaSuccess) return MOE_ERR_CUDA;
+    uint8_t *ws = nullptr;
+    const moe_status_t s = static_workspace_of_current_device(&ws);
+    if (s != MOE_OK) return s;
+    // The error word is the first word of the scratch's header, as in a caller workspace.
+    return moe_check_device_error(ws, stream);
+}

@@ -15,8 +15,10 @@ def pytest_configure(config):
 def pytest_collection_modifyitems(config, items):
     # The expert-parallel tests run the single-GPU layer inside every rank, so
     # they come after every test of the layer's own entry points (a layer
-    # failure is reported as such first).
-    rank = {"test_gpu_ep": 1}
+    # failure is reported as such first).  The entry point without a caller
+    # workspace comes last of all: a run that stops at its first failure has
+    # then run everything else.
+    rank = {"test_gpu_ep": 1, "test_zz_no_alloc": 2}
     items.sort(key=lambda it: rank.get(getattr(it.module, "__name__", ""), 0))
 
 

@@ -4,9 +4,13 @@ plug-ins without access to their host framework's allocator): its scratch is a
 fixed device array inside the library instead of a caller workspace.
 
 Checked through the C ABI against moe_forward (the entry point with a caller
-workspace) on the same inputs, within the layer's per-row tolerance, on two
-calls in a row (the array keeps the previous call's contents), and the
-rejection of a size beyond the array.  This file is collected last on purpose.
+workspace) on the same inputs on two calls in a row (the array keeps the
+previous call's contents): both run the same deterministic kernels, so the
+outputs must be equal bit for bit, which also implies the layer's per-row
+tolerance.  Also: the array's error word (moe_check_device_error_static)
+reports a dropped out-of-range expert id and is cleared by the next call, and
+a size beyond the array is rejected.  The conftest hook runs this file after
+every other test.
 """
 import numpy as np
 import pytest
@@ -46,8 +50,25 @@ def test_static_matches_workspace_entry_point_two_calls_in_a_row(moe, w):
     first = moe.forward_static(*args)
     second = moe.forward_static(*args)
     torch.cuda.synchronize()
+    assert moe.check_device_error_static() == 0
+    assert torch.equal(first, ref)
+    assert torch.equal(second, ref)
     within_tolerance(first, ref)
-    within_tolerance(second, ref)
+
+
+def test_static_error_word_reports_dropped_ids(moe):
+    w = W.WORKLOADS[0]
+    g = gpu_layer(w)
+    bad = g["idx"].clone()
+    bad[3, 1] = w.E + 5  # out of range: dropped from routing and reported
+    args = (g["xq"], g["xs"], bad, g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I)
+    ref = moe.forward(*args)
+    got = moe.forward_static(*args)
+    assert moe.check_device_error_static() == 5  # MOE_ERR_BAD_ROUTING
+    assert torch.equal(got, ref)
+    moe.forward_static(g["xq"], g["xs"], g["idx"], g["tw"], g["l1_t"], g["l2_t"], w.E, w.H, w.I)
+    assert moe.check_device_error_static() == 0
+    assert moe.load().moe_check_device_error_static(-1, None) == 1  # MOE_ERR_INVALID_ARG
 
 
 def test_static_rejects_sizes_beyond_its_array(moe):
