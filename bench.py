@@ -44,6 +44,9 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="b200", choices=["b200", "reference"])
     p.add_argument("--workload", type=int, default=1)
+    p.add_argument("--also", default=None,
+                   help="comma-separated workload ids measured after the headline one in the same run "
+                        "(default: 2,3,4 when the headline is the decode workload; '' for none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-tokens", type=int, default=8, help="tokens in the oracle's timed sample")
     p.add_argument("--experts", type=int, default=0,
@@ -357,7 +360,8 @@ def run_reference(args, w, rank, world):
         "metric": METRIC, "impl": "reference", "value": value, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")}},
+        "config": workload_config(w, args, world, len(W.touched_experts(torch.from_numpy(s["idx"]), w.E)),
+                                  expert_bytes(w, args.format)),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -477,7 +481,7 @@ def run_ep(args, w, rank, world, local_rank):
         stop.record(stream)
         barrier()
     ms = max_over_ranks(start.elapsed_time(stop) / args.steps, device)
-    st = moe.check_device_error(layer.ws)
+    st = layer.check()  # the dispatch's error word, then the expert layer's
     if st != 0:
         raise RuntimeError(f"device error: {moe.STATUS.get(st, st)}")
     # kernels of this library per step: routing (one block up to 1024 rows,
@@ -533,17 +537,22 @@ def run_shared_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
-def run_b200(args, w, rank, world, local_rank):
+def workload_config(w, args, world, touched=None, b12=None):
+    """The `config` object of a bench line (the same keys in both arms)."""
+    cfg = {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")},
+           "parallelism": f"replicas x{world}", "weight_layout": args.layout}
+    if touched is not None:
+        cfg["l2"] = ("inputs larger than L2 (touched expert weights per step >> 126 MB)"
+                     if touched * sum(b12) > 256e6 else "inputs fit in L2 (not flushed)")
+    return cfg
+
+
+def time_layer(args, w, device, world):
+    """Seeded inputs and weights of workload w resident in HBM, W warm-up
+    layer calls, then K calls back to back timed with CUDA events on the launch
+    stream (barrier + synchronize on both sides), then the same K calls again
+    with an event between kernels for the per-kernel times."""
     import moe_expert_layer_08_b200 as moe
-    from moe_expert_layer_08_b200 import build as mbuild
-    if rank == 0:
-        mbuild.build()
-    if world > 1:
-        torch.distributed.barrier()
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    if args.format == "nvfp4" and args.layout != "packets":
-        raise SystemExit("the NVFP4 variant takes packet weights")
     g = build_layer(w, device, args.layout, args.format)
     layer = moe.MoELayer(g["l1_t"], g["l2_t"], w.E, w.k, w.H, w.I, T_max=w.T, device=device, weights=g["rm"],
                          fmt=args.format)
@@ -586,8 +595,98 @@ def run_b200(args, w, rank, world, local_rank):
         stop.record(stream)
         barrier()
         staged_ms = start.elapsed_time(stop) / args.steps
+    st = moe.check_device_error(layer.workspace)
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {moe.STATUS.get(st, st)}")
     stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(moe.NUM_STAGE_EVENTS - 1)] for e in ev])
     ms = max_over_ranks(total_ms / args.steps, device)
+    return dict(g=g, layer=layer, out=out, stream=stream, ms=ms, staged_ms=staged_ms, stage_ms=stage_ms,
+                clocks=clocks.summary(), barrier=barrier)
+
+
+def layer_figures(args, w, r, world):
+    """Throughput, per-kernel times and rooflines of one timed workload."""
+    import moe_expert_layer_08_b200 as moe
+    g, ms, stage_ms = r["g"], r["ms"], r["stage_ms"]
+    # roofline of the dominant kernel (GEMM1 or GEMM2), timed by the stage events
+    touched = len(W.touched_experts(g["idx"].cpu(), w.E))
+    b1, b2 = expert_bytes(w, args.format)
+    g1_ms, g2_ms = float(stage_ms[:, 1].mean()), float(stage_ms[:, 2].mean())
+    pk = peaks()
+    if g1_ms >= g2_ms:
+        kname, kms, kbytes = "moe_gemm_kernel<gemm1>", g1_ms, touched * b1
+    else:
+        kname, kms, kbytes = "moe_gemm_kernel<gemm2>", g2_ms, touched * b2
+    achieved = kbytes / (kms * 1e-3) / 1e9
+    traffic = measured_traffic(w, touched, g1_ms >= g2_ms, args.format)
+    roofline = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "peak_source": pk["source"], "algorithmic_bytes": kbytes,
+                "traffic": traffic, "spec": {"peak": SPEC_HBM_GBPS, "frac": achieved / SPEC_HBM_GBPS}}
+    # tensor peaks: FP8 = 2 x measured bf16, FP4 (NVFP4) = 4 x (the nominal
+    # dense ratios); the block-scaled FP8 x FP4 MMA runs at the FP8 rate
+    ratio = 2.0 if args.format == "mx" else 4.0
+    spec_tc = SPEC_FP8_TFLOPS * ratio / 2.0
+    if w.T * w.k > 8 * w.E:
+        # large batches: each weight byte feeds ~T*k/E rows, and the tensor
+        # pipe binds as much as HBM.  The denominator is the sustained peak
+        # (the power-capped regime of a long run); the burst and spec
+        # fractions are given beside it, and "clocks" shows the regime the
+        # timed region actually ran in.
+        kflops = 2.0 * w.T * w.k * (2 * w.I if g1_ms >= g2_ms else w.H) * (w.H if g1_ms >= g2_ms else w.I)
+        peak_s, peak_b = ratio * pk["bf16_sustained"], ratio * pk["bf16"]
+        tflops = kflops / (kms * 1e-3) / 1e12
+        roofline = {"kernel": kname, "bound": "tensor", "achieved": tflops, "peak": peak_s, "unit": "TFLOP/s",
+                    "frac": tflops / peak_s,
+                    "peak_source": pk["source"] + f" sustained ({ratio:g} x bf16_tflops_sustained)",
+                    "frac_of_burst": tflops / peak_b,
+                    "burst_peak": peak_b,
+                    "spec": {"peak": spec_tc, "frac": tflops / spec_tc},
+                    "algorithmic_flops": kflops,
+                    "traffic": traffic, "hbm": {"achieved_GBps": achieved, "frac": achieved / pk["hbm"]}}
+        if cublas_fp8() and args.format == "mx":
+            roofline["cublas_fp8"] = {arm: {"sustained": c["sustained"], "frac": tflops / c["sustained"],
+                                            "burst": c["burst"], "frac_of_burst": tflops / c["burst"]}
+                                      for arm, c in cublas_fp8().items()}
+    x_bytes = w.T * w.H * 33 // 32 if args.format == "mx" else w.T * w.H * 9 // 16
+    layer_bytes = touched * (b1 + b2) + x_bytes + w.T * w.k * 12 + w.T * w.H * 2
+    tflops_layer = w.flops / (ms * 1e-3) / 1e12
+    layer_tc = {"sustained": tflops_layer / (ratio * pk["bf16_sustained"]),
+                "burst": tflops_layer / (ratio * pk["bf16"]),
+                "spec": tflops_layer / spec_tc}
+    if cublas_fp8() and args.format == "mx":
+        layer_tc["cublas_fp8_sustained"] = {arm: tflops_layer / c["sustained"] for arm, c in cublas_fp8().items()}
+    return {
+        "value": world * tflops_layer, "ms_per_step": ms, "touched": touched, "b12": (b1, b2),
+        "us_per_layer": ms * 1e3,
+        "effective_GBps": layer_bytes / (ms * 1e-3) / 1e9,
+        "hbm_frac_layer": layer_bytes / (ms * 1e-3) / 1e9 / pk["hbm"],
+        "touched_experts": touched,
+        "stage_us": {"route_gather": float(stage_ms[:, 0].mean() * 1e3), "gemm1": g1_ms * 1e3,
+                     "gemm2": g2_ms * 1e3, "combine": float(stage_ms[:, 3].mean() * 1e3)},
+        "stage_timing": {"how": "second pass of the same K steps with a CUDA event on the launch stream "
+                                "between kernels; the roofline's kernel duration comes from it",
+                         "us_per_layer": r["staged_ms"] * 1e3},
+        "roofline": roofline,
+        "layer_frac_of_tensor_peak": layer_tc,
+        "layer_frac_of_hbm_spec": layer_bytes / (ms * 1e-3) / 1e9 / SPEC_HBM_GBPS,
+        "gpu_launches": args.steps * moe.forward_kernel_launches(w.T, w.E, w.k, w.H, w.I),
+        "clocks": r["clocks"],
+    }
+
+
+def run_b200(args, w, rank, world, local_rank):
+    import moe_expert_layer_08_b200 as moe
+    from moe_expert_layer_08_b200 import build as mbuild
+    if rank == 0:
+        mbuild.build()
+    if world > 1:
+        torch.distributed.barrier()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if args.format == "nvfp4" and args.layout != "packets":
+        raise SystemExit("the NVFP4 variant takes packet weights")
+    r = time_layer(args, w, device, world)
+    g, layer, out, stream, barrier = r["g"], r["layer"], r["out"], r["stream"], r["barrier"]
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host output.
     # The step's four inputs sit in one pinned staging buffer (256-byte aligned
@@ -618,6 +717,7 @@ def run_b200(args, w, rank, world, local_rank):
         layer(d_xq, d_xs, d_idx, d_tw, out=out, stream=stream)
         h_out.copy_(out, non_blocking=True)
 
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(args.warmup):
         e2e_step()
     barrier()
@@ -633,81 +733,19 @@ def run_b200(args, w, rank, world, local_rank):
 
     if rank != 0:
         return
-    # roofline of the dominant kernel (GEMM1 or GEMM2), timed by the stage events
-    touched = len(W.touched_experts(g["idx"].cpu(), w.E))
-    b1, b2 = expert_bytes(w, args.format)
-    g1_ms, g2_ms = float(stage_ms[:, 1].mean()), float(stage_ms[:, 2].mean())
-    pk = peaks()
-    if g1_ms >= g2_ms:
-        kname, kms, kbytes = "moe_gemm_kernel<gemm1>", g1_ms, touched * b1
-    else:
-        kname, kms, kbytes = "moe_gemm_kernel<gemm2>", g2_ms, touched * b2
-    achieved = kbytes / (kms * 1e-3) / 1e9
-    traffic = measured_traffic(w, touched, g1_ms >= g2_ms, args.format)
-    roofline = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "peak_source": pk["source"], "algorithmic_bytes": kbytes,
-                "traffic": traffic, "spec": {"peak": SPEC_HBM_GBPS, "frac": achieved / SPEC_HBM_GBPS}}
-    # tensor peaks: FP8 = 2 x measured bf16, FP4 (NVFP4) = 4 x (the nominal
-    # dense ratios); the block-scaled FP8 x FP4 MMA runs at the FP8 rate
-    ratio = 2.0 if args.format == "mx" else 4.0
-    spec_tc = SPEC_FP8_TFLOPS * ratio / 2.0
-    if w.T * w.k > 8 * w.E:
-        # large batches: each weight byte feeds ~T*k/E rows, and the tensor
-        # pipe binds as much as HBM.  The kernel is timed inside the layer
-        # step, run back to back for the whole timed region (under the power
-        # cap: see "clocks"), so the denominator is the sustained peak; the
-        # burst and spec fractions are given beside it.
-        kflops = 2.0 * w.T * w.k * (2 * w.I if g1_ms >= g2_ms else w.H) * (w.H if g1_ms >= g2_ms else w.I)
-        peak_s, peak_b = ratio * pk["bf16_sustained"], ratio * pk["bf16"]
-        tflops = kflops / (kms * 1e-3) / 1e12
-        roofline = {"kernel": kname, "bound": "tensor", "achieved": tflops, "peak": peak_s, "unit": "TFLOP/s",
-                    "frac": tflops / peak_s,
-                    "peak_source": pk["source"] + f" sustained ({ratio:g} x bf16_tflops_sustained)",
-                    "frac_of_burst": tflops / peak_b,
-                    "burst_peak": peak_b,
-                    "spec": {"peak": spec_tc, "frac": tflops / spec_tc},
-                    "algorithmic_flops": kflops,
-                    "traffic": traffic, "hbm": {"achieved_GBps": achieved, "frac": achieved / pk["hbm"]}}
-        if cublas_fp8() and args.format == "mx":
-            roofline["cublas_fp8"] = {arm: {"sustained": c["sustained"], "frac": tflops / c["sustained"],
-                                            "burst": c["burst"], "frac_of_burst": tflops / c["burst"]}
-                                      for arm, c in cublas_fp8().items()}
-    x_bytes = w.T * w.H * 33 // 32 if args.format == "mx" else w.T * w.H * 9 // 16
-    layer_bytes = touched * (b1 + b2) + x_bytes + w.T * w.k * 12 + w.T * w.H * 2
-    flops = w.flops
-    value = world * flops / (ms * 1e-3) / 1e12
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
-    layer_tc = {"sustained": value / world / (ratio * pk["bf16_sustained"]),
-                "burst": value / world / (ratio * pk["bf16"]),
-                "spec": value / world / spec_tc}
-    if cublas_fp8() and args.format == "mx":
-        layer_tc["cublas_fp8_sustained"] = {arm: value / world / c["sustained"]
-                                            for arm, c in cublas_fp8().items()}
+    f = layer_figures(args, w, r, world)
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": f["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": f["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "data": "synthetic",
         "dtype": "fp8xfp4 (fp32 accumulate)" if args.format == "mx" else "nvfp4 e2m1xe2m1 (fp32 accumulate)",
-        "config": {"workload": w.name, **{k: getattr(w, k) for k in ("T", "E", "k", "H", "I", "seed", "routing")},
-                   "parallelism": f"replicas x{world}", "weight_layout": args.layout,
-                   "l2": "inputs larger than L2 (touched expert weights per step >> 126 MB)"
-                   if touched * (b1 + b2) > 256e6 else "inputs fit in L2 (not flushed)"},
-        "us_per_layer": ms * 1e3,
-        "effective_GBps": layer_bytes / (ms * 1e-3) / 1e9,
-        "hbm_frac_layer": layer_bytes / (ms * 1e-3) / 1e9 / pk["hbm"],
-        "touched_experts": touched,
-        "stage_us": {"route_gather": float(stage_ms[:, 0].mean() * 1e3), "gemm1": g1_ms * 1e3,
-                     "gemm2": g2_ms * 1e3, "combine": float(stage_ms[:, 3].mean() * 1e3)},
-        "stage_timing": {"how": "second pass of the same K steps with a CUDA event on the launch stream "
-                                "between kernels; the roofline's kernel duration comes from it",
-                         "us_per_layer": staged_ms * 1e3},
-        "roofline": roofline,
-        "layer_frac_of_tensor_peak": layer_tc,
-        "layer_frac_of_hbm_spec": layer_bytes / (ms * 1e-3) / 1e9 / SPEC_HBM_GBPS,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * moe.forward_kernel_launches(w.T, w.E, w.k, w.H, w.I),
-        "clocks": clocks.summary(),
+        "config": workload_config(w, args, world, f["touched"], f["b12"]),
+        **{k: f[k] for k in ("us_per_layer", "effective_GBps", "hbm_frac_layer", "touched_experts", "stage_us",
+                             "stage_timing", "roofline", "layer_frac_of_tensor_peak", "layer_frac_of_hbm_spec")},
+        "e2e": {"value": world * w.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": f["gpu_launches"],
+        "clocks": f["clocks"],
     }
     if not args.no_cpu_baseline:
         s = oracle_sample(w, args.cpu_tokens, device, args.format)
@@ -715,6 +753,30 @@ def run_b200(args, w, rank, world, local_rank):
         line["cpu_baseline"] = {"value": cflops / times[0] / 1e12, "unit": "TFLOP/s", "cores": threads,
                                 "kind": "oracle", "seconds": times[0],
                                 "sample": f"first {len(s['tokens'])} of {w.T} tokens, all {w.k} experts each"}
+    # The other workloads of the table, measured in the same run (one GPU
+    # only): the same K timed calls after W warm-up calls each, with their own
+    # clocks.  No end-to-end pass and no oracle timing for these (the
+    # headline workload above carries both).
+    extra = [int(x) for x in args.also.split(",") if x.strip()] if args.also else []
+    if world == 1 and extra and not (args.experts or args.tokens):
+        del r, g, layer, out, h_in, d_in, h_out, d_xq, d_xs, d_idx, d_tw
+        torch.cuda.empty_cache()
+        line["workloads"] = {}
+        for wid in extra:
+            wx = W.WORKLOADS[wid]
+            rx = time_layer(args, wx, device, world)
+            fx = layer_figures(args, wx, rx, world)
+            line["workloads"][wx.name] = {
+                "config": workload_config(wx, args, world, fx["touched"], fx["b12"]),
+                "tflops": fx["value"], "us_per_layer": fx["us_per_layer"],
+                **{k: fx[k] for k in ("effective_GBps", "hbm_frac_layer", "touched_experts", "stage_us",
+                                      "roofline", "layer_frac_of_tensor_peak", "gpu_launches", "clocks")},
+                "not_measured_here": "e2e and the oracle's cpu_baseline (headline workload only)",
+            }
+            del rx
+            torch.cuda.empty_cache()
+        line["gpu_launches"] += sum(v["gpu_launches"] for v in line["workloads"].values())
+        line["gpu_launches_note"] = "headline timed region plus the timed regions of `workloads`"
     print(json.dumps(line), flush=True)
 
 
@@ -727,6 +789,9 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl" if args.impl == "b200" else "gloo",
                                              timeout=datetime.timedelta(seconds=120))
+    if args.also is None:
+        args.also = "2,3,4" if args.workload == 1 and not (args.experts or args.tokens) and \
+            args.format == "mx" and args.layout == "packets" else ""
     w = W.WORKLOADS[args.workload]
     if args.experts or args.tokens:
         E, T = args.experts or w.E, args.tokens or w.T

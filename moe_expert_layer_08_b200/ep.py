@@ -27,7 +27,7 @@ from __future__ import annotations
 
 import torch
 
-from . import ep_combine, ep_dispatch, ep_workspace_bytes, forward, workspace_bytes
+from . import check_device_error, ep_combine, ep_dispatch, ep_workspace_bytes, forward, workspace_bytes
 
 __all__ = ["ExpertParallelLayer"]
 
@@ -74,6 +74,9 @@ class ExpertParallelLayer:
         self.y_loc = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
         self.y_back = torch.empty((n, H), dtype=torch.bfloat16, device=dev)
         self.ws_loc = torch.empty(workspace_bytes(self.recv_max, self.E_loc, 1, H, I), dtype=u8, device=dev)
+        # error words start clean (a step with no received rows runs no layer on ws_loc)
+        self.ws[:4].zero_()
+        self.ws_loc[:4].zero_()
         self.last_n_recv = 0  # rows the expert layer ran over in the last step
 
     # ---------------------------------------------------------------- phases
@@ -106,6 +109,14 @@ class ExpertParallelLayer:
     def combine(self, topk_w, out=None, stream=None):
         """Step 5: out (bf16 [T, H]) from the returned rows in y_back."""
         return ep_combine(self.y_back, topk_w, self.E, self.ws, out=out, stream=stream)
+
+    def check(self, stream=None) -> int:
+        """Synchronises the stream and returns the device status of the last
+        step: the dispatch workspace's error word (dropped expert ids) or, if
+        that is clean, the expert layer's (its bounded waits record timeouts
+        there); 0 when both are clean."""
+        st = check_device_error(self.ws, stream=stream)
+        return st if st != 0 else check_device_error(self.ws_loc, stream=stream)
 
     # ------------------------------------------------------------- one step
     def _exchange(self, dst, src, out_splits, in_splits):

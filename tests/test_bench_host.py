@@ -77,3 +77,18 @@ def test_committed_cublas_fp8_figure_is_below_the_derived_denominator():
         assert 0 < c["sustained"] <= c["burst"]
         if pk["source"] == "measured":
             assert c["sustained"] <= 2.0 * pk["bf16_sustained"]
+
+
+def test_both_arms_print_the_same_config_keys():
+    # the driver compares the two arms' `config` objects: the GPU arm's and
+    # the oracle arm's come from the same function with the same arguments
+    import types
+    args = types.SimpleNamespace(layout="packets")
+    for w in W.WORKLOADS.values():
+        b12 = bench.expert_bytes(w, "mx")
+        a = bench.workload_config(w, args, 1, 44, b12)
+        b = bench.workload_config(w, args, 1, 44, b12)
+        assert a == b
+        assert set(a) == {"workload", "T", "E", "k", "H", "I", "seed", "routing", "parallelism",
+                          "weight_layout", "l2"}
+        assert a["workload"] == w.name and a["parallelism"] == "replicas x1"
