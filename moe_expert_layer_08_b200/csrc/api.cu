@@ -4,6 +4,7 @@
 // the launch sequence of one layer.
 #include <cmath>
 #include <mutex>
+#include <vector>
 
 #include "moe.h"
 #include "moe_common.cuh"
@@ -193,6 +194,24 @@ int num_sms() {
         cache[dev] = n > 0 ? n : 148;
     }
     return cache[dev];
+}
+
+cudaError_t set_max_dynamic_smem(const void *kernel, int bytes) {
+    struct Done {
+        const void *kernel;
+        int dev, bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Done> done;
+    int dev = 0;
+    const cudaError_t ge = cudaGetDevice(&dev);
+    if (ge != cudaSuccess) return ge;
+    std::lock_guard<std::mutex> g(mu);
+    for (const Done &d : done)
+        if (d.kernel == kernel && d.dev == dev && d.bytes >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.push_back({kernel, dev, bytes});
+    return e;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

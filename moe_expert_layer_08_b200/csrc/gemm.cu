@@ -545,9 +545,25 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                     for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(v1[j]));
                 }
             };
-            // GEMM1 epilogue of 32 tokens: activation, scale, requantised h
-            auto finish1 = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], int cb) {
-            float h[32], amx[32];
+            // GEMM1: gate and up accumulators of column block cb (K split: both halves added)
+            auto load_gu = [&](int cb, uint32_t (&g)[32], uint32_t (&u)[32]) {
+                tmem_ld_32x32(acc + uint32_t(cb * 32), g);
+                tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
+                tmem_ld_wait();
+                if (add_split) {
+                    uint32_t g1[32], u1[32];
+                    tmem_ld_32x32(acc + uint32_t(2 * kN + cb * 32), g1);
+                    tmem_ld_32x32(acc + uint32_t(3 * kN + cb * 32), u1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g1[j]));
+                        u[j] = __float_as_uint(__uint_as_float(u[j]) + __uint_as_float(u1[j]));
+                    }
+                }
+            };
+            // h = act(gate, up) of 32 tokens of this lane's intermediate row
+            auto activate = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], float (&h)[32]) {
             if (args.act_kind == MOE_ACT_SWIGLU) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
@@ -568,9 +584,59 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                     h[j] = __fdividef(args.beta * tanhf(gv * args.inv_beta), 1.0f + __expf(-gv)) * up;
                 }
             }
+            };
+            // FP8 requantisation of 32 tokens of h (this lane's row): the scale
+            // byte of token cb*32 + lane (the amax over the warp's 32 rows, one
+            // UE8M0 group of GEMM2's K) and the 32 codes, four tokens per word
+            // (byte b of word m: token 4m + b)
+            auto quantize8 = [&](float (&h)[32], uint32_t (&pq)[8], uint32_t &sfb) {
+                float amx[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
+                for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
+                const int e = scale_exponent<true>(warp_transpose_max(amx, lane));
+                const float mult = exp2_neg(e);
+                sfb = uint32_t(e + 127);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    uint32_t w = 0;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const float mj = __shfl_sync(0xFFFFFFFFu, mult, 4 * m + b);
+                        w |= to_e4m3(h[4 * m + b] * mj) << (8 * b);
+                    }
+                    pq[m] = w;
+                }
+            };
+            // Stores of quantize8's results for column block cb: the scale byte,
+            // then the codes.  Lanes 4G .. 4G+3 hold rows 4G .. 4G+3; a 4 x 4
+            // byte transpose among them gives lane 4G + r the four row bytes of
+            // token 4m + r, one 4-byte store per token and word.
+            auto store8 = [&](const uint32_t (&pq)[8], uint32_t sfb, int cb) {
+                const int tok = cb * 32 + lane;
+                if (tok < ch.z)
+                    args.out_sf[(int64_t(c) * n_tiles + it) * C::kActSf + act_sf_offset(tok, q)] = uint8_t(sfb);
+                const int G = lane >> 2, r = lane & 3;
+                const uint32_t sel = uint32_t(r) | (uint32_t(4 + r) << 4);
+                uint8_t *qrow = args.out_q + (int64_t(it) * args.rows + ch.y + cb * 32) * kTileK + q * 32 + 4 * G;
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const uint32_t v0 = __shfl_sync(0xFFFFFFFFu, pq[m], 4 * G);
+                    const uint32_t v1 = __shfl_sync(0xFFFFFFFFu, pq[m], 4 * G + 1);
+                    const uint32_t v2 = __shfl_sync(0xFFFFFFFFu, pq[m], 4 * G + 2);
+                    const uint32_t v3 = __shfl_sync(0xFFFFFFFFu, pq[m], 4 * G + 3);
+                    const uint32_t w = __byte_perm(__byte_perm(v0, v1, sel), __byte_perm(v2, v3, sel), 0x5410);
+                    const int t = 4 * m + r;
+                    if (cb * 32 + t < ch.z) *reinterpret_cast<uint32_t *>(qrow + int64_t(t) * kTileK) = w;
+                }
+            };
+            // GEMM1 epilogue of 32 tokens: activation, scale, requantised h
+            auto finish1 = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], int cb) {
+            float h[32];
+            activate(g, u, h);
             if constexpr (kNv) {
+                float amx[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
                 // NVFP4: groups of 16 rows of h = the two half-warps.  Lane l
                 // gets the amax of tokens cb*32 + l%16 and cb*32 + 16 + l%16 over
                 // its half-warp, and their UE4M3 scale codes.
@@ -599,33 +665,58 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         qbase[int64_t(cb * 32 + j) * kTileK] = uint8_t(code | (partner << 4));
                 }
             } else {
-            // lane l: amax of token cb*32+l over this warp's 32 rows of h
-            const float amax = warp_transpose_max(amx, lane);
-            const int e = scale_exponent<true>(amax);
-            const float mult = exp2_neg(e);
-            const int tok = cb * 32 + lane;
-            if (tok < ch.z)
-                args.out_sf[(int64_t(c) * n_tiles + it) * C::kActSf + act_sf_offset(tok, q)] =
-                    uint8_t(e + 127);
-            // K-block-major [I/128][rows][128]: this warp's 32 codes of a row are
-            // bytes q*32 .. q*32+31 of row (ch.y + token) in K block `it`
-            uint8_t *qbase = args.out_q + (int64_t(it) * args.rows + ch.y) * kTileK + q * 32;
-            // one store per token: the warp's 32 lanes write 32 contiguous bytes
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float mj = __shfl_sync(0xFFFFFFFFu, mult, j);
-                const uint32_t code = to_e4m3(h[j] * mj);
-                if (cb * 32 + j < ch.z) qbase[int64_t(cb * 32 + j) * kTileK + lane] = uint8_t(code);
-            }
+                uint32_t pq[8], sfb;
+                quantize8(h, pq, sfb);
+                store8(pq, sfb, cb);
             }
             };
-            // GEMM2 epilogue of 32 tokens of output tile 2 * it + a: bf16 Y rows
-            auto finish2 = [&](const uint32_t (&g)[32], int a, int cb) {
+            // GEMM2: 32 fp32 accumulator words (tokens) -> 16 words of bf16 pairs
+            // (word m: token 2m in the low half, 2m + 1 in the high half)
+            auto pack2 = [&](const uint32_t (&g)[32], uint32_t (&pk)[16]) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const __nv_bfloat162 b2 =
+                        __floats2bfloat162_rn(__uint_as_float(g[2 * m]), __uint_as_float(g[2 * m + 1]));
+                    pk[m] = *reinterpret_cast<const uint32_t *>(&b2);
+                }
+            };
+            // GEMM2 stores of 32 tokens of output tile 2 * it + a: bf16 Y rows
+            auto store2 = [&](const uint32_t (&pk)[16], int a, int cb) {
                 const int tile = 2 * it + a;
             __nv_bfloat16 *ybase = args.out_y + int64_t(ch.y + cb * 32) * args.out_ld + tile * kTileRows + q * 32;
             if constexpr (C::kStaged) {
                 // two passes of 16 rows: stage [row][32 columns] bf16 (1 KB), then
                 // 16-byte stores, four lanes per 64-byte row piece
+                uint16_t *sb = reinterpret_cast<uint16_t *>(my_stage);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        sb[j * 32 + lane] = uint16_t(pk[hh * 8 + j / 2] >> (16 * (j & 1)));
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int cidx = i * 32 + lane;  // row hh*16 + cidx / 4, columns (cidx % 4) * 8 ..
+                        const int r = hh * 16 + (cidx >> 2);
+                        if (cb * 32 + r < ch.z)
+                            *reinterpret_cast<uint4 *>(ybase + int64_t(r) * args.out_ld + (cidx & 3) * 8) =
+                                *reinterpret_cast<const uint4 *>(my_stage + cidx * 16);
+                    }
+                    __syncwarp();
+                }
+            } else {
+                uint16_t *yb = reinterpret_cast<uint16_t *>(ybase);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (cb * 32 + j < ch.z) yb[int64_t(j) * args.out_ld + lane] = uint16_t(pk[j / 2] >> (16 * (j & 1)));
+            }
+            };
+            // GEMM2 epilogue of 32 tokens of output tile 2 * it + a (NVFP4, split
+            // units): bf16 Y rows straight from the accumulator words
+            auto finish2 = [&](const uint32_t (&g)[32], int a, int cb) {
+                const int tile = 2 * it + a;
+            __nv_bfloat16 *ybase = args.out_y + int64_t(ch.y + cb * 32) * args.out_ld + tile * kTileRows + q * 32;
+            if constexpr (C::kStaged) {
                 __nv_bfloat16 *sb = reinterpret_cast<__nv_bfloat16 *>(my_stage);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -635,7 +726,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                     __syncwarp();
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
-                        const int cidx = i * 32 + lane;  // row hh*16 + cidx / 4, columns (cidx % 4) * 8 ..
+                        const int cidx = i * 32 + lane;
                         const int r = hh * 16 + (cidx >> 2);
                         if (cb * 32 + r < ch.z)
                             *reinterpret_cast<uint4 *>(ybase + int64_t(r) * args.out_ld + (cidx & 3) * 8) =
@@ -657,23 +748,62 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) p[j * kTileRows] = __uint_as_float(v[j]);
             };
+            // Whole items (FP8 x FP4): only the work that reads the accumulator
+            // runs while the MMAs wait for it.  Each unit's results go to a few
+            // registers (GEMM1: 8 words of codes + the scale byte; GEMM2: 16
+            // words of bf16 pairs), the accumulator is released to the issuers,
+            // and then the units' global stores run, overlapping the next
+            // item's MMAs.
+            if (!kNv && !is_unit) {
+                if constexpr (kGemm1) {
+                    constexpr int kU = ((kN + 31) / 32 + kCbStep - 1) / kCbStep;
+                    uint32_t pq[kU][8], sfb[kU];
+#pragma unroll
+                    for (int i = 0; i < kU; ++i) {
+                        const int cb = half + i * kCbStep;
+                        if (cb < ncb) {
+                            uint32_t g[32], u[32];
+                            float h[32];
+                            load_gu(cb, g, u);
+                            activate(g, u, h);
+                            quantize8(h, pq[i], sfb[i]);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+#pragma unroll
+                    for (int i = 0; i < kU; ++i) {
+                        const int cb = half + i * kCbStep;
+                        if (cb < ncb) store8(pq[i], sfb[i], cb);
+                    }
+                } else {
+                    constexpr int kU = (kNumA * ((kN + 31) / 32) + kCbStep - 1) / kCbStep;
+                    uint32_t pk[kU][16];
+#pragma unroll
+                    for (int i = 0; i < kU; ++i) {
+                        const int u = half + i * kCbStep, a = u % kNumA, cb = u / kNumA;
+                        if (cb < ncb && 2 * it + a < n_tiles) {
+                            uint32_t g[32];
+                            load_tile(a, cb, g);
+                            pack2(g, pk[i]);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tmem_empty[buf]);
+#pragma unroll
+                    for (int i = 0; i < kU; ++i) {
+                        const int u = half + i * kCbStep, a = u % kNumA, cb = u / kNumA;
+                        if (cb < ncb && 2 * it + a < n_tiles) store2(pk[i], a, cb);
+                    }
+                }
+                continue;
+            }
             if constexpr (kGemm1) {
                 for (int cb = half; cb < ncb; cb += kCbStep) {
                     uint32_t g[32], u[32];
-                    tmem_ld_32x32(acc + uint32_t(cb * 32), g);
-                    tmem_ld_32x32(acc + uint32_t(kN + cb * 32), u);
-                    tmem_ld_wait();
-                    if (add_split) {
-                        uint32_t g1[32], u1[32];
-                        tmem_ld_32x32(acc + uint32_t(2 * kN + cb * 32), g1);
-                        tmem_ld_32x32(acc + uint32_t(3 * kN + cb * 32), u1);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g1[j]));
-                            u[j] = __float_as_uint(__uint_as_float(u[j]) + __uint_as_float(u1[j]));
-                        }
-                    }
+                    load_gu(cb, g, u);
                     if (is_unit) {
                         put_part(0, cb, g);
                         put_part(1, cb, u);
@@ -761,15 +891,9 @@ static cudaError_t launch_gemm_t(const CUtensorMap &tmap_w, const CUtensorMap &t
                                  const CUtensorMap &tmap_act_full, const GemmArgs &args, int grid,
                                  cudaStream_t stream) {
     using C = GemmCfg<kGemm1, kN, kNv>;
-    static int configured_for = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_for != dev) {
-        const cudaError_t e = cudaFuncSetAttribute(moe_gemm_kernel<kGemm1, kN, kNv>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured_for = dev;
-    }
+    const cudaError_t e =
+        set_max_dynamic_smem(reinterpret_cast<const void *>(moe_gemm_kernel<kGemm1, kN, kNv>), C::kSmemBytes);
+    if (e != cudaSuccess) return e;
     return launch_pdl(moe_gemm_kernel<kGemm1, kN, kNv>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
                       tmap_w, tmap_wsf, tmap_act, tmap_act_full, args);
 }

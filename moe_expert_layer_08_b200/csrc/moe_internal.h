@@ -105,6 +105,9 @@ bool encode_bf16_rows(CUtensorMap *m, const void *base, uint64_t cols, uint64_t 
 
 // Multiprocessors of the current device (cached per device).
 int num_sms();
+// Opts `kernel` in to `bytes` of dynamic shared memory on the current device,
+// once per (kernel, device); safe to call from several host threads.
+cudaError_t set_max_dynamic_smem(const void *kernel, int bytes);
 
 // Argument checks shared by the entry points.
 bool aligned(const void *p, uintptr_t a);

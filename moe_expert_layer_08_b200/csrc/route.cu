@@ -362,15 +362,9 @@ cudaError_t launch_routing(const int64_t *topk_idx, int k, int E, uint8_t *ws, c
     cudaError_t e;
     if (R <= kRouteSmallMax) {
         const size_t smem = size_t(32) * E * sizeof(int);
-        static int configured_for = -1;
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (configured_for != dev) {
-            e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     32 * kMaxExperts * int(sizeof(int)));
-            if (e != cudaSuccess) return e;
-            configured_for = dev;
-        }
+        e = set_max_dynamic_smem(reinterpret_cast<const void *>(route_small_kernel),
+                                 32 * kMaxExperts * int(sizeof(int)));
+        if (e != cudaSuccess) return e;
         e = launch_pdl(route_small_kernel, dim3(1), dim3(1024), smem, stream, topk_idx, R, k, E, cr, side, count,
                        offset, chunk_base, chunks, chunks_s, perm, inv, rowinfo, hdr, expert_stats);
     } else {

@@ -359,15 +359,9 @@ template <bool kGemm1, int kN>
 static cudaError_t launch_shared_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, const SharedArgs &a,
                                    int items, cudaStream_t stream) {
     using C = SharedCfg<kN>;
-    static int configured_for = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_for != dev) {
-        const cudaError_t e = cudaFuncSetAttribute(shared_gemm_kernel<kGemm1, kN>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        configured_for = dev;
-    }
+    const cudaError_t e =
+        set_max_dynamic_smem(reinterpret_cast<const void *>(shared_gemm_kernel<kGemm1, kN>), C::kSmemBytes);
+    if (e != cudaSuccess) return e;
     const int sms = num_sms();
     const int grid = items < sms ? (items > 0 ? items : 1) : sms;
     return launch_pdl(shared_gemm_kernel<kGemm1, kN>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
