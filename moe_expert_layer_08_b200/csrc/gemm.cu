@@ -410,6 +410,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 const int it = item % n_items;
                 const bool valid = kGemm1 || 2 * it + a < n_tiles;  // GEMM2's last pair may hold one tile
                 const uint32_t n = uint32_t((ch.z + 15) / 16 * 16);
+                // activation scale images the MMAs read: one per 128 of the N rows
+                const int sfb_images = int(n + 127) / 128;
                 const int buf = li % kBufs;
                 const uint32_t use = uint32_t(li / kBufs) & 1u;  // how often this buffer was used, mod 2
                 if (!mbar_wait(&tmem_empty[buf], use ^ 1u, abort_flag, err, 2)) break;
@@ -450,8 +452,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                             tc_cp_sf(col + j * 4, smem_desc_sf(smem_u32(sfa + (a * kNvImages + sI) * kSfBlockBytes)));
 #pragma unroll
                             for (int im = 0; im < C::kSfbImages; ++im)
-                                tc_cp_sf(colb + (j * C::kSfbImages + im) * 4,
-                                         smem_desc_sf(smem_u32(sfb + sI * C::kActSf + im * kSfBlockBytes)));
+                                if (im < sfb_images)
+                                    tc_cp_sf(colb + (j * C::kSfbImages + im) * 4,
+                                             smem_desc_sf(smem_u32(sfb + sI * C::kActSf + im * kSfBlockBytes)));
                         }
                         const uint64_t adesc = smem_desc_sw128(smem_u32(st + a * C::kATile));
                         const uint64_t bdesc = smem_desc_sw128(smem_u32(bt));
@@ -478,8 +481,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                             const uint32_t sfb_col = col + 4;
 #pragma unroll
                             for (int im = 0; im < C::kSfbImages; ++im)
-                                tc_cp_sf(sfb_col + im * 4,
-                                         smem_desc_sf(smem_u32(sfb + b * C::kActSf + im * kSfBlockBytes)));
+                                if (im < sfb_images)
+                                    tc_cp_sf(sfb_col + im * 4,
+                                             smem_desc_sf(smem_u32(sfb + b * C::kActSf + im * kSfBlockBytes)));
                             const uint64_t adesc = smem_desc_sw128(smem_u32(st + slot * C::kATile));
                             const uint64_t bdesc = smem_desc_sw128(smem_u32(bt + b * C::kBTile));
 #pragma unroll
@@ -598,13 +602,10 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 sfb = uint32_t(e + 127);
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
-                    uint32_t w = 0;
+                    float v[4];
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const float mj = __shfl_sync(0xFFFFFFFFu, mult, 4 * m + b);
-                        w |= to_e4m3(h[4 * m + b] * mj) << (8 * b);
-                    }
-                    pq[m] = w;
+                    for (int b = 0; b < 4; ++b) v[b] = h[4 * m + b] * __shfl_sync(0xFFFFFFFFu, mult, 4 * m + b);
+                    pq[m] = to_e4m3x4(v);
                 }
             };
             // Stores of quantize8's results for column block cb: the scale byte,

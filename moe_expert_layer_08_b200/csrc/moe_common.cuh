@@ -107,6 +107,17 @@ __device__ __forceinline__ uint32_t to_e4m3(float v) {
     return uint32_t(m) | ((__float_as_uint(v) >> 24) & 0x80u);
 }
 
+// The E4M3 codes of four scaled values, v[b] in byte b, two conversions per
+// instruction; as in to_e4m3 the sign bit of every code is the sign bit of
+// its value (a value that rounds to zero keeps its sign).
+__device__ __forceinline__ uint32_t to_e4m3x4(const float (&v)[4]) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[0], v[1]), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[2], v[3]), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t sign = ((__float_as_uint(v[0]) >> 24) & 0x80u) | ((__float_as_uint(v[1]) >> 16) & 0x8000u) |
+                          ((__float_as_uint(v[2]) >> 8) & 0x800000u) | (__float_as_uint(v[3]) & 0x80000000u);
+    return (lo | (hi << 16)) | sign;
+}
+
 // E2M1 code (4 bits) of v (|v| <= 6), round to nearest even, sign from v.
 __device__ __forceinline__ uint32_t to_e2m1(float v) {
     const __nv_fp4_storage_t m = __nv_cvt_float_to_fp4(fabsf(v), __NV_E2M1, cudaRoundNearest);
