@@ -534,6 +534,30 @@ moe_status_t moe_ep_combine_peers(const void *const *peer_y, const int64_t *recv
                                   const float *topk_w, int T, int E, int k, int H, int ranks, const void *workspace,
                                   size_t ws_bytes, void *out_bf16, moe_stream_t stream);
 
+/*
+ * Peer buffers for the two entry points above (no counterpart on the pages,
+ * which leave the symmetric-memory set-up to the serving system): CUDA IPC
+ * over one process per GPU.
+ *
+ * moe_ipc_handle -- the IPC handle (MOE_IPC_HANDLE_BYTES bytes, written to
+ *   `handle`) of the device allocation that holds device pointer `ptr`, and
+ *   ptr's byte offset inside that allocation (`offset`), to be sent to the
+ *   other ranks.  `ptr` may point anywhere inside an allocation (framework
+ *   allocators sub-allocate).  Host-side only; enqueues nothing.
+ * moe_ipc_open -- maps another process's allocation, given its handle, into
+ *   this process on CUDA device `device` (peer access enabled as needed);
+ *   `*base` receives the mapped base, to which the sender's offset is added.
+ *   A process cannot open a handle of its own allocations (use the pointer).
+ * moe_ipc_close -- unmaps a base returned by moe_ipc_open.  The mapping must
+ *   outlive every kernel that reads or writes through it.
+ * Errors: MOE_ERR_INVALID_ARG for null arguments or a negative device;
+ * MOE_ERR_CUDA when CUDA refuses (the CUDA error is cleared).
+ */
+#define MOE_IPC_HANDLE_BYTES 64
+moe_status_t moe_ipc_handle(const void *ptr, void *handle, size_t *offset);
+moe_status_t moe_ipc_open(const void *handle, int device, void **base);
+moe_status_t moe_ipc_close(void *base);
+
 #ifdef __cplusplus
 }
 #endif

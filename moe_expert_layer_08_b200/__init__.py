@@ -23,9 +23,11 @@ __all__ = [
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
     "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
     "ep_workspace_bytes", "ep_dispatch", "ep_combine", "ep_combine_peers", "ep_route", "ep_dispatch_peers",
+    "ipc_handle", "ipc_open", "ipc_close", "IPC_HANDLE_BYTES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+IPC_HANDLE_BYTES = 64  # MOE_IPC_HANDLE_BYTES
 NUM_STAGE_EVENTS = 5
 STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024  # MOE_STATIC_WORKSPACE_BYTES
 STATUS = {
@@ -115,6 +117,9 @@ def _declare(lib):
         "moe_ep_combine_peers": (I32, [P, P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P]),
         "moe_ep_route": (I32, [P, I32, I32, I32, I32, I32, P, SZ, P, P]),
         "moe_ep_dispatch_peers": (I32, [P, P, P, I32, I32, I32, I32, I32, P, SZ, P, P, P, P, P]),
+        "moe_ipc_handle": (I32, [P, P, c.POINTER(SZ)]),
+        "moe_ipc_open": (I32, [P, I32, c.POINTER(P)]),
+        "moe_ipc_close": (I32, [P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -658,3 +663,31 @@ def ep_dispatch_peers(x_fp8, x_sf, topk_idx, E: int, workspace, peer_x, peer_sf,
     _check(load().moe_ep_dispatch_peers(_ptr(x_fp8), _ptr(x_sf), _ptr(topk_idx), T, E, k, H, ranks, _ptr(workspace),
                                         workspace.numel(), _ptr(peer_x), _ptr(peer_sf), _ptr(peer_eid),
                                         _ptr(recv_base), _stream(stream)), "moe_ep_dispatch_peers")
+
+
+# ------------------------------------------------------------ peer buffers (CUDA IPC)
+def ipc_handle(t: torch.Tensor):
+    """(handle bytes, byte offset) of device tensor t's allocation, for
+    another process's ipc_open (moe_ipc_handle)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("ipc_handle takes a CUDA tensor")
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_size_t()
+    _check(load().moe_ipc_handle(_ptr(t), buf, ctypes.byref(off)), "moe_ipc_handle")
+    return buf.raw, off.value
+
+
+def ipc_open(handle: bytes, device: int) -> int:
+    """Maps another process's allocation into this one on CUDA device
+    ``device``; returns the mapped base address (moe_ipc_open)."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has IPC_HANDLE_BYTES bytes")
+    base = ctypes.c_void_p()
+    _check(load().moe_ipc_open(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES), int(device),
+                               ctypes.byref(base)), "moe_ipc_open")
+    return int(base.value)
+
+
+def ipc_close(base: int) -> None:
+    """Unmaps a base returned by ipc_open (moe_ipc_close)."""
+    _check(load().moe_ipc_close(ctypes.c_void_p(base)), "moe_ipc_close")

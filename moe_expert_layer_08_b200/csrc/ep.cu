@@ -14,6 +14,8 @@
 // forms out[t] = bf16(sum_j w[t, j] * Y[inv[t*k + j]]) with the layer's own
 // combine kernel through the inverse permutation the dispatch left in the
 // workspace.
+#include <cstring>
+
 #include "ep_internal.h"
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -327,6 +329,63 @@ moe_status_t moe_ep_dispatch_peers(const void *x_fp8, const void *x_sf, const in
         static_cast<const uint4 *>(x_fp8), static_cast<const uint32_t *>(x_sf),
         reinterpret_cast<uint4 *const *>(peer_x), reinterpret_cast<uint32_t *const *>(peer_sf), peer_eid, recv_base);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ peer buffers
+// Mapping the ranks' receive and output buffers into each other's address
+// space with CUDA IPC (for moe_ep_dispatch_peers / moe_ep_combine_peers).  A
+// buffer may sit anywhere inside its allocation (framework allocators hand
+// out pieces of larger blocks): the handle names the whole allocation and the
+// offset locates the buffer in it.
+
+static_assert(sizeof(cudaIpcMemHandle_t) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+
+moe_status_t moe_ipc_handle(const void *ptr, void *handle, size_t *offset) {
+    if (!ptr || !handle || !offset) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = use_device_of(ptr);
+    if (s != MOE_OK) return s;
+    typedef CUresult (*RangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+    static RangeFn range = []() -> RangeFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<RangeFn>(p);
+    }();
+    if (!range) return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t bytes = 0;
+    if (range(&base, &bytes, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    memcpy(handle, &h, sizeof(h));
+    *offset = size_t(reinterpret_cast<CUdeviceptr>(ptr) - base);
+    return MOE_OK;
+}
+
+moe_status_t moe_ipc_open(const void *handle, int device, void **base) {
+    if (!handle || !base || device < 0) return MOE_ERR_INVALID_ARG;
+    if (cudaSetDevice(device) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof(h));
+    if (cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}
+
+moe_status_t moe_ipc_close(void *base) {
+    if (!base) return MOE_ERR_INVALID_ARG;
+    if (cudaIpcCloseMemHandle(base) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
 }
 
 }  // extern "C"

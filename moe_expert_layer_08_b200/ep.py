@@ -17,7 +17,17 @@ on each rank:
    permutation of step 1.
 
 Every step of the computation runs in the CUDA library; this module sizes the
-buffers and issues the collectives.  Every rank takes the same collective
+buffers and issues the collectives.
+
+``forward_peers`` is the same step over peer memory: the ranks' receive and
+output buffers are mapped into every rank's address space once
+(``enable_peers``: CUDA IPC handles exchanged over the process group, see
+``PeerBuffers``), the dispatch writes each routed row straight into the
+receive buffers of the rank that holds its expert (``moe_ep_dispatch_peers``)
+and the combine reads each expert output where it was computed
+(``moe_ep_combine_peers``), with stream-ordered barriers (an all-reduce of one
+element on the step's stream) between the phases instead of the row
+all-to-alls.  Every rank takes the same collective
 steps in the same order, whatever its row counts.  The row counts are needed
 on the host for the split sizes, so ``forward`` synchronises once per step
 after the count exchange (an all-gather of every rank's per-destination
@@ -27,9 +37,69 @@ from __future__ import annotations
 
 import torch
 
-from . import check_device_error, ep_combine, ep_dispatch, ep_workspace_bytes, forward, workspace_bytes
+from . import (check_device_error, ep_combine, ep_combine_peers, ep_dispatch, ep_dispatch_peers, ep_route,
+               ep_workspace_bytes, forward, ipc_close, ipc_handle, ipc_open, workspace_bytes)
 
-__all__ = ["ExpertParallelLayer"]
+__all__ = ["ExpertParallelLayer", "PeerBuffers", "CudaIpc"]
+
+
+class CudaIpc:
+    """The library's CUDA IPC entry points (moe_ipc_handle / _open / _close)."""
+
+    def export(self, t):
+        return ipc_handle(t)
+
+    def open(self, handle: bytes, device: int) -> int:
+        return ipc_open(handle, device)
+
+    def close(self, base: int) -> None:
+        ipc_close(base)
+
+
+class PeerBuffers:
+    """Named buffers of every rank of ``group``, addressable from this process.
+
+    Every rank passes its own buffers (same names on every rank); each is
+    exported as (IPC handle of its allocation, byte offset in it), the records
+    are all-gathered, and every other rank's allocation is opened once (two
+    buffers in one allocation share a handle).  ``tables[name]`` is an i64
+    [ranks] tensor on ``device``: entry d is the address of rank d's buffer in
+    this process (this rank's own buffer's address for d = rank).  A
+    collective: every rank of the group constructs it at the same point.
+    ``ipc`` is the mapping backend (default: CUDA IPC through the library).
+    """
+
+    def __init__(self, buffers: dict, group=None, ipc=None, device=None):
+        import torch.distributed as dist
+        self.ipc = ipc if ipc is not None else CudaIpc()
+        self.rank, self.ranks = dist.get_rank(group), dist.get_world_size(group)
+        names = sorted(buffers)
+        first = buffers[names[0]]
+        dev_index = first.device.index if first.device.type == "cuda" else -1
+        mine = {n: self.ipc.export(buffers[n]) for n in names}
+        everyone = [None] * self.ranks
+        dist.all_gather_object(everyone, {"device": dev_index, "names": names, "records": mine}, group=group)
+        if any(r["names"] != names for r in everyone):
+            raise ValueError("every rank must pass the same buffer names")
+        self.opened = {}  # handle bytes -> mapped base
+        addr = {n: [0] * self.ranks for n in names}
+        for d in range(self.ranks):
+            for n in names:
+                if d == self.rank:
+                    addr[n][d] = buffers[n].data_ptr()
+                    continue
+                handle, offset = everyone[d]["records"][n]
+                if handle not in self.opened:
+                    self.opened[handle] = self.ipc.open(handle, dev_index)
+                addr[n][d] = self.opened[handle] + offset
+        dev = device if device is not None else first.device
+        self.tables = {n: torch.tensor(addr[n], dtype=torch.int64, device=dev) for n in names}
+
+    def close(self):
+        """Unmaps the other ranks' allocations (after every kernel that uses them)."""
+        for base in self.opened.values():
+            self.ipc.close(base)
+        self.opened = {}
 
 
 class ExpertParallelLayer:
@@ -109,6 +179,60 @@ class ExpertParallelLayer:
     def combine(self, topk_w, out=None, stream=None):
         """Step 5: out (bf16 [T, H]) from the returned rows in y_back."""
         return ep_combine(self.y_back, topk_w, self.E, self.ws, out=out, stream=stream)
+
+    # ------------------------------------------------------------- peer memory
+    def enable_peers(self, ipc=None):
+        """Maps every rank's receive buffers and expert-layer output into this
+        rank's address space (a collective over the group; see PeerBuffers)."""
+        self.peers = PeerBuffers({"x": self.recv_x, "sf": self.recv_sf, "eid": self.recv_eid, "y": self.y_loc},
+                                 group=self.group, ipc=ipc)
+        self._flag = torch.zeros(1, dtype=torch.float32, device=self.recv_x.device)
+        return self.peers
+
+    def _barrier(self):
+        # stream-ordered: work enqueued after it on this rank's stream starts
+        # only once every rank has reached it
+        import torch.distributed as dist
+        dist.all_reduce(self._flag, group=self.group)
+
+    def _route(self, topk_idx):
+        return ep_route(topk_idx, self.E, self.H, self.ranks, self.ws, self.send_counts)
+
+    def _push(self, x_fp8, x_sf, topk_idx, recv_base):
+        t = self.peers.tables
+        ep_dispatch_peers(x_fp8, x_sf, topk_idx, self.E, self.ws, t["x"], t["sf"], t["eid"], recv_base)
+
+    def _pull(self, topk_idx, topk_w, recv_base, out):
+        return ep_combine_peers(self.peers.tables["y"], recv_base, topk_idx, topk_w, self.E, self.H, self.ws,
+                                out=out)
+
+    def forward_peers(self, x_fp8, x_sf, topk_idx, topk_w, out=None):
+        """One layer step over peer memory (after ``enable_peers`` on every
+        rank); the same result as ``forward`` bit for bit."""
+        import torch.distributed as dist
+        if getattr(self, "peers", None) is None:
+            raise RuntimeError("enable_peers() first (on every rank)")
+        if x_fp8.shape[0] > self.T_max:
+            raise ValueError(f"{x_fp8.shape[0]} tokens > T_max = {self.T_max}")
+        counts = self._route(topk_idx)
+        rows = [torch.empty_like(counts) for _ in range(self.ranks)]
+        dist.all_gather(rows, counts, group=self.group)
+        matrix = torch.stack(rows).tolist()
+        most = max(sum(matrix[src][dst] for src in range(self.ranks)) for dst in range(self.ranks))
+        if most > self.recv_max:
+            raise ValueError(f"a rank would receive {most} rows > recv_max = {self.recv_max}")
+        # this rank's first row in rank d's receive buffers: what ranks 0..rank-1 send to d
+        base = [sum(matrix[src][d] for src in range(self.rank)) for d in range(self.ranks)]
+        recv_base = torch.tensor(base, dtype=torch.int64, device=counts.device)
+        n_recv = sum(matrix[src][self.rank] for src in range(self.ranks))
+        self.last_n_recv = n_recv
+        self._push(x_fp8, x_sf, topk_idx, recv_base)
+        self._barrier()   # every rank's rows are in every receive buffer
+        self.expert(n_recv)
+        self._barrier()   # every rank's expert outputs are complete
+        out = self._pull(topk_idx, topk_w, recv_base, out)
+        self._barrier()   # nobody still reads a rank's buffers when the next step writes them
+        return out
 
     def check(self, stream=None) -> int:
         """Synchronises the stream and returns the device status of the last
