@@ -101,7 +101,10 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    pdl_wait();
+    // GEMM2's weights do not depend on GEMM1: its weight producer fills the
+    // ring before GEMM1 has finished; every other access to memory written by
+    // earlier kernels comes after pdl_wait
+    if (kGemm1 || warp != 0) pdl_wait();
     if (threadIdx.x == 32) pdl_trigger();
 
     const int n_items = args.n_items, n_tiles = args.n_tiles;
@@ -223,29 +226,38 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
         const int half = warp >= 8 ? 1 : 0;
         constexpr int kCbStep = C::kEpiWarps / 4;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        // GEMM1: h of 32 tokens of intermediate tile `it` from gate g and up u
-        auto finish1 = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], int tok0, int nrows, int it) {
+        // GEMM1: h of kJ tokens of intermediate tile `it` from gate g and up u
+        // (the linear layer's bf16 output, then the activation in fp32)
+        auto finish1 = [&](const auto &g, const auto &u, int tok0, int nrows, int it) {
+            constexpr int kJ = int(sizeof(g) / sizeof(g[0]));
             __nv_bfloat16 *hb = args.out + int64_t(tok0) * args.out_ld + it * kTileRows + q * 32 + lane;
+            float h[kJ];
+            if (args.act_kind == MOE_ACT_SWIGLU) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                // the linear layer's bf16 output, then the activation in fp32
-                const float gv = bf16_round_f(__uint_as_float(g[j]));
-                const float uv = bf16_round_f(__uint_as_float(u[j]));
-                float hv;
-                if (args.act_kind == MOE_ACT_SWIGLU) {
-                    hv = gv / (1.0f + expf(-gv)) * uv;
-                } else {
-                    const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
-                    hv = (1.0f / (1.0f + expf(-gv))) * (args.beta * tanhf(gv * args.inv_beta)) * up;
+                for (int j = 0; j < kJ; ++j) {
+                    const float gv = bf16_round_f(__uint_as_float(g[j]));
+                    const float uv = bf16_round_f(__uint_as_float(u[j]));
+                    h[j] = gv / (1.0f + expf(-gv)) * uv;
                 }
-                if (j < nrows) hb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(hv);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kJ; ++j) {
+                    const float gv = bf16_round_f(__uint_as_float(g[j]));
+                    const float uv = bf16_round_f(__uint_as_float(u[j]));
+                    const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
+                    h[j] = (1.0f / (1.0f + expf(-gv))) * (args.beta * tanhf(gv * args.inv_beta)) * up;
+                }
             }
+#pragma unroll
+            for (int j = 0; j < kJ; ++j)
+                if (j < nrows) hb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(h[j]);
         };
-        // GEMM2: y of 32 tokens of output tile `tile`
-        auto finish2 = [&](const uint32_t (&v)[32], int tok0, int nrows, int tile) {
+        // GEMM2: y of kJ tokens of output tile `tile`
+        auto finish2 = [&](const auto &v, int tok0, int nrows, int tile) {
+            constexpr int kJ = int(sizeof(v) / sizeof(v[0]));
             __nv_bfloat16 *yb = args.out + int64_t(tok0) * args.out_ld + tile * kTileRows + q * 32 + lane;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
+            for (int j = 0; j < kJ; ++j)
                 if (j < nrows) yb[int64_t(j) * args.out_ld] = __float2bfloat16_rn(__uint_as_float(v[j]));
         };
         int li = 0, nsplit = 0;
@@ -284,9 +296,10 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 continue;
             }
             // K part of an item (32-token blocks: one column block): write this
-            // part's fp32 accumulators; the item's last part to finish adds the
-            // parts 0 .. split-1 in that order and runs the epilogue, so the
-            // result does not depend on which part ends last
+            // part's fp32 accumulators of the block's real tokens; the item's
+            // last part to finish adds the parts 0 .. split-1 in that order and
+            // runs the epilogue, so the result does not depend on which part
+            // ends last
             if constexpr (kN == 32) {
                 float *pu = args.part + size_t(uu) * kPartUnitFloats + q * 32 + lane;
 #pragma unroll 1
@@ -295,7 +308,8 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                     tmem_ld_32x32(acc + uint32_t(a * kN), v);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) pu[(a * 32 + j) * kTileRows] = __uint_as_float(v[j]);
+                    for (int j = 0; j < 32; ++j)
+                        if (j < rows) pu[(a * 32 + j) * kTileRows] = __uint_as_float(v[j]);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -317,32 +331,51 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 if (!mbar_wait(epi_go, uint32_t(nsplit & 1), abort_flag, err, 16)) break;
                 ++nsplit;
                 if (!*epi_last) continue;
+                // the parts' sums, 8 tokens at a time, added in part order 0 ..
+                // split-1 (two parts' loads in flight); then the block's epilogue
                 const float *p0 = args.part + size_t(item) * split * kPartUnitFloats + q * 32 + lane;
-                auto sum_part = [&](int a, uint32_t (&v)[32]) {
-                    float s_[32];
+#pragma unroll 1
+                for (int jb = 0; jb * 8 < rows; ++jb) {
+                    const float *pj = p0 + jb * 8 * kTileRows;
+                    uint32_t sv[2][8];
+                    float s_[2][8];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) s_[j] = __ldcg(p0 + (a * 32 + j) * kTileRows);
-                    for (int sp = 1; sp < split; ++sp) {
-                        const float *p = p0 + size_t(sp) * kPartUnitFloats;
+                    for (int a = 0; a < 2; ++a)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) s_[j] += __ldcg(p + (a * 32 + j) * kTileRows);
+                        for (int j = 0; j < 8; ++j) s_[a][j] = __ldcg(pj + (a * 32 + j) * kTileRows);
+#pragma unroll 1
+                    for (int sp = 1; sp < split; sp += 2) {
+                        const float *pa = pj + size_t(sp) * kPartUnitFloats;
+                        const bool two = sp + 1 < split;
+                        float t0[2][8], t1[2][8];
+#pragma unroll
+                        for (int a = 0; a < 2; ++a)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                t0[a][j] = __ldcg(pa + (a * 32 + j) * kTileRows);
+                                t1[a][j] = two ? __ldcg(pa + kPartUnitFloats + (a * 32 + j) * kTileRows) : 0.0f;
+                            }
+#pragma unroll
+                        for (int a = 0; a < 2; ++a)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) s_[a][j] += t0[a][j];
+                        if (two) {
+#pragma unroll
+                            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) s_[a][j] += t1[a][j];
+                        }
                     }
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(s_[j]);
-                };
-                const int tok0 = blk * kN;
-                if constexpr (kGemm1) {
-                    uint32_t g[32], u[32];
-                    sum_part(0, g);
-                    sum_part(1, u);
-                    finish1(g, u, tok0, rows, it);
-                } else {
-#pragma unroll 1
-                    for (int a = 0; a < 2; ++a) {
-                        if (2 * it + a >= n_tiles) break;
-                        uint32_t v[32];
-                        sum_part(a, v);
-                        finish2(v, tok0, rows, 2 * it + a);
+                    for (int a = 0; a < 2; ++a)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) sv[a][j] = __float_as_uint(s_[a][j]);
+                    const int tok0 = blk * kN + jb * 8;
+                    if constexpr (kGemm1) {
+                        finish1(sv[0], sv[1], tok0, rows - jb * 8, it);
+                    } else {
+                        finish2(sv[0], tok0, rows - jb * 8, 2 * it);
+                        if (2 * it + 1 < n_tiles) finish2(sv[1], tok0, rows - jb * 8, 2 * it + 1);
                     }
                 }
             }

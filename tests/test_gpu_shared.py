@@ -67,3 +67,15 @@ def test_shared_full_size_sampled(moe):
 def test_shared_decode_size(moe):
     """T = 8 tokens (32-token blocks, most SMs idle), SH = 7168, SI = 2048."""
     run_and_compare(moe, 8, 7168, 2048, 7)
+
+
+def test_shared_decode_size_situ(moe):
+    """T = 8, full size, SiTU: the K-split path's last part runs the SiTU
+    activation."""
+    run_and_compare(moe, 8, 7168, 2048, 9, situ=(1.25, 1.5))
+
+
+def test_shared_split_ragged_blocks(moe):
+    """T = 40 at full size: two 32-token blocks (32 and 8 rows), each item's K
+    cut into an even number of parts."""
+    run_and_compare(moe, 40, 7168, 2048, 10)
