@@ -237,7 +237,9 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 for (int j = 0; j < kJ; ++j) {
                     const float gv = bf16_round_f(__uint_as_float(g[j]));
                     const float uv = bf16_round_f(__uint_as_float(u[j]));
-                    h[j] = gv / (1.0f + expf(-gv)) * uv;
+                    // silu(g) * u with the fast exponential and division, as in the
+                    // routed experts' epilogue (0 where 1 + e^-g overflows: the limit)
+                    h[j] = __fdividef(gv * uv, 1.0f + __expf(-gv));
                 }
             } else {
 #pragma unroll
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                     const float gv = bf16_round_f(__uint_as_float(g[j]));
                     const float uv = bf16_round_f(__uint_as_float(u[j]));
                     const float up = args.inv_lbeta != 0.0f ? args.lbeta * tanhf(uv * args.inv_lbeta) : uv;
-                    h[j] = (1.0f / (1.0f + expf(-gv))) * (args.beta * tanhf(gv * args.inv_beta)) * up;
+                    h[j] = __fdividef(args.beta * tanhf(gv * args.inv_beta), 1.0f + __expf(-gv)) * up;
                 }
             }
 #pragma unroll
@@ -332,39 +334,36 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 ++nsplit;
                 if (!*epi_last) continue;
                 // the parts' sums, 8 tokens at a time, added in part order 0 ..
-                // split-1 (two parts' loads in flight); then the block's epilogue
+                // split-1 (the loads of four parts in flight together); then the
+                // block's epilogue
                 const float *p0 = args.part + size_t(item) * split * kPartUnitFloats + q * 32 + lane;
 #pragma unroll 1
                 for (int jb = 0; jb * 8 < rows; ++jb) {
                     const float *pj = p0 + jb * 8 * kTileRows;
                     uint32_t sv[2][8];
                     float s_[2][8];
-#pragma unroll
-                    for (int a = 0; a < 2; ++a)
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) s_[a][j] = __ldcg(pj + (a * 32 + j) * kTileRows);
 #pragma unroll 1
-                    for (int sp = 1; sp < split; sp += 2) {
-                        const float *pa = pj + size_t(sp) * kPartUnitFloats;
-                        const bool two = sp + 1 < split;
-                        float t0[2][8], t1[2][8];
+                    for (int sp0 = 0; sp0 < split; sp0 += 4) {
+                        float t[4][2][8];
 #pragma unroll
-                        for (int a = 0; a < 2; ++a)
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                t0[a][j] = __ldcg(pa + (a * 32 + j) * kTileRows);
-                                t1[a][j] = two ? __ldcg(pa + kPartUnitFloats + (a * 32 + j) * kTileRows) : 0.0f;
-                            }
-#pragma unroll
-                        for (int a = 0; a < 2; ++a)
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) s_[a][j] += t0[a][j];
-                        if (two) {
+                        for (int i = 0; i < 4; ++i)
 #pragma unroll
                             for (int a = 0; a < 2; ++a)
 #pragma unroll
-                                for (int j = 0; j < 8; ++j) s_[a][j] += t1[a][j];
-                        }
+                                for (int j = 0; j < 8; ++j)
+                                    t[i][a][j] = sp0 + i < split ? __ldcg(pj + size_t(sp0 + i) * kPartUnitFloats +
+                                                                          (a * 32 + j) * kTileRows)
+                                                                 : 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    if (sp0 + i == 0)
+                                        s_[a][j] = t[i][a][j];
+                                    else if (sp0 + i < split)
+                                        s_[a][j] += t[i][a][j];
                     }
 #pragma unroll
                     for (int a = 0; a < 2; ++a)
