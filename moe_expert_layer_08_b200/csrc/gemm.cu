@@ -630,41 +630,61 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                     if (cb * 32 + t < ch.z) *reinterpret_cast<uint32_t *>(qrow + int64_t(t) * kTileK) = w;
                 }
             };
+            // NVFP4 requantisation of 32 tokens of h (this lane's row): groups of
+            // 16 rows of h are the two half-warps; lane l gets the UE4M3 scale
+            // codes of tokens cb*32 + l%16 (byte 0 of sc) and cb*32 + 16 + l%16
+            // (byte 1), and its 32 E2M1 codes, eight per word (nibble j % 8 of
+            // word j / 8: token j)
+            auto quantize4 = [&](float (&h)[32], uint32_t (&cq)[4], uint32_t &sc) {
+                float amx[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
+                float amA, amB;
+                halfwarp_transpose_max(amx, lane, amA, amB);
+                const uint32_t cA = nvfp4_scale_code(amA), cB = nvfp4_scale_code(amB);
+                const float sA = e4m3_mag_value(cA), sB = e4m3_mag_value(cB);
+                sc = cA | (cB << 8);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) cq[m] = 0u;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, (lane & 16) | (j & 15));
+                    cq[j >> 3] |= to_e2m1(__fdiv_rn(h[j], sj)) << (4 * (j & 7));
+                }
+            };
+            // Stores of quantize4's results for column block cb: the two scale
+            // bytes, then one byte per token from each even lane (its own code in
+            // the low nibble, the next row's in the high one).  GEMM2 reads h in
+            // 256-K blocks: this item's 128 rows are half `it % 2` of block it / 2,
+            // and the warp's 32 rows are groups g4 = (q % 2) * 2 + half-warp of
+            // image (it % 2) * 2 + q / 2.
+            auto store4 = [&](const uint32_t (&cq)[4], uint32_t sc, int cb) {
+                const int img = (it & 1) * 2 + (q >> 1), g4 = (q & 1) * 2 + (lane >> 4);
+                uint8_t *sfo = args.out_sf + ((int64_t(c) * (n_tiles / 2) + it / 2) * kNvImages + img) * C::kActSf;
+                const int tA = cb * 32 + (lane & 15), tB = tA + 16;
+                if (tA < ch.z) sfo[act_sf_offset(tA, g4)] = uint8_t(sc & 0xFFu);
+                if (tB < ch.z) sfo[act_sf_offset(tB, g4)] = uint8_t(sc >> 8);
+                uint32_t pc[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) pc[m] = __shfl_xor_sync(0xFFFFFFFFu, cq[m], 1);
+                uint8_t *qbase = args.out_q + (int64_t(it >> 1) * args.rows + ch.y) * kTileK + (it & 1) * 64 +
+                                 q * 16 + (lane >> 1);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t code = (cq[j >> 3] >> (4 * (j & 7))) & 0xFu;
+                    const uint32_t partner = (pc[j >> 3] >> (4 * (j & 7))) & 0xFu;
+                    if (!(lane & 1) && cb * 32 + j < ch.z)
+                        qbase[int64_t(cb * 32 + j) * kTileK] = uint8_t(code | (partner << 4));
+                }
+            };
             // GEMM1 epilogue of 32 tokens: activation, scale, requantised h
             auto finish1 = [&](const uint32_t (&g)[32], const uint32_t (&u)[32], int cb) {
             float h[32];
             activate(g, u, h);
             if constexpr (kNv) {
-                float amx[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) amx[j] = fabsf(h[j]);
-                // NVFP4: groups of 16 rows of h = the two half-warps.  Lane l
-                // gets the amax of tokens cb*32 + l%16 and cb*32 + 16 + l%16 over
-                // its half-warp, and their UE4M3 scale codes.
-                float amA, amB;
-                halfwarp_transpose_max(amx, lane, amA, amB);
-                const uint32_t cA = nvfp4_scale_code(amA), cB = nvfp4_scale_code(amB);
-                const float sA = e4m3_mag_value(cA), sB = e4m3_mag_value(cB);
-                // GEMM2 reads h in 256-K blocks: this item's 128 rows are half
-                // `it % 2` of block it / 2; the warp's 32 rows are groups g4 =
-                // (q % 2) * 2 + half-warp of image (it % 2) * 2 + q / 2
-                const int img = (it & 1) * 2 + (q >> 1), g4 = (q & 1) * 2 + (lane >> 4);
-                uint8_t *sfo = args.out_sf + ((int64_t(c) * (n_tiles / 2) + it / 2) * kNvImages + img) * C::kActSf;
-                const int tA = cb * 32 + (lane & 15), tB = tA + 16;
-                if (tA < ch.z) sfo[act_sf_offset(tA, g4)] = uint8_t(cA);
-                if (tB < ch.z) sfo[act_sf_offset(tB, g4)] = uint8_t(cB);
-                // codes: row (ch.y + token) of block it / 2 holds this warp's 32
-                // values as bytes (it % 2) * 64 + q * 16 .. + 15, two per byte
-                uint8_t *qbase = args.out_q + (int64_t(it >> 1) * args.rows + ch.y) * kTileK + (it & 1) * 64 +
-                                 q * 16 + (lane >> 1);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, (lane & 16) | (j & 15));
-                    const uint32_t code = to_e2m1(__fdiv_rn(h[j], sj));
-                    const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
-                    if (!(lane & 1) && cb * 32 + j < ch.z)
-                        qbase[int64_t(cb * 32 + j) * kTileK] = uint8_t(code | (partner << 4));
-                }
+                uint32_t cq[4], sc;
+                quantize4(h, cq, sc);
+                store4(cq, sc, cb);
             } else {
                 uint32_t pq[8], sfb;
                 quantize8(h, pq, sfb);
@@ -749,16 +769,20 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) p[j * kTileRows] = __uint_as_float(v[j]);
             };
-            // Whole items (FP8 x FP4): only the work that reads the accumulator
-            // runs while the MMAs wait for it.  Each unit's results go to a few
-            // registers (GEMM1: 8 words of codes + the scale byte; GEMM2: 16
-            // words of bf16 pairs), the accumulator is released to the issuers,
-            // and then the units' global stores run, overlapping the next
-            // item's MMAs.
-            if (!kNv && !is_unit) {
+            // Whole items: only the work that reads the accumulator runs while
+            // the MMAs wait for it.  Each unit's results go to a few registers
+            // (GEMM1: the requantised codes and scales; GEMM2: 16 words of bf16
+            // pairs), the accumulator is released to the issuers, and then the
+            // units' global stores run, overlapping the next item's MMAs.
+            // (NVFP4's GEMM2 with 32-row chunks adds two K-split accumulators and
+            // keeps the per-unit path: no registers to spare.)
+            if (!is_unit && (!kNv || kGemm1 || !C::kSmall)) {
                 if constexpr (kGemm1) {
+                    // FP8: 8 words of codes + the scale byte per column block;
+                    // NVFP4: 4 words of codes + the two scale codes
                     constexpr int kU = ((kN + 31) / 32 + kCbStep - 1) / kCbStep;
-                    uint32_t pq[kU][8], sfb[kU];
+                    constexpr int kW = kNv ? 4 : 8;
+                    uint32_t pq[kU][kW], sfb[kU];
 #pragma unroll
                     for (int i = 0; i < kU; ++i) {
                         const int cb = half + i * kCbStep;
@@ -767,7 +791,10 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                             float h[32];
                             load_gu(cb, g, u);
                             activate(g, u, h);
-                            quantize8(h, pq[i], sfb[i]);
+                            if constexpr (kNv)
+                                quantize4(h, pq[i], sfb[i]);
+                            else
+                                quantize8(h, pq[i], sfb[i]);
                         }
                     }
                     tc_fence_before();
@@ -776,7 +803,12 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < kU; ++i) {
                         const int cb = half + i * kCbStep;
-                        if (cb < ncb) store8(pq[i], sfb[i], cb);
+                        if (cb < ncb) {
+                            if constexpr (kNv)
+                                store4(pq[i], sfb[i], cb);
+                            else
+                                store8(pq[i], sfb[i], cb);
+                        }
                     }
                 } else {
                     constexpr int kU = (kNumA * ((kN + 31) / 32) + kCbStep - 1) / kCbStep;
