@@ -90,7 +90,17 @@ struct GemmCfg {
     static constexpr int kSfColsIssuer = kNv ? (kImg / kKSplit) * (1 + kSfbImages) * 4
                                              : (kKB / kKSplit) * kImg * (1 + kSfbImages) * 4;
     static constexpr int kSfRegions = kNv ? 2 : kStages;
-    static constexpr int kSfCols = kSfRegions * kIssuers * kSfColsIssuer;
+    // NVFP4 with large chunks: a tcgen05 instruction costs its issuing thread
+    // a fixed time whatever its N, and a 256-K stage takes each issuer four
+    // MMAs and twelve scale copies, so the chunk's eight activation images
+    // leave the two MMA issuers: warp 6 copies them (the weight producer, warp
+    // 0, also loads the activations) into one TMEM region per stage slot that
+    // both issuers read; each issuer still copies its own tile's four images
+    // into the same region.  (The FP8 x FP4 kernels, with three copies per
+    // issuer and stage, measured no faster this way.)
+    static constexpr bool kCopier = !kSmall && kNv;
+    static constexpr int kSfColsSlot = kImg * kKB * (kNumA + kSfbImages) * 4;
+    static constexpr int kSfCols = kCopier ? kStages * kSfColsSlot : kSfRegions * kIssuers * kSfColsIssuer;
     static constexpr int kAccBufs = (2 * kAccCols + kSfCols) <= 512 ? 2 : 1;
     static constexpr int kTmemUsed = kAccBufs * kAccCols + kSfCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
@@ -104,7 +114,8 @@ struct GemmCfg {
     static constexpr int kBoxPackets = kNumA * kKB;
     static_assert(kTmemUsed <= 512, "TMEM budget");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
-    static_assert(8 * (2 * kStages + 10) + 12 <= kSmemMisc, "barriers and flags");
+    static_assert(8 * (3 * kStages + 11) + 12 <= kSmemMisc, "barriers and flags");
+    static_assert(!kCopier || (kNv && kKB == 1 && kKSplit == 1), "the copier's regions hold one K block per stage");
     static_assert(!kSmall || kN * kNumA * kTileRows == kPartUnitFloats, "split-unit partial size");
     static_assert(kBTile % 1024 == 0, "swizzle atoms");
     static_assert(kKB == 1 || kN == kActBoxRows, "one activation box per stage when a stage spans K blocks");
@@ -250,7 +261,9 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     uint64_t *mma_done = tmem_empty + 2;     // [kIssuers]
     uint64_t *epi_bar = mma_done + 4;        // split unit: epilogue warps' partials written
     uint64_t *epi_go = epi_bar + 1;          // split unit: the finishing decision taken
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(epi_go + 1);
+    uint64_t *sf_ready = epi_go + 1;         // [kStages] large chunks: the stage's scale images in TMEM
+    uint64_t *cp_done = sf_ready + kStages;  // large chunks: all of the copier's copies complete
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(cp_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     volatile int *epi_last = abort_flag + 1;
     uint8_t *epi_stage = reinterpret_cast<uint8_t *>(full) + C::kSmemMisc;  // [kEpiWarps][1024] (large chunks)
@@ -258,9 +271,11 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 2);  // weight producer + activation producer
+            mbar_init(&full[s], 2);  // weight copies + activation copies
             mbar_init(&empty[s], kIssuers);
+            mbar_init(&sf_ready[s], 1);
         }
+        mbar_init(cp_done, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tmem_full[b], kIssuers);
             mbar_init(&tmem_empty[b], C::kEpiWarps);
@@ -304,14 +319,15 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     const int issuer = warp == 1 ? 0 : warp == 7 ? 1 : (kIssuers == 4 && warp == 8) ? 2
                      : (kIssuers == 4 && warp == 9) ? 3 : -1;
 
-    if (warp == 0 || warp == 6) {
+    if (warp == 0 || (warp == 6 && !C::kCopier)) {
         if (lane == 0) {
             // ------------------------------------------------------------ producers
-            // warp 0: weight packets and their scale blocks (one box each per
-            // stage); warp 6: the chunk's activation K blocks (one 3D box of
-            // kKB K blocks x 32 rows per 32 rows) and their scale blocks.
-            const bool weights = warp == 0;
-            const uint64_t pol = weights ? policy_evict_first() : policy_evict_last();
+            // weight packets and their scale blocks (one box each per stage;
+            // warp 0), the chunk's activation K blocks (one 3D box of kKB K
+            // blocks x 32 rows per 32 rows) and their scale blocks (warp 6, or
+            // warp 0 as well with large chunks)
+            const bool weights = warp == 0, acts = C::kCopier || warp == 6;
+            const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0, fill_parity = 0;
@@ -329,7 +345,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 for (int step = s0; step < s1; ++step) {
                     const int kb0 = step * kKB;
                     const int nkb = min(kKB, KB - kb0);
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, weights ? 1 : 5)) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, acts && !weights ? 5 : 1)) {
                         ok = false;
                         break;
                     }
@@ -343,17 +359,18 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         const int pkt = int((int64_t(ch.x) * groups + it) * KB * 2 + int64_t(kb0) * 2);
                         if (kNv) {
                             // packed E2M1 bodies as bytes; scale images (128 words, image, packet)
-                            tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol);
-                            tma_load_3d(sf, &tmap_wsf, &full[stage], 0, 0, pkt, pol);
+                            tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol_w);
+                            tma_load_3d(sf, &tmap_wsf, &full[stage], 0, 0, pkt, pol_w);
                         } else {
                             if (args.w_rowmajor)
                                 tma_load_4d(st, &tmap_w, &full[stage], 0,
-                                            ch.x * args.w_rows_per_expert + it * args.w_item_rows, 0, kb0, pol);
+                                            ch.x * args.w_rows_per_expert + it * args.w_item_rows, 0, kb0, pol_w);
                             else
-                                tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol);
-                            tma_load_2d(sf, &tmap_wsf, &full[stage], args.w_sf_x0, pkt, pol);
+                                tma_load_4d(st, &tmap_w, &full[stage], 0, 0, 0, pkt / 2, pol_w);
+                            tma_load_2d(sf, &tmap_wsf, &full[stage], args.w_sf_x0, pkt, pol_w);
                         }
-                    } else {
+                    }
+                    if (acts) {
                         // the activation box always moves kKB K blocks (a K
                         // block past the end reads zeros); a nearly full large
                         // chunk takes one kN-row box instead of several 32-row ones
@@ -363,15 +380,15 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                                               uint32_t(rows_moved * kKB * kTileK + nkb * C::kImg * C::kActSf));
                         uint8_t *bt = st + kNumA * kKB * C::kATile;
                         if (one_box) {
-                            tma_load_3d(bt, &tmap_act_full, &full[stage], 0, ch.y, kb0, pol);
+                            tma_load_3d(bt, &tmap_act_full, &full[stage], 0, ch.y, kb0, pol_a);
                         } else {
                             for (int j = 0; j < nbox; ++j)
                                 tma_load_3d(bt + j * kActBoxRows * kTileK, &tmap_act, &full[stage], 0,
-                                            ch.y + j * kActBoxRows, kb0, pol);
+                                            ch.y + j * kActBoxRows, kb0, pol_a);
                         }
                         bulk_load(sf + C::kImg * kNumA * kKB * kSfBlockBytes,
                                   args.act_sf + (int64_t(c) * KB + kb0) * C::kImg * C::kActSf,
-                                  nkb * C::kImg * C::kActSf, &full[stage], pol);
+                                  nkb * C::kImg * C::kActSf, &full[stage], pol_a);
                     }
                     filled |= 1u << stage;
                     fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
@@ -388,6 +405,52 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 const unsigned long long t0 = global_timer_ns();
                 while (!mbar_try_wait(&full[s], par) && global_timer_ns() - t0 < kWaitTimeoutNs) {
                 }
+            }
+        }
+        __syncwarp();
+    } else if (C::kCopier && warp == 6) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ scale copier
+            // For every stage: once its data has landed, the chunk's activation
+            // scale images of the four 64-K steps go to the stage slot's TMEM
+            // region; the slot's previous MMAs are complete by then (the
+            // producer refilled it after their commits).
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int wk = 0; ok && wk < n_works; ++wk) {
+                int item, s0, s1;
+                work_of(P, wk, n_steps, item, s0, s1);
+                const int4 ch = __ldcg(args.chunks + item / n_items);
+                const int sfb_images = (ch.z + 15) / 16 * 16 > 128 ? 2 : 1;
+                for (int step = s0; step < s1; ++step) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, err, 9)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t *sfa = sfs + stage * C::kStageSf;
+                    const uint32_t col = tmem + uint32_t(kBufs * C::kAccCols + stage * C::kSfColsSlot);
+                    const uint8_t *sfb = sfa + kNumA * kNvImages * kSfBlockBytes;
+                    const uint32_t colb = col + kNumA * kNvImages * 4;
+#pragma unroll
+                    for (int j = 0; j < kNvImages; ++j)
+#pragma unroll
+                        for (int im = 0; im < C::kSfbImages; ++im)
+                            if (im < sfb_images)
+                                tc_cp_sf(colb + (j * C::kSfbImages + im) * 4,
+                                         smem_desc_sf(smem_u32(sfb + j * C::kActSf + im * kSfBlockBytes)));
+                    tc_commit(&sf_ready[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // the copies must be complete before TMEM is released
+            tc_commit(cp_done);
+            const unsigned long long t0 = global_timer_ns();
+            while (!mbar_try_wait(cp_done, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
             }
         }
         __syncwarp();
@@ -424,8 +487,33 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (C::kCopier && !mbar_wait(&sf_ready[stage], phase, abort_flag, err, 10)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    if (kNv && valid && gstage >= 2) {
+                    if (C::kCopier) {
+                        // this stage slot's region: the A images of both tiles (this
+                        // issuer copies its own four here), then the chunk's
+                        // activation images (from the copier)
+                        const uint8_t *st = tiles + stage * C::kStageTiles;
+                        const uint32_t col = tmem + uint32_t(kBufs * C::kAccCols + stage * C::kSfColsSlot);
+                        const uint64_t adesc = smem_desc_sw128(smem_u32(st + a * C::kATile));
+                        const uint64_t bdesc = smem_desc_sw128(smem_u32(st + kNumA * C::kATile));
+                        if (valid) {
+                            const uint8_t *sfa = sfs + stage * C::kStageSf;
+                            const uint32_t cola = col + a * kNvImages * 4, colb = col + kNumA * kNvImages * 4;
+#pragma unroll
+                            for (int j = 0; j < kNvImages; ++j)
+                                tc_cp_sf(cola + j * 4, smem_desc_sf(smem_u32(sfa + (a * kNvImages + j) * kSfBlockBytes)));
+#pragma unroll
+                            for (int j = 0; j < kNvImages; ++j)
+                                // 64 K (32 bytes) per step inside the 128-byte swizzled row, one image each
+                                tc_mma_nvf4(acc, adesc + uint64_t(2 * j), bdesc + uint64_t(2 * j), idesc_nvf4(n),
+                                            cola + j * 4, colb + j * C::kSfbImages * 4,
+                                            (step == s0 && j == 0) ? 0u : 1u);
+                        }
+                    } else if (kNv && valid && gstage >= 2) {
                         // this issuer's scale region was last read by the MMAs of stage
                         // gstage - 2: their commit has completed that stage's `empty` phase
                         const int g2 = gstage - 2;
@@ -435,7 +523,8 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                         }
                         tc_fence_after();
                     }
-                    if (kNv && valid) {
+                    if (C::kCopier) {
+                    } else if (kNv && valid) {
                         // this issuer's MMA steps ks = h * kSteps .. (h + 1) * kSteps - 1
                         // of the four, each with its weight and activation scale image
                         constexpr int kSteps = kNvImages / C::kKSplit;
