@@ -853,10 +853,13 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             };
             // a split unit's partial: [tile][kN columns][128 rows] fp32
             float *part = is_unit ? args.part + size_t(P.unit) * kPartUnitFloats : nullptr;
+            // (the chunk's real rows only: the item's last unit reads no others)
             auto put_part = [&](int a, int cb, const uint32_t (&v)[32]) {
                 float *p = part + size_t(a * kN + cb * 32) * kTileRows + q * 32 + lane;
+                const int nr = ch.z - cb * 32;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) p[j * kTileRows] = __uint_as_float(v[j]);
+                for (int j = 0; j < 32; ++j)
+                    if (j < nr) p[j * kTileRows] = __uint_as_float(v[j]);
             };
             // Whole items: only the work that reads the accumulator runs while
             // the MMAs wait for it.  Each unit's results go to a few registers
@@ -970,15 +973,45 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
             if (!mbar_wait(epi_go, 0, abort_flag, err, 8)) break;
             if (!*epi_last) continue;
             const float *p0 = args.part + size_t(P.unit / P.split) * P.split * kPartUnitFloats;
+            // tile a's sum over the units of column block cb, added in unit order;
+            // rows past the chunk's end read as zero.  A block of at most 8 real
+            // rows (decode) takes four units' loads per round.
             auto sum_part = [&](int a, int cb, uint32_t (&v)[32]) {
-                float acc_v[32];
                 const float *p = p0 + size_t(a * kN + cb * 32) * kTileRows + q * 32 + lane;
+                const int nr = ch.z - cb * 32;
+                if (nr <= 8) {
+                    float s8[8];
+#pragma unroll 1
+                    for (int sp0 = 0; sp0 < P.split; sp0 += 4) {
+                        float t[4][8];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc_v[j] = __ldcg(p + j * kTileRows);
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                t[i][j] = (sp0 + i < P.split && j < nr)
+                                              ? __ldcg(p + size_t(sp0 + i) * kPartUnitFloats + j * kTileRows)
+                                              : 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                if (sp0 + i == 0)
+                                    s8[j] = t[i][j];
+                                else if (sp0 + i < P.split)
+                                    s8[j] += t[i][j];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(j < 8 ? s8[j & 7] : 0.0f);
+                    return;
+                }
+                float acc_v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc_v[j] = j < nr ? __ldcg(p + j * kTileRows) : 0.0f;
                 for (int sp = 1; sp < P.split; ++sp) {
                     p += kPartUnitFloats;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc_v[j] += __ldcg(p + j * kTileRows);
+                    for (int j = 0; j < 32; ++j)
+                        if (j < nr) acc_v[j] += __ldcg(p + j * kTileRows);
                 }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(acc_v[j]);
