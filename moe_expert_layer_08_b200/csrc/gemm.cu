@@ -299,12 +299,16 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    // GEMM2's weights do not depend on GEMM1, so its producer streams the
-    // first stages' weight tiles before waiting for GEMM1 to finish; every
-    // other access to memory written by earlier kernels comes after pdl_wait.
-    const bool early_weights = !kGemm1;
-    const bool is_w_producer = warp == 0 && lane == 0;
-    if (!(early_weights && is_w_producer)) pdl_wait();
+    // The weights depend on neither kernel before this one (GEMM1: the gather;
+    // GEMM2: GEMM1), and the routing's chunk list had been written when that
+    // kernel started (it waited for the routing before letting this one
+    // launch), so the weight producer's warp streams its first stages before
+    // waiting; every other access to memory written by earlier kernels comes
+    // after pdl_wait.  The whole warp skips the wait: a lane waiting alone would
+    // hold lane 0 at the warp's reconvergence.  (With the scale-copy warp,
+    // warp 0 also loads the activations and waits.)
+    const bool early_weights = warp == 0 && !C::kCopier;
+    if (!early_weights) pdl_wait();
     if (threadIdx.x == 32) pdl_trigger();
 
     const int n_tiles = args.n_tiles, n_items = args.n_items;
