@@ -151,6 +151,9 @@ struct GemmArgs {
     int act_kind;              // GEMM1: MOE_ACT_SWIGLU or MOE_ACT_SITU
     float beta, inv_beta;      // SiTU coefficients (inv_lbeta = 0: no linear coefficient)
     float lbeta, inv_lbeta;
+    // 1: the previous kernel is the main list's launch of this GEMM, which writes
+    // nothing this launch reads: wait for it at the end, not the start
+    int overlap_prev;
 };
 
 // After the call lane l holds, over the 16 lanes of its half-warp, the max of
@@ -307,8 +310,12 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
     // after pdl_wait.  The whole warp skips the wait: a lane waiting alone would
     // hold lane 0 at the warp's reconvergence.  (With the scale-copy warp,
     // warp 0 also loads the activations and waits.)
+    // A side-list launch (after the main list's launch of the same GEMM) uses
+    // nothing that launch writes: it starts at once, overlapping its tail, and
+    // waits at its end instead, so that it completes after it (what the next
+    // kernel's wait relies on).
     const bool early_weights = warp == 0 && !C::kCopier;
-    if (!early_weights) pdl_wait();
+    if (!early_weights && !args.overlap_prev) pdl_wait();
     if (threadIdx.x == 32) pdl_trigger();
 
     const int n_tiles = args.n_tiles, n_items = args.n_items;
@@ -1039,6 +1046,7 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
         }
     }
 
+    if (args.overlap_prev) pdl_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1103,6 +1111,7 @@ cudaError_t launch_gemm(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap
     a.chunks = reinterpret_cast<const int4 *>(ws + (side ? L.off_chunks_s : L.off_chunks));
     a.hdr = reinterpret_cast<int *>(ws);
     a.chunks_word = side ? kHdrNumChunksSide : kHdrNumChunks;
+    a.overlap_prev = side ? 1 : 0;
     a.part = reinterpret_cast<float *>(ws + L.off_part);
     a.split_cnt = a.hdr + (gemm1 ? kHdrSplitCnt1 : kHdrSplitCnt2);
     a.rows = int(L.Rp);
