@@ -743,13 +743,16 @@ __global__ void __launch_bounds__(GemmCfg<kGemm1, kN, kNv>::kThreads, 1)
                 halfwarp_transpose_max(amx, lane, amA, amB);
                 const uint32_t cA = nvfp4_scale_code(amA), cB = nvfp4_scale_code(amB);
                 const float sA = e4m3_mag_value(cA), sB = e4m3_mag_value(cB);
+                const float rA = __frcp_rn(sA), rB = __frcp_rn(sB);
                 sc = cA | (cB << 8);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) cq[m] = 0u;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, (lane & 16) | (j & 15));
-                    cq[j >> 3] |= to_e2m1(__fdiv_rn(h[j], sj)) << (4 * (j & 7));
+                    const int src = (lane & 16) | (j & 15);
+                    const float sj = __shfl_sync(0xFFFFFFFFu, j < 16 ? sA : sB, src);
+                    const float rj = __shfl_sync(0xFFFFFFFFu, j < 16 ? rA : rB, src);
+                    cq[j >> 3] |= to_e2m1(nvfp4_quotient(h[j], sj, rj)) << (4 * (j & 7));
                 }
             };
             // Stores of quantize4's results for column block cb: the two scale

@@ -153,6 +153,25 @@ __device__ __forceinline__ uint32_t nvfp4_scale_code(float amax) {
     return c;
 }
 
+// h / s rounded to nearest (the fp32 quotient an E2M1 code is taken from),
+// for an UE4M3 scale s > 0 and r = RN(1 / s), without a division per value:
+// q0 = RN(h r), then one correction from the exact remainder h - q0 s (an
+// FMA), q = RN(q0 + (h - q0 s) r) -- the reciprocal-based correction step of
+// P. Markstein, "IA-64 and Elementary Functions" (2000), ch. 8.  An exhaustive
+// GPU comparison with the IEEE division (all 126 nonzero UE4M3 magnitudes,
+// every fp32 h with 2^-60 <= |h| < 2^101) found no difference.  Outside that
+// range, and where |q0| >= 8, the last bits cannot change the E2M1 code:
+// there q0 itself is used (|h / s| < 2^-51 rounds to a zero code with the sign
+// of h), clamped to +-8 (which saturates to the largest code like any
+// quotient above 6).
+__device__ __forceinline__ float nvfp4_quotient(float h, float s, float r) {
+    const float q0 = __fmul_rn(h, r);
+    const float rem = __fmaf_rn(-q0, s, h);
+    const float q = __fmaf_rn(rem, r, q0);
+    const bool exact = fabsf(h) >= 0x1p-60f && fabsf(q0) < 8.0f;
+    return exact ? q : fminf(fmaxf(q0, -8.0f), 8.0f);
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
