@@ -17,12 +17,16 @@
 //   warp 6 (one thread): activation producer.  The chunk's FP8 rows, stored
 //     K-block-major, as 3D boxes (32-row boxes, or one kN-row box for a nearly
 //     full large chunk) and the chunk's scale images by a bulk copy; they are
-//     re-read by every tile of the chunk (evict-last).
+//     re-read by every tile of the chunk (evict-last).  NVFP4 with large
+//     chunks: warp 0 loads the activations too, and warp 6 copies each
+//     stage's activation scale images into TMEM for both issuers.
 //   warps 1 and 7 (and 8, 9 with K split; one thread each): MMA issuers, one
 //     per tile (and K half): tcgen05.cp of the stage's scale images into TMEM,
 //     then tcgen05.mma.kind::mxf8f6f4.block_scale (K = 32 each) or
 //     kind::mxf4nvf4 (K = 64); tcgen05.commit releases the stage and, after
 //     the item's last stage, hands the accumulator to the epilogue.
+//   The weight producer's warp streams before the grid-dependency wait; a
+//   side-list launch waits at its end instead of its start.
 //   warps 2-5 (and 8-11 for large chunks): epilogue, TMEM -> registers (thread
 //     = weight row, registers = 32 tokens).  GEMM1: h = silu(gate) * up (or
 //     SiTU), per-token amax over each 32-row group (a warp) by a transposing
