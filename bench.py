@@ -85,7 +85,7 @@ def run_shared(args, rank, world, local_rank):
     T = args.shared_expert
     SH, SI = (int(v) for v in args.shared_dims.split(","))
     x, l1, l2 = W.gen_shared(T, SH, SI, 1, device)
-    ws = torch.empty(moe.shared_workspace_bytes(T, SH, SI), dtype=torch.uint8, device=device)
+    ws = moe.shared_workspace(T, SH, SI, device)
     out = torch.empty((T, SH), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -430,11 +430,16 @@ moe_status_t moe_probe_wait_timeout(void *workspace, size_t ws_bytes, unsigned t
  *   aligned; workspace 256-byte aligned, ws_bytes >= moe_shared_workspace_bytes
  *   (T, SH, SI) (else MOE_ERR_WORKSPACE_TOO_SMALL).  activation NULL means
  *   SwiGLU.  The caller owns every buffer; the call allocates nothing,
- *   enqueues a 2 KiB memset of the workspace header and two kernels on
- *   `stream`, and does not synchronise.  T = 0 enqueues nothing.  Argument
- *   errors (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE) are returned
- *   before any CUDA call; a device-side wait that times out is reported by
- *   moe_check_device_error(workspace) as MOE_ERR_DEVICE_TIMEOUT.
+ *   enqueues two kernels on `stream` (nothing else, so the first can start
+ *   under the tail of the preceding kernel), and does not synchronise.
+ *   T = 0 enqueues nothing.  The workspace must be zero-filled (e.g. by
+ *   cudaMemsetAsync) before its first use by this entry point, and again
+ *   after any other use of the same memory; every call leaves it ready for
+ *   the next one, a call that timed out included.  Argument errors
+ *   (MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE) are returned before any
+ *   CUDA call; a device-side wait that times out is reported by
+ *   moe_check_device_error(workspace) as MOE_ERR_DEVICE_TIMEOUT (the word
+ *   holds the status of the last call).
  */
 moe_status_t moe_shared_workspace_bytes(int T_max, int SH, int SI, size_t *bytes);
 moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const void *l2_bf16,

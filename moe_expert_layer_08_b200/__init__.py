@@ -21,7 +21,7 @@ __all__ = [
     "forward_static", "check_device_error_static", "STATIC_WORKSPACE_BYTES", "Activation", "activation", "forward_kernel_launches",
     "Weights", "RowMajorWeights", "transformed_scale_bytes", "transform_scales", "LAYOUT_PACKETS",
     "LAYOUT_ROW_MAJOR", "quantize_nvfp4", "transformed_weight_bytes_nvfp4", "transform_weights_nvfp4",
-    "forward_nvfp4", "shared_workspace_bytes", "shared_forward", "probe_wait_timeout",
+    "forward_nvfp4", "shared_workspace_bytes", "shared_workspace", "shared_forward", "probe_wait_timeout",
     "ep_workspace_bytes", "ep_dispatch", "ep_combine", "ep_combine_peers", "ep_route", "ep_dispatch_peers",
     "ipc_handle", "ipc_open", "ipc_close", "IPC_HANDLE_BYTES",
 ]
@@ -419,10 +419,17 @@ def shared_workspace_bytes(T_max: int, SH: int, SI: int) -> int:
     return n.value
 
 
+def shared_workspace(T_max: int, SH: int, SI: int, device):
+    """A zero-filled workspace for shared_forward (the state its first use
+    needs; every call leaves it ready for the next)."""
+    return torch.zeros(shared_workspace_bytes(T_max, SH, SI), dtype=torch.uint8, device=device)
+
+
 def shared_forward(x, l1, l2, out=None, workspace=None, act=None, stream=None):
     """The BF16 shared expert: x [T, SH], l1 [2 SI, SH] (gate rows first), l2
     [SH, SI], all bf16; returns y (bf16 [T, SH]).  ``act``: an Activation, None
-    = SwiGLU."""
+    = SwiGLU.  ``workspace``: from shared_workspace (zero-filled before its
+    first use); None allocates one for this call."""
     _need(x, torch.bfloat16, "x", 2)
     _need(l1, torch.bfloat16, "l1", 2)
     _need(l2, torch.bfloat16, "l2", 2)
@@ -435,7 +442,7 @@ def shared_forward(x, l1, l2, out=None, workspace=None, act=None, stream=None):
     else:
         _need(out, torch.bfloat16, "out", 2)
     if workspace is None:
-        workspace = torch.empty(shared_workspace_bytes(T, SH, SI), dtype=torch.uint8, device=x.device)
+        workspace = shared_workspace(T, SH, SI, x.device)
     else:
         _need(workspace, torch.uint8, "workspace")
     st = load().moe_shared_forward(_ptr(x), _ptr(l1), _ptr(l2), _ptr(out), T, SH, SI,

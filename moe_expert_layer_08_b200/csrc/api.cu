@@ -683,9 +683,10 @@ moe_status_t moe_shared_forward(const void *x_bf16, const void *l1_bf16, const v
         return MOE_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int *hdr = reinterpret_cast<int *>(ws);
-    cudaError_t e = cudaMemsetAsync(ws, 0, kHdrBytes, st);  // error word of this call
+    // no memset: GEMM1 clears the error word, each GEMM the other's split
+    // counters (the workspace is zero-filled before its first use)
     float *part = reinterpret_cast<float *>(ws + kHdrBytes + shared_h_bytes(T, SI));
-    if (e == cudaSuccess) e = launch_shared(true, tm_l1, tm_x, T, SH, SI, h, hdr, part, act, st);
+    cudaError_t e = launch_shared(true, tm_l1, tm_x, T, SH, SI, h, hdr, part, act, st);
     if (e == cudaSuccess) e = launch_shared(false, tm_l2, tm_h, T, SH, SI, out_bf16, hdr, part, act, st);
     return cuda_status(e);
 }

@@ -50,6 +50,8 @@ struct SharedArgs {
     int split;         // K parts per item (1: none); parts > 1 only with 32-token blocks
     float *part;       // split: fp32 partial accumulators [unit][tile][32 tokens][128 rows]
     int *cnt;          // split: per item, parts finished (the last resets it)
+    int *cnt_clear;    // the other GEMM's split counters (kHdrSplitWords), zeroed here
+    int clear_err;     // GEMM1: zero the error word of this call
     int act_kind;      // GEMM1: MOE_ACT_SWIGLU or MOE_ACT_SITU
     float beta, inv_beta, lbeta, inv_lbeta;
 };
@@ -105,6 +107,23 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     // ring before GEMM1 has finished; every other access to memory written by
     // earlier kernels comes after pdl_wait
     if (kGemm1 || warp != 0) pdl_wait();
+    if (blockIdx.x == 0 && warp == 1) {
+        // The call's header upkeep, in place of a memset before the first
+        // kernel (which would keep GEMM1 from starting under the previous
+        // kernel's tail): GEMM1 clears the error word of this call, and each
+        // GEMM clears the other's split counters (nonzero only after a call
+        // that timed out). The kernel that used them last has completed
+        // (griddepcontrol.wait above), and the next one to use them reads them
+        // only after its own wait; the stores are fenced before the trigger
+        // that lets the next kernel launch.
+        for (int i = lane; i < kHdrSplitWords; i += 32) args.cnt_clear[i] = 0;
+        if (args.clear_err && lane == 0) {
+            args.hdr[kHdrError] = 0;
+            args.hdr[kHdrTimeoutWhere] = 0;
+        }
+        __threadfence();
+        __syncwarp();
+    }
     if (threadIdx.x == 32) pdl_trigger();
 
     const int n_items = args.n_items, n_tiles = args.n_tiles;
@@ -408,7 +427,11 @@ cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorM
     a.T = T;
     a.hdr = hdr;
     a.part = part;
-    a.cnt = hdr + kHdrSplitCnt1;  // per item; zeroed with the header, reset by each item's last part
+    // per item, reset by each item's last part; the other GEMM's counters are
+    // cleared by this one (see the kernel)
+    a.cnt = hdr + (gemm1 ? kHdrSplitCnt1 : kHdrSplitCnt2);
+    a.cnt_clear = hdr + (gemm1 ? kHdrSplitCnt2 : kHdrSplitCnt1);
+    a.clear_err = gemm1 ? 1 : 0;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.act_kind = act.kind;
     a.beta = act.beta;

@@ -28,7 +28,7 @@ def bits(t: torch.Tensor) -> np.ndarray:
 def run_and_compare(moe, T, SH, SI, seed, tokens=None, situ=None, repeat=True):
     x, l1, l2 = W.gen_shared(T, SH, SI, seed, "cuda")
     act = None if situ is None else moe.activation("situ", situ[0], situ[1])
-    ws = torch.empty(moe.shared_workspace_bytes(T, SH, SI), dtype=torch.uint8, device="cuda")
+    ws = moe.shared_workspace(T, SH, SI, "cuda")
     y = moe.shared_forward(x, l1, l2, workspace=ws, act=act)
     assert moe.check_device_error(ws) == 0
     if repeat:
@@ -79,3 +79,30 @@ def test_shared_split_ragged_blocks(moe):
     """T = 40 at full size: two 32-token blocks (32 and 8 rows), each item's K
     cut into an even number of parts."""
     run_and_compare(moe, 40, 7168, 2048, 10)
+
+
+def test_shared_workspace_reuse(moe):
+    """One zero-filled workspace through calls of different token counts
+    (K-split and unsplit, both token-block sizes) and activations, then
+    through a header as a call whose GEMM2 timed out leaves it (error word
+    set, GEMM2's split counters at header words 192..319 nonzero): every
+    result is bit-identical to a call on a fresh workspace, and the error word
+    reports each call's own status."""
+    SH, SI = 1024, 512
+    ws = moe.shared_workspace(1100, SH, SI, "cuda")
+    situ = moe.activation("situ", 1.25, 1.5)
+    for T, act, seed in [(8, None, 11), (300, situ, 12), (8, situ, 13), (40, None, 14), (1100, None, 15),
+                         (1, None, 16), (8, None, 11)]:
+        x, l1, l2 = W.gen_shared(T, SH, SI, seed, "cuda")
+        fresh = moe.shared_forward(x, l1, l2, workspace=moe.shared_workspace(T, SH, SI, "cuda"), act=act)
+        got = moe.shared_forward(x, l1, l2, workspace=ws, act=act)
+        assert moe.check_device_error(ws) == 0
+        assert torch.equal(got.view(torch.int16), fresh.view(torch.int16)), f"T={T}"
+    hdr = ws[:2048].view(torch.int32)
+    hdr[0] = 2  # the timeout bit
+    hdr[192:320] = 7
+    x, l1, l2 = W.gen_shared(8, SH, SI, 17, "cuda")
+    fresh = moe.shared_forward(x, l1, l2, workspace=moe.shared_workspace(8, SH, SI, "cuda"))
+    got = moe.shared_forward(x, l1, l2, workspace=ws)
+    assert moe.check_device_error(ws) == 0
+    assert torch.equal(got.view(torch.int16), fresh.view(torch.int16))
