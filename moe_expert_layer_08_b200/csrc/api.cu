@@ -638,9 +638,7 @@ moe_status_t moe_probe_wait_timeout(void *workspace, size_t ws_bytes, unsigned t
 // ---------------------------------------------------------------- BF16 shared expert
 // header (error word, split counters), h [T][SI] bf16, K-split partial sums
 static size_t shared_h_bytes(int T, int SI) { return align_up(size_t(T) * size_t(SI) * 2, 256); }
-static size_t shared_ws_bytes(int T, int SI) {
-    return kHdrBytes + shared_h_bytes(T, SI) + size_t(kMaxSplitUnits) * kPartUnitFloats * sizeof(float);
-}
+static size_t shared_ws_bytes(int T, int SI) { return kHdrBytes + shared_h_bytes(T, SI) + shared_part_bytes(T); }
 
 moe_status_t moe_shared_workspace_bytes(int T_max, int SH, int SI, size_t *bytes) {
     if (!bytes || T_max < 0 || SH <= 0 || SI <= 0) return MOE_ERR_INVALID_ARG;

@@ -94,9 +94,10 @@ cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *to
 // else 128) and the launch of GEMM1 (tmap_w over L1 [2SI][SH], tmap_act over x
 // [T][SH], out = h [T][SI]) or GEMM2 (L2 [SH][SI], h, out = y [T][SH]); the
 // maps' boxes are 128 / shared_block_rows(T) rows of 64 bf16.  part: scratch
-// of kMaxSplitUnits x kPartUnitFloats floats for K-split partial sums.
-constexpr int kSharedSmallT = 256;
+// of shared_part_bytes(T) bytes for K-split partial sums.
+constexpr int kSharedSmallT = 128;
 int shared_block_rows(int T);
+size_t shared_part_bytes(int T);
 cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, int T, int SH, int SI,
                           void *out, int *hdr, float *part, const moe_activation_t &act, cudaStream_t stream);
 // Tensor map of a row-major bf16 matrix [rows][cols]: boxes of 64 columns

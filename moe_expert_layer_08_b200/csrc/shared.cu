@@ -38,6 +38,17 @@ struct SharedCfg {
     static_assert(8 * (2 * kStages + 8) + 12 <= kSmemMisc, "barriers and flags");
 };
 
+// K-split partial sums: one unit holds a part's fp32 accumulators of both
+// tiles of its item, [tile][token][128 rows]; the scratch holds 256 units of
+// 32-token blocks (8 MiB) or 160 of 128-token blocks (20 MiB), and no split
+// needs more (about one unit per SM)
+template <int kN>
+constexpr int kSharedPartUnitFloats = 2 * kN * kTileRows;
+constexpr int kSharedMaxUnits32 = 256;
+constexpr int kSharedMaxUnits128 = 160;
+static_assert(kSharedMaxUnits32 / 2 <= kHdrSplitWords && kSharedMaxUnits128 / 2 <= kHdrSplitWords,
+              "a split item's counter in the header");
+
 struct SharedArgs {
     int T;             // tokens
     int K;             // reduction length (SH for GEMM1, SI for GEMM2)
@@ -47,8 +58,8 @@ struct SharedArgs {
     int out_ld;        // row length of the output (SI or SH)
     __nv_bfloat16 *out;
     int *hdr;          // workspace header (error word)
-    int split;         // K parts per item (1: none); parts > 1 only with 32-token blocks
-    float *part;       // split: fp32 partial accumulators [unit][tile][32 tokens][128 rows]
+    int split;         // K parts per item (1: none)
+    float *part;       // split: fp32 partial accumulators [unit][tile][kN tokens][128 rows]
     int *cnt;          // split: per item, parts finished (the last resets it)
     int *cnt_clear;    // the other GEMM's split counters (kHdrSplitWords), zeroed here
     int clear_err;     // GEMM1: zero the error word of this call
@@ -58,7 +69,7 @@ struct SharedArgs {
 
 __device__ __forceinline__ float bf16_round_f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
-template <bool kGemm1, int kN>
+template <bool kGemm1, int kN, bool kSplit>
 __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     shared_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_act,
                        const SharedArgs args) {
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     const int num_items = n_blocks * n_items;
     const int KB = args.K / 64;  // K blocks of 64 bf16 (128 bytes)
     // work units: item u / split, K blocks [kb_lo(u), kb_hi(u)) of its K
-    const int split = kN == 32 ? args.split : 1;
+    const int split = kSplit ? args.split : 1;
     const int num_units = num_items * split;
     auto kb_lo = [&](int u) { return (u % split) * KB / split; };
     auto kb_hi = [&](int u) { return (u % split + 1) * KB / split; };
@@ -316,21 +327,26 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 if (lane == 0) mbar_arrive(&tmem_empty[buf]);
                 continue;
             }
-            // K part of an item (32-token blocks: one column block): write this
-            // part's fp32 accumulators of the block's real tokens; the item's
-            // last part to finish adds the parts 0 .. split-1 in that order and
-            // runs the epilogue, so the result does not depend on which part
-            // ends last
-            if constexpr (kN == 32) {
-                float *pu = args.part + size_t(uu) * kPartUnitFloats + q * 32 + lane;
+            // K part of an item: write this part's fp32 accumulators of the
+            // block's real tokens (each warp its lane quarter of its column
+            // blocks); the item's last part to finish adds the parts 0 ..
+            // split-1 in that order and runs the epilogue, so the result does
+            // not depend on which part ends last
+            if constexpr (kSplit) {
+                constexpr int kUnit = kSharedPartUnitFloats<kN>;
+                const int ncb = (rows + 31) / 32;
+                float *pu = args.part + size_t(uu) * kUnit + q * 32 + lane;
 #pragma unroll 1
-                for (int a = 0; a < 2; ++a) {
-                    uint32_t v[32];
-                    tmem_ld_32x32(acc + uint32_t(a * kN), v);
-                    tmem_ld_wait();
+                for (int cb = half; cb < ncb; cb += kCbStep) {
+#pragma unroll 1
+                    for (int a = 0; a < 2; ++a) {
+                        uint32_t v[32];
+                        tmem_ld_32x32(acc + uint32_t(a * kN + cb * 32), v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (j < rows) pu[(a * 32 + j) * kTileRows] = __uint_as_float(v[j]);
+                        for (int j = 0; j < 32; ++j)
+                            if (cb * 32 + j < rows) pu[(a * kN + cb * 32 + j) * kTileRows] = __uint_as_float(v[j]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -355,10 +371,10 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                 // the parts' sums, 8 tokens at a time, added in part order 0 ..
                 // split-1 (the loads of four parts in flight together); then the
                 // block's epilogue
-                const float *p0 = args.part + size_t(item) * split * kPartUnitFloats + q * 32 + lane;
+                const float *p0 = args.part + size_t(item) * split * kUnit + q * 32 + lane;
 #pragma unroll 1
-                for (int jb = 0; jb * 8 < rows; ++jb) {
-                    const float *pj = p0 + jb * 8 * kTileRows;
+                for (int jt = half * 32; jt < rows; jt += (jt & 31) == 24 ? 8 + 32 * (kCbStep - 1) : 8) {
+                    const float *pj = p0 + jt * kTileRows;
                     uint32_t sv[2][8];
                     float s_[2][8];
 #pragma unroll 1
@@ -370,8 +386,8 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                             for (int a = 0; a < 2; ++a)
 #pragma unroll
                                 for (int j = 0; j < 8; ++j)
-                                    t[i][a][j] = sp0 + i < split ? __ldcg(pj + size_t(sp0 + i) * kPartUnitFloats +
-                                                                          (a * 32 + j) * kTileRows)
+                                    t[i][a][j] = sp0 + i < split ? __ldcg(pj + size_t(sp0 + i) * kUnit +
+                                                                          (a * kN + j) * kTileRows)
                                                                  : 0.0f;
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
@@ -388,12 +404,12 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
                     for (int a = 0; a < 2; ++a)
 #pragma unroll
                         for (int j = 0; j < 8; ++j) sv[a][j] = __float_as_uint(s_[a][j]);
-                    const int tok0 = blk * kN + jb * 8;
+                    const int tok0 = blk * kN + jt;
                     if constexpr (kGemm1) {
-                        finish1(sv[0], sv[1], tok0, rows - jb * 8, it);
+                        finish1(sv[0], sv[1], tok0, rows - jt, it);
                     } else {
-                        finish2(sv[0], tok0, rows - jb * 8, 2 * it);
-                        if (2 * it + 1 < n_tiles) finish2(sv[1], tok0, rows - jb * 8, 2 * it + 1);
+                        finish2(sv[0], tok0, rows - jt, 2 * it);
+                        if (2 * it + 1 < n_tiles) finish2(sv[1], tok0, rows - jt, 2 * it + 1);
                     }
                 }
             }
@@ -406,20 +422,25 @@ __global__ void __launch_bounds__(SharedCfg<kN>::kThreads, 1)
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <bool kGemm1, int kN>
+template <bool kGemm1, int kN, bool kSplit>
 static cudaError_t launch_shared_t(const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, const SharedArgs &a,
                                    int items, cudaStream_t stream) {
     using C = SharedCfg<kN>;
     const cudaError_t e =
-        set_max_dynamic_smem(reinterpret_cast<const void *>(shared_gemm_kernel<kGemm1, kN>), C::kSmemBytes);
+        set_max_dynamic_smem(reinterpret_cast<const void *>(shared_gemm_kernel<kGemm1, kN, kSplit>), C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int sms = num_sms();
     const int grid = items < sms ? (items > 0 ? items : 1) : sms;
-    return launch_pdl(shared_gemm_kernel<kGemm1, kN>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
+    return launch_pdl(shared_gemm_kernel<kGemm1, kN, kSplit>, dim3(grid), dim3(C::kThreads), size_t(C::kSmemBytes), stream,
                       tmap_w, tmap_act, a);
 }
 
 int shared_block_rows(int T) { return T <= kSharedSmallT ? 32 : 128; }
+
+size_t shared_part_bytes(int T) {
+    return shared_block_rows(T) == 32 ? size_t(kSharedMaxUnits32) * kSharedPartUnitFloats<32> * sizeof(float)
+                                      : size_t(kSharedMaxUnits128) * kSharedPartUnitFloats<128> * sizeof(float);
+}
 
 cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, int T, int SH, int SI,
                           void *out, int *hdr, float *part, const moe_activation_t &act, cudaStream_t stream) {
@@ -453,22 +474,29 @@ cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorM
     }
     const int kn = shared_block_rows(T);
     const int items = (T + kn - 1) / kn * a.n_items;
-    // 32-token blocks with fewer items than SMs: cut each item's K into parts
-    // (at least four 64-element K blocks each) so that about every SM works
+    // fewer items than SMs: cut each item's K into parts (at least four
+    // 64-element K blocks each) so that about every SM works, as many units
+    // as the partial-sum scratch holds
     const int sms = num_sms();
+    const int max_units = kn == 32 ? kSharedMaxUnits32 : kSharedMaxUnits128;
     a.split = 1;
-    if (kn == 32 && items < sms) {
+    if (items < sms) {
         int s = sms / items;
         if (s > (a.K / 64) / 4) s = (a.K / 64) / 4;
-        if (s > kMaxSplitUnits / items) s = kMaxSplitUnits / items;
+        if (s > max_units / items) s = max_units / items;
         a.split = s > 1 ? s : 1;
     }
     const int units = items * a.split;
+    // 32-token blocks: one kernel for both; 128-token blocks: the K-split
+    // epilogue only in the kernel that needs it
     if (kn == 32)
-        return gemm1 ? launch_shared_t<true, 32>(tmap_w, tmap_act, a, units, stream)
-                     : launch_shared_t<false, 32>(tmap_w, tmap_act, a, units, stream);
-    return gemm1 ? launch_shared_t<true, 128>(tmap_w, tmap_act, a, items, stream)
-                 : launch_shared_t<false, 128>(tmap_w, tmap_act, a, items, stream);
+        return gemm1 ? launch_shared_t<true, 32, true>(tmap_w, tmap_act, a, units, stream)
+                     : launch_shared_t<false, 32, true>(tmap_w, tmap_act, a, units, stream);
+    if (a.split > 1)
+        return gemm1 ? launch_shared_t<true, 128, true>(tmap_w, tmap_act, a, units, stream)
+                     : launch_shared_t<false, 128, true>(tmap_w, tmap_act, a, units, stream);
+    return gemm1 ? launch_shared_t<true, 128, false>(tmap_w, tmap_act, a, units, stream)
+                 : launch_shared_t<false, 128, false>(tmap_w, tmap_act, a, units, stream);
 }
 
 }  // namespace moe

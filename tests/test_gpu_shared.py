@@ -1,8 +1,9 @@
 """GPU parity of the BF16 shared expert (moe_shared_forward through the C ABI)
 against the oracle, per token row: rel L2 <= 1e-2 and max abs <= 5e-2 *
 max|row| (the DeepGEMM PR #416 test body bounds the shared output's relative
-L2 by 1e-2).  Small cases on every token, with both token-block sizes (32 up
-to 256 tokens, else 128), ragged token counts and an odd output-tile count;
+L2 by 1e-2).  Small cases on every token, with both token-block sizes (32-token
+blocks up to T = 128, else 128-token blocks), with and without a K split,
+ragged token counts and an odd output-tile count;
 the full-size case on sampled tokens."""
 import numpy as np
 import pytest
@@ -46,7 +47,7 @@ def run_and_compare(moe, T, SH, SI, seed, tokens=None, situ=None, repeat=True):
     (37, 512, 256, 2),       # ragged 32-token blocks
     (300, 384, 256, 3),      # odd output-tile count: GEMM2's last pair holds one tile
     (1100, 256, 128, 4),     # 128-token blocks, ragged last block
-    (250, 256, 256, 8),      # 32-token blocks at the largest such T
+    (128, 256, 256, 8),      # 32-token blocks at the largest such T
 ])
 def test_shared_small(moe, T, SH, SI, seed):
     run_and_compare(moe, T, SH, SI, seed)
@@ -106,3 +107,24 @@ def test_shared_workspace_reuse(moe):
     got = moe.shared_forward(x, l1, l2, workspace=ws)
     assert moe.check_device_error(ws) == 0
     assert torch.equal(got.view(torch.int16), fresh.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,SH,SI,seed,situ", [
+    (300, 1024, 512, 18, None),          # 128-token blocks (128, 128, 44 rows), both GEMMs K-split
+    (600, 640, 384, 19, None),           # odd output-tile count, GEMM1 split in two
+    (290, 512, 1024, 20, (1.25, 1.5)),   # SiTU on the 128-token split path
+    (129, 1024, 512, 22, None),          # the smallest such T: a last block of one token
+])
+def test_shared_split_128_token_blocks(moe, T, SH, SI, seed, situ):
+    """More than 128 tokens (128-token blocks) with fewer work items than SMs:
+    each item's K is cut into parts whose fp32 partials (128 tokens per block)
+    the item's last part adds in part order; every token checked."""
+    run_and_compare(moe, T, SH, SI, seed, situ=situ)
+
+
+def test_shared_split_128_full_size_sampled(moe):
+    """T = 300 at SH = 7168, SI = 2048 (GEMM1 split three ways over 48 items),
+    16 sampled tokens from every block, the last included."""
+    T = 300
+    tokens = sorted(set(np.random.default_rng(21).choice(T, 13, replace=False).tolist()) | {0, 255, T - 1})
+    run_and_compare(moe, T, 7168, 2048, 21, tokens=tokens)
