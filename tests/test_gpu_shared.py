@@ -128,3 +128,10 @@ def test_shared_split_128_full_size_sampled(moe):
     T = 300
     tokens = sorted(set(np.random.default_rng(21).choice(T, 13, replace=False).tolist()) | {0, 255, T - 1})
     run_and_compare(moe, T, 7168, 2048, 21, tokens=tokens)
+
+
+def test_shared_split_global_partials(moe):
+    """An item cut into more K parts than a thread-block cluster holds (T = 8,
+    SH = 7168, SI = 128: one GEMM1 item in 28 parts) adds its partials through
+    global memory, the last part to finish reducing them."""
+    run_and_compare(moe, 8, 7168, 128, 23)
