@@ -92,3 +92,27 @@ def test_both_arms_print_the_same_config_keys():
         assert set(a) == {"workload", "T", "E", "k", "H", "I", "seed", "routing", "parallelism",
                           "weight_layout", "l2"}
         assert a["workload"] == w.name and a["parallelism"] == "replicas x1"
+
+
+def test_shared_roofline_takes_the_binding_bound():
+    """The shared expert's roofline: HBM (its bf16 weights read once) while
+    that takes longer than the FLOPs at the tensor peak, else the tensor pipe;
+    the fraction is achieved / peak in the bound's unit, the other beside it."""
+    pk = dict(hbm=6000.0, bf16=1600.0, bf16_sustained=1200.0, source="measured")
+    wbytes = 3 * 7168 * 2048 * 2
+    for T, us in [(8, 40.0), (8192, 600.0)]:
+        flops = 2.0 * T * 3 * 7168 * 2048
+        r = bench.shared_roofline(flops, wbytes, us * 1e-3, pk)
+        t_hbm, t_tc = wbytes / 6000e9, flops / 1200e12
+        assert r["bound"] == ("hbm" if t_hbm > t_tc else "tensor")
+        assert r["other"]["bound"] == ("tensor" if t_hbm > t_tc else "hbm")
+        tf = flops / (us * 1e-6) / 1e12
+        gbps = wbytes / (us * 1e-6) / 1e9
+        if r["bound"] == "hbm":
+            assert r["unit"] == "GB/s" and r["frac"] == pytest.approx(gbps / 6000.0)
+            assert r["other"]["frac"] == pytest.approx(tf / 1200.0)
+        else:
+            assert r["unit"] == "TFLOP/s" and r["frac"] == pytest.approx(tf / 1200.0)
+            assert r["other"]["frac"] == pytest.approx(gbps / 6000.0)
+    assert bench.shared_roofline(2.0 * 8 * 3 * 7168 * 2048, wbytes, 0.04, pk)["bound"] == "hbm"
+    assert bench.shared_roofline(2.0 * 8192 * 3 * 7168 * 2048, wbytes, 0.6, pk)["bound"] == "tensor"
