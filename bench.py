@@ -692,15 +692,19 @@ def layer_figures(args, w, r, world):
     # dense ratios); the block-scaled FP8 x FP4 MMA runs at the FP8 rate
     ratio = 2.0 if args.format == "mx" else 4.0
     spec_tc = SPEC_FP8_TFLOPS * ratio / 2.0
-    if w.T * w.k > 8 * w.E:
-        # large batches: each weight byte feeds ~T*k/E rows, and the tensor
-        # pipe binds as much as HBM.  The denominator is the sustained peak
-        # (the power-capped regime of a long run); the burst and spec
-        # fractions are given beside it, and "clocks" shows the regime the
-        # timed region actually ran in.
-        kflops = 2.0 * w.T * w.k * (2 * w.I if g1_ms >= g2_ms else w.H) * (w.H if g1_ms >= g2_ms else w.I)
-        peak_s, peak_b = ratio * pk["bf16_sustained"], ratio * pk["bf16"]
-        tflops = kflops / (kms * 1e-3) / 1e12
+    # the binding roofline of the dominant kernel: its algorithmic FLOPs at the
+    # sustained tensor peak (the power-capped regime of a long run; burst and
+    # spec beside it, and "clocks" shows the regime the timed region ran in)
+    # against its algorithmic bytes at the measured HBM bandwidth, whichever
+    # takes longer; the other fraction is reported beside it
+    kflops = 2.0 * w.T * w.k * (2 * w.I if g1_ms >= g2_ms else w.H) * (w.H if g1_ms >= g2_ms else w.I)
+    peak_s, peak_b = ratio * pk["bf16_sustained"], ratio * pk["bf16"]
+    tflops = kflops / (kms * 1e-3) / 1e12
+    tensor_frac = {"achieved": tflops, "peak": peak_s, "unit": "TFLOP/s", "frac": tflops / peak_s,
+                   "frac_of_burst": tflops / peak_b, "algorithmic_flops": kflops}
+    if kflops / (peak_s * 1e12) <= kbytes / (pk["hbm"] * 1e9):
+        roofline["tensor"] = tensor_frac
+    else:
         roofline = {"kernel": kname, "bound": "tensor", "achieved": tflops, "peak": peak_s, "unit": "TFLOP/s",
                     "frac": tflops / peak_s,
                     "peak_source": pk["source"] + f" sustained ({ratio:g} x bf16_tflops_sustained)",

@@ -116,3 +116,34 @@ def test_shared_roofline_takes_the_binding_bound():
             assert r["other"]["frac"] == pytest.approx(gbps / 6000.0)
     assert bench.shared_roofline(2.0 * 8 * 3 * 7168 * 2048, wbytes, 0.04, pk)["bound"] == "hbm"
     assert bench.shared_roofline(2.0 * 8192 * 3 * 7168 * 2048, wbytes, 0.6, pk)["bound"] == "tensor"
+
+
+def test_layer_roofline_takes_the_binding_bound():
+    """The layer's roofline is the dominant GEMM's binding one: HBM when its
+    algorithmic bytes at the measured bandwidth take longer than its FLOPs at
+    the sustained tensor peak (decode; NVFP4 at prefill, whose FP4 MMA runs at
+    twice the FP8 rate), else the tensor pipe (FP8 x FP4 prefill), with the
+    other fraction beside it."""
+    import types
+
+    import numpy as np
+    import torch
+    pk = bench.peaks()
+    for wi, fmt, want in [(1, "mx", "hbm"), (3, "mx", "tensor"), (3, "nvfp4", "hbm"), (4, "mx", "tensor")]:
+        w = W.WORKLOADS[wi]
+        idx = (torch.arange(w.T * w.k) % w.E).view(w.T, w.k)
+        r = dict(g={"idx": idx}, ms=2.0, stage_ms=np.array([[0.01, 1.2, 0.6, 0.05]]), staged_ms=2.0, clocks={})
+        f = bench.layer_figures(types.SimpleNamespace(format=fmt, steps=1), w, r, 1)
+        ro = f["roofline"]
+        b1, _ = bench.expert_bytes(w, fmt)
+        kbytes = min(w.T * w.k, w.E) * b1  # the experts the routing touches
+        kflops = 2.0 * w.T * w.k * 2 * w.I * w.H
+        peak_tc = (2.0 if fmt == "mx" else 4.0) * pk["bf16_sustained"]
+        assert ro["bound"] == want, (w.name, fmt)
+        assert want == ("hbm" if kbytes / (pk["hbm"] * 1e9) >= kflops / (peak_tc * 1e12) else "tensor")
+        if want == "hbm":
+            assert ro["frac"] == pytest.approx(kbytes / 1.2e-3 / 1e9 / pk["hbm"])
+            assert ro["tensor"]["frac"] == pytest.approx(kflops / 1.2e-3 / 1e12 / peak_tc)
+        else:
+            assert ro["frac"] == pytest.approx(kflops / 1.2e-3 / 1e12 / peak_tc)
+            assert ro["hbm"]["frac"] == pytest.approx(kbytes / 1.2e-3 / 1e9 / pk["hbm"])
