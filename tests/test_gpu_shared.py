@@ -48,6 +48,7 @@ def run_and_compare(moe, T, SH, SI, seed, tokens=None, situ=None, repeat=True):
     (300, 384, 256, 3),      # odd output-tile count: GEMM2's last pair holds one tile
     (1100, 256, 128, 4),     # 128-token blocks, ragged last block
     (128, 256, 256, 8),      # 32-token blocks at the largest such T
+    (5, 128, 128, 24),       # the smallest shapes: one intermediate tile, one output tile (GEMM2 pair half empty)
 ])
 def test_shared_small(moe, T, SH, SI, seed):
     run_and_compare(moe, T, SH, SI, seed)
@@ -55,6 +56,13 @@ def test_shared_small(moe, T, SH, SI, seed):
 
 def test_shared_situ(moe):
     run_and_compare(moe, 70, 256, 256, 5, situ=(1.25, 1.5))
+
+
+def test_shared_situ_without_linear_term(moe):
+    """SiTU with no linear_beta: the up projection enters unclipped, on the
+    K-split cluster path (T = 8) and with 128-token blocks (T = 200)."""
+    run_and_compare(moe, 8, 1024, 512, 25, situ=(2.0, None))
+    run_and_compare(moe, 200, 512, 256, 26, situ=(0.75, None))
 
 
 def test_shared_full_size_sampled(moe):
