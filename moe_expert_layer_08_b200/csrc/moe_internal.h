@@ -90,11 +90,13 @@ constexpr int kActBoxRows = 32;  // activation rows per TMA box
 cudaError_t launch_combine(const uint8_t *ws, const WsLayout &L, const float *topk_w, int T, int k, int H,
                            void *out, cudaStream_t stream);
 
-// BF16 shared expert: tokens per work item (32 up to kSharedSmallT tokens,
-// else 128) and the launch of GEMM1 (tmap_w over L1 [2SI][SH], tmap_act over x
-// [T][SH], out = h [T][SI]) or GEMM2 (L2 [SH][SI], h, out = y [T][SH]); the
-// maps' boxes are 128 / shared_block_rows(T) rows of 64 bf16.  part: scratch
-// of shared_part_bytes(T) bytes for K-split partial sums.
+// BF16 shared expert: tokens per work item (32 up to kSharedTinyT tokens, 64
+// up to kSharedSmallT, else 128) and the launch of GEMM1 (tmap_w over L1
+// [2SI][SH], tmap_act over x [T][SH], out = h [T][SI]) or GEMM2 (L2 [SH][SI],
+// h, out = y [T][SH]); the maps' boxes are 128 / shared_block_rows(T) rows of
+// 64 bf16.  part: scratch of shared_part_bytes(T) bytes for K-split partial
+// sums.
+constexpr int kSharedTinyT = 64;
 constexpr int kSharedSmallT = 128;
 int shared_block_rows(int T);
 size_t shared_part_bytes(int T);

@@ -29,14 +29,14 @@ namespace moe {
 
 template <int kN>
 struct SharedCfg {
-    static constexpr int kStages = kN == 128 ? 4 : 6;
+    static constexpr int kStages = kN == 128 ? 4 : (kN == 64 ? 5 : 6);
     static constexpr int kATile = kTileRows * kTileK;  // 16 KB: 128 rows x 64 bf16
     static constexpr int kBTile = kN * kTileK;
     static constexpr int kStageBytes = 2 * kATile + kBTile;
     static constexpr int kSmemMisc = 256;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kSmemMisc;
     static constexpr int kAccCols = 2 * kN;  // one accumulator buffer: tile 0, tile 1
-    static constexpr int kTmemCols = 4 * kN <= 128 ? 128 : 512;
+    static constexpr int kTmemCols = 4 * kN <= 128 ? 128 : (4 * kN <= 256 ? 256 : 512);
     static constexpr int kEpiWarps = kN == 128 ? 8 : 4;
     static constexpr int kThreads = 32 * (kEpiWarps == 8 ? 12 : 8);
     static_assert(4 * kN <= kTmemCols, "two accumulator buffers");
@@ -47,18 +47,20 @@ struct SharedCfg {
 
 // K-split partial sums: one unit holds a part's fp32 accumulators of both
 // tiles of its item, [tile][token][128 rows]; the scratch holds 256 units of
-// 32-token blocks (8 MiB) or 160 of 128-token blocks (20 MiB), and no split
-// needs more (about one unit per SM)
+// 32-token blocks (8 MiB), 256 of 64-token blocks (16 MiB) or 160 of
+// 128-token blocks (20 MiB), and no split needs more (about one unit per SM)
 template <int kN>
 constexpr int kSharedPartUnitFloats = 2 * kN * kTileRows;
 constexpr int kSharedMaxUnits32 = 256;
+constexpr int kSharedMaxUnits64 = 256;
 constexpr int kSharedMaxUnits128 = 160;
 // the most parts of one item that run as a thread-block cluster (above 8 the
 // cluster size is non-portable: used where the device can hold the clusters),
 // and how many parts the split may drop so that its clusters fit at once
 constexpr int kSharedMaxClusterParts = 16;
 constexpr int kSharedClusterShrink = 2;
-static_assert(kSharedMaxUnits32 / 2 <= kHdrSplitWords && kSharedMaxUnits128 / 2 <= kHdrSplitWords,
+static_assert(kSharedMaxUnits32 / 2 <= kHdrSplitWords && kSharedMaxUnits64 / 2 <= kHdrSplitWords &&
+                  kSharedMaxUnits128 / 2 <= kHdrSplitWords,
               "a split item's counter in the header");
 
 struct SharedArgs {
@@ -610,11 +612,13 @@ static cudaError_t launch_shared_t(const CUtensorMap &tmap_w, const CUtensorMap 
     return cudaLaunchKernelEx(&cfg, shared_gemm_kernel<kGemm1, kN, kSplit>, tmap_w, tmap_act, a);
 }
 
-int shared_block_rows(int T) { return T <= kSharedSmallT ? 32 : 128; }
+int shared_block_rows(int T) { return T <= kSharedTinyT ? 32 : T <= kSharedSmallT ? 64 : 128; }
 
 size_t shared_part_bytes(int T) {
-    return shared_block_rows(T) == 32 ? size_t(kSharedMaxUnits32) * kSharedPartUnitFloats<32> * sizeof(float)
-                                      : size_t(kSharedMaxUnits128) * kSharedPartUnitFloats<128> * sizeof(float);
+    const int kn = shared_block_rows(T);
+    return kn == 32   ? size_t(kSharedMaxUnits32) * kSharedPartUnitFloats<32> * sizeof(float)
+           : kn == 64 ? size_t(kSharedMaxUnits64) * kSharedPartUnitFloats<64> * sizeof(float)
+                      : size_t(kSharedMaxUnits128) * kSharedPartUnitFloats<128> * sizeof(float);
 }
 
 cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorMap &tmap_act, int T, int SH, int SI,
@@ -653,7 +657,7 @@ cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorM
     // 64-element K blocks each) so that about every SM works, as many units
     // as the partial-sum scratch holds
     const int sms = num_sms();
-    const int max_units = kn == 32 ? kSharedMaxUnits32 : kSharedMaxUnits128;
+    const int max_units = kn == 32 ? kSharedMaxUnits32 : kn == 64 ? kSharedMaxUnits64 : kSharedMaxUnits128;
     a.split = 1;
     if (items < sms) {
         int s = sms / items;
@@ -661,11 +665,14 @@ cudaError_t launch_shared(bool gemm1, const CUtensorMap &tmap_w, const CUtensorM
         if (s > max_units / items) s = max_units / items;
         a.split = s > 1 ? s : 1;
     }
-    // 32-token blocks: one kernel for both; 128-token blocks: the K-split
-    // epilogue only in the kernel that needs it
+    // 32- and 64-token blocks: one kernel with and without a split; 128-token
+    // blocks: the K-split epilogue only in the kernel that needs it
     if (kn == 32)
         return gemm1 ? launch_shared_t<true, 32, true>(tmap_w, tmap_act, a, items, stream)
                      : launch_shared_t<false, 32, true>(tmap_w, tmap_act, a, items, stream);
+    if (kn == 64)
+        return gemm1 ? launch_shared_t<true, 64, true>(tmap_w, tmap_act, a, items, stream)
+                     : launch_shared_t<false, 64, true>(tmap_w, tmap_act, a, items, stream);
     if (a.split > 1)
         return gemm1 ? launch_shared_t<true, 128, true>(tmap_w, tmap_act, a, items, stream)
                      : launch_shared_t<false, 128, true>(tmap_w, tmap_act, a, items, stream);

@@ -183,17 +183,21 @@ def test_nvfp4_entry_points_validate_on_the_host(moelib):
 
 def test_shared_expert_entry_points_validate_on_the_host(moelib):
     """Workspace size = 2 KiB header + h [T, SI] bf16 (256-aligned) + the
-    K-split partial sums (up to 128 tokens: 256 units of 32-token blocks, 8
-    MiB; above: 160 units of 128-token blocks, 20 MiB); shapes, token counts,
-    activations and sizes are checked before any CUDA call."""
+    K-split partial sums (up to 64 tokens: 256 units of 32-token blocks, 8
+    MiB; up to 128: 256 units of 64-token blocks, 16 MiB; above: 160 units of
+    128-token blocks, 20 MiB); shapes, token counts, activations and sizes are
+    checked before any CUDA call."""
     import ctypes
     import moe_expert_layer_08_b200 as m
     lib = m.load()
     scratch32 = 256 * 2 * 32 * 128 * 4
+    scratch64 = 256 * 2 * 64 * 128 * 4
     scratch128 = 160 * 2 * 128 * 128 * 4
     assert m.shared_workspace_bytes(8192, 7168, 2048) == 2048 + 8192 * 2048 * 2 + scratch128
     assert m.shared_workspace_bytes(129, 7168, 2048) == 2048 + 129 * 2048 * 2 + scratch128
-    assert m.shared_workspace_bytes(128, 7168, 2048) == 2048 + 128 * 2048 * 2 + scratch32
+    assert m.shared_workspace_bytes(128, 7168, 2048) == 2048 + 128 * 2048 * 2 + scratch64
+    assert m.shared_workspace_bytes(65, 7168, 2048) == 2048 + 65 * 2048 * 2 + scratch64
+    assert m.shared_workspace_bytes(64, 7168, 2048) == 2048 + 64 * 2048 * 2 + scratch32
     assert m.shared_workspace_bytes(3, 256, 128) == 2048 + 768 + scratch32
     assert m.shared_workspace_bytes(0, 256, 128) == 2048 + scratch32
     n = ctypes.c_size_t()

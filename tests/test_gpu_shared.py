@@ -1,8 +1,9 @@
 """GPU parity of the BF16 shared expert (moe_shared_forward through the C ABI)
 against the oracle, per token row: rel L2 <= 1e-2 and max abs <= 5e-2 *
 max|row| (the DeepGEMM PR #416 test body bounds the shared output's relative
-L2 by 1e-2).  Small cases on every token, with both token-block sizes (32-token
-blocks up to T = 128, else 128-token blocks), with and without a K split,
+L2 by 1e-2).  Small cases on every token, with every token-block size (32-token
+blocks up to T = 64, 64-token blocks up to 128, else 128-token blocks), with
+and without a K split,
 ragged token counts and an odd output-tile count;
 the full-size case on sampled tokens."""
 import numpy as np
@@ -45,9 +46,11 @@ def run_and_compare(moe, T, SH, SI, seed, tokens=None, situ=None, repeat=True):
 @pytest.mark.parametrize("T,SH,SI,seed", [
     (1, 256, 128, 1),        # one token
     (37, 512, 256, 2),       # ragged 32-token blocks
+    (64, 512, 256, 27),      # 32-token blocks at the largest such T
+    (100, 384, 256, 28),     # two 64-token blocks (64, 36 rows), odd output-tile count
     (300, 384, 256, 3),      # odd output-tile count: GEMM2's last pair holds one tile
     (1100, 256, 128, 4),     # 128-token blocks, ragged last block
-    (128, 256, 256, 8),      # 32-token blocks at the largest such T
+    (128, 256, 256, 8),      # 64-token blocks at the largest such T
     (5, 128, 128, 24),       # the smallest shapes: one intermediate tile, one output tile (GEMM2 pair half empty)
 ])
 def test_shared_small(moe, T, SH, SI, seed):
@@ -86,7 +89,7 @@ def test_shared_decode_size_situ(moe):
 
 def test_shared_split_ragged_blocks(moe):
     """T = 40 at full size: two 32-token blocks (32 and 8 rows), each item's K
-    cut into an even number of parts."""
+    cut into parts across a cluster."""
     run_and_compare(moe, 40, 7168, 2048, 10)
 
 
@@ -143,3 +146,19 @@ def test_shared_split_global_partials(moe):
     SH = 7168, SI = 128: one GEMM1 item in 28 parts) adds its partials through
     global memory, the last part to finish reducing them."""
     run_and_compare(moe, 8, 7168, 128, 23)
+
+
+@pytest.mark.parametrize("T,SH,SI,seed,situ", [
+    (96, 1024, 512, 29, None),           # 64-token blocks (64, 32 rows), both GEMMs K-split
+    (65, 768, 384, 30, (1.25, 1.5)),     # the smallest such T: a last block of one token, SiTU
+])
+def test_shared_split_64_token_blocks(moe, T, SH, SI, seed, situ):
+    """65 to 128 tokens: 64-token blocks, each item's K cut into parts; every
+    token checked."""
+    run_and_compare(moe, T, SH, SI, seed, situ=situ)
+
+
+def test_shared_64_token_blocks_full_size(moe):
+    """T = 96 at SH = 7168, SI = 2048 (two 64-token blocks, 32 GEMM1 items
+    split four ways), every token."""
+    run_and_compare(moe, 96, 7168, 2048, 31)
