@@ -421,8 +421,8 @@ moe_status_t moe_probe_wait_timeout(void *workspace, size_t ws_bytes, unsigned t
  * moe_shared_workspace_bytes -- bytes of device workspace moe_shared_forward
  *   needs for up to T_max tokens (a 2 KiB header with the device error word,
  *   then h [T, SI] bf16, then the fp32 partial sums of the K split that
- *   token counts with fewer work items than SMs use: 8 MiB up to 128 tokens,
- *   20 MiB above; the size never falls as T_max grows).
+ *   token counts with fewer work items than SMs use: 8 MiB up to 64 tokens,
+ *   16 MiB up to 128, 20 MiB above; the size never falls as T_max grows).
  *   MOE_ERR_UNSUPPORTED_SHAPE unless SH and SI are multiples of 128.
  *
  * moe_shared_forward -- y for T tokens.  All pointers are device pointers on
