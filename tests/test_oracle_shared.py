@@ -1,7 +1,7 @@
 """Pins of the oracle's BF16 shared expert (DeepGEMM PR #416, BF16 shared-expert
 test body): against an independent float64 numpy evaluation with torch's bf16
-rounding between the steps, its SiTU form, a closed-form special case and
-token-permutation equivariance."""
+rounding between the steps, its SiTU form with and without the linear term,
+a closed-form special case and token-permutation equivariance."""
 import numpy as np
 import pytest
 import torch
@@ -67,6 +67,20 @@ def test_shared_situ_matches_float64_reference():
     y_ref, h_ref = reference(x, l1, l2, situ(1.25, 1.5))
     assert_close_bits(got["h"], h_ref, "h")
     assert_close_bits(got["y"], y_ref, "y")
+
+
+def test_shared_situ_without_linear_term_matches_float64_reference():
+    """SiTU with no linear_beta: the up projection enters as it is,
+    sigmoid(g) * beta * tanh(g / beta) * u (and differs from the form with a
+    linear term)."""
+    x, l1, l2 = draws(4, 128, 64, 8)
+    got = oracle.shared_forward(x, l1, l2, activation="situ", beta=2.0, linear_beta=None, intermediates=True)
+    plain = lambda g, u: (1.0 / (1.0 + np.exp(-g))) * (2.0 * np.tanh(g / 2.0)) * u
+    y_ref, h_ref = reference(x, l1, l2, plain)
+    assert_close_bits(got["h"], h_ref, "h")
+    assert_close_bits(got["y"], y_ref, "y")
+    clipped = oracle.shared_forward(x, l1, l2, activation="situ", beta=2.0, linear_beta=0.05)["y"]
+    assert not np.array_equal(clipped, got["y"])
 
 
 def test_shared_gate_first_and_orientation():
