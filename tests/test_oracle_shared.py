@@ -83,6 +83,16 @@ def test_shared_situ_without_linear_term_matches_float64_reference():
     assert not np.array_equal(clipped, got["y"])
 
 
+def test_shared_situ_with_large_betas_is_swiglu():
+    """beta * tanh(g / beta) -> g and lbeta * tanh(u / lbeta) -> u as the betas
+    grow, so SiTU with betas of 1e9 gives SwiGLU's bits."""
+    x, l1, l2 = draws(5, 128, 64, 9)
+    swig = oracle.shared_forward(x, l1, l2, intermediates=True)
+    big = oracle.shared_forward(x, l1, l2, activation="situ", beta=1e9, linear_beta=1e9, intermediates=True)
+    assert_close_bits(big["h"], swig["h"], "h")
+    assert_close_bits(big["y"], swig["y"], "y")
+
+
 def test_shared_gate_first_and_orientation():
     """Swapping the gate and up halves, or transposing L2's role, changes the
     result (the reference above takes gate = first SI rows of L1)."""
