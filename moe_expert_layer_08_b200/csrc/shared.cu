@@ -29,7 +29,7 @@ namespace moe {
 
 // kN = tokens per block (32 up to 64 tokens, 64 up to 128, else 128): a stage
 // holds the item's two 128-row weight tiles and the block's token tile of one
-// 64-element K block, as many stages as fit about 205-220 KB of shared memory.
+// 64-element K block; as many stages as fit (192-216 KB of shared memory).
 template <int kN>
 struct SharedCfg {
     static constexpr int kStages = kN == 128 ? 4 : (kN == 64 ? 5 : 6);
